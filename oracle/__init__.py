@@ -1,0 +1,206 @@
+"""CPU oracle for the activation-sparsified linear layer (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA
+library ``sparse_linear_b200`` and never imports it.
+
+``oracle.c`` holds the float64 definitions (plus the float32 score/selection
+decision); this module compiles it with gcc on first use, loads it with
+ctypes and wraps each function for numpy arrays.  ``brute.py`` holds an
+independent pure-Python enumerator for tiny cases.
+
+Functions and the passages they follow (page title, section):
+
+* ``weight_prep``   WiSparse page §2.1 eq. (4) (g) and activation-sparsity
+                    overview §3.1 (rowsum for the mean shift).
+* ``token_mean``    overview §3.1 (D-PTS eta).
+* ``token_var``     overview §3.2 (VAR, unbiased variance).
+* ``channel_energy``/``clact_full``  overview §2.2.3 (CLACT).
+* ``score``         overview §2.2.1, §2.2.3, §3.1; WiSparse eq. (4).
+* ``select_nm``     overview §2.1 / §2.2.1 (block top-N).
+* ``select_topk``   WiSparse §2.2 (per-layer keep fraction).
+* ``var_scale``     overview §3.2.
+* ``linear``        overview §3.1 / §3.2 and the layer definition y = prune(x) W^T.
+* ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+          "-fno-fast-math", "-Wall"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (gcc, no CUDA)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            D = ctypes.c_double
+            sig = {
+                "or_weight_prep": [P, I, I, D, P, P],
+                "or_token_mean": [P, I, I, P],
+                "or_token_var": [P, I, I, P],
+                "or_channel_energy": [P, I, I, P],
+                "or_clact_full": [P, I, I, P],
+                "or_score": [P, I, I, P, P, P],
+                "or_select_nm": [P, I, I, I, I, P],
+                "or_select_topk": [P, I, I, I, P],
+                "or_var_scale": [P, P, I, I, P, D, D, P, P, P, P],
+                "or_linear": [P, P, I, I, P, P, I, P, P, P, I, P],
+                "or_compress_nm": [P, P, I, I, I, I, P, P],
+            }
+            for name, args in sig.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = None
+            _lib = lib
+    return _lib
+
+
+def _f32(a):
+    a = a.float().numpy() if hasattr(a, "numpy") and not isinstance(a, np.ndarray) else a
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def weight_prep(W, alpha: float):
+    """g [k] = ||W[:,i]||_2^alpha and rowsum [n_out], float64."""
+    W = _f32(W)
+    n_out, k = W.shape
+    g = np.empty(k, np.float64)
+    rs = np.empty(n_out, np.float64)
+    _load().or_weight_prep(_ptr(W), n_out, k, float(alpha), _ptr(g), _ptr(rs))
+    return g, rs
+
+
+def token_mean(x):
+    x = _f32(x)
+    T, k = x.shape
+    out = np.empty(T, np.float64)
+    _load().or_token_mean(_ptr(x), T, k, _ptr(out))
+    return out
+
+
+def token_var(x):
+    x = _f32(x)
+    T, k = x.shape
+    out = np.empty(T, np.float64)
+    _load().or_token_var(_ptr(x), T, k, _ptr(out))
+    return out
+
+
+def channel_energy(x):
+    x = _f32(x)
+    T, k = x.shape
+    out = np.empty(k, np.float64)
+    _load().or_channel_energy(_ptr(x), T, k, _ptr(out))
+    return out
+
+
+def clact_full(x):
+    x = _f32(x)
+    T, k = x.shape
+    out = np.empty((T, k), np.float64)
+    _load().or_clact_full(_ptr(x), T, k, _ptr(out))
+    return out
+
+
+def score(x, eta=None, f=None):
+    """float32 score: fl32(|fl32(x - eta)| * f) (eta, f optional, float32)."""
+    x = _f32(x)
+    T, k = x.shape
+    e = None if eta is None else np.ascontiguousarray(eta, np.float32).reshape(T)
+    ff = None if f is None else np.ascontiguousarray(f, np.float32).reshape(k)
+    s = np.empty((T, k), np.float32)
+    _load().or_score(_ptr(x), T, k, _ptr(e), _ptr(ff), _ptr(s))
+    return s
+
+
+def select_nm(s, n: int, m: int):
+    s = np.ascontiguousarray(s, np.float32)
+    T, k = s.shape
+    if k % m:
+        raise ValueError("k must be a multiple of m")
+    mask = np.empty((T, k), np.uint8)
+    _load().or_select_nm(_ptr(s), T, k, int(n), int(m), _ptr(mask))
+    return mask
+
+
+def select_topk(s, kk: int):
+    s = np.ascontiguousarray(s, np.float32)
+    T, k = s.shape
+    mask = np.empty((T, k), np.uint8)
+    _load().or_select_topk(_ptr(s), T, k, int(kk), _ptr(mask))
+    return mask
+
+
+def var_scale(x, mask, running_in=None, momentum: float = 0.9, eps: float = 1e-6):
+    """Returns dict var_dense, var_kept, running, nu (float64 [T])."""
+    x = _f32(x)
+    T, k = x.shape
+    mask = np.ascontiguousarray(mask, np.uint8)
+    rin = None if running_in is None else np.ascontiguousarray(running_in, np.float64)
+    out = {n: np.empty(T, np.float64) for n in ("var_dense", "var_kept", "running", "nu")}
+    _load().or_var_scale(_ptr(x), _ptr(mask), T, k, _ptr(rin), float(momentum), float(eps),
+                         _ptr(out["var_dense"]), _ptr(out["var_kept"]),
+                         _ptr(out["running"]), _ptr(out["nu"]))
+    return out
+
+
+def linear(x, mask, W, eta=None, rowsum=None, nu=None, rows=None):
+    """float64 y[r, o] over the kept channels (see oracle.c)."""
+    x = _f32(x)
+    W = _f32(W)
+    T, k = x.shape
+    n_out = W.shape[0]
+    mask = np.ascontiguousarray(mask, np.uint8)
+    e = None if eta is None else np.ascontiguousarray(eta, np.float64)
+    rs = None if rowsum is None else np.ascontiguousarray(rowsum, np.float64)
+    if e is not None and rs is None:
+        raise ValueError("eta needs rowsum")
+    nv = None if nu is None else np.ascontiguousarray(nu, np.float64)
+    rr = None if rows is None else np.ascontiguousarray(rows, np.int32)
+    n_rows = T if rr is None else len(rr)
+    y = np.empty((n_rows, n_out), np.float64)
+    _load().or_linear(_ptr(x), _ptr(mask), T, k, _ptr(e), _ptr(W), n_out, _ptr(rs),
+                      _ptr(nv), _ptr(rr), n_rows, _ptr(y))
+    return y
+
+
+def compress_nm(v, mask, n: int, m: int):
+    """Kept values of each block, contiguous in channel order, and positions."""
+    v = _f32(v)
+    T, k = v.shape
+    mask = np.ascontiguousarray(mask, np.uint8)
+    kc = k // m * n
+    vals = np.empty((T, kc), np.float32)
+    pos = np.empty((T, kc), np.uint8)
+    _load().or_compress_nm(_ptr(v), _ptr(mask), T, k, int(n), int(m), _ptr(vals), _ptr(pos))
+    return vals, pos

@@ -1,0 +1,298 @@
+/*
+ * Reference oracle for the activation-sparsified linear layer y = prune(x) W^T.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code with the CUDA library.
+ *
+ * Plain, slow, obviously correct: every quantity is computed from its
+ * definition, statistics and contractions in float64, with no blocking,
+ * fusion or reordering.  The only float32 arithmetic is the channel score,
+ * because the selection decision is taken in float32 on both sides (one
+ * float32 subtraction for the mean shift, one float32 multiply for the
+ * score).  Build with -ffp-contract=off and without fast-math.
+ *
+ * Sources (page title, section):
+ *   [OVW]  "激活稀疏化技术：提升LLM推理效率的动态剪枝方法"
+ *          (activation-sparsity overview): section 2.1 N:M patterns,
+ *          2.2.1 magnitude pruning, 2.2.3 CLACT score, 3.1 D-PTS,
+ *          3.2 VAR variance correction.
+ *   [WIS]  "大模型推理优化：WiSparse激活稀疏化技术解析": section 2.1, eq. (4),
+ *          weight-aware score s_i = |x_i| * ||W[:,i]||_2^alpha; section 2.2
+ *          per-layer keep fraction (top-k).
+ *   [SQR]  "利用2:4稀疏性与Squared-ReLU加速Transformer训练与推理": section 2.1
+ *          2:4 pattern, 2.3 dropping the smallest of a 3-nonzero block,
+ *          3.3 compressed layout with the kept values stored contiguously.
+ *
+ * Readings where the pages are silent or disagree (all listed in the design
+ * notes): exactly N per M-block (or exactly k per token), equal float32
+ * scores broken towards the lower channel index; blocks are [jM, jM+M);
+ * the weight norm runs over the output rows of input column i; the CLACT
+ * row factor is constant within a token and so the ranking uses |x_ij| * c_j;
+ * D-PTS adds eta back to every channel, i.e. y = (xhat*m) W^T + eta*rowsum(W);
+ * VAR: unbiased variances, running variance initialised to the first batch's
+ * dense variance and updated with momentum before the scale is formed, scale
+ * = sqrt(running / (Var[x*m] + eps)), applied to the whole output row.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------------------
+ * Weight preparation.  [WIS] section 2.1, eq. (4): g_i = (||W[:,i]||_2)^alpha,
+ * the norm taken over the n_out output rows of input column i; precomputed
+ * once per layer.  [OVW] section 3.1: rowsum_o = sum_i W[o,i], the term that
+ * restores the shifted-out mean (y = (x_sparse + eta) W^T).
+ * W is [n_out, k] row-major (PyTorch Linear layout).
+ * ------------------------------------------------------------------------- */
+void or_weight_prep(const float *W, int n_out, int k, double alpha,
+                    double *g, double *rowsum)
+{
+    if (g) {
+        #pragma omp parallel for schedule(static)
+        for (int i = 0; i < k; i++) {
+            double ss = 0.0;
+            for (int o = 0; o < n_out; o++) {
+                double w = (double)W[(size_t)o * k + i];
+                ss += w * w;
+            }
+            g[i] = pow(sqrt(ss), alpha);
+        }
+    }
+    if (rowsum) {
+        #pragma omp parallel for schedule(static)
+        for (int o = 0; o < n_out; o++) {
+            double s = 0.0;
+            for (int i = 0; i < k; i++) s += (double)W[(size_t)o * k + i];
+            rowsum[o] = s;
+        }
+    }
+}
+
+/* [OVW] section 3.1: eta_t = mean over the channels of token t. */
+void or_token_mean(const float *x, int T, int k, double *eta)
+{
+    for (int t = 0; t < T; t++) {
+        double s = 0.0;
+        for (int i = 0; i < k; i++) s += (double)x[(size_t)t * k + i];
+        eta[t] = s / (double)k;
+    }
+}
+
+/* Unbiased variance of each token's k channels (two-pass, float64). */
+void or_token_var(const float *x, int T, int k, double *var)
+{
+    for (int t = 0; t < T; t++) {
+        double mean = 0.0;
+        for (int i = 0; i < k; i++) mean += (double)x[(size_t)t * k + i];
+        mean /= (double)k;
+        double ss = 0.0;
+        for (int i = 0; i < k; i++) {
+            double d = (double)x[(size_t)t * k + i] - mean;
+            ss += d * d;
+        }
+        var[t] = ss / (double)(k - 1);
+    }
+}
+
+/* [OVW] section 2.2.3: column energy c_j = sqrt(sum_p x_pj^2) over the T
+ * tokens of the call. */
+void or_channel_energy(const float *x, int T, int k, double *c)
+{
+    for (int j = 0; j < k; j++) {
+        double s = 0.0;
+        for (int p = 0; p < T; p++) {
+            double v = (double)x[(size_t)p * k + j];
+            s += v * v;
+        }
+        c[j] = sqrt(s);
+    }
+}
+
+/* [OVW] section 2.2.3, full CLACT score in float64:
+ * S_ij = |x_ij| / sqrt(sum_k x_ik^2) * sqrt(sum_p x_pj^2). */
+void or_clact_full(const float *x, int T, int k, double *S)
+{
+    double *c = (double *)malloc(sizeof(double) * (size_t)k);
+    or_channel_energy(x, T, k, c);
+    for (int t = 0; t < T; t++) {
+        double r = 0.0;
+        for (int i = 0; i < k; i++) {
+            double v = (double)x[(size_t)t * k + i];
+            r += v * v;
+        }
+        r = sqrt(r);
+        for (int j = 0; j < k; j++)
+            S[(size_t)t * k + j] = fabs((double)x[(size_t)t * k + j]) / r * c[j];
+    }
+    free(c);
+}
+
+/* ---------------------------------------------------------------------------
+ * Channel score in float32, the precision the selection decision is taken in.
+ *   xhat = fl32(x - eta_t)         when eta is given (D-PTS, [OVW] 3.1),
+ *          x                        otherwise;
+ *   s    = fl32(|xhat| * f_i)       f = g ([WIS] eq. 4), c (CLACT, [OVW]
+ *                                   2.2.3, row factor dropped), or 1 when
+ *                                   f is NULL (magnitude, [OVW] 2.2.1).
+ * ------------------------------------------------------------------------- */
+void or_score(const float *x, int T, int k, const float *eta, const float *f,
+              float *s)
+{
+    for (int t = 0; t < T; t++) {
+        for (int i = 0; i < k; i++) {
+            float xh = x[(size_t)t * k + i];
+            if (eta) xh = xh - eta[t];
+            float a = fabsf(xh);
+            s[(size_t)t * k + i] = f ? a * f[i] : a;
+        }
+    }
+}
+
+/* Strict ranking order: higher score first, equal scores by lower index. */
+static int ahead(float sj, int j, float si, int i)
+{
+    return (sj > si) || (sj == si && j < i);
+}
+
+/* [OVW] section 2.1 / 2.2.1: in every block of m consecutive channels
+ * [jm, jm+m) keep the n with the largest score (exactly n; ties to the lower
+ * index).  mask is [T, k] of 0/1. */
+void or_select_nm(const float *s, int T, int k, int n, int m, uint8_t *mask)
+{
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; t++) {
+        const float *st = s + (size_t)t * k;
+        for (int b = 0; b < k; b += m) {
+            for (int i = b; i < b + m; i++) {
+                int rank = 0;
+                for (int j = b; j < b + m; j++)
+                    if (j != i && ahead(st[j], j, st[i], i)) rank++;
+                mask[(size_t)t * k + i] = (uint8_t)(rank < n);
+            }
+        }
+    }
+}
+
+typedef struct { float s; int i; } keyed;
+
+static int cmp_keyed(const void *a, const void *b)
+{
+    const keyed *p = (const keyed *)a, *q = (const keyed *)b;
+    if (p->s > q->s) return -1;
+    if (p->s < q->s) return 1;
+    return (p->i < q->i) ? -1 : (p->i > q->i);
+}
+
+/* [WIS] section 2.2: per-layer keep fraction, i.e. keep the kk channels of
+ * largest score per token (exactly kk; ties to the lower index). */
+void or_select_topk(const float *s, int T, int k, int kk, uint8_t *mask)
+{
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; t++) {
+        keyed *v = (keyed *)malloc(sizeof(keyed) * (size_t)k);
+        for (int i = 0; i < k; i++) { v[i].s = s[(size_t)t * k + i]; v[i].i = i; }
+        qsort(v, (size_t)k, sizeof(keyed), cmp_keyed);
+        memset(mask + (size_t)t * k, 0, (size_t)k);
+        for (int r = 0; r < kk; r++) mask[(size_t)t * k + v[r].i] = 1;
+        free(v);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * [OVW] section 3.2, variance correction:
+ *   var_dense_t = Var[x_t]            (unbiased)
+ *   var_kept_t  = Var[x_t * m_t]      (zeros included, unbiased)
+ *   running_t   = var_dense_t                         on the first batch,
+ *                 mom*running_in_t + (1-mom)*var_dense_t  afterwards
+ *   nu_t        = sqrt(running_t / (var_kept_t + eps))
+ * ------------------------------------------------------------------------- */
+void or_var_scale(const float *x, const uint8_t *mask, int T, int k,
+                  const double *running_in, double momentum, double eps,
+                  double *var_dense, double *var_kept, double *running_out,
+                  double *nu)
+{
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; t++) {
+        double *xm = (double *)malloc(sizeof(double) * (size_t)k);
+        double mean = 0.0, mk = 0.0;
+        for (int i = 0; i < k; i++) {
+            double v = (double)x[(size_t)t * k + i];
+            xm[i] = mask[(size_t)t * k + i] ? v : 0.0;
+            mean += v;
+            mk += xm[i];
+        }
+        mean /= (double)k;
+        mk /= (double)k;
+        double sd = 0.0, sk = 0.0;
+        for (int i = 0; i < k; i++) {
+            double d = (double)x[(size_t)t * k + i] - mean;
+            double e = xm[i] - mk;
+            sd += d * d;
+            sk += e * e;
+        }
+        double vd = sd / (double)(k - 1), vk = sk / (double)(k - 1);
+        double run = running_in ? momentum * running_in[t] + (1.0 - momentum) * vd : vd;
+        if (var_dense) var_dense[t] = vd;
+        if (var_kept) var_kept[t] = vk;
+        if (running_out) running_out[t] = run;
+        if (nu) nu[t] = sqrt(run / (vk + eps));
+        free(xm);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Contraction over the kept channels, float64:
+ *   y[r,o] = nu_t * ( sum_i xhat_ti * m_ti * W[o,i]  +  eta_t * rowsum_o )
+ * with t = rows[r] (all tokens when rows is NULL), xhat = x - eta when eta is
+ * given (D-PTS, [OVW] 3.1: y = (x_sparse + eta) W^T, the eta added back to
+ * every channel) else x, the rowsum term only with eta, and nu only when
+ * given (VAR, [OVW] 3.2: y = scale * (x_sparse W^T)).
+ * ------------------------------------------------------------------------- */
+void or_linear(const float *x, const uint8_t *mask, int T, int k,
+               const double *eta, const float *W, int n_out,
+               const double *rowsum, const double *nu, const int *rows,
+               int n_rows, double *y)
+{
+    (void)T;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n_rows; r++) {
+        double *xv = (double *)malloc(sizeof(double) * (size_t)k);
+        int t = rows ? rows[r] : r;
+        for (int i = 0; i < k; i++) {
+            double v = (double)x[(size_t)t * k + i];
+            if (eta) v -= eta[t];
+            xv[i] = mask[(size_t)t * k + i] ? v : 0.0;
+        }
+        for (int o = 0; o < n_out; o++) {
+            const float *wr = W + (size_t)o * k;
+            double acc = 0.0;
+            for (int i = 0; i < k; i++) acc += xv[i] * (double)wr[i];
+            if (eta) acc += eta[t] * rowsum[o];
+            if (nu) acc *= nu[t];
+            y[(size_t)r * n_out + o] = acc;
+        }
+        free(xv);
+    }
+}
+
+/* [SQR] section 3.3: compressed N:M layout, the kept values of every block
+ * stored contiguously in ascending channel order, with their positions
+ * inside the block.  values/pos are [T, k/m*n].  The mask must hold exactly n
+ * per block. */
+void or_compress_nm(const float *v, const uint8_t *mask, int T, int k, int n,
+                    int m, float *values, uint8_t *pos)
+{
+    size_t kc = (size_t)k / (size_t)m * (size_t)n;
+    for (int t = 0; t < T; t++) {
+        size_t w = 0;
+        for (int b = 0; b < k; b += m)
+            for (int i = b; i < b + m; i++)
+                if (mask[(size_t)t * k + i]) {
+                    values[(size_t)t * kc + w] = v[(size_t)t * k + i];
+                    pos[(size_t)t * kc + w] = (uint8_t)(i - b);
+                    w++;
+                }
+    }
+}

@@ -1,0 +1,340 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself (a value the pages print, a closed form, an invariant, a special case
+that reduces to a plain library routine, or brute-force enumeration), chosen
+so that a dropped term, a wrong sign or index, or a transposed operand in the
+oracle fails at least one of them.  No GPU needed."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _bf16(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+# --------------------------------------------------------------------------
+# Page-printed values: the N:M pattern table (overview page, section 2.1).
+# --------------------------------------------------------------------------
+def _table():
+    rows = []
+    with open(os.path.join(GOLDEN, "nm_table.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            pat, cnt, bits = line.split()
+            n, m = map(int, pat.split(":"))
+            rows.append((n, m, float(cnt), float(bits)))
+    return rows
+
+
+def _count_dp(m, n):
+    # Pascal's rule, a different route from enumeration.
+    row = [1]
+    for _ in range(m):
+        row = [1] + [row[i] + row[i + 1] for i in range(len(row) - 1)] + [1]
+    return row[n]
+
+
+def test_nm_table_keep_pattern_counts():
+    for n, m, cnt, _ in _table():
+        if m <= 16:
+            assert brute.count_subsets(m, n) == int(cnt)
+        else:  # printed to one significant digit
+            c = _count_dp(m, n)
+            assert round(c / 1e8) == round(cnt / 1e8)
+
+
+def test_nm_table_metadata_bits():
+    for n, m, cnt, bits in _table():
+        if (n, m) == (4, 8):
+            continue  # printed 0.81, ceil(log2 70)/8 = 0.875: garbled row
+        c = brute.count_subsets(m, n) if m <= 16 else _count_dp(m, n)
+        assert round(math.ceil(math.log2(c)) / m, 2) == round(bits, 2)
+
+
+# --------------------------------------------------------------------------
+# Selection: brute-force enumeration of every C(M,N) subset.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (3, 4), (4, 8), (2, 8)])
+def test_select_nm_matches_enumeration(oracle_lib, n, m):
+    r = _rng(10 + n * 100 + m)
+    for quant in (None, 4):  # quantised scores force ties
+        s = r.random((3, 8 * m)).astype(np.float32)
+        if quant:
+            s = (np.floor(s * quant) / quant).astype(np.float32)
+        np.testing.assert_array_equal(oracle_lib.select_nm(s, n, m), brute.select_nm(s, n, m))
+
+
+def test_select_8of16_matches_enumeration(oracle_lib):
+    r = _rng(7)
+    s = (np.floor(r.random((1, 32)) * 6) / 6).astype(np.float32)
+    np.testing.assert_array_equal(oracle_lib.select_nm(s, 8, 16), brute.select_nm(s, 8, 16))
+
+
+def test_tiny_layer_all_c42_subsets(oracle_lib):
+    """Tiny layer (x f32 [4,256], 2:4 magnitude): every block checked against
+    all C(4,2)=6 subsets."""
+    x, _ = synth.tiny_layer()
+    s = oracle_lib.score(x.numpy())
+    np.testing.assert_array_equal(oracle_lib.select_nm(s, 2, 4), brute.select_nm(s, 2, 4))
+
+
+@pytest.mark.parametrize("kk", [0, 1, 3, 5, 9, 10])
+def test_select_topk_matches_enumeration(oracle_lib, kk):
+    r = _rng(kk)
+    s = (np.floor(r.random((4, 10)) * 5) / 5).astype(np.float32)
+    np.testing.assert_array_equal(oracle_lib.select_topk(s, kk), brute.select_topk(s, kk))
+
+
+def test_select_invariants(oracle_lib):
+    """Exactly N per block; every kept score >= every dropped score in its
+    block; equal scores kept from the lower index first."""
+    r = _rng(3)
+    x = _bf16(r.laplace(0, 0.3, size=(5, 1024)))
+    s = oracle_lib.score(x)
+    for n, m in [(2, 4), (8, 16), (16, 32)]:
+        mask = oracle_lib.select_nm(s, n, m)
+        blocks = mask.reshape(5, -1, m)
+        assert (blocks.sum(-1) == n).all()
+        sb = s.reshape(5, -1, m)
+        kept_min = np.where(blocks == 1, sb, np.inf).min(-1)
+        drop_max = np.where(blocks == 0, sb, -np.inf).max(-1)
+        assert (kept_min >= drop_max).all()
+    for kk in (0, 1, 400, 1024):
+        mask = oracle_lib.select_topk(s, kk)
+        assert (mask.sum(1) == kk).all()
+    # all-equal scores: the lowest indices win
+    s0 = np.ones((1, 16), np.float32)
+    np.testing.assert_array_equal(oracle_lib.select_nm(s0, 2, 4)[0], [1, 1, 0, 0] * 4)
+    np.testing.assert_array_equal(oracle_lib.select_topk(s0, 3)[0], [1] * 3 + [0] * 13)
+
+
+def test_zero_block_keeps_lowest_indices(oracle_lib):
+    """A block [0, 0, 0, v] under 2:4 keeps {0, 3} (zeros are eligible)."""
+    s = oracle_lib.score(np.array([[0, 0, 0, 0.5, 0, -2, 0, 0]], np.float32))
+    np.testing.assert_array_equal(oracle_lib.select_nm(s, 2, 4)[0], [1, 0, 0, 1, 1, 1, 0, 0])
+
+
+def test_three_nonzero_block_drops_smallest(oracle_lib):
+    """2:4 + Squared-ReLU page, section 2.3: a 4-block with 3 nonzeros drops the
+    smallest-magnitude one."""
+    x = np.array([[0.0, 3.0, 1.0, 2.0, 5.0, 0.0, 0.25, 4.0]], np.float32)
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    np.testing.assert_array_equal(mask[0], [0, 1, 0, 1, 1, 0, 0, 1])
+
+
+# --------------------------------------------------------------------------
+# Scores
+# --------------------------------------------------------------------------
+def test_score_definition_special_cases(oracle_lib):
+    x = np.array([[1.5, -2.0, 0.25, -0.75]], np.float32)
+    np.testing.assert_array_equal(oracle_lib.score(x)[0], np.abs(x[0]))
+    eta = np.array([0.5], np.float32)
+    np.testing.assert_array_equal(oracle_lib.score(x, eta=eta)[0], [1.0, 2.5, 0.25, 1.25])
+    f = np.array([2.0, 0.5, 4.0, 1.0], np.float32)
+    np.testing.assert_array_equal(oracle_lib.score(x, f=f)[0], [3.0, 1.0, 1.0, 0.75])
+
+
+def test_weight_aware_alpha0_is_magnitude(oracle_lib):
+    r = _rng(5)
+    x = _bf16(r.laplace(0, 0.3, size=(3, 512)))
+    W = _bf16(r.normal(0, 0.02, size=(300, 512)))
+    g, _ = oracle_lib.weight_prep(W, 0.0)
+    np.testing.assert_array_equal(g, np.ones(512))
+    s_w = oracle_lib.score(x, f=g.astype(np.float32))
+    np.testing.assert_array_equal(oracle_lib.select_nm(s_w, 8, 16),
+                                  oracle_lib.select_nm(oracle_lib.score(x), 8, 16))
+
+
+def test_clact_single_token_is_magnitude(oracle_lib):
+    """With T=1, c_j = |x_j|, so |x_j| c_j = x_j^2 (exact in fp32 for bf16
+    inputs) ranks like |x_j|."""
+    r = _rng(6)
+    x = _bf16(r.standard_t(3, size=(1, 1024)) * 0.5)
+    c = oracle_lib.channel_energy(x).astype(np.float32)
+    np.testing.assert_array_equal(c, np.abs(x[0]))
+    s = oracle_lib.score(x, f=c)
+    for n, m in [(2, 4), (16, 32)]:
+        np.testing.assert_array_equal(oracle_lib.select_nm(s, n, m),
+                                      oracle_lib.select_nm(oracle_lib.score(x), n, m))
+
+
+def test_clact_row_factor_is_constant_per_token(oracle_lib):
+    """The full CLACT score divided by |x_ij| c_j equals 1/||x_t|| for every
+    channel of token t (overview page §2.2.3), which is why ranking by
+    |x_ij| c_j gives the same per-token order."""
+    r = _rng(8)
+    x = _bf16(r.standard_t(3, size=(6, 256)) * 0.5)
+    S = oracle_lib.clact_full(x)
+    c = np.sqrt((x.astype(np.float64) ** 2).sum(0))
+    rn = np.sqrt((x.astype(np.float64) ** 2).sum(1))
+    np.testing.assert_allclose(S, np.abs(x) * c[None, :] / rn[:, None], rtol=1e-13)
+    np.testing.assert_allclose(oracle_lib.channel_energy(x), c, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Statistics and weight preparation: closed forms
+# --------------------------------------------------------------------------
+def test_token_stats_closed_forms(oracle_lib):
+    k = 1000
+    x = np.stack([np.full(k, 0.75), np.arange(k) * 0.5 - 3.0]).astype(np.float32)
+    eta = oracle_lib.token_mean(x)
+    np.testing.assert_allclose(eta, [0.75, (k - 1) / 2 * 0.5 - 3.0], rtol=1e-15)
+    var = oracle_lib.token_var(x)
+    np.testing.assert_allclose(var, [0.0, 0.25 * k * (k + 1) / 12], rtol=1e-13)
+
+
+def test_weight_prep_closed_form(oracle_lib):
+    """W[o, i] = a_i * b_o with known column norms |a_i| ||b|| and row sums
+    b_o * sum(a): a transposed norm axis or a dropped exponent fails."""
+    a = np.array([0.5, -1.0, 2.0, 0.25, 4.0], np.float64)
+    b = np.array([1.0, -0.5, 0.25, 2.0, 0.125, -1.0, 0.5], np.float64)
+    W = np.outer(b, a).astype(np.float32)  # [n_out=7, k=5]
+    for alpha in (0.0, 0.5, 1.0, 1.7):
+        g, rs = oracle_lib.weight_prep(W, alpha)
+        np.testing.assert_allclose(g, (np.abs(a) * np.linalg.norm(b)) ** alpha, rtol=1e-14)
+        np.testing.assert_allclose(rs, b * a.sum(), rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Contraction
+# --------------------------------------------------------------------------
+def test_linear_keep_all_is_dense_matmul(oracle_lib):
+    r = _rng(11)
+    x = _bf16(r.laplace(0, 0.3, size=(5, 96)))
+    W = _bf16(r.normal(0, 0.02, size=(40, 96)))
+    y = oracle_lib.linear(x, np.ones_like(x, np.uint8), W)
+    np.testing.assert_allclose(y, x.astype(np.float64) @ W.astype(np.float64).T, rtol=1e-12, atol=1e-15)
+
+
+def test_linear_masked_and_rows(oracle_lib):
+    r = _rng(12)
+    x = _bf16(r.laplace(0, 0.3, size=(6, 64)))
+    W = _bf16(r.normal(0, 0.02, size=(33, 64)))
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    ref = (x.astype(np.float64) * mask) @ W.astype(np.float64).T
+    np.testing.assert_allclose(oracle_lib.linear(x, mask, W), ref, rtol=1e-12, atol=1e-15)
+    rows = [5, 0, 3]
+    np.testing.assert_allclose(oracle_lib.linear(x, mask, W, rows=rows), ref[rows], rtol=1e-12, atol=1e-15)
+
+
+def test_dpts_identity(oracle_lib):
+    """(xhat*m + eta) W^T computed densely equals (xhat*m) W^T + eta*rowsum(W)
+    (overview page §3.1)."""
+    r = _rng(13)
+    x = _bf16(r.laplace(0.2, 0.3, size=(4, 128)))
+    W = _bf16(r.normal(0, 0.02, size=(50, 128)))
+    eta = oracle_lib.token_mean(x)
+    eta32 = eta.astype(np.float32)
+    mask = oracle_lib.select_nm(oracle_lib.score(x, eta=eta32), 8, 16)
+    _, rs = oracle_lib.weight_prep(W, 1.0)
+    y = oracle_lib.linear(x, mask, W, eta=eta, rowsum=rs)
+    xhat = x.astype(np.float64) - eta[:, None]
+    dense = (xhat * mask + eta[:, None]) @ W.astype(np.float64).T
+    np.testing.assert_allclose(y, dense, rtol=1e-11, atol=1e-14)
+    # and the shift really matters: without eta the result differs
+    assert not np.allclose(oracle_lib.linear(x, mask, W), dense, rtol=1e-6)
+
+
+def test_var_closed_form(oracle_lib):
+    """Blocks [a, -a, b, -b] with |a| > |b| under 2:4: dense and kept sums are
+    zero, so nu = sqrt(sum x^2 / (sum_kept x^2 + eps (K-1))) on the first
+    batch (overview page §3.2)."""
+    r = _rng(14)
+    k = 256
+    a = r.uniform(1.0, 2.0, size=k // 4)
+    b = r.uniform(0.0, 0.9, size=k // 4)
+    x = np.stack([a, -a, b, -b], 1).reshape(1, k).astype(np.float32)
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    np.testing.assert_array_equal(mask.reshape(-1, 4), np.tile([1, 1, 0, 0], (k // 4, 1)))
+    eps = 1e-6
+    out = oracle_lib.var_scale(x, mask, None, 0.9, eps)
+    x64 = x.astype(np.float64)[0]
+    nu = math.sqrt((x64 ** 2).sum() / ((x64[mask[0] == 1] ** 2).sum() + eps * (k - 1)))
+    np.testing.assert_allclose(out["nu"], [nu], rtol=1e-12)
+    np.testing.assert_allclose(out["var_dense"], [(x64 ** 2).sum() / (k - 1)], rtol=1e-12)
+    # keep-all: nu = sqrt(v / (v + eps))
+    out = oracle_lib.var_scale(x, np.ones_like(mask), None, 0.9, eps)
+    v = out["var_dense"][0]
+    np.testing.assert_allclose(out["nu"], [math.sqrt(v / (v + eps))], rtol=1e-12)
+
+
+def test_var_running_average_over_batches(oracle_lib):
+    """Eight batches chained through the oracle equal a scalar recomputation
+    of running <- 0.9 running + 0.1 var_dense (first batch: var_dense)."""
+    r = _rng(15)
+    T, k = 3, 64
+    run = None
+    scal = [None] * T
+    for b in range(8):
+        x = _bf16(r.standard_t(3, size=(T, k)) * 0.5)
+        mask = oracle_lib.select_nm(oracle_lib.score(x), 16, 32)
+        out = oracle_lib.var_scale(x, mask, run, 0.9, 1e-6)
+        for t in range(T):
+            vd = np.var(x[t].astype(np.float64), ddof=1)
+            vk = np.var(x[t].astype(np.float64) * mask[t], ddof=1)
+            scal[t] = vd if scal[t] is None else 0.9 * scal[t] + 0.1 * vd
+            np.testing.assert_allclose(out["running"][t], scal[t], rtol=1e-12)
+            np.testing.assert_allclose(out["nu"][t], math.sqrt(scal[t] / (vk + 1e-6)), rtol=1e-12)
+        run = out["running"]
+
+
+def test_vr_scale_applies_to_whole_row(oracle_lib):
+    r = _rng(16)
+    x = _bf16(r.laplace(0, 0.3, size=(3, 64)))
+    W = _bf16(r.normal(0, 0.02, size=(20, 64)))
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 16, 32)
+    nu = np.array([1.5, 0.5, 2.0])
+    np.testing.assert_allclose(oracle_lib.linear(x, mask, W, nu=nu),
+                               oracle_lib.linear(x, mask, W) * nu[:, None], rtol=1e-13)
+
+
+def test_compress_roundtrip(oracle_lib):
+    r = _rng(17)
+    x = _bf16(r.laplace(0, 0.3, size=(3, 64)))
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    vals, pos = oracle_lib.compress_nm(x, mask, 2, 4)
+    assert vals.shape == (3, 32)
+    back = np.zeros_like(x)
+    for t in range(3):
+        for j in range(32):
+            back[t, (j // 2) * 4 + pos[t, j]] = vals[t, j]
+    np.testing.assert_array_equal(back, x * mask)
+    assert (pos.reshape(3, -1, 2)[:, :, 0] < pos.reshape(3, -1, 2)[:, :, 1]).all()
+
+
+# --------------------------------------------------------------------------
+# Squared-ReLU workload: closed-form sparsity statistics
+# --------------------------------------------------------------------------
+def test_sqrelu_sparsity_closed_form(oracle_lib):
+    """z ~ N(-1.2, 1): natural zeros Phi(1.2) = 0.88493; enforcing 2:4 by
+    magnitude drops (4p^3(1-p) + 2p^4) / (4p) = 1.248% of the nonzeros,
+    p = 1 - Phi(1.2) (2:4 + Squared-ReLU page §2.2-2.3 report ~1% at high
+    natural sparsity)."""
+    _, x, _ = synth.prefill_sqrelu(T=256, with_weight=False)
+    xf = x.float().numpy()
+    n = xf.size
+    p = 0.5 * math.erfc(1.2 / math.sqrt(2))
+    zero = (xf == 0).mean()
+    assert abs(zero - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
+    mask = oracle_lib.select_nm(oracle_lib.score(xf), 2, 4)
+    nz = xf != 0
+    dropped = (nz & (mask == 0)).sum() / nz.sum()
+    expect = (4 * p ** 3 * (1 - p) + 2 * p ** 4) / (4 * p)
+    # per-block variance of the dropped count, delta method on the ratio
+    blocks = nz.reshape(-1, 4).sum(1)
+    d = np.maximum(blocks - 2, 0)
+    sig = math.sqrt(np.var(d - expect * blocks) / len(blocks)) / (4 * p)
+    assert abs(dropped - expect) < 5 * sig, (dropped, expect, sig)
