@@ -1,0 +1,218 @@
+/*
+ * actsparse.h -- C ABI of the activation-sparsified linear layer
+ *                y = prune(x) W^T  on NVIDIA B200 (sm_100a).
+ *
+ * The layer keeps, per token, a subset of the input channels of x and
+ * contracts only those against W.  Sources (page title, section):
+ *   [OVW] "激活稀疏化技术：提升LLM推理效率的动态剪枝方法" (activation-sparsity
+ *         overview): 2.1 N:M patterns, 2.2.1 magnitude score, 2.2.3 CLACT
+ *         score, 3.1 D-PTS mean shift, 3.2 VAR variance correction.
+ *   [WIS] "大模型推理优化：WiSparse激活稀疏化技术解析": 2.1 eq. (4) weight-aware
+ *         score, 2.2 per-layer keep fraction, 3.1 fused sparse operator.
+ *   [SQR] "利用2:4稀疏性与Squared-ReLU加速Transformer训练与推理": 2.1 2:4 on
+ *         tensor cores, 2.3 3-nonzero blocks, 3.3 compressed layout.
+ *
+ * Conventions for every entry point
+ *   - Layouts are row-major.  x is [T, K] (T tokens, K input channels),
+ *     W is [n_out, K] (PyTorch Linear layout), Wt is [K, n_out], y is
+ *     [T, n_out].  All pointers are DEVICE pointers owned by the caller
+ *     unless stated otherwise; the library never allocates and never frees.
+ *   - Every call is asynchronous and ordered on `stream` (0 = legacy default
+ *     stream).  Scratch memory is passed in as `workspace`, sized with
+ *     as_workspace_size().  Workspace must be zero-filled once before its
+ *     first use; every call leaves it zero-filled again.  Calls that share a
+ *     workspace must not run concurrently.
+ *   - Errors are returned, never raised: arguments are validated on the host
+ *     and an invalid call launches nothing.  A kernel that gives up a bounded
+ *     wait records AS_ERR_TIMEOUT in a device status word that
+ *     as_stream_status() reports.  No entry point aborts, exits or traps.
+ *   - Device pointers must be 16-byte aligned (AS_ERR_ALIGN otherwise).
+ *   - Channel selection is deterministic: exactly N per M-block (or exactly
+ *     k_keep per token), equal float32 scores broken towards the lower channel
+ *     index; repeated calls give bitwise-identical results.
+ */
+#ifndef ACTSPARSE_H
+#define ACTSPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define AS_ABI_VERSION 1
+#define AS_MAX_DECODE_T 16
+
+typedef enum as_status {
+    AS_OK = 0,
+    AS_ERR_INVALID_ARG = 1,  /* NULL where a buffer is required, bad enum */
+    AS_ERR_SHAPE = 2,        /* K % M != 0, N > M, k_keep > K, T out of range */
+    AS_ERR_DTYPE = 3,        /* dtype not supported by this operation */
+    AS_ERR_ALIGN = 4,        /* pointer or row stride not 16-byte aligned */
+    AS_ERR_UNSUPPORTED = 5,  /* valid but unsupported combination */
+    AS_ERR_WORKSPACE = 6,    /* workspace NULL or smaller than required */
+    AS_ERR_CUDA = 7,         /* a CUDA runtime/driver call failed */
+    AS_ERR_TIMEOUT = 8       /* a device-side bounded wait gave up */
+} as_status;
+
+typedef enum as_dtype { AS_F32 = 0, AS_BF16 = 1 } as_dtype;
+
+/* Channel score s_ti, taken in float32 ([OVW] 2.2.1, 2.2.3; [WIS] eq. 4):
+ *   xhat = fl32(x - eta_t) with D-PTS, x otherwise;  s = fl32(|xhat| * f_i)
+ *   AS_SCORE_MAG:    f_i = 1
+ *   AS_SCORE_WEIGHT: f_i = g_i = ||W[:,i]||_2^alpha (from as_weight_prep)
+ *   AS_SCORE_CLACT:  f_i = c_i = sqrt(sum over the T tokens of the call of
+ *                    x_ti^2); the CLACT row factor 1/||x_t|| is the same for
+ *                    every channel of a token and does not change the ranking. */
+typedef enum as_score { AS_SCORE_MAG = 0, AS_SCORE_WEIGHT = 1, AS_SCORE_CLACT = 2 } as_score;
+
+/* Selection ([OVW] 2.1; [WIS] 2.2):
+ *   AS_SEL_NM:   in every block of m consecutive channels [jm, jm+m) keep the
+ *                n largest scores; m in {1,2,4,8,16,32}, 1 <= n <= m, K % m == 0.
+ *   AS_SEL_TOPK: keep the k_keep largest scores of each token, 0 <= k_keep <= K.
+ *   AS_SEL_ALL:  keep every channel (dense layer, for baselines and checks). */
+typedef enum as_sel { AS_SEL_NM = 0, AS_SEL_TOPK = 1, AS_SEL_ALL = 2 } as_sel;
+
+typedef struct as_config {
+    int32_t score;        /* as_score */
+    int32_t sel;          /* as_sel */
+    int32_t n, m;         /* N:M pattern (AS_SEL_NM) */
+    int32_t k_keep;       /* kept channels per token (AS_SEL_TOPK) */
+    int32_t dpts;         /* 1: D-PTS, [OVW] 3.1: score and keep xhat = x - eta_t,
+                             eta_t = mean_i x_ti, and add eta_t * rowsum_o back:
+                             y = (xhat*m) W^T + eta * rowsum(W). */
+    int32_t var;          /* 1: VAR, [OVW] 3.2 (prefill only; not with dpts):
+                             running_t <- var_dense_t on the first batch, else
+                             mom*running_t + (1-mom)*var_dense_t; then
+                             nu_t = sqrt(running_t / (Var[x_t*m_t] + eps)),
+                             y_t <- nu_t * y_t.  Variances are unbiased. */
+    float var_momentum;   /* mom, 0.9 on the page */
+    float var_eps;        /* eps, 1e-6 on the page */
+    int32_t out_dtype;    /* as_dtype of y */
+} as_config;
+
+/* Outputs of as_select.  Every pointer is optional (NULL = not written) unless
+ * the operation needs it; all are device memory. */
+typedef struct as_select_out {
+    uint32_t *bitmask;   /* [T, ceil(K/32)]: bit (i % 32) of word i/32 = channel i kept */
+    float *eta;          /* [T]  D-PTS mean (float32, the value the score used) */
+    float *colnorm;      /* [K]  CLACT c_i (float32, the value the score used) */
+    float *var_dense;    /* [T]  Var[x_t] (VAR) */
+    float *var_kept;     /* [T]  Var[x_t * m_t] (VAR) */
+    float *nu;           /* [T]  VAR scale */
+    void *x_masked;      /* [T, K] in x's dtype: xhat*m, zeros where dropped */
+    void *x_compact;     /* 2:4 only, bf16 [T, K/2]: the two kept values of every
+                            4-block in ascending channel order ([SQR] 3.3) */
+    uint32_t *meta24;    /* 2:4 only: positions of the kept values in the
+                            tcgen05 sparse-MMA metadata layout; size in 32-bit
+                            words is as_meta24_words(T, K).  Layout: tiles of
+                            128 tokens x 128 channels, tile (r, c) at word offset
+                            (r * ceil(K/128) + c) * 512; inside a tile, word
+                            lane*4 + j holds MMA step j (channels 32j..32j+31 of
+                            the tile) for TMEM lane
+                                lane = 16*(p/16) + 8*(q/16) + p%8
+                            (p = token within the tile, q = channel within the
+                            32-channel step): bits [16*((p%16)/8) + 4*((q%16)/4),
+                            +4) of that word hold the 4-block's two positions
+                            i0 | i1 << 2, i0 < i1.  Padding blocks hold 0x4. */
+} as_select_out;
+
+/* --------------------------------------------------------------------------
+ * Weight preparation, once per layer ([WIS] 2.1: norms precomputed; [OVW] 3.1).
+ *   W      [n_out, K] in dtype `dt` (input).
+ *   Wt     [K, n_out] in `dt` (output, optional): channel-major copy that the
+ *          decode path streams, one contiguous row per kept channel.
+ *   g      [K] float32 (optional): ||W[:,i]||_2^alpha, accumulated in float64.
+ *   rowsum [n_out] float32 (optional): sum_i W[o,i], accumulated in float64.
+ *   Workspace: as_workspace_size(AS_OP_WEIGHT_PREP, 0, K, n_out, NULL).
+ * ------------------------------------------------------------------------ */
+as_status as_weight_prep(const void *W, as_dtype dt, int n_out, int K, float alpha,
+                         void *Wt, float *g, float *rowsum,
+                         void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Score + selection + compensation statistics for T tokens (prefill side, or
+ * to inspect a decode selection).  x [T, K] in `dt`.
+ *   chan_factor: g [K] for AS_SCORE_WEIGHT (required); ignored otherwise
+ *                (CLACT computes c over the T tokens and writes out->colnorm
+ *                when given).
+ *   running_var: [T] float32 in/out, required when cfg->var; when
+ *                var_first_batch != 0 it is overwritten with var_dense.
+ *   out:         see as_select_out.  2:4 outputs need dt == AS_BF16 and
+ *                K % 16 == 0.  x_masked is written in x's dtype.
+ *   Workspace: as_workspace_size(AS_OP_SELECT, T, K, 0, cfg).
+ * ------------------------------------------------------------------------ */
+as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *cfg,
+                    const float *chan_factor, float *running_var, int var_first_batch,
+                    const as_select_out *out, void *workspace, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Decode: 1 <= T <= 16 tokens against the channel-major weight Wt [K, n_out].
+ * For N:M selection the score, block top-N, D-PTS mean and the contraction
+ * run in one kernel that streams only the union over the T tokens of the
+ * kept rows of Wt ([WIS] 3.1: sparsify fused with the matmul, no
+ * intermediate activation written); top-k runs a per-token selection kernel
+ * first.  Accumulation is float32 in a fixed order (deterministic).
+ *   x [T, K] and Wt in `dt`; g [K] float32 for AS_SCORE_WEIGHT; rowsum
+ *   [n_out] float32 when cfg->dpts.  y [T, n_out] in cfg->out_dtype.
+ *   mask_out [T, ceil(K/32)] (optional): the selection bitmask.
+ *   eta_out [T] (optional): the float32 D-PTS mean the score used.
+ *   colnorm_out [K] (optional): the float32 CLACT c the score used.
+ *   Requires n_out % 8 == 0.  cfg->var is not supported (AS_ERR_UNSUPPORTED).
+ *   Workspace: as_workspace_size(AS_OP_DECODE, T, K, n_out, cfg).
+ * ------------------------------------------------------------------------ */
+as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out,
+                           const void *Wt, const float *g, const float *rowsum,
+                           const as_config *cfg, void *y, uint32_t *mask_out,
+                           float *eta_out, float *colnorm_out,
+                           void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Prefill contraction on the tensor cores (bf16 in, float32 accumulate in
+ * tensor memory, output in cfg->out_dtype) over a selection made by
+ * as_select with the same cfg:
+ *   cfg->sel == AS_SEL_NM with n=2, m=4: sel->x_compact + sel->meta24 are
+ *     the sparse A operand of tcgen05.mma.sp ([SQR] 2.1: the tensor core
+ *     skips the dropped half of the multiply-adds).
+ *   any other selection: sel->x_masked is the A operand of a dense
+ *     tcgen05.mma GEMM (tensor cores support 2:4 only).
+ *   AS_SEL_ALL: x itself (sel->x_masked may point at x).
+ *   W [n_out, K] bf16 (K-major, the PyTorch layout).  Epilogue:
+ *   y = nu_t * acc (cfg->var, nu from as_select) or acc + eta_t * rowsum_o
+ *   (cfg->dpts), then rounding to the output dtype.
+ *   Requires K % 8 == 0 (K % 16 == 0 for 2:4) and n_out % 8 == 0.
+ *   Workspace: as_workspace_size(AS_OP_PREFILL, T, K, n_out, cfg) (zero).
+ * ------------------------------------------------------------------------ */
+as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int K,
+                            int n_out, const float *rowsum, const float *eta,
+                            const float *nu, const as_config *cfg, void *y,
+                            void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Which operation a workspace size is asked for. */
+enum { AS_OP_WEIGHT_PREP = 0, AS_OP_SELECT = 1, AS_OP_DECODE = 2, AS_OP_PREFILL = 3 };
+
+/* Bytes of workspace the operation needs (0 if none); (size_t)-1 if the
+ * arguments are invalid. */
+size_t as_workspace_size(int op, int T, int K, int n_out, const as_config *cfg);
+
+/* Number of 32-bit metadata words of a 2:4 selection of T tokens x K channels. */
+size_t as_meta24_words(int T, int K);
+
+/* Synchronises `stream`, then reports (and clears) a device-side error such
+ * as AS_ERR_TIMEOUT recorded by a kernel of this library, or AS_ERR_CUDA if
+ * the stream itself failed. */
+as_status as_stream_status(cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *as_status_string(as_status s);
+
+/* AS_ABI_VERSION of the loaded library. */
+int as_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ACTSPARSE_H */

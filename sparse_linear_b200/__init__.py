@@ -1,0 +1,185 @@
+"""Python binding of libactsparse, the B200 activation-sparsified linear layer.
+
+Argument marshalling only: every step of the layer (weight preparation,
+scores, selection, compensation statistics, the contraction) runs in the CUDA
+kernels of ``libactsparse.so``; this module passes device pointers, sizes and
+the current CUDA stream through the C ABI declared in ``include/actsparse.h``
+and raises ``ASError`` for a non-zero status.  The functions keep the C names.
+
+There is no CPU fallback: importing this package on a machine where the
+library cannot be loaded raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libactsparse.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python sparse_linear_b200/build.py` "
+        "(nvcc, sm_100a) before using sparse_linear_b200")
+_lib = ctypes.CDLL(LIB_PATH)
+
+# ---------------------------------------------------------------- constants
+AS_OK, AS_ERR_INVALID_ARG, AS_ERR_SHAPE, AS_ERR_DTYPE, AS_ERR_ALIGN = 0, 1, 2, 3, 4
+AS_ERR_UNSUPPORTED, AS_ERR_WORKSPACE, AS_ERR_CUDA, AS_ERR_TIMEOUT = 5, 6, 7, 8
+AS_F32, AS_BF16 = 0, 1
+AS_SCORE_MAG, AS_SCORE_WEIGHT, AS_SCORE_CLACT = 0, 1, 2
+AS_SEL_NM, AS_SEL_TOPK, AS_SEL_ALL = 0, 1, 2
+AS_OP_WEIGHT_PREP, AS_OP_SELECT, AS_OP_DECODE, AS_OP_PREFILL = 0, 1, 2, 3
+AS_MAX_DECODE_T = 16
+
+EXPORTS = [
+    "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
+    "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
+    "as_abi_version",
+]
+
+
+class as_config(ctypes.Structure):
+    _fields_ = [("score", ctypes.c_int32), ("sel", ctypes.c_int32), ("n", ctypes.c_int32),
+                ("m", ctypes.c_int32), ("k_keep", ctypes.c_int32), ("dpts", ctypes.c_int32),
+                ("var", ctypes.c_int32), ("var_momentum", ctypes.c_float),
+                ("var_eps", ctypes.c_float), ("out_dtype", ctypes.c_int32)]
+
+
+class as_select_out(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "bitmask", "eta", "colnorm", "var_dense", "var_kept", "nu", "x_masked",
+        "x_compact", "meta24")]
+
+
+_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_sig = {
+    "as_weight_prep": ([_P, _I, _I, _I, _F, _P, _P, _P, _P, _S, _P], _I),
+    "as_select": ([_P, _I, _I, _I, ctypes.POINTER(as_config), _P, _P, _I,
+                   ctypes.POINTER(as_select_out), _P, _S, _P], _I),
+    "as_linear_decode": ([_P, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(as_config), _P, _P, _P, _P,
+                          _P, _S, _P], _I),
+    "as_linear_prefill": ([ctypes.POINTER(as_select_out), _P, _I, _I, _I, _P, _P, _P,
+                           ctypes.POINTER(as_config), _P, _P, _S, _P], _I),
+    "as_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(as_config)], _S),
+    "as_meta24_words": ([_I, _I], _S),
+    "as_stream_status": ([_P], _I),
+    "as_status_string": ([_I], ctypes.c_char_p),
+    "as_abi_version": ([], _I),
+}
+for _name, (_args, _res) in _sig.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+class ASError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_lib.as_status_string(code).decode()}")
+
+
+def _check(code: int, where: str) -> None:
+    if code != AS_OK:
+        raise ASError(code, where)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libactsparse takes device tensors; got a CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError("libactsparse takes contiguous (row-major) tensors")
+    return t.data_ptr()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return AS_BF16
+    if t.dtype == torch.float32:
+        return AS_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def config(score: int = AS_SCORE_MAG, sel: int = AS_SEL_NM, n: int = 2, m: int = 4, k_keep: int = 0,
+           dpts: bool = False, var: bool = False, var_momentum: float = 0.9, var_eps: float = 1e-6,
+           out_dtype: int = AS_BF16) -> as_config:
+    return as_config(score, sel, n, m, k_keep, int(dpts), int(var), var_momentum, var_eps, out_dtype)
+
+
+def select_out(**bufs) -> as_select_out:
+    o = as_select_out()
+    for k, v in bufs.items():
+        setattr(o, k, _ptr(v))
+    return o
+
+
+# ---------------------------------------------------------------- entry points
+def as_abi_version() -> int:
+    return _lib.as_abi_version()
+
+
+def as_status_string(code: int) -> str:
+    return _lib.as_status_string(code).decode()
+
+
+def as_workspace_size(op: int, T: int, K: int, n_out: int, cfg: as_config | None) -> int:
+    r = _lib.as_workspace_size(op, T, K, n_out, ctypes.byref(cfg) if cfg is not None else None)
+    if r == ctypes.c_size_t(-1).value:
+        raise ASError(AS_ERR_INVALID_ARG, "as_workspace_size")
+    return r
+
+
+def as_meta24_words(T: int, K: int) -> int:
+    return _lib.as_meta24_words(T, K)
+
+
+def as_weight_prep(W, alpha: float, Wt=None, g=None, rowsum=None, workspace=None, stream=None) -> None:
+    n_out, K = W.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_weight_prep(_ptr(W), _dt(W), n_out, K, float(alpha), _ptr(Wt), _ptr(g), _ptr(rowsum),
+                               _ptr(workspace), ws_bytes, _stream(stream)), "as_weight_prep")
+
+
+def as_select(x, cfg: as_config, out: as_select_out, chan_factor=None, running_var=None,
+              var_first_batch: bool = False, workspace=None, stream=None) -> None:
+    T, K = x.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_select(_ptr(x), _dt(x), T, K, ctypes.byref(cfg), _ptr(chan_factor), _ptr(running_var),
+                          int(var_first_batch), ctypes.byref(out), _ptr(workspace), ws_bytes,
+                          _stream(stream)), "as_select")
+
+
+def as_linear_decode(x, Wt, cfg: as_config, y, g=None, rowsum=None, mask_out=None, eta_out=None,
+                     colnorm_out=None, workspace=None, stream=None) -> None:
+    T, K = x.shape
+    n_out = Wt.shape[1]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_linear_decode(_ptr(x), _dt(x), T, K, n_out, _ptr(Wt), _ptr(g), _ptr(rowsum),
+                                 ctypes.byref(cfg), _ptr(y), _ptr(mask_out), _ptr(eta_out),
+                                 _ptr(colnorm_out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "as_linear_decode")
+
+
+def as_linear_prefill(sel: as_select_out, W, T: int, cfg: as_config, y, rowsum=None, eta=None, nu=None,
+                      workspace=None, stream=None) -> None:
+    n_out, K = W.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_linear_prefill(ctypes.byref(sel), _ptr(W), T, K, n_out, _ptr(rowsum), _ptr(eta), _ptr(nu),
+                                  ctypes.byref(cfg), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "as_linear_prefill")
+
+
+def as_stream_status(stream=None) -> int:
+    return _lib.as_stream_status(_stream(stream))

@@ -1,0 +1,304 @@
+// extern "C" entry points of libactsparse (declared in include/actsparse.h).
+//
+// Every entry point validates its arguments on the host and launches nothing
+// when they are invalid; CUDA launch errors are mapped to AS_ERR_CUDA.  No
+// entry point allocates device memory: scratch space is the caller's
+// workspace, sized by as_workspace_size().
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace as;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool valid_m(int m) { return m == 1 || m == 2 || m == 4 || m == 8 || m == 16 || m == 32; }
+
+as_status check_cfg(const as_config *cfg, int K)
+{
+    if (!cfg) return AS_ERR_INVALID_ARG;
+    if (cfg->score < AS_SCORE_MAG || cfg->score > AS_SCORE_CLACT) return AS_ERR_INVALID_ARG;
+    if (cfg->sel < AS_SEL_NM || cfg->sel > AS_SEL_ALL) return AS_ERR_INVALID_ARG;
+    if (cfg->out_dtype != AS_F32 && cfg->out_dtype != AS_BF16) return AS_ERR_DTYPE;
+    if (cfg->sel == AS_SEL_NM) {
+        if (!valid_m(cfg->m)) return AS_ERR_SHAPE;
+        if (cfg->n < 1 || cfg->n > cfg->m) return AS_ERR_SHAPE;
+        if (K % cfg->m != 0) return AS_ERR_SHAPE;
+    }
+    if (cfg->sel == AS_SEL_TOPK && (cfg->k_keep < 0 || cfg->k_keep > K)) return AS_ERR_SHAPE;
+    if (cfg->dpts && cfg->var) return AS_ERR_UNSUPPORTED;
+    if (cfg->var && !(cfg->var_eps >= 0.0f && cfg->var_momentum >= 0.0f && cfg->var_momentum <= 1.0f))
+        return AS_ERR_INVALID_ARG;
+    return AS_OK;
+}
+
+bool is24(const as_config *cfg) { return cfg->sel == AS_SEL_NM && cfg->n == 2 && cfg->m == 4; }
+
+as_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AS_OK : AS_ERR_CUDA; }
+
+size_t decode_ws(int T, int K, int n_out, const as_config *cfg, int bf16)
+{
+    DecodePlan p = decode_plan(T, K, n_out, bf16);
+    size_t bytes = round_up(p.counter_bytes, 256) + round_up(p.partial_bytes, 256);
+    if (cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL)
+        bytes += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
+    if (cfg->sel == AS_SEL_TOPK && cfg->score == AS_SCORE_CLACT) bytes += round_up(colnorm_workspace(T, K), 256);
+    return bytes;
+}
+
+size_t select_ws(int T, int K, const as_config *cfg)
+{
+    return cfg->score == AS_SCORE_CLACT ? round_up(colnorm_workspace(T, K), 256) : 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int as_abi_version(void) { return AS_ABI_VERSION; }
+
+const char *as_status_string(as_status s)
+{
+    switch (s) {
+    case AS_OK: return "AS_OK";
+    case AS_ERR_INVALID_ARG: return "AS_ERR_INVALID_ARG: missing buffer or bad enum";
+    case AS_ERR_SHAPE: return "AS_ERR_SHAPE: shape not supported (K % M, N > M, k_keep, T range)";
+    case AS_ERR_DTYPE: return "AS_ERR_DTYPE: dtype not supported by this operation";
+    case AS_ERR_ALIGN: return "AS_ERR_ALIGN: pointer or row stride not 16-byte aligned";
+    case AS_ERR_UNSUPPORTED: return "AS_ERR_UNSUPPORTED: combination not supported";
+    case AS_ERR_WORKSPACE: return "AS_ERR_WORKSPACE: workspace missing or too small";
+    case AS_ERR_CUDA: return "AS_ERR_CUDA: a CUDA call failed";
+    case AS_ERR_TIMEOUT: return "AS_ERR_TIMEOUT: a device-side bounded wait gave up";
+    }
+    return "unknown as_status";
+}
+
+size_t as_meta24_words(int T, int K)
+{
+    if (T <= 0 || K <= 0) return 0;
+    return (size_t)((T + 127) / 128) * (size_t)((K + 127) / 128) * 512;
+}
+
+size_t as_workspace_size(int op, int T, int K, int n_out, const as_config *cfg)
+{
+    if (K <= 0) return (size_t)-1;
+    switch (op) {
+    case AS_OP_WEIGHT_PREP:
+        if (n_out <= 0) return (size_t)-1;
+        return weight_prep_workspace(n_out, K);
+    case AS_OP_SELECT:
+        if (T <= 0 || check_cfg(cfg, K) != AS_OK) return (size_t)-1;
+        return select_ws(T, K, cfg);
+    case AS_OP_DECODE:
+        if (T < 1 || T > AS_MAX_DECODE_T || n_out <= 0 || check_cfg(cfg, K) != AS_OK) return (size_t)-1;
+        return decode_ws(T, K, n_out, cfg, 1) > decode_ws(T, K, n_out, cfg, 0) ? decode_ws(T, K, n_out, cfg, 1)
+                                                                                : decode_ws(T, K, n_out, cfg, 0);
+    case AS_OP_PREFILL:
+        if (T <= 0 || n_out <= 0 || check_cfg(cfg, K) != AS_OK) return (size_t)-1;
+        return 0;
+    }
+    return (size_t)-1;
+}
+
+as_status as_weight_prep(const void *W, as_dtype dt, int n_out, int K, float alpha, void *Wt, float *g,
+                         float *rowsum, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!W || n_out <= 0 || K <= 0) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    if (!aligned16(W) || !aligned16(Wt) || !aligned16(g) || !aligned16(rowsum)) return AS_ERR_ALIGN;
+    if (g) {
+        if (!workspace || ws_bytes < weight_prep_workspace(n_out, K)) return AS_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return AS_ERR_ALIGN;
+    }
+    return cuda_status(launch_weight_prep(W, dt == AS_BF16, n_out, K, alpha, Wt, g, rowsum, workspace, stream));
+}
+
+as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *cfg, const float *chan_factor,
+                    float *running_var, int var_first_batch, const as_select_out *out, void *workspace,
+                    size_t ws_bytes, cudaStream_t stream)
+{
+    if (!x || !out || T <= 0 || K <= 0) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    as_status st = check_cfg(cfg, K);
+    if (st != AS_OK) return st;
+    if (K % 8 != 0) return AS_ERR_SHAPE;
+    if (cfg->score == AS_SCORE_WEIGHT && !chan_factor) return AS_ERR_INVALID_ARG;
+    if (cfg->var && !running_var) return AS_ERR_INVALID_ARG;
+    if ((out->x_compact || out->meta24) && (!is24(cfg) || dt != AS_BF16 || K % 16 != 0)) return AS_ERR_UNSUPPORTED;
+    if ((out->x_compact == nullptr) != (out->meta24 == nullptr)) return AS_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, chan_factor, running_var, out->bitmask, out->eta, out->colnorm, out->var_dense,
+                          out->var_kept, out->nu, out->x_masked, out->x_compact, out->meta24, workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return AS_ERR_ALIGN;
+    if (cfg->sel == AS_SEL_TOPK && cfg->k_keep > 0 && cfg->k_keep < K && (size_t)K * 4 > 200 * 1024)
+        return AS_ERR_SHAPE;  // top-k keeps the row's scores in shared memory
+    const size_t need = select_ws(T, K, cfg);
+    if (need && (!workspace || ws_bytes < need)) return AS_ERR_WORKSPACE;
+
+    const float *f = cfg->score == AS_SCORE_WEIGHT ? chan_factor : nullptr;
+    if (cfg->score == AS_SCORE_CLACT) {
+        float *c = out->colnorm;
+        if (!c) c = reinterpret_cast<float *>(static_cast<char *>(workspace) + colnorm_workspace(T, K) -
+                                              (size_t)K * sizeof(float));
+        cudaError_t e = launch_colnorm(x, dt == AS_BF16, T, K, c, workspace, stream);
+        if (e != cudaSuccess) return AS_ERR_CUDA;
+        f = c;
+    }
+    SelectArgs a{};
+    a.x = x;
+    a.bf16 = dt == AS_BF16;
+    a.T = T;
+    a.K = K;
+    a.score = cfg->score;
+    a.sel = cfg->sel;
+    a.n = cfg->n;
+    a.m = cfg->m;
+    a.k_keep = cfg->k_keep;
+    a.dpts = cfg->dpts;
+    a.var = cfg->var;
+    a.first = var_first_batch;
+    a.mom = cfg->var_momentum;
+    a.eps = cfg->var_eps;
+    a.f = f;
+    a.running_var = running_var;
+    a.bitmask = out->bitmask;
+    a.eta = out->eta;
+    a.var_dense = out->var_dense;
+    a.var_kept = out->var_kept;
+    a.nu = out->nu;
+    a.x_masked = out->x_masked;
+    a.x_compact = out->x_compact;
+    a.meta24 = out->meta24;
+    return cuda_status(launch_select(a, stream));
+}
+
+as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, const void *Wt, const float *g,
+                           const float *rowsum, const as_config *cfg, void *y, uint32_t *mask_out, float *eta_out,
+                           float *colnorm_out, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!x || !Wt || !y) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    if (T < 1 || T > AS_MAX_DECODE_T || K <= 0 || n_out <= 0) return AS_ERR_SHAPE;
+    as_status st = check_cfg(cfg, K);
+    if (st != AS_OK) return st;
+    if (cfg->var) return AS_ERR_UNSUPPORTED;
+    if (K % 8 != 0 || n_out % 8 != 0) return AS_ERR_SHAPE;
+    if (cfg->score == AS_SCORE_WEIGHT && !g) return AS_ERR_INVALID_ARG;
+    if (cfg->dpts && !rowsum) return AS_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, Wt, g, rowsum, y, mask_out, eta_out, colnorm_out, workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return AS_ERR_ALIGN;
+    const int bf16 = dt == AS_BF16;
+    const size_t need = decode_ws(T, K, n_out, cfg, bf16);
+    if (!workspace || ws_bytes < need) return AS_ERR_WORKSPACE;
+
+    DecodePlan plan = decode_plan(T, K, n_out, bf16);
+    char *ws = static_cast<char *>(workspace);
+    unsigned *counters = reinterpret_cast<unsigned *>(ws);
+    ws += round_up(plan.counter_bytes, 256);
+    float *partial = reinterpret_cast<float *>(ws);
+    ws += round_up(plan.partial_bytes, 256);
+
+    const uint32_t *mask_in = nullptr;
+    if (cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL) {
+        // per-token selection first (exact top-k needs the whole row)
+        uint32_t *bm = reinterpret_cast<uint32_t *>(ws);
+        ws += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
+        const float *f = cfg->score == AS_SCORE_WEIGHT ? g : nullptr;
+        if (cfg->score == AS_SCORE_CLACT) {
+            float *c = colnorm_out;
+            if (!c) c = reinterpret_cast<float *>(ws + colnorm_workspace(T, K) - (size_t)K * sizeof(float));
+            if (launch_colnorm(x, bf16, T, K, c, ws, stream) != cudaSuccess) return AS_ERR_CUDA;
+            f = c;
+        }
+        SelectArgs s{};
+        s.x = x;
+        s.bf16 = bf16;
+        s.T = T;
+        s.K = K;
+        s.score = cfg->score;
+        s.sel = cfg->sel;
+        s.k_keep = cfg->k_keep;
+        s.dpts = cfg->dpts;
+        s.f = f;
+        s.bitmask = bm;
+        if (cfg->sel == AS_SEL_TOPK && (size_t)K * 4 > 200 * 1024 && cfg->k_keep > 0 && cfg->k_keep < K)
+            return AS_ERR_SHAPE;
+        if (launch_select(s, stream) != cudaSuccess) return AS_ERR_CUDA;
+        mask_in = bm;
+    }
+    DecodeArgs a{};
+    a.x = x;
+    a.Wt = Wt;
+    a.bf16 = bf16;
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.score = mask_in ? AS_SCORE_MAG : cfg->score;
+    a.sel = cfg->sel;
+    a.n = cfg->n;
+    a.m = cfg->m;
+    a.dpts = cfg->dpts;
+    a.g = g;
+    a.rowsum = rowsum;
+    a.mask_in = mask_in;
+    a.y = y;
+    a.out_bf16 = cfg->out_dtype == AS_BF16;
+    a.mask_out = mask_out;
+    a.eta_out = eta_out;
+    a.colnorm_out = mask_in ? nullptr : colnorm_out;
+    a.partial = partial;
+    a.counters = counters;
+    return cuda_status(launch_decode(a, plan, stream));
+}
+
+as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int K, int n_out, const float *rowsum,
+                            const float *eta, const float *nu, const as_config *cfg, void *y, void *workspace,
+                            size_t ws_bytes, cudaStream_t stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (!sel || !W || !y || T <= 0 || K <= 0 || n_out <= 0) return AS_ERR_INVALID_ARG;
+    as_status st = check_cfg(cfg, K);
+    if (st != AS_OK) return st;
+    if (K % 8 != 0 || n_out % 8 != 0) return AS_ERR_SHAPE;
+    const bool sparse = is24(cfg);
+    if (sparse && (K % 16 != 0 || !sel->x_compact || !sel->meta24)) return AS_ERR_INVALID_ARG;
+    if (!sparse && !sel->x_masked) return AS_ERR_INVALID_ARG;
+    if (cfg->dpts && (!rowsum || !eta)) return AS_ERR_INVALID_ARG;
+    if (cfg->var && !nu) return AS_ERR_INVALID_ARG;
+    const void *ptrs[] = {W, rowsum, eta, nu, y, sel->x_compact, sel->meta24, sel->x_masked};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return AS_ERR_ALIGN;
+    GemmArgs a{};
+    a.A = sparse ? sel->x_compact : sel->x_masked;
+    a.meta = sparse ? sel->meta24 : nullptr;
+    a.W = W;
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.sparse = sparse;
+    a.rowsum = cfg->dpts ? rowsum : nullptr;
+    a.eta = cfg->dpts ? eta : nullptr;
+    a.nu = cfg->var ? nu : nullptr;
+    a.y = y;
+    a.out_bf16 = cfg->out_dtype == AS_BF16;
+    return cuda_status(launch_gemm(a, stream));
+}
+
+as_status as_stream_status(cudaStream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return AS_ERR_CUDA;
+    int code = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&code, as::g_status, sizeof(int)) != cudaSuccess) return AS_ERR_CUDA;
+    if (code != 0 && cudaMemcpyToSymbol(as::g_status, &zero, sizeof(int)) != cudaSuccess) return AS_ERR_CUDA;
+    return code == 0 ? AS_OK : static_cast<as_status>(code);
+}
+
+}  // extern "C"

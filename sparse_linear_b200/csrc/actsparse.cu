@@ -1,0 +1,7 @@
+// Single translation unit of libactsparse: the device status word and every
+// kernel live in one module, so no relocatable device code is needed.
+#include "weight_prep.cu"
+#include "select.cu"
+#include "decode.cu"
+#include "gemm.cu"
+#include "abi.cu"

@@ -1,0 +1,357 @@
+// Prefill contraction y = A W^T on the 5th-generation tensor cores.
+//
+// Dense variant (masked activations, any N:M or top-k selection):
+//   tcgen05.mma kind::f16, M=128, N=256, K=16 per instruction.
+// Sparse variant (2:4 selection): the 2:4 + Squared-ReLU page
+// (利用2:4稀疏性与Squared-ReLU加速Transformer训练与推理) section 2.1: when A
+// holds two nonzeros in every four consecutive K elements, the tensor core
+// skips half of the multiply-adds.  A is the compacted half (x_compact) and
+// the positions live in tensor memory; tcgen05.mma.sp kind::f16, M=128,
+// N=128, K=32 (logical) per instruction.
+//
+// Persistent, warp-specialised CTA (one per SM, 192 threads):
+//   warp 0   TMA producer: A and W tiles (128-byte swizzle, K-major) and the
+//            2:4 metadata tile into a STAGES-deep shared-memory ring.
+//   warp 1   allocates tensor memory; one thread issues the MMAs (and, for
+//            the sparse variant, copies each metadata tile into TMEM first).
+//   warps 2-5 epilogue: TMEM -> registers (tcgen05.ld), eta*rowsum or nu
+//            scaling, rounding, stores.  Two accumulator buffers let the
+//            epilogue of one tile overlap the main loop of the next.
+// No cluster multicast is used.  Every mbarrier wait is bounded.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace as {
+
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_GROUP_M = 16;  // tile raster: 16 row tiles share each weight tile
+
+template <bool SPARSE>
+struct GemmCfg;
+template <>
+struct GemmCfg<false> {
+    static constexpr int BN = 256;
+    static constexpr int STAGES = 4;
+    static constexpr int KB = 64;                         // logical K per stage
+    static constexpr int A_BYTES = GEMM_BM * 64 * 2;      // 128 rows x 128 B
+    static constexpr int B_BYTES = BN * 64 * 2;           // 256 rows x 128 B
+    static constexpr int M_BYTES = 0;
+    static constexpr int MMAS = 4;                        // K = 16 each
+    static constexpr int NACC = 2;
+};
+template <>
+struct GemmCfg<true> {
+    static constexpr int BN = 128;
+    static constexpr int STAGES = 4;
+    static constexpr int KB = 128;                        // logical K per stage (64 kept)
+    static constexpr int A_BYTES = GEMM_BM * 64 * 2;      // compact half: 128 rows x 128 B
+    static constexpr int B_BYTES = BN * 128 * 2;          // two 128-byte-wide K sub-tiles
+    static constexpr int M_BYTES = 2048;                  // 128 lanes x 16 B of positions
+    static constexpr int MMAS = 4;                        // K = 32 (logical) each
+    static constexpr int NACC = 2;
+};
+
+template <bool SPARSE>
+constexpr size_t gemm_smem_bytes()
+{
+    using C = GemmCfg<SPARSE>;
+    return 1024 /* alignment slack */ + (size_t)C::STAGES * (C::A_BYTES + C::B_BYTES + C::M_BYTES) + 256;
+}
+
+struct GemmParams {
+    const uint32_t *meta;
+    const float *rowsum, *eta, *nu;
+    void *y;
+    int T, K, n_out, out_bf16;
+    int m_tiles, n_tiles, k_blocks, meta_kt;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int &mt, int &nt)
+{
+    const int per_group = GEMM_GROUP_M * n_tiles;
+    const int group = tile / per_group, rem = tile % per_group;
+    const int gm = min(GEMM_GROUP_M, m_tiles - group * GEMM_GROUP_M);
+    mt = group * GEMM_GROUP_M + rem % gm;
+    nt = rem / gm;
+}
+
+template <bool SPARSE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p)
+{
+    using C = GemmCfg<SPARSE>;
+    constexpr int BN = C::BN, S = C::STAGES;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~uintptr_t(1023));
+    unsigned char *sA = smem;
+    unsigned char *sB = sA + S * C::A_BYTES;
+    unsigned char *sM = sB + S * C::B_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sM + S * C::M_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 2;
+    uint64_t *drain = bars + 2 * S + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*(volatile int *)abort_flag; tile += gridDim.x) {
+                int mt, nt;
+                tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                    mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + C::M_BYTES);
+                    unsigned char *a_dst = sA + stage * C::A_BYTES;
+                    unsigned char *b_dst = sB + stage * C::B_BYTES;
+                    tma_load_2d(a_dst, &tmA, &full[stage], kb * 64, mt * GEMM_BM);
+                    if constexpr (SPARSE) {
+                        tma_load_2d(b_dst, &tmB, &full[stage], kb * 128, nt * BN);
+                        tma_load_2d(b_dst + BN * 128, &tmB, &full[stage], kb * 128 + 64, nt * BN);
+                        const uint32_t *src = p.meta + ((size_t)mt * p.meta_kt + kb) * 512;
+                        bulk_load(sM + stage * C::M_BYTES, src, C::M_BYTES, &full[stage]);
+                    } else {
+                        tma_load_2d(b_dst, &tmB, &full[stage], kb * 64, nt * BN);
+                    }
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(GEMM_BM, BN, SPARSE);
+            const uint32_t meta_tmem = tmem + C::NACC * BN;
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*(volatile int *)abort_flag; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
+                    const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+                    const uint64_t a_desc = sdesc_kmajor_sw128(a_addr);
+                    if constexpr (SPARSE) {
+                        const uint32_t e_tmem = meta_tmem + stage * 4;
+                        tmem_cp_128x128b(e_tmem, sdesc_rows16(smem_u32(sM + stage * C::M_BYTES)));
+#pragma unroll
+                        for (int j = 0; j < C::MMAS; ++j) {
+                            // step j: kept K elements [16j, 16j+16) of A (32 bytes in),
+                            // logical K [32j, 32j+32) of W: sub-tile j/2, 64 bytes in
+                            const uint64_t a_j = a_desc + (uint64_t)((32 * j) >> 4);
+                            const uint64_t b_j =
+                                sdesc_kmajor_sw128(b_addr + (j >> 1) * (BN * 128) + (j & 1) * 64);
+                            // metadata column e_tmem + j, addressed as the even column
+                            // plus the selector (bit 0 of the instruction descriptor)
+                            mma_sp_bf16(d_tmem, a_j, b_j, idesc | (uint32_t)(j & 1), e_tmem + (j & ~1),
+                                        (kb | j) != 0);
+                        }
+                    } else {
+                        const uint64_t b_desc = sdesc_kmajor_sw128(b_addr);
+#pragma unroll
+                        for (int j = 0; j < C::MMAS; ++j)
+                            mma_bf16(d_tmem, a_desc + (uint64_t)((32 * j) >> 4), b_desc + (uint64_t)((32 * j) >> 4),
+                                     idesc, (kb | j) != 0);
+                    }
+                    tc_commit(&empty[stage]);  // frees the stage when these MMAs finish
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) { *(volatile int *)abort_flag = 1; break; }
+                tc_commit(&acc_full[acc]);
+            }
+            // drain: wait until every MMA issued above has completed
+            tc_commit(drain);
+            mbar_wait(drain, 0);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;  // TMEM lanes 32q..32q+31
+        int it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && !*(volatile int *)abort_flag; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            int mt, nt;
+            tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
+            if (!mbar_wait(&acc_full[acc], acc_phase)) { *(volatile int *)abort_flag = 1; break; }
+            tc_fence_after();
+            const int row = mt * GEMM_BM + 32 * q + lane;
+            const bool row_ok = row < p.T;
+            float rscale = 1.0f, reta = 0.0f;
+            if (row_ok) {
+                if (p.nu) rscale = p.nu[row];
+                if (p.eta) reta = p.eta[row];
+            }
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + acc * BN + ch * 32, r);
+                tmem_ld_wait();
+                const int col0 = nt * BN + ch * 32;
+                if (!row_ok || col0 >= p.n_out) continue;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float f = __uint_as_float(r[i]);
+                    if (p.nu) f *= rscale;
+                    if (p.eta) {
+                        const int c = min(col0 + i, p.n_out - 1);
+                        f = fmaf(reta, p.rowsum[c], f);
+                    }
+                    v[i] = f;
+                }
+                if (p.out_bf16) {
+                    __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(p.y) + (size_t)row * p.n_out + col0;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        if (col0 + 8 * c8 < p.n_out) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * c8 + 2 * i], v[8 * c8 + 2 * i + 1]);
+                                w[i] = *reinterpret_cast<uint32_t *>(&h);
+                            }
+                            *reinterpret_cast<uint4 *>(yr + 8 * c8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                } else {
+                    float *yr = static_cast<float *>(p.y) + (size_t)row * p.n_out + col0;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        if (col0 + 4 * c4 < p.n_out)
+                            *reinterpret_cast<float4 *>(yr + 4 * c4) =
+                                make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                      const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled_t encode_fn()
+{
+    static PFN_encodeTiled_t fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled_t>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous), box {64 cols, box_rows}.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    PFN_encodeTiled_t enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <bool SPARSE>
+static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
+{
+    using C = GemmCfg<SPARSE>;
+    CUtensorMap mA, mB;
+    const uint64_t ka = SPARSE ? (uint64_t)a.K / 2 : (uint64_t)a.K;
+    if (!make_map(&mA, a.A, (uint64_t)a.T, ka, GEMM_BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, C::BN)) return cudaErrorInvalidValue;
+    GemmParams p{};
+    p.meta = a.meta;
+    p.rowsum = a.rowsum;
+    p.eta = a.eta;
+    p.nu = a.nu;
+    p.y = a.y;
+    p.T = a.T;
+    p.K = a.K;
+    p.n_out = a.n_out;
+    p.out_bf16 = a.out_bf16;
+    p.m_tiles = (a.T + GEMM_BM - 1) / GEMM_BM;
+    p.n_tiles = (a.n_out + C::BN - 1) / C::BN;
+    p.k_blocks = (a.K + C::KB - 1) / C::KB;
+    p.meta_kt = (a.K + 127) / 128;
+    const size_t smem = gemm_smem_bytes<SPARSE>();
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int grid = std::min(tiles, sm_count());
+    k_gemm<SPARSE><<<grid, GEMM_THREADS, smem, st>>>(mA, mB, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st)
+{
+    return a.sparse ? launch_gemm_t<true>(a, st) : launch_gemm_t<false>(a, st);
+}
+
+}  // namespace as

@@ -1,0 +1,73 @@
+// Host-side launchers of the kernels (internal to libactsparse).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace as {
+
+// ------------------------------------------------------------ weight prep
+size_t weight_prep_workspace(int n_out, int k);
+cudaError_t launch_weight_prep(const void *W, int bf16, int n_out, int k, float alpha, void *Wt, float *g,
+                               float *rowsum, void *ws, cudaStream_t st);
+
+// ------------------------------------------------------------ select
+struct SelectArgs {
+    const void *x;
+    int bf16;
+    int T, K;
+    int score, sel, n, m, k_keep, dpts, var, first;
+    float mom, eps;
+    const float *f;  // channel factor (g or c) or nullptr
+    float *running_var;
+    uint32_t *bitmask;
+    float *eta, *var_dense, *var_kept, *nu;
+    void *x_masked;
+    void *x_compact;
+    uint32_t *meta24;
+};
+// CLACT column energy c_j = sqrt(sum_t x_tj^2), float64 partials in ws.
+size_t colnorm_workspace(int T, int K);
+cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void *ws, cudaStream_t st);
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+
+// ------------------------------------------------------------ decode
+struct DecodeArgs {
+    const void *x;
+    const void *Wt;
+    int bf16;
+    int T, K, n_out;
+    int score, sel, n, m, dpts;
+    const float *g;
+    const float *rowsum;
+    const uint32_t *mask_in;  // precomputed selection (top-k / all), or nullptr for fused N:M
+    void *y;
+    int out_bf16;
+    uint32_t *mask_out;
+    float *eta_out;
+    float *colnorm_out;
+    float *partial;     // split-K partial sums
+    unsigned *counters; // one per N-slice, zero between calls
+};
+struct DecodePlan {
+    int n_slices, k_splits, words_per_split, tpad;
+    size_t partial_bytes, counter_bytes, smem_bytes;
+};
+DecodePlan decode_plan(int T, int K, int n_out, int bf16);
+cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st);
+
+// ------------------------------------------------------------ prefill GEMM
+struct GemmArgs {
+    const void *A;        // bf16 [T, Ka] K-major (x_masked, x or x_compact)
+    const uint32_t *meta; // 2:4 metadata (sparse only)
+    const void *W;        // bf16 [n_out, K] K-major
+    int T, K, n_out;
+    int sparse;
+    const float *rowsum, *eta, *nu;  // epilogue terms (optional)
+    void *y;
+    int out_bf16;
+};
+cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
+
+}  // namespace as

@@ -1,0 +1,350 @@
+// Per-token score, selection and compensation statistics (as_select).
+//
+// One CTA of 256 threads per token row.  Sources (page title, section):
+//  - 激活稀疏化技术：提升LLM推理效率的动态剪枝方法 (activation-sparsity overview):
+//    2.1 N:M patterns; 2.2.1 magnitude score; 2.2.3 CLACT score; 3.1 D-PTS
+//    (eta = token mean, prune x - eta, add eta back); 3.2 VAR (variance ratio
+//    with a running average).
+//  - 大模型推理优化：WiSparse激活稀疏化技术解析: 2.1 eq. (4) weight-aware score;
+//    2.2 per-layer keep fraction (exact top-k per token here).
+//  - 利用2:4稀疏性与Squared-ReLU加速Transformer训练与推理: 3.3 compressed
+//    layout with the kept values contiguous, plus position metadata.
+//
+// Row statistics accumulate in float64 (fixed order: per-thread strided sums,
+// warp tree, then the eight warps in order), the score is one float32
+// subtraction and one float32 multiply, and the decision compares float32
+// bit patterns (scores are >= 0) with ties to the lower index.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "select_util.cuh"
+
+namespace as {
+
+constexpr int SEL_THREADS = 256;
+
+// Block-wide sum of two float64 values (deterministic order).
+__device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[SEL_THREADS / 32])
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    a = warp_sum_f64(a);
+    b = warp_sum_f64(b);
+    if (lane == 0) { red[0][warp] = a; red[1][warp] = b; }
+    __syncthreads();
+    double sa = 0.0, sb = 0.0;
+#pragma unroll
+    for (int w = 0; w < SEL_THREADS / 32; ++w) { sa += red[0][w]; sb += red[1][w]; }
+    a = sa;
+    b = sb;
+    __syncthreads();
+}
+
+// Exclusive prefix sum over the block in thread order; returns the prefix,
+// `total` receives the block total.
+__device__ __forceinline__ int block_excl_scan(int v, int &total, int *wsum)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < SEL_THREADS / 32; ++w) {
+        if (w < warp) base += wsum[w];
+        tot += wsum[w];
+    }
+    __syncthreads();
+    total = tot;
+    return base + inc - v;
+}
+
+// 2:4 metadata byte address (see the meta24 layout in actsparse.h).
+__device__ __forceinline__ uint8_t *meta_byte(uint32_t *meta, int t, int c0, int kt)
+{
+    const int p = t & 127, tile = (t >> 7) * kt + (c0 >> 7);
+    const int j = (c0 & 127) >> 5, q = c0 & 31;
+    const int lane = 16 * (p >> 4) + 8 * (q >> 4) + (p & 7);
+    const int byte = 2 * ((p & 15) >> 3) + ((q & 15) >> 3);
+    return reinterpret_cast<uint8_t *>(meta) + (size_t)tile * 2048 + lane * 16 + j * 4 + byte;
+}
+
+template <typename TX>
+__device__ __forceinline__ void store8(TX *p, const float (&v)[8]);
+
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16 *p, const float (&v)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <>
+__device__ __forceinline__ void store8<float>(float *p, const float (&v)[8])
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
+{
+    extern __shared__ __align__(16) uint32_t keys[];  // [K] score bits (top-k only)
+    __shared__ double red[2][SEL_THREADS / 32];
+    __shared__ int wsum[SEL_THREADS / 32];
+    __shared__ uint32_t hist[256];
+    __shared__ uint32_t s_digit, s_remaining;
+
+    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int K = a.K, ngroups = K >> 3, ntiles = (ngroups + SEL_THREADS - 1) / SEL_THREADS;
+    const int kt = (K + 127) >> 7;
+
+    if (t >= a.T) {  // padding rows of the 2:4 metadata tiles
+        if (a.meta24)
+            for (int g = tid; g < kt * 16; g += SEL_THREADS) *meta_byte(a.meta24, t, 8 * g, kt) = 0x44;
+        return;
+    }
+    const TX *xr = static_cast<const TX *>(a.x) + (size_t)t * K;
+
+    // ---- row statistics: sum x, sum x^2 (float64)
+    double sx = 0.0, sxx = 0.0;
+    if (a.dpts || a.var) {
+        for (int g = tid; g < ngroups; g += SEL_THREADS) {
+            float v[8];
+            load8(xr + 8 * g, v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                sx += (double)v[e];
+                sxx += (double)v[e] * (double)v[e];
+            }
+        }
+        block_sum2(sx, sxx, red);
+    }
+    const float eta = a.dpts ? (float)(sx / (double)K) : 0.0f;
+    if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
+
+    // ---- top-k: scores to shared memory, then an MSB-first radix select of
+    // the k-th largest key and the number of equal keys to keep.
+    uint32_t tau = 0;
+    int need = 0;
+    const bool topk = a.sel == AS_SEL_TOPK;
+    const int kk = a.k_keep;
+    if (topk && kk > 0 && kk < K) {
+        for (int g = tid; g < ngroups; g += SEL_THREADS) {
+            float v[8], xh[8], s[8];
+            load8(xr + 8 * g, v);
+            score8(v, a.dpts, eta, a.f, 8 * g, xh, s);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) keys[8 * g + e] = __float_as_uint(s[e]);
+        }
+        uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)kk;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            hist[tid] = 0;
+            __syncthreads();
+            for (int i = tid; i < K; i += SEL_THREADS) {
+                uint32_t key = keys[i];
+                if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (tid < 32) {
+                // lane l owns digits 255-8l .. 248-8l (highest first)
+                uint32_t c = 0;
+#pragma unroll
+                for (int d = 0; d < 8; ++d) c += hist[255 - 8 * lane - d];
+                uint32_t inc = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    uint32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += u;
+                }
+                unsigned hit = __ballot_sync(0xffffffffu, inc >= remaining);
+                int L = __ffs(hit) - 1;
+                if (lane == L) {
+                    uint32_t cum = inc - c;
+                    for (int d = 0; d < 8; ++d) {
+                        uint32_t h = hist[255 - 8 * lane - d];
+                        if (cum + h >= remaining) {
+                            s_digit = 255 - 8 * lane - d;
+                            s_remaining = remaining - cum;
+                            break;
+                        }
+                        cum += h;
+                    }
+                }
+            }
+            __syncthreads();
+            prefix |= s_digit << shift;
+            pmask |= 255u << shift;
+            remaining = s_remaining;
+            __syncthreads();
+        }
+        tau = prefix;
+        need = (int)remaining;
+    }
+
+    // ---- decisions and outputs, 2048 channels (8 per thread) per tile
+    const int words = (K + 31) >> 5;
+    double skm = 0.0, skmm = 0.0;
+    int eq_base = 0;
+    for (int tile = 0; tile < ntiles; ++tile) {
+        const int g = tile * SEL_THREADS + tid, c0 = 8 * g;
+        const bool act = g < ngroups;
+        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, xh[8], s[8];
+        if (act) load8(xr + c0, v);
+        score8(v, a.dpts, eta, act ? a.f : nullptr, c0, xh, s);
+        uint32_t keep;
+        if (a.sel == AS_SEL_NM) {
+            keep = nm_keep_dispatch(s, lane, a.n, a.m);
+        } else if (topk) {
+            if (kk <= 0) keep = 0;
+            else if (kk >= K) keep = 0xFF;
+            else {
+                uint32_t gt = 0, eq = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    uint32_t key = act ? keys[c0 + e] : 0u;
+                    gt |= (uint32_t)(act && key > tau) << e;
+                    eq |= (uint32_t)(act && key == tau) << e;
+                }
+                int total;
+                int before = eq_base + block_excl_scan(__popc(eq), total, wsum);
+                eq_base += total;
+                keep = gt;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if ((eq >> e) & 1u) {
+                        keep |= (uint32_t)(before < need) << e;
+                        ++before;
+                    }
+            }
+        } else {
+            keep = 0xFF;
+        }
+        if (!act) continue;
+
+        if (a.bitmask) {
+            uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
+            bm[g] = (uint8_t)keep;
+            if (g == ngroups - 1)
+                for (int b = ngroups; b < words * 4; ++b) bm[b] = 0;
+        }
+        float km[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) km[e] = ((keep >> e) & 1u) ? xh[e] : 0.0f;
+        if (a.var) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                skm += (double)km[e];
+                skmm += (double)km[e] * (double)km[e];
+            }
+        }
+        if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
+        if (a.x_compact) {
+            // two 4-blocks per thread, two kept values each (exactly 2:4)
+            float cv[4];
+            uint32_t nib[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t b = (keep >> (4 * h)) & 0xFu;
+                int i0 = __ffs(b) - 1;
+                int i1 = 31 - __clz(b);
+                cv[2 * h] = xh[4 * h + i0];
+                cv[2 * h + 1] = xh[4 * h + i1];
+                nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
+            }
+            __nv_bfloat162 p0 = __floats2bfloat162_rn(cv[0], cv[1]);
+            __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
+            uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1));
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) = pk;
+            if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
+        }
+    }
+    if (a.meta24 && tid < 16 * kt - ngroups)  // channel padding of the last 128-channel tile
+        *meta_byte(a.meta24, t, 8 * (ngroups + tid), kt) = 0x44;
+
+    // ---- VAR: variances, running average, scale
+    if (a.var) {
+        block_sum2(skm, skmm, red);
+        if (tid == 0) {
+            const double Kd = (double)K;
+            double vd = (sxx - sx * sx / Kd) / (Kd - 1.0);
+            double vk = (skmm - skm * skm / Kd) / (Kd - 1.0);
+            double run = a.first ? vd : (double)a.mom * (double)a.running_var[t] + (1.0 - (double)a.mom) * vd;
+            a.running_var[t] = (float)run;
+            if (a.var_dense) a.var_dense[t] = (float)vd;
+            if (a.var_kept) a.var_kept[t] = (float)vk;
+            if (a.nu) a.nu[t] = (float)sqrt(run / (vk + (double)a.eps));
+        }
+    }
+}
+
+// ---------------------------------------------------------------- CLACT
+template <typename TX>
+__global__ void k_colsq_rows(const TX *__restrict__ x, int T, int K, int rows_per, double *__restrict__ part)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x, s = blockIdx.y;
+    if (i >= K) return;
+    const int t0 = s * rows_per, t1 = min(T, t0 + rows_per);
+    double acc = 0.0;
+    for (int t = t0; t < t1; ++t) {
+        double v = (double)Elem<TX>::to_f32(x[(size_t)t * K + i]);
+        acc += v * v;
+    }
+    part[(size_t)s * K + i] = acc;
+}
+
+__global__ void k_colnorm_final(const double *__restrict__ part, int slabs, int K, float *__restrict__ c)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= K) return;
+    double s = 0.0;
+    for (int j = 0; j < slabs; ++j) s += part[(size_t)j * K + i];
+    c[i] = (float)sqrt(s);
+}
+
+static int colnorm_slabs(int T) { return (T + 127) / 128; }
+
+size_t colnorm_workspace(int T, int K)
+{
+    return (size_t)colnorm_slabs(T) * (size_t)K * sizeof(double) + (size_t)K * sizeof(float);
+}
+
+cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void *ws, cudaStream_t st)
+{
+    const int slabs = colnorm_slabs(T);
+    double *part = static_cast<double *>(ws);
+    dim3 grid((K + 127) / 128, slabs);
+    if (bf16)
+        k_colsq_rows<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), T, K, 128, part);
+    else
+        k_colsq_rows<float><<<grid, 128, 0, st>>>(static_cast<const float *>(x), T, K, 128, part);
+    k_colnorm_final<<<(K + 255) / 256, 256, 0, st>>>(part, slabs, K, c);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st)
+{
+    const bool topk = a.sel == AS_SEL_TOPK && a.k_keep > 0 && a.k_keep < a.K;
+    const size_t smem = topk ? (size_t)a.K * sizeof(uint32_t) : 0;
+    const int grid = a.meta24 ? ((a.T + 127) / 128) * 128 : a.T;
+    if (a.bf16) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(k_select<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_select<__nv_bfloat16><<<grid, SEL_THREADS, smem, st>>>(a);
+    } else {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(k_select<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_select<float><<<grid, SEL_THREADS, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace as

@@ -1,0 +1,103 @@
+// Selection helpers shared by the select and decode kernels.
+//
+// Activation-sparsity overview page (激活稀疏化技术：提升LLM推理效率的动态剪枝方法)
+// section 2.1 / 2.2.1: keep N of every M consecutive channels by score; the
+// page's snippet keeps everything >= the N-th value, which can keep more
+// than N on ties.  Here exactly N are kept and equal float32 scores go to the
+// lower channel index, so the result is unique.
+#pragma once
+
+#include "common.cuh"
+
+namespace as {
+
+// Eight consecutive channels of one token, converted to float32 (exact).
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8])
+{
+    uint4 r = *reinterpret_cast<const uint4 *>(p);
+    uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ void load8(const float *p, float (&v)[8])
+{
+    float4 a = *reinterpret_cast<const float4 *>(p);
+    float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8f(const float *p, float (&v)[8]) { load8(p, v); }
+
+// Score of eight channels: s = fl32(|xhat| * f), xhat = fl32(x - eta) when
+// shift != 0.  Explicit round-to-nearest intrinsics keep the compiler from
+// contracting or reassociating (the selection decision depends on the bits).
+__device__ __forceinline__ void score8(const float (&x)[8], bool shift, float eta, const float *f, int c0,
+                                       float (&xh)[8], float (&s)[8])
+{
+    float fv[8];
+    if (f) load8f(f + c0, fv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        xh[e] = shift ? __fsub_rn(x[e], eta) : x[e];
+        float a = fabsf(xh[e]);
+        s[e] = f ? __fmul_rn(a, fv[e]) : a;
+    }
+}
+
+// "j ranks ahead of i": higher score, or equal score and lower index.
+__device__ __forceinline__ int ahead(float sj, int j, float si, int i) { return (sj > si) | ((sj == si) & (j < i)); }
+
+// Keep bits (bit e = channel 8*lane_group + e) of exactly-N-per-M selection.
+// The lane holds channels [8g, 8g+8); blocks of M > 8 span M/8 consecutive
+// lanes, whose scores are exchanged with shuffles (all 32 lanes must call).
+template <int M>
+__device__ __forceinline__ uint32_t nm_keep(const float (&s)[8], int lane, int n)
+{
+    uint32_t keep = 0;
+    if constexpr (M <= 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int b0 = (e / M) * M;
+            int rank = 0;
+#pragma unroll
+            for (int j = 0; j < M; ++j) rank += (j + b0 != e) & ahead(s[b0 + j], b0 + j, s[e], e);
+            keep |= (uint32_t)(rank < n) << e;
+        }
+    } else {
+        constexpr int G = M / 8;
+        float blk[M];
+        const int base = lane & ~(G - 1);
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) blk[q * 8 + e] = __shfl_sync(0xffffffffu, s[e], base + q);
+        const int pe0 = (lane & (G - 1)) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            int rank = 0;
+#pragma unroll
+            for (int j = 0; j < M; ++j) rank += (j != pe0 + e) & ahead(blk[j], j, s[e], pe0 + e);
+            keep |= (uint32_t)(rank < n) << e;
+        }
+    }
+    return keep;
+}
+
+__device__ __forceinline__ uint32_t nm_keep_dispatch(const float (&s)[8], int lane, int n, int m)
+{
+    switch (m) {
+    case 1: return nm_keep<1>(s, lane, n);
+    case 2: return nm_keep<2>(s, lane, n);
+    case 4: return nm_keep<4>(s, lane, n);
+    case 8: return nm_keep<8>(s, lane, n);
+    case 16: return nm_keep<16>(s, lane, n);
+    default: return nm_keep<32>(s, lane, n);
+    }
+}
+
+}  // namespace as

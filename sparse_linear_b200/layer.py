@@ -1,0 +1,104 @@
+"""Buffer management around the C ABI: a prepared sparse linear layer.
+
+``SparseLinear`` owns the per-layer tensors (channel-major weight copy,
+weight-aware channel factors, row sums) and a zero-filled workspace, all
+allocated through torch on the current CUDA device, and calls the C entry
+points.  It performs no arithmetic of its own.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (AS_BF16, AS_F32, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_SELECT, AS_OP_WEIGHT_PREP,
+               AS_SCORE_CLACT, AS_SEL_NM, as_linear_decode, as_linear_prefill, as_meta24_words,
+               as_select, as_weight_prep, as_workspace_size, select_out)
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """Zero-filled byte buffer (the ABI requires zeros before first use)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+class SparseLinear:
+    """One activation-sparsified linear layer y = prune(x) W^T.
+
+    W: [n_out, K] bf16 or f32 CUDA tensor (PyTorch Linear layout).
+    cfg: ``as_config``; ``alpha`` is the weight-aware exponent.
+    ``keep_wt`` builds the channel-major copy needed by the decode path.
+    """
+
+    def __init__(self, W: torch.Tensor, cfg, alpha: float = 0.0, keep_wt: bool = True):
+        self.W = W.contiguous()
+        self.cfg = cfg
+        self.alpha = float(alpha)
+        self.n_out, self.K = W.shape
+        dev = W.device
+        self.g = torch.empty(self.K, dtype=torch.float32, device=dev)
+        self.rowsum = torch.empty(self.n_out, dtype=torch.float32, device=dev)
+        self.Wt = torch.empty(self.K, self.n_out, dtype=W.dtype, device=dev) if keep_wt else None
+        ws = workspace(as_workspace_size(AS_OP_WEIGHT_PREP, 0, self.K, self.n_out, None), dev)
+        as_weight_prep(self.W, self.alpha, Wt=self.Wt, g=self.g, rowsum=self.rowsum, workspace=ws)
+        self._ws = {}
+
+    def _workspace(self, op: int, T: int) -> torch.Tensor:
+        key = (op, T)
+        if key not in self._ws:
+            self._ws[key] = workspace(as_workspace_size(op, T, self.K, self.n_out, self.cfg), self.W.device)
+        return self._ws[key]
+
+    def out_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.cfg.out_dtype == AS_BF16 else torch.float32
+
+    # ---------------------------------------------------------------- decode
+    def decode(self, x: torch.Tensor, y: torch.Tensor | None = None, mask_out=None, eta_out=None,
+               colnorm_out=None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=x.device)
+        as_linear_decode(x, self.Wt, self.cfg, y, g=self.g, rowsum=self.rowsum, mask_out=mask_out,
+                         eta_out=eta_out, colnorm_out=colnorm_out,
+                         workspace=self._workspace(AS_OP_DECODE, T), stream=stream)
+        return y
+
+    # ---------------------------------------------------------------- prefill
+    def select_buffers(self, T: int, device=None) -> dict:
+        """Device buffers for every as_select output this layer's cfg uses."""
+        dev = device or self.W.device
+        K = self.K
+        c = self.cfg
+        b = dict(bitmask=torch.empty(T, (K + 31) // 32, dtype=torch.int32, device=dev),
+                 eta=torch.empty(T, dtype=torch.float32, device=dev),
+                 colnorm=torch.empty(K, dtype=torch.float32, device=dev))
+        if c.var:
+            for k in ("var_dense", "var_kept", "nu"):
+                b[k] = torch.empty(T, dtype=torch.float32, device=dev)
+        if c.sel == AS_SEL_NM and c.n == 2 and c.m == 4 and self.W.dtype == torch.bfloat16:
+            b["x_compact"] = torch.empty(T, K // 2, dtype=torch.bfloat16, device=dev)
+            b["meta24"] = torch.empty(as_meta24_words(T, K), dtype=torch.int32, device=dev)
+        else:
+            b["x_masked"] = torch.empty(T, K, dtype=self.W.dtype, device=dev)
+        return b
+
+    def select(self, x: torch.Tensor, bufs: dict, running_var=None, first_batch: bool = False,
+               stream=None) -> None:
+        T = x.shape[0]
+        chan = self.g if self.cfg.score != AS_SCORE_CLACT else None
+        as_select(x, self.cfg, select_out(**bufs), chan_factor=chan, running_var=running_var,
+                  var_first_batch=first_batch, workspace=self._workspace(AS_OP_SELECT, T), stream=stream)
+
+    def prefill_from(self, bufs: dict, T: int, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=self.W.device)
+        as_linear_prefill(select_out(**{k: v for k, v in bufs.items()
+                                        if k in ("x_masked", "x_compact", "meta24")}),
+                          self.W, T, self.cfg, y, rowsum=self.rowsum, eta=bufs.get("eta"),
+                          nu=bufs.get("nu"), workspace=self._workspace(AS_OP_PREFILL, T), stream=stream)
+        return y
+
+    def prefill(self, x: torch.Tensor, running_var=None, first_batch: bool = False, stream=None):
+        bufs = self.select_buffers(x.shape[0], x.device)
+        self.select(x, bufs, running_var=running_var, first_batch=first_batch, stream=stream)
+        return self.prefill_from(bufs, x.shape[0], stream=stream), bufs
+
+
+__all__ = ["SparseLinear", "workspace", "AS_F32", "AS_BF16"]

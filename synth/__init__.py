@@ -63,11 +63,13 @@ def tiny_layer(seed: int = 0):
     return x, w
 
 
-def decode_downproj(T: int = 16, seed: int = 1, k: int = 11008, n_out: int = 4096):
+def decode_downproj(T: int = 16, seed: int = 1, k: int = 11008, n_out: int = 4096,
+                    with_weight: bool = True):
     """Decode down-projection activations and weight.
 
     Returns ``(x, W, outlier_channels)``; ``x`` is the first ``T`` of 16 drawn
-    tokens, so the T=1/8/16 cases are nested.
+    tokens, so the T=1/8/16 cases are nested.  ``W`` is None when
+    ``with_weight`` is False.
     """
     if not 1 <= T <= 16:
         raise ValueError("T must be in [1, 16]")
@@ -77,7 +79,7 @@ def decode_downproj(T: int = 16, seed: int = 1, k: int = 11008, n_out: int = 409
     x64 = rx.laplace(0.0, 0.3, size=(16, k))
     x64[:, outl] *= 20.0
     x = to_dtype(x64[:T], torch.bfloat16)
-    w = _normal(rw, (n_out, k), 0.02, torch.bfloat16)
+    w = _normal(rw, (n_out, k), 0.02, torch.bfloat16) if with_weight else None
     return x, w, torch.from_numpy(outl)
 
 

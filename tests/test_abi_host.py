@@ -1,0 +1,137 @@
+"""Host-only checks of the C-ABI library: it loads without a GPU, exports
+every entry point include/actsparse.h declares, and its argument validation
+rejects invalid calls with the documented status before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "actsparse.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_as_build", os.path.join(ROOT, "sparse_linear_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()
+    import sparse_linear_b200 as sl
+    return sl
+
+
+def declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(as_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for n in ("as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
+              "as_workspace_size", "as_stream_status", "as_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in declared():
+        assert hasattr(raw, n), n
+    assert set(lib.EXPORTS) == set(declared())
+    assert lib.as_abi_version() == 1
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        assert lib.as_status_string(code).startswith("AS_")
+
+
+def test_workspace_sizes(lib):
+    cfg = lib.config(score=lib.AS_SCORE_WEIGHT, sel=lib.AS_SEL_NM, n=8, m=16, dpts=True)
+    ws = lib.as_workspace_size(lib.AS_OP_DECODE, 1, 11008, 4096, cfg)
+    assert ws > 0
+    assert lib.as_workspace_size(lib.AS_OP_WEIGHT_PREP, 0, 4096, 1024, None) == 4 * 4096 * 8
+    assert lib.as_workspace_size(lib.AS_OP_PREFILL, 4096, 14336, 4096, lib.config()) == 0
+    bad = lib.config(sel=lib.AS_SEL_NM, n=2, m=4)
+    with pytest.raises(lib.ASError):
+        lib.as_workspace_size(lib.AS_OP_DECODE, 17, 1024, 64, bad)  # T > 16
+    with pytest.raises(lib.ASError):
+        lib.as_workspace_size(lib.AS_OP_SELECT, 4, 1022, 0, bad)  # K % M
+    assert lib.as_meta24_words(4096, 14336) == 32 * 112 * 512
+    assert lib.as_meta24_words(1, 16) == 512
+
+
+def _call_decode(lib, x, K, n_out, cfg, T=1, dt=None, y=16, wt=16, ws=16, ws_bytes=1 << 20):
+    f = lib._lib.as_linear_decode
+    return f(x, lib.AS_BF16 if dt is None else dt, T, K, n_out, wt, None, None, ctypes.byref(cfg), y,
+             None, None, None, ws, ws_bytes, None)
+
+
+def test_decode_validation_launches_nothing(lib):
+    """Invalid calls are rejected on the host (fake, never-dereferenced
+    16-byte-aligned addresses: a launch would fault, so any call reaching
+    the GPU would fail here without a GPU)."""
+    fake = 1 << 20
+    ok = lib.config(sel=lib.AS_SEL_NM, n=2, m=4)
+    assert _call_decode(lib, fake, 1000, 64, ok, T=0) == lib.AS_ERR_SHAPE
+    assert _call_decode(lib, fake, 1000, 64, ok, T=17) == lib.AS_ERR_SHAPE
+    assert _call_decode(lib, fake, 1002, 64, ok) == lib.AS_ERR_SHAPE                # K % M
+    assert _call_decode(lib, fake, 1024, 60, ok) == lib.AS_ERR_SHAPE                # n_out % 8
+    assert _call_decode(lib, fake, 1024, 64, lib.config(n=5, m=4)) == lib.AS_ERR_SHAPE
+    assert _call_decode(lib, fake, 1024, 64, lib.config(n=2, m=3)) == lib.AS_ERR_SHAPE
+    assert _call_decode(lib, fake, 1024, 64, lib.config(sel=lib.AS_SEL_TOPK, k_keep=2000)) == lib.AS_ERR_SHAPE
+    assert _call_decode(lib, fake, 1024, 64, ok, dt=7) == lib.AS_ERR_DTYPE
+    assert _call_decode(lib, fake + 4, 1024, 64, ok) == lib.AS_ERR_ALIGN
+    assert _call_decode(lib, None, 1024, 64, ok) == lib.AS_ERR_INVALID_ARG
+    assert _call_decode(lib, fake, 1024, 64, lib.config(var=True)) == lib.AS_ERR_UNSUPPORTED
+    assert _call_decode(lib, fake, 1024, 64, lib.config(dpts=True)) == lib.AS_ERR_INVALID_ARG  # no rowsum
+    assert _call_decode(lib, fake, 1024, 64, lib.config(score=lib.AS_SCORE_WEIGHT)) == lib.AS_ERR_INVALID_ARG
+    assert _call_decode(lib, fake, 1024, 64, ok, ws=None) == lib.AS_ERR_WORKSPACE
+    assert _call_decode(lib, fake, 1024, 64, ok, ws_bytes=0) == lib.AS_ERR_WORKSPACE
+
+
+def test_select_and_prefill_validation(lib):
+    fake = 1 << 20
+    sel = lib._lib.as_select
+    cfg24 = lib.config(sel=lib.AS_SEL_NM, n=2, m=4)
+    out = lib.as_select_out()
+    out.x_compact = fake
+    out.meta24 = fake
+    # compact 2:4 operand needs bf16 and K % 16 == 0
+    assert sel(fake, lib.AS_F32, 4, 64, ctypes.byref(cfg24), None, None, 0, ctypes.byref(out), None, 0,
+               None) == lib.AS_ERR_UNSUPPORTED
+    assert sel(fake, lib.AS_BF16, 4, 72, ctypes.byref(cfg24), None, None, 0, ctypes.byref(out), None, 0,
+               None) == lib.AS_ERR_UNSUPPORTED
+    cfg816 = lib.config(sel=lib.AS_SEL_NM, n=8, m=16)
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(cfg816), None, None, 0, ctypes.byref(out), None, 0,
+               None) == lib.AS_ERR_UNSUPPORTED
+    both = lib.config(dpts=True, var=True)
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(both), None, fake, 1, ctypes.byref(lib.as_select_out()),
+               None, 0, None) == lib.AS_ERR_UNSUPPORTED
+    var = lib.config(var=True)
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(var), None, None, 1, ctypes.byref(lib.as_select_out()),
+               None, 0, None) == lib.AS_ERR_INVALID_ARG  # no running_var
+    clact = lib.config(score=lib.AS_SCORE_CLACT, n=16, m=32)
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(clact), None, None, 0, ctypes.byref(lib.as_select_out()),
+               None, 0, None) == lib.AS_ERR_WORKSPACE
+    pre = lib._lib.as_linear_prefill
+    empty = lib.as_select_out()
+    assert pre(ctypes.byref(empty), fake, 4, 64, 64, None, None, None, ctypes.byref(cfg816), fake, None, 0,
+               None) == lib.AS_ERR_INVALID_ARG  # no x_masked
+    assert pre(ctypes.byref(empty), fake, 4, 64, 64, None, None, None, ctypes.byref(cfg24), fake, None, 0,
+               None) == lib.AS_ERR_INVALID_ARG  # no compact operand
+    masked = lib.as_select_out()
+    masked.x_masked = fake
+    assert pre(ctypes.byref(masked), fake, 4, 60, 64, None, None, None, ctypes.byref(lib.config(n=2, m=2)),
+               fake, None, 0, None) == lib.AS_ERR_SHAPE  # K % 8
+    assert pre(ctypes.byref(masked), fake, 4, 64, 64, None, None, None, ctypes.byref(lib.config(dpts=True, n=8, m=16)),
+               fake, None, 0, None) == lib.AS_ERR_INVALID_ARG  # dpts needs eta and rowsum
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lib.as_linear_decode(x, x, lib.config(), x)

@@ -1,0 +1,303 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Masks and indices must match bit-exactly (the oracle's selection is run on
+the float32 statistics the GPU exported: eta, g, c); statistics within the
+stated relative bounds of the oracle's float64 values; outputs within
+relative L2 error 2e-3 (float32 output) or 1e-2 (bf16 output)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import decode_meta24, f32, rel_l2, unpack_bitmask
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32, TOL_BF16 = 2e-3, 1e-2
+
+
+@pytest.fixture(scope="module")
+def sl():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import sparse_linear_b200 as m
+    return m
+
+
+def dev(t):
+    return t.cuda().contiguous()
+
+
+def layer(sl, W, cfg, alpha=0.0):
+    from sparse_linear_b200.layer import SparseLinear
+    return SparseLinear(dev(W), cfg, alpha=alpha)
+
+
+# ---------------------------------------------------------------- weight prep
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 1.0])
+def test_weight_prep(sl, alpha):
+    _, W = synth.random_layer(1, 520, 1000, seed=21)
+    L = layer(sl, W, sl.config(), alpha)
+    g_ref, rs_ref = oracle.weight_prep(W.float().numpy(), alpha)
+    np.testing.assert_allclose(f32(L.g), g_ref, rtol=1e-6)
+    scale = np.sqrt((W.double().numpy() ** 2).sum(1))
+    assert (np.abs(f32(L.rowsum) - rs_ref) <= 1e-6 * scale + 1e-30).all()
+    assert torch.equal(L.Wt.cpu(), W.t().contiguous())
+
+
+# ---------------------------------------------------------------- decode
+def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None):
+    """Runs as_linear_decode; checks eta, mask (bit-exact) and y."""
+    T, K = x.shape
+    L = layer(sl, W, cfg, alpha)
+    xd = dev(x)
+    words = (K + 31) // 32
+    mask_d = torch.zeros(T, words, dtype=torch.int32, device="cuda")
+    eta_d = torch.zeros(T, dtype=torch.float32, device="cuda")
+    c_d = torch.zeros(K, dtype=torch.float32, device="cuda")
+    y = L.decode(xd, mask_out=mask_d, eta_out=eta_d, colnorm_out=c_d)
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    xf = x.float().numpy()
+    eta32 = None
+    eta64 = None
+    if cfg.dpts:
+        eta64 = oracle.token_mean(xf)
+        eta32 = f32(eta_d)
+        assert (np.abs(eta32 - eta64) <= 1e-6 * np.abs(xf).mean(1)).all()
+    if cfg.score == sl.AS_SCORE_WEIGHT:
+        f = f32(L.g)
+    elif cfg.score == sl.AS_SCORE_CLACT:
+        f = f32(c_d)
+        np.testing.assert_allclose(f, oracle.channel_energy(xf), rtol=1e-6)
+    else:
+        f = None
+    s = oracle.score(xf, eta=eta32, f=f)
+    if cfg.sel == sl.AS_SEL_NM:
+        ref_mask = oracle.select_nm(s, cfg.n, cfg.m)
+    elif cfg.sel == sl.AS_SEL_TOPK:
+        ref_mask = oracle.select_topk(s, cfg.k_keep)
+    else:
+        ref_mask = np.ones_like(s, np.uint8)
+    got = unpack_bitmask(mask_d, K)
+    np.testing.assert_array_equal(got, ref_mask)
+    _, rs = oracle.weight_prep(W.float().numpy(), 1.0)
+    ref = oracle.linear(xf, ref_mask, W.float().numpy(), eta=eta64, rowsum=rs if cfg.dpts else None)
+    if tol is None:
+        tol = TOL_BF16 if cfg.out_dtype == sl.AS_BF16 else TOL_F32
+    err = rel_l2(f32(y), ref)
+    assert err <= tol, err
+    return y, got
+
+
+def test_decode_tiny_layer(sl):
+    """x f32 [4,256], W f32 [512,256], 2:4 magnitude, no compensation."""
+    x, W = synth.tiny_layer()
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, out_dtype=sl.AS_F32)
+    check_decode(sl, x, W, cfg)
+
+
+@pytest.mark.parametrize("T", [1, 8, 16])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_decode_downproj(sl, T, out):
+    """Llama-7B down-projection: 8:16 weight-aware alpha=0.5 with D-PTS."""
+    x, W, _ = synth.decode_downproj(T)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True,
+                    out_dtype=sl.AS_BF16 if out == "bf16" else sl.AS_F32)
+    check_decode(sl, x, W, cfg, alpha=0.5)
+
+
+@pytest.mark.parametrize("T,K,n_out,n,m,score,dpts,ties", [
+    (3, 1040, 264, 2, 4, 0, False, 0),
+    (5, 1040, 264, 8, 16, 1, True, 0),
+    (2, 2048, 520, 16, 32, 2, False, 0),
+    (7, 1056, 72, 1, 4, 0, True, 3),
+    (16, 512, 256, 4, 8, 1, False, 2),
+    (4, 4096, 1024, 16, 32, 0, True, 2),
+    (11, 8192, 136, 8, 16, 2, True, 0),
+    (1, 96, 8, 2, 4, 0, False, 1),
+])
+def test_decode_ragged(sl, T, K, n_out, n, m, score, dpts, ties):
+    x, W = synth.random_layer(T, K, n_out, seed=T * 1000 + K + m, ties=ties)
+    cfg = sl.config(score=score, sel=sl.AS_SEL_NM, n=n, m=m, dpts=dpts, out_dtype=sl.AS_F32)
+    check_decode(sl, x, W, cfg, alpha=0.5)
+
+
+def test_decode_fp32_weights(sl):
+    x, W = synth.random_layer(6, 1024, 264, seed=5, dtype=torch.float32)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True, out_dtype=sl.AS_F32)
+    check_decode(sl, x, W, cfg, alpha=1.0)
+
+
+def test_decode_block_topk(sl):
+    """Llama3.1-8B block at one token: per-layer exact top-k keep fraction and
+    weight-aware exponent."""
+    blk = synth.decode_block()
+    for ly in blk["layers"]:
+        K = ly["k"]
+        kk = int(math.floor(ly["keep_frac"] * K + 0.5))
+        cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_TOPK, k_keep=kk)
+        check_decode(sl, blk["x"][ly["x_key"]], ly["W"], cfg, alpha=ly["alpha"])
+
+
+@pytest.mark.parametrize("kk", [0, 1, 100, 1023, 1024])
+def test_decode_topk_edges(sl, kk):
+    x, W = synth.random_layer(3, 1024, 64, seed=kk, ties=2)
+    cfg = sl.config(score=sl.AS_SCORE_MAG, sel=sl.AS_SEL_TOPK, k_keep=kk, dpts=True, out_dtype=sl.AS_F32)
+    check_decode(sl, x, W, cfg)
+
+
+def test_decode_keep_all_is_dense(sl):
+    x, W = synth.random_layer(4, 1024, 136, seed=9)
+    cfg = sl.config(sel=sl.AS_SEL_ALL, out_dtype=sl.AS_F32)
+    y, mask = check_decode(sl, x, W, cfg)
+    assert mask.all()
+
+
+def test_decode_deterministic(sl):
+    x, W, _ = synth.decode_downproj(8)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
+    L = layer(sl, W, cfg, 0.5)
+    xd = dev(x)
+    y1 = L.decode(xd).clone()
+    y2 = L.decode(xd).clone()
+    assert torch.equal(y1, y2)
+
+
+# ---------------------------------------------------------------- prefill
+def check_select_24(sl, x, bufs, rows):
+    """2:4 select outputs on the given rows: bitmask, compact values, metadata."""
+    T, K = x.shape
+    xf = x.float().numpy()[rows]
+    ref_mask = oracle.select_nm(oracle.score(xf), 2, 4)
+    got = unpack_bitmask(bufs["bitmask"], K)[rows]
+    np.testing.assert_array_equal(got, ref_mask)
+    vals, pos = oracle.compress_nm(xf, ref_mask, 2, 4)
+    np.testing.assert_array_equal(f32(bufs["x_compact"])[rows], vals)  # exact: x is bf16, no shift
+    meta = decode_meta24(bufs["meta24"], T, K)[rows]
+    np.testing.assert_array_equal(meta.reshape(len(rows), -1), pos.astype(np.int64))
+    return ref_mask
+
+
+@pytest.mark.parametrize("T,K,n_out", [(300, 1024, 520), (128, 14336, 256), (5, 256, 64), (1000, 2048, 1024)])
+def test_prefill_24(sl, T, K, n_out):
+    x, W = synth.random_layer(T, K, n_out, seed=T + K, dist="sqrelu")
+    for out in (sl.AS_BF16, sl.AS_F32):
+        cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, out_dtype=out)
+        L = layer(sl, W, cfg)
+        y, bufs = L.prefill(dev(x))
+        torch.cuda.synchronize()
+        assert sl.as_stream_status() == sl.AS_OK
+        rows = np.arange(T)
+        mask = check_select_24(sl, x, bufs, rows)
+        ref = oracle.linear(x.float().numpy(), mask, W.float().numpy())
+        err = rel_l2(f32(y), ref)
+        assert err <= (TOL_BF16 if out == sl.AS_BF16 else TOL_F32), err
+
+
+def test_prefill_24_full_size(sl):
+    """FFN down-projection at prefill: squared-ReLU activations [4096, 14336],
+    2:4 by magnitude on the sparse tensor-core path; sampled rows."""
+    _, x, W = synth.prefill_sqrelu()
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4)
+    L = layer(sl, W, cfg)
+    y, bufs = L.prefill(dev(x))
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    rows = np.array([0, 1, 127, 128, 1000, 2047, 2048, 3071, 4094, 4095])
+    mask = check_select_24(sl, x, bufs, rows)
+    ref = oracle.linear(x.float().numpy()[rows], mask, W.float().numpy())
+    assert rel_l2(f32(y)[rows], ref) <= TOL_BF16
+    # property over the whole output: the share of natural nonzeros that the
+    # 2:4 enforcement drops matches its closed form (2:4 + Squared-ReLU page, 2.3)
+    nzm = unpack_bitmask(bufs["bitmask"], x.shape[1])
+    nz = x.float().numpy() != 0
+    dropped = (nz & (nzm == 0)).sum() / nz.sum()
+    p = 0.5 * math.erfc(1.2 / math.sqrt(2))
+    assert abs(dropped - (4 * p ** 3 * (1 - p) + 2 * p ** 4) / (4 * p)) < 2e-4
+
+
+def check_prefill_masked(sl, xs, W, cfg, alpha=0.0, rows=None):
+    """Runs select + prefill over a list of batches (VAR running state
+    carried); checks statistics, masks and outputs on `rows`."""
+    L = layer(sl, W, cfg, alpha)
+    T, K = xs[0].shape
+    running = torch.zeros(T, dtype=torch.float32, device="cuda")
+    run_ref = None
+    rows = np.arange(T) if rows is None else rows
+    for b, x in enumerate(xs):
+        y, bufs = L.prefill(dev(x), running_var=running, first_batch=(b == 0))
+        torch.cuda.synchronize()
+        assert sl.as_stream_status() == sl.AS_OK
+        xf = x.float().numpy()
+        if cfg.score == sl.AS_SCORE_CLACT:
+            f = f32(bufs["colnorm"])
+            np.testing.assert_allclose(f, oracle.channel_energy(xf), rtol=1e-6)
+        elif cfg.score == sl.AS_SCORE_WEIGHT:
+            f = f32(L.g)
+        else:
+            f = None
+        eta32 = f32(bufs["eta"])[rows] if cfg.dpts else None
+        eta64 = oracle.token_mean(xf[rows]) if cfg.dpts else None
+        if cfg.dpts:
+            assert (np.abs(eta32 - eta64) <= 1e-6 * np.abs(xf[rows]).mean(1)).all()
+        s = oracle.score(xf[rows], eta=eta32, f=f)
+        ref_mask = (oracle.select_nm(s, cfg.n, cfg.m) if cfg.sel == sl.AS_SEL_NM
+                    else oracle.select_topk(s, cfg.k_keep) if cfg.sel == sl.AS_SEL_TOPK
+                    else np.ones_like(s, np.uint8))
+        np.testing.assert_array_equal(unpack_bitmask(bufs["bitmask"], K)[rows], ref_mask)
+        nu = None
+        if cfg.var:
+            st = oracle.var_scale(xf[rows], ref_mask, None if run_ref is None else run_ref[rows],
+                                  cfg.var_momentum, cfg.var_eps)
+            if run_ref is None:
+                run_ref = np.zeros(T)
+            run_ref[rows] = st["running"]
+            np.testing.assert_allclose(f32(bufs["var_dense"])[rows], st["var_dense"], rtol=1e-6)
+            np.testing.assert_allclose(f32(bufs["var_kept"])[rows], st["var_kept"], rtol=1e-6)
+            np.testing.assert_allclose(f32(running)[rows], st["running"], rtol=1e-5)
+            np.testing.assert_allclose(f32(bufs["nu"])[rows], st["nu"], rtol=1e-5)
+            nu = st["nu"]
+        _, rs = oracle.weight_prep(W.float().numpy(), 1.0)
+        ref = oracle.linear(xf[rows], ref_mask, W.float().numpy(), eta=eta64,
+                            rowsum=rs if cfg.dpts else None, nu=nu)
+        tol = TOL_BF16 if cfg.out_dtype == sl.AS_BF16 else TOL_F32
+        if cfg.dpts:
+            tol = max(tol, TOL_BF16)  # the shifted kept values enter the tensor cores as bf16
+        err = rel_l2(f32(y)[rows], ref)
+        assert err <= tol, (b, err)
+
+
+def test_prefill_clact_var_small(sl):
+    T, K, n_out = 264, 1024, 264
+    xs = [synth.random_layer(T, K, n_out, seed=100 + b, dist="t3")[0] for b in range(3)]
+    W = synth.random_layer(1, K, n_out, seed=99)[1]
+    cfg = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)
+    check_prefill_masked(sl, xs, W, cfg)
+
+
+@pytest.mark.parametrize("n,m,score,dpts", [(8, 16, 1, True), (4, 8, 0, False), (1, 4, 2, False)])
+def test_prefill_dense_path(sl, n, m, score, dpts):
+    T, K, n_out = 200, 2048, 392
+    x, W = synth.random_layer(T, K, n_out, seed=n * m, dist="laplace")
+    cfg = sl.config(score=score, sel=sl.AS_SEL_NM, n=n, m=m, dpts=dpts, out_dtype=sl.AS_F32)
+    check_prefill_masked(sl, [x], W, cfg, alpha=0.5)
+
+
+def test_prefill_topk_and_all(sl):
+    T, K, n_out = 130, 1024, 256
+    x, W = synth.random_layer(T, K, n_out, seed=3)
+    check_prefill_masked(sl, [x], W, sl.config(sel=sl.AS_SEL_TOPK, k_keep=600))
+    check_prefill_masked(sl, [x], W, sl.config(sel=sl.AS_SEL_ALL, out_dtype=sl.AS_F32))
+
+
+def test_prefill_clact_var_full_size(sl):
+    """CLACT + VAR at 16:32 on [8192, 8192] (masked dense tensor-core GEMM):
+    two of the eight batches, sampled rows."""
+    W = synth.prefill_clact_weight()
+    xs = [synth.prefill_clact_batch(b) for b in range(2)]
+    cfg = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)
+    rows = np.array([0, 127, 128, 4097, 8190, 8191])
+    check_prefill_masked(sl, xs, W, cfg, rows=rows)
