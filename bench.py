@@ -140,9 +140,9 @@ def kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kind: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+def recorded_traffic():
+    """Mean per-launch DRAM bytes over T = 1, 8, 16 from the committed ncu
+    summary, if every T was captured on the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "decode_downproj_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -153,8 +153,10 @@ def recorded_traffic(kind: str):
             kv[k.strip()] = v.strip()
     if kv.get("kernel_source_sha256_16") != kernel_hash():
         return None
-    v = kv.get(kind)
-    return float(v) if v else None
+    vals = [kv.get(f"dram_bytes_T{T}") for T in DECODE_TS]
+    if not all(vals):
+        return None
+    return sum(float(v) for v in vals) / len(vals)
 
 
 # ---------------------------------------------------------------- decode
@@ -237,17 +239,17 @@ def bench_decode(sl, dev, steps, warmup, world):
         barrier(world)
         return s.elapsed_time(e) / 1e3
 
+    clk = Clocks(torch.cuda.current_device()).__enter__()
     for j in range(max(3, warmup)):
         with torch.cuda.stream(stream):
             graphs[j % N_ROT].replay()
     torch.cuda.synchronize()
-    with Clocks(torch.cuda.current_device()) as clk:
-        t_local = timed(lambda j: graphs[j % N_ROT].replay(), steps)
-        # per-T kernel durations (each graph holds one decode launch)
-        per_t = {}
-        reps = max(4 * N_ROT, steps)
-        for T in DECODE_TS:
-            per_t[T] = timed(lambda j, T=T: per_t_graphs[T][j % N_ROT].replay(), reps) / reps
+    t_local = timed(lambda j: graphs[j % N_ROT].replay(), steps)
+    # per-T kernel durations (each graph holds one decode launch)
+    per_t = {}
+    reps = max(4 * N_ROT, steps)
+    for T in DECODE_TS:
+        per_t[T] = timed(lambda j, T=T: per_t_graphs[T][j % N_ROT].replay(), reps) / reps
     t_max = max_over_ranks(t_local, world)
 
     # end to end through host buffers: pinned host x -> device, decode, y -> pinned host
@@ -268,6 +270,7 @@ def bench_decode(sl, dev, steps, warmup, world):
             e2e_step(j)
     torch.cuda.synchronize()
     t_e2e = max_over_ranks(timed(e2e_step, steps), world)
+    clk.__exit__(None, None, None)
     h2d = sum(T * K_DOWN * 2 for T in DECODE_TS)
     d2h = sum(T * N_DOWN * 2 for T in DECODE_TS)
     assert sl.as_stream_status(stream) == sl.AS_OK
@@ -313,6 +316,8 @@ def bench_prefill(sl, dev, pk):
     for _ in range(3):
         L.select(x, bufs)
         L.prefill_from(bufs, T, y)
+    for _ in range(3):
+        torch.matmul(x, W.t())  # cuBLAS handle, workspace and heuristics outside the timing
     t_sel = ev_time(lambda: L.select(x, bufs), 10)
     t_gemm = ev_time(lambda: L.prefill_from(bufs, T, y), 10)
     t_dense = ev_time(lambda: torch.matmul(x, W.t()), 10)
@@ -341,6 +346,8 @@ def bench_prefill(sl, dev, pk):
     for _ in range(2):
         L.select(x, bufs, running_var=run)
         L.prefill_from(bufs, T, y)
+    for _ in range(3):
+        torch.matmul(x, W.t())
     t_sel = ev_time(lambda: L.select(x, bufs, running_var=run), 5)
     t_gemm = ev_time(lambda: L.prefill_from(bufs, T, y), 5)
     t_dense = ev_time(lambda: torch.matmul(x, W.t()), 5)
@@ -382,6 +389,42 @@ def oracle_decode_sample(budget_s: float):
     return tokens / el, threads, f"{reps} oracle decode steps (T=1,8,16 of the down-projection), {el:.1f} s"
 
 
+# ---------------------------------------------------------------- profiling cases
+def run_case(args):
+    """A few eager launches of one operation (the small commands the ncu
+    summaries under profiles/ were taken on); prints per-launch times."""
+    import sparse_linear_b200 as sl
+    from sparse_linear_b200.layer import SparseLinear
+    dev = torch.device("cuda", 0)
+    times = []
+    if args.case == "decode":
+        x, W, _ = synth.decode_downproj(16)
+        cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
+        L = SparseLinear(W.to(dev), cfg, alpha=0.5)
+        xd = x[:args.T].contiguous().to(dev)
+        fn = lambda: L.decode(xd)  # noqa: E731
+    elif args.case in ("sqrelu24", "dense"):
+        _, x, W = synth.prefill_sqrelu(T=args.T)
+        cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4) if args.case == "sqrelu24" else \
+            sl.config(sel=sl.AS_SEL_NM, n=1, m=2)
+        L = SparseLinear(W.to(dev), cfg, keep_wt=False)
+        xd = x.to(dev)
+        bufs = L.select_buffers(args.T)
+        L.select(xd, bufs)
+        fn = lambda: L.prefill_from(bufs, args.T)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    for _ in range(args.reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e) * 1e3)
+    assert sl.as_stream_status() == sl.AS_OK
+    print(json.dumps({"case": args.case, "T": args.T, "us_per_launch": times}))
+
+
 # ---------------------------------------------------------------- main
 def run_reference(args, world, rank):
     if rank != 0:
@@ -401,12 +444,18 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--case", default=None, help="profiling case: decode | sqrelu24 | dense")
+    ap.add_argument("--T", type=int, default=1)
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
@@ -435,7 +484,7 @@ def main():
     if rank != 0:
         return
     peak = pk["hbm_gbs"]
-    traffic = recorded_traffic("dram_bytes_per_launch")
+    traffic = recorded_traffic()
     line = {
         "metric": METRIC, "value": d["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": d["t"] / args.steps * 1e3,
