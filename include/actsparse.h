@@ -191,6 +191,38 @@ as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int 
                             const float *nu, const as_config *cfg, void *y,
                             void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* --------------------------------------------------------------------------
+ * as_linear_decode_noalloc: as_linear_decode for callers that cannot
+ * allocate device memory.  (The pages have no counterpart; this is a
+ * deployment variant of the same decode.)
+ *
+ * Some callers cannot call cudaMalloc, for example code running inside a
+ * host framework that owns all device memory through its own pool and
+ * forbids allocations from outside it, or a process held to a device-memory
+ * budget fixed at start-up.  This entry point takes no workspace: its scratch
+ * (split-K partial sums, arrival counters, the top-k bitmask) lives in one
+ * file-scope device array of AS_NOALLOC_SCRATCH_BYTES, which every GPU that
+ * loads the library holds until the process exits.  The caller still passes
+ * inputs and outputs, with the meaning, layouts and errors of
+ * as_linear_decode.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     routine.  Calls whose scratch need (as_workspace_size(AS_OP_DECODE, ...))
+ *     exceeds AS_NOALLOC_SCRATCH_BYTES return AS_ERR_WORKSPACE and launch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents.  The
+ *     part that must start at zero is cleared on `stream` at every call.
+ *     Calls whose executions overlap on the GPU (different streams without
+ *     ordering, or several host threads) race on the array and give
+ *     undefined results: order them on one stream.
+ * ------------------------------------------------------------------------ */
+#define AS_NOALLOC_SCRATCH_BYTES (8u << 20)
+as_status as_linear_decode_noalloc(const void *x, as_dtype dt, int T, int K, int n_out,
+                                   const void *Wt, const float *g, const float *rowsum,
+                                   const as_config *cfg, void *y, uint32_t *mask_out,
+                                   float *eta_out, float *colnorm_out, cudaStream_t stream);
+
 /* Which operation a workspace size is asked for. */
 enum { AS_OP_WEIGHT_PREP = 0, AS_OP_SELECT = 1, AS_OP_DECODE = 2, AS_OP_PREFILL = 3 };
 

@@ -37,8 +37,9 @@ AS_MAX_DECODE_T = 16
 EXPORTS = [
     "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
-    "as_abi_version",
+    "as_abi_version", "as_linear_decode_noalloc",
 ]
+AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class as_config(ctypes.Structure):
@@ -63,6 +64,8 @@ _sig = {
                           _P, _S, _P], _I),
     "as_linear_prefill": ([ctypes.POINTER(as_select_out), _P, _I, _I, _I, _P, _P, _P,
                            ctypes.POINTER(as_config), _P, _P, _S, _P], _I),
+    "as_linear_decode_noalloc": ([_P, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(as_config), _P, _P, _P,
+                                  _P, _P], _I),
     "as_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(as_config)], _S),
     "as_meta24_words": ([_I, _I], _S),
     "as_stream_status": ([_P], _I),
@@ -170,6 +173,18 @@ def as_linear_decode(x, Wt, cfg: as_config, y, g=None, rowsum=None, mask_out=Non
                                  ctypes.byref(cfg), _ptr(y), _ptr(mask_out), _ptr(eta_out),
                                  _ptr(colnorm_out), _ptr(workspace), ws_bytes, _stream(stream)),
            "as_linear_decode")
+
+
+def as_linear_decode_noalloc(x, Wt, cfg: as_config, y, g=None, rowsum=None, mask_out=None, eta_out=None,
+                             colnorm_out=None, stream=None) -> None:
+    """as_linear_decode without a workspace argument: the scratch is the
+    library's own fixed device array (see include/actsparse.h)."""
+    T, K = x.shape
+    n_out = Wt.shape[1]
+    _check(_lib.as_linear_decode_noalloc(_ptr(x), _dt(x), T, K, n_out, _ptr(Wt), _ptr(g), _ptr(rowsum),
+                                         ctypes.byref(cfg), _ptr(y), _ptr(mask_out), _ptr(eta_out),
+                                         _ptr(colnorm_out), _stream(stream)),
+           "as_linear_decode_noalloc")
 
 
 def as_linear_prefill(sel: as_select_out, W, T: int, cfg: as_config, y, rowsum=None, eta=None, nu=None,

@@ -5,3 +5,4 @@
 #include "decode.cu"
 #include "gemm.cu"
 #include "abi.cu"
+#include "noalloc.cu"
