@@ -200,31 +200,41 @@ def bench_decode(sl, dev, steps, warmup, world):
         bytes_call[T] = tot / N_ROT
     torch.cuda.synchronize()
 
-    # one CUDA graph per rotation index, each one full step (T = 1, 8, 16)
+    # CUDA graphs: one holding a full rotation of 8 steps (T = 1, 8, 16 each),
+    # one per rotation index holding a single step (for step counts that are
+    # not a multiple of 8), and one per T holding 8 calls of that T
     stream = torch.cuda.Stream()
-    graphs = []
     with torch.cuda.stream(stream):
         for i in range(N_ROT):
             for T in DECODE_TS:  # warm the launch path outside capture
                 call(i, T, stream=stream)
         stream.synchronize()
+        big = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(big, stream=stream):
+            for i in range(N_ROT):
+                for T in DECODE_TS:
+                    call(i, T, stream=stream)
+        graphs = []
         for i in range(N_ROT):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for T in DECODE_TS:
                     call(i, T, stream=stream)
             graphs.append(g)
-    per_t_graphs = {}
-    with torch.cuda.stream(stream):
+        per_t_graphs = {}
         for T in DECODE_TS:
-            gl = []
-            for i in range(N_ROT):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(N_ROT):
                     call(i, T, stream=stream)
-                gl.append(g)
-            per_t_graphs[T] = gl
+            per_t_graphs[T] = g
     torch.cuda.synchronize()
+
+    def run_steps(n):
+        for _ in range(n // N_ROT):
+            big.replay()
+        for j in range(n % N_ROT):
+            graphs[j].replay()
 
     def timed(run, n):
         barrier(world)
@@ -240,16 +250,15 @@ def bench_decode(sl, dev, steps, warmup, world):
         return s.elapsed_time(e) / 1e3
 
     clk = Clocks(torch.cuda.current_device()).__enter__()
-    for j in range(max(3, warmup)):
-        with torch.cuda.stream(stream):
-            graphs[j % N_ROT].replay()
+    with torch.cuda.stream(stream):
+        run_steps(max(3, warmup))
     torch.cuda.synchronize()
-    t_local = timed(lambda j: graphs[j % N_ROT].replay(), steps)
-    # per-T kernel durations (each graph holds one decode launch)
+    t_local = timed(lambda j: run_steps(steps) if j == 0 else None, 1)
+    # per-T kernel durations: graphs of 8 back-to-back calls of one T
     per_t = {}
-    reps = max(4 * N_ROT, steps)
+    reps = max(8, steps // N_ROT)
     for T in DECODE_TS:
-        per_t[T] = timed(lambda j, T=T: per_t_graphs[T][j % N_ROT].replay(), reps) / reps
+        per_t[T] = timed(lambda j, T=T: per_t_graphs[T].replay(), reps) / (reps * N_ROT)
     t_max = max_over_ranks(t_local, world)
 
     # end to end through host buffers: pinned host x -> device, decode, y -> pinned host
@@ -276,6 +285,7 @@ def bench_decode(sl, dev, steps, warmup, world):
     assert sl.as_stream_status(stream) == sl.AS_OK
 
     tokens = sum(DECODE_TS)
+    launches_per_step = sum(sl.as_decode_launches(T, K_DOWN, N_DOWN, sl.AS_BF16, cfg) for T in DECODE_TS)
     step_bytes = sum(bytes_call.values())
     kern_time = sum(per_t.values())
     return dict(
@@ -286,7 +296,7 @@ def bench_decode(sl, dev, steps, warmup, world):
                for T in DECODE_TS},
         achieved_gbs=step_bytes / kern_time / 1e9, bytes_per_step=step_bytes,
         bytes_per_launch=step_bytes / len(DECODE_TS),
-        clocks=clk.summary(), launches=steps * len(DECODE_TS))
+        clocks=clk.summary(), launches=steps * launches_per_step)
 
 
 # ---------------------------------------------------------------- prefill

@@ -230,6 +230,11 @@ enum { AS_OP_WEIGHT_PREP = 0, AS_OP_SELECT = 1, AS_OP_DECODE = 2, AS_OP_PREFILL 
  * arguments are invalid. */
 size_t as_workspace_size(int op, int T, int K, int n_out, const as_config *cfg);
 
+/* Number of kernels one as_linear_decode call with these arguments launches
+ * (for sizing CUDA graphs and counting launches); -1 if the arguments are
+ * invalid.  Host-only. */
+int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cfg);
+
 /* Number of 32-bit metadata words of a 2:4 selection of T tokens x K channels. */
 size_t as_meta24_words(int T, int K);
 

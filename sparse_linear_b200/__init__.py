@@ -37,7 +37,7 @@ AS_MAX_DECODE_T = 16
 EXPORTS = [
     "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
-    "as_abi_version", "as_linear_decode_noalloc",
+    "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -68,6 +68,7 @@ _sig = {
                                   _P, _P], _I),
     "as_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(as_config)], _S),
     "as_meta24_words": ([_I, _I], _S),
+    "as_decode_launches": ([_I, _I, _I, _I, ctypes.POINTER(as_config)], _I),
     "as_stream_status": ([_P], _I),
     "as_status_string": ([_I], ctypes.c_char_p),
     "as_abi_version": ([], _I),
@@ -142,6 +143,10 @@ def as_workspace_size(op: int, T: int, K: int, n_out: int, cfg: as_config | None
     if r == ctypes.c_size_t(-1).value:
         raise ASError(AS_ERR_INVALID_ARG, "as_workspace_size")
     return r
+
+
+def as_decode_launches(T: int, K: int, n_out: int, dtype: int, cfg: as_config) -> int:
+    return _lib.as_decode_launches(T, K, n_out, dtype, ctypes.byref(cfg))
 
 
 def as_meta24_words(T: int, K: int) -> int:

@@ -44,10 +44,11 @@ as_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AS_OK : AS_ERR_
 size_t decode_ws(int T, int K, int n_out, const as_config *cfg, int bf16)
 {
     DecodePlan p = decode_plan(T, K, n_out, bf16);
-    size_t bytes = round_up(p.counter_bytes, 256) + round_up(p.partial_bytes, 256);
-    if (cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL)
-        bytes += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
-    if (cfg->sel == AS_SEL_TOPK && cfg->score == AS_SCORE_CLACT) bytes += round_up(colnorm_workspace(T, K), 256);
+    size_t bytes = round_up(p.counter_bytes, 256) + round_up(p.partial_bytes, 256) + round_up(p.eta_bytes, 256);
+    // the bf16 path always selects in a separate kernel; float32 only for top-k / keep-all
+    const bool sel_kernel = bf16 || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL;
+    if (sel_kernel) bytes += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
+    if (sel_kernel && cfg->score == AS_SCORE_CLACT) bytes += round_up(colnorm_workspace(T, K), 256);
     return bytes;
 }
 
@@ -203,10 +204,12 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     ws += round_up(plan.counter_bytes, 256);
     float *partial = reinterpret_cast<float *>(ws);
     ws += round_up(plan.partial_bytes, 256);
+    float *eta_ws = reinterpret_cast<float *>(ws);
+    ws += round_up(plan.eta_bytes, 256);
 
     const uint32_t *mask_in = nullptr;
-    if (cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL) {
-        // per-token selection first (exact top-k needs the whole row)
+    if (bf16 || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL) {
+        // per-token selection kernel first (bf16: always; float32: top-k needs the whole row)
         uint32_t *bm = reinterpret_cast<uint32_t *>(ws);
         ws += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
         const float *f = cfg->score == AS_SCORE_WEIGHT ? g : nullptr;
@@ -223,13 +226,18 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
         s.K = K;
         s.score = cfg->score;
         s.sel = cfg->sel;
+        s.n = cfg->n;
+        s.m = cfg->m;
         s.k_keep = cfg->k_keep;
         s.dpts = cfg->dpts;
         s.f = f;
         s.bitmask = bm;
+        s.eta = cfg->dpts ? eta_ws : nullptr;  // the decode kernel reuses the means the selection used
         if (cfg->sel == AS_SEL_TOPK && (size_t)K * 4 > 200 * 1024 && cfg->k_keep > 0 && cfg->k_keep < K)
             return AS_ERR_SHAPE;
-        if (launch_select(s, stream) != cudaSuccess) return AS_ERR_CUDA;
+        const cudaError_t se = (cfg->sel == AS_SEL_NM) ? launch_select_nm_decode(s, stream)
+                                                       : launch_select(s, stream, /*wide=*/1);
+        if (se != cudaSuccess) return AS_ERR_CUDA;
         mask_in = bm;
     }
     DecodeArgs a{};
@@ -254,6 +262,7 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     a.colnorm_out = mask_in ? nullptr : colnorm_out;
     a.partial = partial;
     a.counters = counters;
+    a.eta_in = eta_ws;
     return cuda_status(launch_decode(a, plan, stream));
 }
 
@@ -289,6 +298,23 @@ as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int 
     a.y = y;
     a.out_bf16 = cfg->out_dtype == AS_BF16;
     return cuda_status(launch_gemm(a, stream));
+}
+
+int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cfg)
+{
+    if (as_workspace_size(AS_OP_DECODE, T, K, n_out, cfg) == (size_t)-1) return -1;
+    const int bf16 = dt == AS_BF16;
+    DecodePlan plan = decode_plan(T, K, n_out, bf16);
+    DecodeArgs a{};
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.dpts = cfg->dpts;
+    a.bf16 = bf16;
+    int n = 0;
+    if (bf16 || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL)
+        n += 1 + (cfg->score == AS_SCORE_CLACT ? 2 : 0);  // select kernel (+ column energy)
+    return n + decode_launch_count(a, plan);
 }
 
 as_status as_stream_status(cudaStream_t stream)

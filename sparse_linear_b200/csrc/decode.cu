@@ -347,6 +347,325 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
     if (tid == 0) a.counters[slice] = 0u;  // leave the workspace zeroed for the next call
 }
 
+// ============================================================================
+// bf16 path: tensor-core decode kernel, D-PTS mean kernel, split-K reduction
+// ============================================================================
+//
+// bf16 decode = three kernels chained by programmatic dependent launch:
+//   k_select (one CTA of 1024 threads per token, select.cu): D-PTS mean,
+//     score, exact N:M or top-k selection -> keep words [T, K/32] and eta;
+//   k_decode_tc: CTA (slice, split) owns NS = 512 output columns and a range
+//     of up to 1024 channels.  It loads its activation chunk while the
+//     selection finishes, then reads the keep words and eta, compacts the
+//     union over tokens of the kept channels (ascending) with the kept values
+//     split into bf16 hi + lo (xhat = hi + lo to about 2^-16 relative), and
+//     streams those rows of Wt: each of the 8 warps owns 64 output columns
+//     and runs its own cp.async ring over the 128-byte pieces of the kept rows
+//     it multiplies (no block-wide barrier in the loop).  Each staged
+//     16-channel slab goes through ldmatrix.trans into A fragments and the
+//     tensor cores (mma.sync m16n8k16, bf16 in, float32 accumulate; once for
+//     hi, once for lo).  It writes y directly (one split) or its split-K
+//     partial sums;
+//   k_decode_reduce: adds the partials in split order, with eta*rowsum.
+
+constexpr int TC_WARPS = 8;
+constexpr int TC_THREADS = TC_WARPS * 32;
+constexpr int TC_NS = 512;                     // output columns per CTA
+constexpr int TC_WCOLS = TC_NS / TC_WARPS;     // 64 columns (128 bytes) per warp
+constexpr int TC_WROWP = TC_WCOLS * 2 + 16;    // 144-byte padded row piece (ldmatrix: no bank conflicts)
+constexpr int TC_KS = 16;                      // rows per stage = one mma k-step
+constexpr int TC_MAXW = 32;                    // 32-channel words per CTA
+constexpr int TC_MAXL = TC_MAXW * 32;          // 1024 channels
+constexpr int TC_XP = TC_MAXL + 24;            // token-value row stride (bf16): no bank conflicts
+
+template <int TP>
+struct TcCfg {
+    static constexpr int NS = TC_NS;
+    static constexpr int MT = TC_WCOLS / 16;            // 16-output m-tiles per warp
+    static constexpr int STAGES = TP <= 4 ? 4 : 6;
+    static constexpr int NT = (TP + 7) / 8;             // 8-token n-tiles
+    static constexpr size_t wstage = (size_t)TC_KS * TC_WROWP;
+    static constexpr size_t ring = (size_t)TC_WARPS * STAGES * wstage;
+    static constexpr size_t xchunk = (size_t)TP * TC_MAXL * 2;   // bf16 activation chunk; aliases the ring
+    static constexpr size_t red = (size_t)TP * NS * 4;           // aliases the ring
+    static constexpr size_t big = ring > xchunk ? (ring > red ? ring : red) : (xchunk > red ? xchunk : red);
+    static constexpr size_t lists = (size_t)TC_MAXL * 4 + (size_t)2 * TP * TC_XP * 2;
+    static constexpr size_t smem = big + lists;
+    static constexpr int TARGET = TP <= 4 ? 296 : 148;
+    static constexpr int MINB = TP <= 4 ? 2 : 1;
+};
+
+// y = sum of the split-K partials in split order (+ eta*rowsum), 4 columns a thread.
+__global__ void __launch_bounds__(256) k_decode_reduce(const float *__restrict__ partial, int k_splits, int T,
+                                                       int n_out, const float *__restrict__ eta,
+                                                       const float *__restrict__ rowsum, void *__restrict__ y,
+                                                       int out_bf16)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const int n4 = T * n_out / 4;
+    if (i >= n4) return;
+    const float4 *p = reinterpret_cast<const float4 *>(partial);
+    float4 s = __ldcg(p + i);
+    for (int k = 1; k < k_splits; ++k) {
+        const float4 v = __ldcg(p + (size_t)k * n4 + i);
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    const int t = (4 * i) / n_out, o = (4 * i) % n_out;
+    if (eta) {
+        const float e = eta[t];
+        s.x = fmaf(e, rowsum[o], s.x);
+        s.y = fmaf(e, rowsum[o + 1], s.y);
+        s.z = fmaf(e, rowsum[o + 2], s.z);
+        s.w = fmaf(e, rowsum[o + 3], s.w);
+    }
+    if (out_bf16) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(s.x, s.y), b = __floats2bfloat162_rn(s.z, s.w);
+        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(y) + (size_t)t * n_out + o) =
+            make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+    } else {
+        *reinterpret_cast<float4 *>(static_cast<float *>(y) + (size_t)t * n_out + o) = s;
+    }
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int TP>
+__global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
+    k_decode_tc(DecodeArgs a, int words_per_split)
+{
+    using C = TcCfg<TP>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char *ring = smem;
+    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(smem);  // [TP][TC_MAXL] activation chunk
+    float *red = reinterpret_cast<float *>(smem);                  // [TP][NS] after the main loop
+    unsigned char *lists = smem + C::big;
+    int *list_ch = reinterpret_cast<int *>(lists);
+    __nv_bfloat16 *xh_hi = reinterpret_cast<__nv_bfloat16 *>(lists + TC_MAXL * 4);  // [TP][TC_XP]
+    __nv_bfloat16 *xh_lo = xh_hi + TP * TC_XP;
+
+    __shared__ float s_eta[TP];
+    __shared__ uint32_t s_keep[TP][TC_MAXW];
+    __shared__ int s_wbase[TC_MAXW + 1];
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int slice = blockIdx.x, split = blockIdx.y;
+    const int T = a.T, K = a.K, n_out = a.n_out;
+    const int nwords = (K + 31) >> 5;
+    const int w0 = split * words_per_split, w1 = min(nwords, w0 + words_per_split);
+    const int nw = max(0, w1 - w0);
+    const int c_begin = 32 * w0, c_end = min(32 * w1, K);
+    const int nch = max(0, c_end - c_begin);  // multiple of 8
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
+
+    // ---- 1. activation chunk (issued before waiting for the selection
+    // kernel), then the keep words and D-PTS means it wrote
+    const int ngc = nch >> 3;
+    uint4 chv[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int i = tid + r * TC_THREADS;
+        if (i < TP * ngc) {
+            const int t = i / ngc, g = i % ngc;
+            chv[r] = t < T ? *reinterpret_cast<const uint4 *>(x + (size_t)t * K + c_begin + 8 * g)
+                           : make_uint4(0, 0, 0, 0);
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // selection kernel complete
+    if (tid < TP) s_eta[tid] = (a.dpts && tid < T) ? a.eta_in[tid] : 0.0f;
+    if (a.eta_out && a.dpts && slice == 0 && split == 0 && tid < T) a.eta_out[tid] = a.eta_in[tid];
+    for (int i = tid; i < T * nw; i += TC_THREADS) {
+        const int t = i / nw, wl = i % nw;
+        const uint32_t word = a.mask_in[(size_t)t * nwords + w0 + wl];
+        s_keep[t][wl] = word;
+        if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int i = tid + r * TC_THREADS;
+        if (i < TP * ngc) *reinterpret_cast<uint4 *>(xs + (i / ngc) * TC_MAXL + 8 * (i % ngc)) = chv[r];
+    }
+    __syncthreads();
+
+    // ---- 3. union list, values split into bf16 hi + lo, [token][position]
+    if (warp == 0) {
+        int cnt = 0;
+        if (lane < nw) {
+            uint32_t u = 0;
+            for (int t = 0; t < T; ++t) u |= s_keep[t][lane];
+            cnt = __popc(u);
+        }
+        int inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        s_wbase[lane] = inc - cnt;
+        if (lane == 31) s_wbase[TC_MAXW] = inc;
+    }
+    __syncthreads();
+    const int L = s_wbase[TC_MAXW];
+    const int Lp = (L + TC_KS - 1) / TC_KS * TC_KS;
+    for (int wl = warp; wl < nw; wl += TC_WARPS) {
+        uint32_t u = 0;
+        for (int t = 0; t < T; ++t) u |= s_keep[t][wl];
+        if ((u >> lane) & 1u) {
+            const int pos = s_wbase[wl] + __popc(u & ((1u << lane) - 1u));
+            const int cl = 32 * wl + lane;
+            list_ch[pos] = c_begin + cl;
+#pragma unroll
+            for (int t = 0; t < TP; ++t) {
+                float v = 0.0f;
+                if (t < T && ((s_keep[t][wl] >> lane) & 1u)) {
+                    const float xv = __bfloat162float(xs[t * TC_MAXL + cl]);
+                    v = a.dpts ? __fsub_rn(xv, s_eta[t]) : xv;
+                }
+                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+                xh_hi[t * TC_XP + pos] = hi;
+                xh_lo[t * TC_XP + pos] = __float2bfloat16_rn(v - __bfloat162float(hi));
+            }
+        }
+    }
+    for (int i = L + tid; i < Lp; i += TC_THREADS) {  // padding positions of the last k-step
+        list_ch[i] = -1;
+#pragma unroll
+        for (int t = 0; t < TP; ++t) {
+            xh_hi[t * TC_XP + i] = __float2bfloat16_rn(0.0f);
+            xh_lo[t * TC_XP + i] = __float2bfloat16_rn(0.0f);
+        }
+    }
+    __syncthreads();  // the activation chunk is dead: the rings reuse its space
+
+    // ---- 4. per-warp cp.async ring over this warp's 64 columns + tensor cores
+    const int nst = Lp / TC_KS;
+    const int col0 = slice * C::NS + warp * TC_WCOLS;
+    const __nv_bfloat16 *wt = static_cast<const __nv_bfloat16 *>(a.Wt);
+    const uint32_t wring = smem_u32(ring) + (uint32_t)(warp * C::STAGES * C::wstage);
+    auto issue = [&](int st) {
+        const uint32_t base = wring + (uint32_t)((st % C::STAGES) * C::wstage);
+#pragma unroll
+        for (int r = 0; r < (TC_KS * TC_WCOLS * 2 / 16) / 32; ++r) {
+            const int id = lane + 32 * r;
+            const int row = id >> 3, c16 = id & 7;
+            const int ch = list_ch[st * TC_KS + row];
+            const int col = col0 + 8 * c16;
+            const bool ok = ch >= 0 && col < n_out;
+            const void *src = ok ? (const void *)(wt + (size_t)ch * n_out + col) : (const void *)wt;
+            cp_async16(base + row * TC_WROWP + c16 * 16, src, ok ? 16u : 0u);  // 0 bytes: zero fill
+        }
+    };
+    float acc[C::MT][C::NT][4];
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
+#pragma unroll
+    for (int st = 0; st < C::STAGES - 1; ++st) {
+        if (st < nst) issue(st);
+        cp_async_commit();
+    }
+    const int g8 = lane >> 2, q4 = lane & 3;
+    const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index, row within it
+    for (int st = 0; st < nst; ++st) {
+        cp_async_wait<C::STAGES - 2>();
+        __syncwarp();  // every lane's pieces of stage st have landed
+        if (st + C::STAGES - 1 < nst) issue(st + C::STAGES - 1);  // into the slot read at st-1
+        cp_async_commit();
+        const uint32_t base = wring + (uint32_t)((st % C::STAGES) * C::wstage);
+        const int pk = st * TC_KS;
+        uint32_t bh[C::NT][2], bl[C::NT][2];
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+            const int t = nt * 8 + g8;
+            if (t < TP) {
+                bh[nt][0] = *reinterpret_cast<const uint32_t *>(xh_hi + t * TC_XP + pk + 2 * q4);
+                bh[nt][1] = *reinterpret_cast<const uint32_t *>(xh_hi + t * TC_XP + pk + 2 * q4 + 8);
+                bl[nt][0] = *reinterpret_cast<const uint32_t *>(xh_lo + t * TC_XP + pk + 2 * q4);
+                bl[nt][1] = *reinterpret_cast<const uint32_t *>(xh_lo + t * TC_XP + pk + 2 * q4 + 8);
+            } else {
+                bh[nt][0] = bh[nt][1] = bl[nt][0] = bl[nt][1] = 0u;
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+            const uint32_t addr = base + (uint32_t)(((mi >> 1) * 8 + mr) * TC_WROWP + (mt * 16 + (mi & 1) * 8) * 2);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_trans(addr, a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < C::NT; ++nt) {
+                mma_16816(acc[mt][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+                mma_16816(acc[mt][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();  // every warp done with its ring: the space becomes the reduction buffer
+
+    // ---- 5. fragments -> shared [token][column] -> y or split-K partials
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+            const int o = warp * TC_WCOLS + mt * 16 + g8;
+            const int t = nt * 8 + 2 * q4;
+            if (t < TP) {
+                red[t * C::NS + o] = acc[mt][nt][0];
+                red[t * C::NS + o + 8] = acc[mt][nt][2];
+            }
+            if (t + 1 < TP) {
+                red[(t + 1) * C::NS + o] = acc[mt][nt][1];
+                red[(t + 1) * C::NS + o + 8] = acc[mt][nt][3];
+            }
+        }
+    __syncthreads();
+    const int k_splits = gridDim.y;
+    const int ocol0 = slice * C::NS;
+    for (int i = tid; i < T * C::NS; i += TC_THREADS) {
+        const int t = i / C::NS, c = i % C::NS, o = ocol0 + c;
+        if (o >= n_out) continue;
+        float v = red[t * C::NS + c];
+        if (k_splits > 1) {
+            a.partial[((size_t)split * T + t) * n_out + o] = v;
+        } else {
+            if (a.dpts) v = fmaf(s_eta[t], a.rowsum[o], v);
+            if (a.out_bf16)
+                static_cast<__nv_bfloat16 *>(a.y)[(size_t)t * n_out + o] = __float2bfloat16_rn(v);
+            else
+                static_cast<float *>(a.y)[(size_t)t * n_out + o] = v;
+        }
+    }
+}
+
+// ============================================================================
+// planning and launch
+// ============================================================================
 static int tpad_of(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16; }
 
 static int vec_of(int tp, int bf16)
@@ -355,32 +674,48 @@ static int vec_of(int tp, int bf16)
     return tp <= 8 ? 4 : 2;
 }
 
-template <typename TW, int TP, int VEC>
-static size_t smem_of()
+static size_t tc_smem(int tp)
 {
-    return DecCfg<TP, VEC, TW>::smem;
+    switch (tp) {
+    case 1: return TcCfg<1>::smem;
+    case 2: return TcCfg<2>::smem;
+    case 4: return TcCfg<4>::smem;
+    case 8: return TcCfg<8>::smem;
+    default: return TcCfg<16>::smem;
+    }
 }
+
+static int tc_ns(int) { return TC_NS; }
 
 DecodePlan decode_plan(int T, int K, int n_out, int bf16)
 {
     DecodePlan p{};
     p.tpad = tpad_of(T);
+    p.tc = bf16 ? 1 : 0;
     const int nwords = (K + 31) / 32;
-    p.n_slices = (n_out + DEC_NS - 1) / DEC_NS;
-    int want = DEC_TARGET_CTAS / p.n_slices;
+    const int ns = p.tc ? tc_ns(p.tpad) : DEC_NS;
+    const int maxw = p.tc ? TC_MAXW : DEC_MAX_WORDS;
+    const int target = p.tc ? (p.tpad <= 4 ? 296 : 148) : DEC_TARGET_CTAS;
+    p.n_slices = (n_out + ns - 1) / ns;
+    int want = target / p.n_slices;
     if (want < 1) want = 1;
     int wps = (nwords + want - 1) / want;
-    if (wps > DEC_MAX_WORDS) wps = DEC_MAX_WORDS;
+    if (wps > maxw) wps = maxw;
     if (wps < 1) wps = 1;
     p.words_per_split = wps;
     p.k_splits = (nwords + wps - 1) / wps;
     p.partial_bytes = p.k_splits > 1 ? (size_t)p.k_splits * T * n_out * sizeof(float) : 0;
     p.counter_bytes = (size_t)p.n_slices * sizeof(unsigned);
-    const int vec = vec_of(p.tpad, bf16);
-    const int tpr = DEC_NS / vec, rg = DEC_THREADS / tpr;
-    size_t list = (size_t)DEC_MAX_WORDS * 32 * (sizeof(int) + p.tpad * sizeof(float));
-    size_t red = (size_t)rg * p.tpad * DEC_NS * sizeof(float);
-    p.smem_bytes = list > red ? list : red;
+    p.eta_bytes = (size_t)T * sizeof(float);
+    if (p.tc) {
+        p.smem_bytes = tc_smem(p.tpad);
+    } else {
+        const int vec = vec_of(p.tpad, bf16);
+        const int tpr = DEC_NS / vec, rg = DEC_THREADS / tpr;
+        size_t list = (size_t)DEC_MAX_WORDS * 32 * (sizeof(int) + p.tpad * sizeof(float));
+        size_t red = (size_t)rg * p.tpad * DEC_NS * sizeof(float);
+        p.smem_bytes = list > red ? list : red;
+    }
     return p;
 }
 
@@ -398,15 +733,61 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &p, cudaStream
     return cudaGetLastError();
 }
 
+int decode_launch_count(const DecodeArgs &, const DecodePlan &p)
+{
+    if (!p.tc) return 1;
+    return 1 + (p.k_splits > 1 ? 1 : 0);  // decode (+ split-K reduction); the select kernel is counted by the caller
+}
+
+// Programmatic dependent launch: the kernel may start before the previous
+// kernel in the stream finishes and must wait (griddepcontrol.wait) before
+// reading what that kernel writes.
+static void set_pdl(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr)
+{
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
+// The tensor-core decode follows the select kernel (which wrote the keep
+// words and means) and, for several splits, is followed by the reduction;
+// both links are programmatic.
+template <int TP>
+static cudaError_t launch_tc(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
+{
+    const size_t smem = TcCfg<TP>::smem;
+    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<TP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_slices, p.k_splits);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    set_pdl(cfg, attr);
+    e = cudaLaunchKernelEx(&cfg, k_decode_tc<TP>, a, p.words_per_split);
+    if (e != cudaSuccess || p.k_splits == 1) return e;
+    cudaLaunchConfig_t rc = {};
+    const int n4 = a.T * a.n_out / 4;
+    rc.gridDim = dim3((n4 + 255) / 256);
+    rc.blockDim = dim3(256);
+    rc.stream = st;
+    cudaLaunchAttribute rattr[1];
+    set_pdl(rc, rattr);
+    return cudaLaunchKernelEx(&rc, k_decode_reduce, (const float *)a.partial, p.k_splits, a.T, a.n_out,
+                              a.dpts ? (const float *)a.eta_in : (const float *)nullptr, a.rowsum, a.y, a.out_bf16);
+}
+
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
 {
     if (a.bf16) {
         switch (p.tpad) {
-        case 1: return launch_t<__nv_bfloat16, 1, 8>(a, p, st);
-        case 2: return launch_t<__nv_bfloat16, 2, 8>(a, p, st);
-        case 4: return launch_t<__nv_bfloat16, 4, 8>(a, p, st);
-        case 8: return launch_t<__nv_bfloat16, 8, 4>(a, p, st);
-        default: return launch_t<__nv_bfloat16, 16, 2>(a, p, st);
+        case 1: return launch_tc<1>(a, p, st);
+        case 2: return launch_tc<2>(a, p, st);
+        case 4: return launch_tc<4>(a, p, st);
+        case 8: return launch_tc<8>(a, p, st);
+        default: return launch_tc<16>(a, p, st);
         }
     }
     switch (p.tpad) {

@@ -30,7 +30,9 @@ struct SelectArgs {
 // CLACT column energy c_j = sqrt(sum_t x_tj^2), float64 partials in ws.
 size_t colnorm_workspace(int T, int K);
 cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void *ws, cudaStream_t st);
-cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st, int wide = 0);
+// N:M selection of a decode call: keep words and eta only (grid token x chunk).
+cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st);
 
 // ------------------------------------------------------------ decode
 struct DecodeArgs {
@@ -49,12 +51,14 @@ struct DecodeArgs {
     float *colnorm_out;
     float *partial;     // split-K partial sums
     unsigned *counters; // one per N-slice, zero between calls
+    float *eta_in;      // D-PTS means written by the select kernel (bf16 path)
 };
 struct DecodePlan {
-    int n_slices, k_splits, words_per_split, tpad;
-    size_t partial_bytes, counter_bytes, smem_bytes;
+    int n_slices, k_splits, words_per_split, tpad, tc;
+    size_t partial_bytes, counter_bytes, eta_bytes, smem_bytes;
 };
 DecodePlan decode_plan(int T, int K, int n_out, int bf16);
+int decode_launch_count(const DecodeArgs &a, const DecodePlan &p);
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st);
 
 // ------------------------------------------------------------ prefill GEMM

@@ -20,10 +20,9 @@
 
 namespace as {
 
-constexpr int SEL_THREADS = 256;
-
 // Block-wide sum of two float64 values (deterministic order).
-__device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[SEL_THREADS / 32])
+template <int NT>
+__device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[NT / 32])
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     a = warp_sum_f64(a);
@@ -32,7 +31,7 @@ __device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[S
     __syncthreads();
     double sa = 0.0, sb = 0.0;
 #pragma unroll
-    for (int w = 0; w < SEL_THREADS / 32; ++w) { sa += red[0][w]; sb += red[1][w]; }
+    for (int w = 0; w < NT / 32; ++w) { sa += red[0][w]; sb += red[1][w]; }
     a = sa;
     b = sb;
     __syncthreads();
@@ -40,6 +39,7 @@ __device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[S
 
 // Exclusive prefix sum over the block in thread order; returns the prefix,
 // `total` receives the block total.
+template <int NT>
 __device__ __forceinline__ int block_excl_scan(int v, int &total, int *wsum)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -53,7 +53,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int &total, int *wsum)
     __syncthreads();
     int base = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < SEL_THREADS / 32; ++w) {
+    for (int w = 0; w < NT / 32; ++w) {
         if (w < warp) base += wsum[w];
         tot += wsum[w];
     }
@@ -94,22 +94,26 @@ __device__ __forceinline__ void store8<float>(float *p, const float (&v)[8])
     *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <typename TX>
-__global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
+// NT threads per token row: 256 for prefill batches, 1024 for the few rows
+// of a decode call (fewer rounds of loads per row).
+template <typename TX, int NT>
+__global__ void __launch_bounds__(NT) k_select(SelectArgs a)
 {
+    // a decode kernel chained after this one may start its own loads now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(16) uint32_t keys[];  // [K] score bits (top-k only)
-    __shared__ double red[2][SEL_THREADS / 32];
-    __shared__ int wsum[SEL_THREADS / 32];
+    __shared__ double red[2][NT / 32];
+    __shared__ int wsum[NT / 32];
     __shared__ uint32_t hist[256];
     __shared__ uint32_t s_digit, s_remaining;
 
     const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-    const int K = a.K, ngroups = K >> 3, ntiles = (ngroups + SEL_THREADS - 1) / SEL_THREADS;
+    const int K = a.K, ngroups = K >> 3, ntiles = (ngroups + NT - 1) / NT;
     const int kt = (K + 127) >> 7;
 
     if (t >= a.T) {  // padding rows of the 2:4 metadata tiles
         if (a.meta24)
-            for (int g = tid; g < kt * 16; g += SEL_THREADS) *meta_byte(a.meta24, t, 8 * g, kt) = 0x44;
+            for (int g = tid; g < kt * 16; g += NT) *meta_byte(a.meta24, t, 8 * g, kt) = 0x44;
         return;
     }
     const TX *xr = static_cast<const TX *>(a.x) + (size_t)t * K;
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
     // ---- row statistics: sum x, sum x^2 (float64)
     double sx = 0.0, sxx = 0.0;
     if (a.dpts || a.var) {
-        for (int g = tid; g < ngroups; g += SEL_THREADS) {
+        for (int g = tid; g < ngroups; g += NT) {
             float v[8];
             load8(xr + 8 * g, v);
 #pragma unroll
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
                 sxx += (double)v[e] * (double)v[e];
             }
         }
-        block_sum2(sx, sxx, red);
+        block_sum2<NT>(sx, sxx, red);
     }
     const float eta = a.dpts ? (float)(sx / (double)K) : 0.0f;
     if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
@@ -138,7 +142,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
     const bool topk = a.sel == AS_SEL_TOPK;
     const int kk = a.k_keep;
     if (topk && kk > 0 && kk < K) {
-        for (int g = tid; g < ngroups; g += SEL_THREADS) {
+        for (int g = tid; g < ngroups; g += NT) {
             float v[8], xh[8], s[8];
             load8(xr + 8 * g, v);
             score8(v, a.dpts, eta, a.f, 8 * g, xh, s);
@@ -147,9 +151,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
         }
         uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)kk;
         for (int shift = 24; shift >= 0; shift -= 8) {
-            hist[tid] = 0;
+            if (tid < 256) hist[tid] = 0;
             __syncthreads();
-            for (int i = tid; i < K; i += SEL_THREADS) {
+            for (int i = tid; i < K; i += NT) {
                 uint32_t key = keys[i];
                 if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
             }
@@ -195,7 +199,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
     double skm = 0.0, skmm = 0.0;
     int eq_base = 0;
     for (int tile = 0; tile < ntiles; ++tile) {
-        const int g = tile * SEL_THREADS + tid, c0 = 8 * g;
+        const int g = tile * NT + tid, c0 = 8 * g;
         const bool act = g < ngroups;
         float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, xh[8], s[8];
         if (act) load8(xr + c0, v);
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
                     eq |= (uint32_t)(act && key == tau) << e;
                 }
                 int total;
-                int before = eq_base + block_excl_scan(__popc(eq), total, wsum);
+                int before = eq_base + block_excl_scan<NT>(__popc(eq), total, wsum);
                 eq_base += total;
                 keep = gt;
 #pragma unroll
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(SelectArgs a)
 
     // ---- VAR: variances, running average, scale
     if (a.var) {
-        block_sum2(skm, skmm, red);
+        block_sum2<NT>(skm, skmm, red);
         if (tid == 0) {
             const double Kd = (double)K;
             double vd = (sxx - sx * sx / Kd) / (Kd - 1.0);
@@ -330,20 +334,105 @@ cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void
     return cudaGetLastError();
 }
 
-cudaError_t launch_select(const SelectArgs &a, cudaStream_t st)
+template <typename TX, int NT>
+static cudaError_t launch_select_t(const SelectArgs &a, size_t smem, int grid, cudaStream_t st)
+{
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_select<TX, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_select<TX, NT><<<grid, NT, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st, int wide)
 {
     const bool topk = a.sel == AS_SEL_TOPK && a.k_keep > 0 && a.k_keep < a.K;
     const size_t smem = topk ? (size_t)a.K * sizeof(uint32_t) : 0;
     const int grid = a.meta24 ? ((a.T + 127) / 128) * 128 : a.T;
-    if (a.bf16) {
-        if (smem > 48 * 1024)
-            cudaFuncSetAttribute(k_select<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_select<__nv_bfloat16><<<grid, SEL_THREADS, smem, st>>>(a);
-    } else {
-        if (smem > 48 * 1024)
-            cudaFuncSetAttribute(k_select<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_select<float><<<grid, SEL_THREADS, smem, st>>>(a);
+    if (a.bf16)
+        return wide ? launch_select_t<__nv_bfloat16, 1024>(a, smem, grid, st)
+                    : launch_select_t<__nv_bfloat16, 256>(a, smem, grid, st);
+    return wide ? launch_select_t<float, 1024>(a, smem, grid, st) : launch_select_t<float, 256>(a, smem, grid, st);
+}
+
+// ---------------------------------------------------------------- decode N:M
+// Selection for a decode call (few tokens): grid (token, 2048-channel chunk),
+// 256 threads.  Every CTA of a token computes the token mean from the whole
+// row with the same code and order (identical float32 bits in all of them);
+// all loads of a thread are issued before any is used.  Output: the keep
+// words of its chunk and, from chunk 0, eta.
+constexpr int SELD_THREADS = 256;
+constexpr int SELD_CHUNK = 2048;             // channels per CTA: one 256-channel tile per warp
+constexpr int SELD_ROWREG = 8;               // row loads held in registers per thread (K <= 16384)
+
+__global__ void __launch_bounds__(SELD_THREADS) k_select_nm_decode(SelectArgs a)
+{
+    using TX = __nv_bfloat16;  // 16-byte row loads hold 8 channels
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ double red[SELD_THREADS / 32];
+    const int t = blockIdx.x, chunk = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = a.K, ng = K >> 3, words = (K + 31) >> 5;
+    const TX *xr = static_cast<const TX *>(a.x) + (size_t)t * K;
+    const int c0 = chunk * SELD_CHUNK + warp * 256 + 8 * lane;  // this lane's 8 channels
+    const bool act = c0 < K;
+
+    // issue: own channels, their factors, and (D-PTS) the whole row
+    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, f[8];
+    if (act) load8(xr + c0, v);
+    const bool has_f = a.f != nullptr && act;
+    if (has_f) load8f(a.f + c0, f);
+    float eta = 0.0f;
+    if (a.dpts) {
+        uint4 raw[SELD_ROWREG];
+#pragma unroll
+        for (int r = 0; r < SELD_ROWREG; ++r) {
+            const int g = tid + r * SELD_THREADS;
+            if (g < ng) raw[r] = *reinterpret_cast<const uint4 *>(xr + 8 * g);
+        }
+        double sum = 0.0;
+#pragma unroll
+        for (int r = 0; r < SELD_ROWREG; ++r) {
+            const int g = tid + r * SELD_THREADS;
+            if (g < ng) {
+                float w[8];
+                load8(&raw[r], w);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sum += (double)w[e];
+            }
+        }
+        for (int g = tid + SELD_ROWREG * SELD_THREADS; g < ng; g += SELD_THREADS) {  // K > 16384
+            float w[8];
+            load8(xr + 8 * g, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sum += (double)w[e];
+        }
+        sum = warp_sum_f64(sum);
+        if (lane == 0) red[warp] = sum;
+        __syncthreads();
+        double tot = 0.0;
+#pragma unroll
+        for (int w = 0; w < SELD_THREADS / 32; ++w) tot += red[w];
+        eta = (float)(tot / (double)K);
+        if (chunk == 0 && tid == 0 && a.eta) a.eta[t] = eta;
     }
+    float xh[8], sc[8];
+    score8(v, a.dpts, eta, has_f ? f : nullptr, 0, xh, sc);
+    uint32_t keep = nm_keep_dispatch(sc, lane, a.n, a.m);
+    if (!act) keep = 0;
+    uint32_t word = keep << (8 * (lane & 3));
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    const int wi = c0 >> 5;
+    if ((lane & 3) == 0 && act) a.bitmask[(size_t)t * words + wi] = word;
+}
+
+cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st)
+{
+    dim3 grid(a.T, (a.K + SELD_CHUNK - 1) / SELD_CHUNK);
+    if (!a.bf16) return cudaErrorInvalidValue;  // the float32 decode selects inside its kernel
+    k_select_nm_decode<<<grid, SELD_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 

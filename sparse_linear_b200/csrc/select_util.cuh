@@ -33,6 +33,17 @@ __device__ __forceinline__ void load8(const float *p, float (&v)[8])
 
 __device__ __forceinline__ void load8f(const float *p, float (&v)[8]) { load8(p, v); }
 
+// Eight bf16 values held in a 16-byte register vector, converted to float32.
+__device__ __forceinline__ void load8(const uint4 *r, float (&v)[8])
+{
+    const uint32_t w[4] = {r->x, r->y, r->z, r->w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
 // Score of eight channels: s = fl32(|xhat| * f), xhat = fl32(x - eta) when
 // shift != 0.  Explicit round-to-nearest intrinsics keep the compiler from
 // contracting or reassociating (the selection decision depends on the bits).
@@ -97,6 +108,32 @@ __device__ __forceinline__ uint32_t nm_keep_dispatch(const float (&s)[8], int la
     case 8: return nm_keep<8>(s, lane, n);
     case 16: return nm_keep<16>(s, lane, n);
     default: return nm_keep<32>(s, lane, n);
+    }
+}
+
+// Lane `lane` of a warp holds channel `lane` of a 32-channel word whose
+// scores are in sc[0..31] (shared memory); keep it if it ranks among the n
+// best of its M-block (blocks [jm, jm+m) inside the word).
+template <int M>
+__device__ __forceinline__ bool nm_rank_keep_m(const float *sc, int lane, int n)
+{
+    const int b0 = lane & ~(M - 1), i = lane & (M - 1);
+    const float si = sc[lane];
+    int rank = 0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) rank += (j != i) & ahead(sc[b0 + j], j, si, i);
+    return rank < n;
+}
+
+__device__ __forceinline__ bool nm_rank_keep(const float *sc, int lane, int n, int m)
+{
+    switch (m) {
+    case 1: return true;
+    case 2: return nm_rank_keep_m<2>(sc, lane, n);
+    case 4: return nm_rank_keep_m<4>(sc, lane, n);
+    case 8: return nm_rank_keep_m<8>(sc, lane, n);
+    case 16: return nm_rank_keep_m<16>(sc, lane, n);
+    default: return nm_rank_keep_m<32>(sc, lane, n);
     }
 }
 
