@@ -45,8 +45,9 @@ size_t decode_ws(int T, int K, int n_out, const as_config *cfg, int bf16)
 {
     DecodePlan p = decode_plan(T, K, n_out, bf16);
     size_t bytes = round_up(p.counter_bytes, 256) + round_up(p.partial_bytes, 256) + round_up(p.eta_bytes, 256);
-    // the bf16 path always selects in a separate kernel; float32 only for top-k / keep-all
-    const bool sel_kernel = bf16 || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL;
+    // a separate selection kernel: bf16 unless fused (<= 2 tokens, N:M); float32 for top-k / keep-all
+    const bool sel_kernel = (bf16 && !decode_fused(p.tpad, cfg->sel, K)) || cfg->sel == AS_SEL_TOPK ||
+                            cfg->sel == AS_SEL_ALL;
     if (sel_kernel) bytes += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
     if (sel_kernel && cfg->score == AS_SCORE_CLACT) bytes += round_up(colnorm_workspace(T, K), 256);
     return bytes;
@@ -208,7 +209,7 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     ws += round_up(plan.eta_bytes, 256);
 
     const uint32_t *mask_in = nullptr;
-    if (bf16 || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL) {
+    if ((bf16 && !decode_fused(plan.tpad, cfg->sel, K)) || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL) {
         // per-token selection kernel first (bf16: always; float32: top-k needs the whole row)
         uint32_t *bm = reinterpret_cast<uint32_t *>(ws);
         ws += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
@@ -311,8 +312,9 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
     a.n_out = n_out;
     a.dpts = cfg->dpts;
     a.bf16 = bf16;
+    a.sel = cfg->sel;
     int n = 0;
-    if (bf16 || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL)
+    if ((bf16 && !decode_fused(plan.tpad, cfg->sel, K)) || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL)
         n += 1 + (cfg->score == AS_SCORE_CLACT ? 2 : 0);  // select kernel (+ column energy)
     return n + decode_launch_count(a, plan);
 }

@@ -395,6 +395,37 @@ struct TcCfg {
     static constexpr int MINB = TP <= 4 ? 2 : 1;
 };
 
+// Sum of the split-K partials p[0], p[stride], ... in split order, with
+// every load of a batch of TC_SPLIT_BATCH issued before the first add
+// (latency of one L2 round trip per batch instead of one per split).
+constexpr int TC_SPLIT_BATCH = 48;
+
+template <typename V>
+__device__ __forceinline__ void add_to(V &a, const V &b);
+template <>
+__device__ __forceinline__ void add_to<float>(float &a, const float &b) { a += b; }
+template <>
+__device__ __forceinline__ void add_to<float4>(float4 &a, const float4 &b)
+{
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+}
+
+template <typename V, int B>
+__device__ __forceinline__ V sum_splits(const V *p, size_t stride, int k_splits)
+{
+    V s = __ldcg(p);
+    for (int k0 = 1; k0 < k_splits; k0 += B) {
+        V v[B];
+#pragma unroll
+        for (int u = 0; u < B; ++u)
+            if (k0 + u < k_splits) v[u] = __ldcg(p + (size_t)(k0 + u) * stride);
+#pragma unroll
+        for (int u = 0; u < B; ++u)
+            if (k0 + u < k_splits) add_to(s, v[u]);
+    }
+    return s;
+}
+
 // y = sum of the split-K partials in split order (+ eta*rowsum), 4 columns a thread.
 __global__ void __launch_bounds__(256) k_decode_reduce(const float *__restrict__ partial, int k_splits, int T,
                                                        int n_out, const float *__restrict__ eta,
@@ -405,12 +436,7 @@ __global__ void __launch_bounds__(256) k_decode_reduce(const float *__restrict__
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     const int n4 = T * n_out / 4;
     if (i >= n4) return;
-    const float4 *p = reinterpret_cast<const float4 *>(partial);
-    float4 s = __ldcg(p + i);
-    for (int k = 1; k < k_splits; ++k) {
-        const float4 v = __ldcg(p + (size_t)k * n4 + i);
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-    }
+    float4 s = sum_splits<float4, 24>(reinterpret_cast<const float4 *>(partial) + i, (size_t)n4, k_splits);
     const int t = (4 * i) / n_out, o = (4 * i) % n_out;
     if (eta) {
         const float e = eta[t];
@@ -453,7 +479,10 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int TP>
+// FUSED (at most 2 tokens): the kernel computes the means and the selection
+// itself (no select kernel before it).  Otherwise the select kernel precedes
+// it.  With several splits k_decode_reduce follows it in both cases.
+template <int TP, bool FUSED>
 __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     k_decode_tc(DecodeArgs a, int words_per_split)
 {
@@ -470,6 +499,9 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     __shared__ float s_eta[TP];
     __shared__ uint32_t s_keep[TP][TC_MAXW];
     __shared__ int s_wbase[TC_MAXW + 1];
+    __shared__ uint32_t s_union[32];
+    __shared__ __align__(16) float s_f[FUSED ? TC_MAXL : 4];  // channel factors (16-byte loads)
+    __shared__ double s_red[TC_WARPS][TP];
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -482,43 +514,124 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     const int nch = max(0, c_end - c_begin);  // multiple of 8
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
 
-    // ---- 1. activation chunk (issued before waiting for the selection
-    // kernel), then the keep words and D-PTS means it wrote
-    const int ngc = nch >> 3;
-    uint4 chv[8];
+    if constexpr (FUSED) {
+        // ---- 1. whole rows (D-PTS mean), own chunk and channel factors,
+        // every load issued before any is used
+        const int ng = K >> 3, gc0 = c_begin >> 3, ngc = nch >> 3;
+        uint4 rowv[TP][8];
+        float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool want_g = a.score == AS_SCORE_WEIGHT && tid < (nch >> 2);
+        if (want_g) gv = *reinterpret_cast<const float4 *>(a.g + c_begin + 4 * tid);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int i = tid + r * TC_THREADS;
-        if (i < TP * ngc) {
-            const int t = i / ngc, g = i % ngc;
-            chv[r] = t < T ? *reinterpret_cast<const uint4 *>(x + (size_t)t * K + c_begin + 8 * g)
-                           : make_uint4(0, 0, 0, 0);
+        for (int t = 0; t < TP; ++t)
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int g = tid + r * TC_THREADS;
+                if (t < T && g < ng) rowv[t][r] = *reinterpret_cast<const uint4 *>(x + (size_t)t * K + 8 * g);
+            }
+        if (want_g) *reinterpret_cast<float4 *>(s_f + 4 * tid) = gv;
+#pragma unroll
+        for (int t = 0; t < TP; ++t) {
+            double sum = 0.0;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int g = tid + r * TC_THREADS;
+                if (t < T && g < ng) {
+                    float w[8];
+                    load8(&rowv[t][r], w);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sum += (double)w[e];
+                    if (g >= gc0 && g < gc0 + ngc) *reinterpret_cast<uint4 *>(xs + t * TC_MAXL + 8 * (g - gc0)) = rowv[t][r];
+                } else if (t >= T && g >= gc0 && g < gc0 + ngc) {
+                    *reinterpret_cast<uint4 *>(xs + t * TC_MAXL + 8 * (g - gc0)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            sum = warp_sum_f64(sum);
+            if (lane == 0) s_red[warp][t] = sum;
         }
+        __syncthreads();
+        if (tid < TP) {
+            double sum = 0.0;
+            for (int w = 0; w < TC_WARPS; ++w) sum += s_red[w][tid];
+            s_eta[tid] = (a.dpts && tid < T) ? (float)(sum / (double)K) : 0.0f;
+            if (a.dpts && slice == 0 && split == 0 && tid < T) {
+                a.eta_in[tid] = s_eta[tid];  // for the split-K reduction kernel
+                if (a.eta_out) a.eta_out[tid] = s_eta[tid];
+            }
+        }
+        if (a.score == AS_SCORE_CLACT) {
+            for (int i = tid; i < nch; i += TC_THREADS) {
+                double q = 0.0;
+                for (int t = 0; t < T; ++t) {
+                    const double v = (double)__bfloat162float(xs[t * TC_MAXL + i]);
+                    q += v * v;
+                }
+                s_f[i] = (float)sqrt(q);
+                if (slice == 0 && a.colnorm_out) a.colnorm_out[c_begin + i] = s_f[i];
+            }
+        }
+        __syncthreads();
+        // ---- 2. selection: a warp scores a (token, 32-channel word) item, one
+        // channel per lane, ranks each in its M-block; its ballot is the word
+        float *wsc = reinterpret_cast<float *>(smem + (size_t)TP * TC_MAXL * 2) + warp * 32;
+        for (int item = warp; item < T * nw; item += TC_WARPS) {
+            const int t = item / nw, wl = item % nw;
+            const int c = 32 * wl + lane;
+            float sc = 0.0f;
+            if (c < nch) {
+                const float xv = __bfloat162float(xs[t * TC_MAXL + c]);
+                const float xh = a.dpts ? __fsub_rn(xv, s_eta[t]) : xv;
+                sc = a.score != AS_SCORE_MAG ? __fmul_rn(fabsf(xh), s_f[c]) : fabsf(xh);
+            }
+            wsc[lane] = sc;
+            __syncwarp();
+            const bool keep = c < nch && nm_rank_keep(wsc, lane, a.n, a.m);
+            const uint32_t word = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0) {
+                s_keep[t][wl] = word;
+                if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+    } else {
+        // ---- 1. activation chunk (issued before waiting for the selection
+        // kernel), then the keep words and D-PTS means it wrote
+        const int ngc = nch >> 3;
+        uint4 chv[8];
+    #pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = tid + r * TC_THREADS;
+            if (i < TP * ngc) {
+                const int t = i / ngc, g = i % ngc;
+                chv[r] = t < T ? *reinterpret_cast<const uint4 *>(x + (size_t)t * K + c_begin + 8 * g)
+                               : make_uint4(0, 0, 0, 0);
+            }
+        }
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // selection kernel complete
+        if (tid < TP) s_eta[tid] = (a.dpts && tid < T) ? a.eta_in[tid] : 0.0f;
+        if (a.eta_out && a.dpts && slice == 0 && split == 0 && tid < T) a.eta_out[tid] = a.eta_in[tid];
+        for (int i = tid; i < T * nw; i += TC_THREADS) {
+            const int t = i / nw, wl = i % nw;
+            const uint32_t word = a.mask_in[(size_t)t * nwords + w0 + wl];
+            s_keep[t][wl] = word;
+            if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
+        }
+    #pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = tid + r * TC_THREADS;
+            if (i < TP * ngc) *reinterpret_cast<uint4 *>(xs + (i / ngc) * TC_MAXL + 8 * (i % ngc)) = chv[r];
+        }
+        __syncthreads();
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // selection kernel complete
-    if (tid < TP) s_eta[tid] = (a.dpts && tid < T) ? a.eta_in[tid] : 0.0f;
-    if (a.eta_out && a.dpts && slice == 0 && split == 0 && tid < T) a.eta_out[tid] = a.eta_in[tid];
-    for (int i = tid; i < T * nw; i += TC_THREADS) {
-        const int t = i / nw, wl = i % nw;
-        const uint32_t word = a.mask_in[(size_t)t * nwords + w0 + wl];
-        s_keep[t][wl] = word;
-        if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int i = tid + r * TC_THREADS;
-        if (i < TP * ngc) *reinterpret_cast<uint4 *>(xs + (i / ngc) * TC_MAXL + 8 * (i % ngc)) = chv[r];
-    }
-    __syncthreads();
 
-    // ---- 3. union list, values split into bf16 hi + lo, [token][position]
+    // ---- 3. union list (ascending channel order) with the per-token kept
+    // values split into bf16 hi + lo, [token][position]
     if (warp == 0) {
-        int cnt = 0;
-        if (lane < nw) {
-            uint32_t u = 0;
+        uint32_t u = 0;
+        if (lane < nw)
             for (int t = 0; t < T; ++t) u |= s_keep[t][lane];
-            cnt = __popc(u);
-        }
+        const int cnt = __popc(u);
         int inc = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -526,14 +639,14 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             if (lane >= o) inc += v;
         }
         s_wbase[lane] = inc - cnt;
+        s_union[lane] = u;
         if (lane == 31) s_wbase[TC_MAXW] = inc;
     }
     __syncthreads();
     const int L = s_wbase[TC_MAXW];
     const int Lp = (L + TC_KS - 1) / TC_KS * TC_KS;
     for (int wl = warp; wl < nw; wl += TC_WARPS) {
-        uint32_t u = 0;
-        for (int t = 0; t < T; ++t) u |= s_keep[t][wl];
+        const uint32_t u = s_union[wl];
         if ((u >> lane) & 1u) {
             const int pos = s_wbase[wl] + __popc(u & ((1u << lane) - 1u));
             const int cl = 32 * wl + lane;
@@ -647,19 +760,21 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     __syncthreads();
     const int k_splits = gridDim.y;
     const int ocol0 = slice * C::NS;
+    auto emit = [&](int t, int o, float v) {
+        if (a.dpts) v = fmaf(s_eta[t], a.rowsum[o], v);
+        if (a.out_bf16)
+            static_cast<__nv_bfloat16 *>(a.y)[(size_t)t * n_out + o] = __float2bfloat16_rn(v);
+        else
+            static_cast<float *>(a.y)[(size_t)t * n_out + o] = v;
+    };
     for (int i = tid; i < T * C::NS; i += TC_THREADS) {
         const int t = i / C::NS, c = i % C::NS, o = ocol0 + c;
         if (o >= n_out) continue;
-        float v = red[t * C::NS + c];
-        if (k_splits > 1) {
+        const float v = red[t * C::NS + c];
+        if (k_splits > 1)
             a.partial[((size_t)split * T + t) * n_out + o] = v;
-        } else {
-            if (a.dpts) v = fmaf(s_eta[t], a.rowsum[o], v);
-            if (a.out_bf16)
-                static_cast<__nv_bfloat16 *>(a.y)[(size_t)t * n_out + o] = __float2bfloat16_rn(v);
-            else
-                static_cast<float *>(a.y)[(size_t)t * n_out + o] = v;
-        }
+        else
+            emit(t, o, v);
     }
 }
 
@@ -733,6 +848,9 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &p, cudaStream
     return cudaGetLastError();
 }
 
+// whole-row loads for the mean are held in registers: K <= 8 * 256 * 8
+bool decode_fused(int tpad, int sel, int K) { return tpad <= 2 && sel == AS_SEL_NM && K <= 8 * TC_THREADS * 8; }
+
 int decode_launch_count(const DecodeArgs &, const DecodePlan &p)
 {
     if (!p.tc) return 1;
@@ -757,16 +875,29 @@ template <int TP>
 static cudaError_t launch_tc(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
 {
     const size_t smem = TcCfg<TP>::smem;
-    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<TP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.n_slices, p.k_splits);
-    cfg.blockDim = dim3(TC_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    set_pdl(cfg, attr);
-    e = cudaLaunchKernelEx(&cfg, k_decode_tc<TP>, a, p.words_per_split);
+    cudaError_t e;
+    bool fused = false;
+    if constexpr (TP <= 2) fused = decode_fused(TP, a.sel, a.K);
+    if (fused) {  // selection inside the decode kernel
+        if constexpr (TP <= 2) {
+            e = cudaFuncSetAttribute(k_decode_tc<TP, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            dim3 grid(p.n_slices, p.k_splits);
+            k_decode_tc<TP, true><<<grid, TC_THREADS, smem, st>>>(a, p.words_per_split);
+            e = cudaGetLastError();
+        }
+    } else {
+        e = cudaFuncSetAttribute(k_decode_tc<TP, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.n_slices, p.k_splits);
+        cfg.blockDim = dim3(TC_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        set_pdl(cfg, attr);
+        e = cudaLaunchKernelEx(&cfg, k_decode_tc<TP, false>, a, p.words_per_split);
+    }
     if (e != cudaSuccess || p.k_splits == 1) return e;
     cudaLaunchConfig_t rc = {};
     const int n4 = a.T * a.n_out / 4;

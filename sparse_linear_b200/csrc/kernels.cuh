@@ -59,6 +59,8 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(int T, int K, int n_out, int bf16);
 int decode_launch_count(const DecodeArgs &a, const DecodePlan &p);
+// True when a bf16 decode of this token pad and selection is one fused launch.
+bool decode_fused(int tpad, int sel, int K);
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st);
 
 // ------------------------------------------------------------ prefill GEMM

@@ -119,16 +119,22 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
     const TX *xr = static_cast<const TX *>(a.x) + (size_t)t * K;
 
     // ---- row statistics: sum x, sum x^2 (float64)
+    constexpr int U = 1;  // tiles whose loads are in flight together (more costs occupancy)
     double sx = 0.0, sxx = 0.0;
     if (a.dpts || a.var) {
-        for (int g = tid; g < ngroups; g += NT) {
-            float v[8];
-            load8(xr + 8 * g, v);
+        for (int g0 = tid; g0 < ngroups; g0 += U * NT) {
+            float v[U][8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                sx += (double)v[e];
-                sxx += (double)v[e] * (double)v[e];
-            }
+            for (int u = 0; u < U; ++u)
+                if (g0 + u * NT < ngroups) load8(xr + 8 * (g0 + u * NT), v[u]);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (g0 + u * NT < ngroups)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        sx += (double)v[u][e];
+                        sxx += (double)v[u][e] * (double)v[u][e];
+                    }
         }
         block_sum2<NT>(sx, sxx, red);
     }
@@ -198,78 +204,93 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
     const int words = (K + 31) >> 5;
     double skm = 0.0, skmm = 0.0;
     int eq_base = 0;
-    for (int tile = 0; tile < ntiles; ++tile) {
-        const int g = tile * NT + tid, c0 = 8 * g;
-        const bool act = g < ngroups;
-        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, xh[8], s[8];
-        if (act) load8(xr + c0, v);
-        score8(v, a.dpts, eta, act ? a.f : nullptr, c0, xh, s);
-        uint32_t keep;
-        if (a.sel == AS_SEL_NM) {
-            keep = nm_keep_dispatch(s, lane, a.n, a.m);
-        } else if (topk) {
-            if (kk <= 0) keep = 0;
-            else if (kk >= K) keep = 0xFF;
-            else {
-                uint32_t gt = 0, eq = 0;
+    for (int tile0 = 0; tile0 < ntiles; tile0 += U) {
+        float vv[U][8], fv[U][8];
+        const bool has_f = a.f != nullptr;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    uint32_t key = act ? keys[c0 + e] : 0u;
-                    gt |= (uint32_t)(act && key > tau) << e;
-                    eq |= (uint32_t)(act && key == tau) << e;
-                }
-                int total;
-                int before = eq_base + block_excl_scan<NT>(__popc(eq), total, wsum);
-                eq_base += total;
-                keep = gt;
+        for (int u = 0; u < U; ++u) {
+            const int g = (tile0 + u) * NT + tid;
+            if (g < ngroups) {
+                load8(xr + 8 * g, vv[u]);
+                if (has_f) load8f(a.f + 8 * g, fv[u]);
+            }
+        }
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if ((eq >> e) & 1u) {
-                        keep |= (uint32_t)(before < need) << e;
-                        ++before;
+        for (int u = 0; u < U; ++u) {
+            if (tile0 + u >= ntiles) break;  // uniform across the block
+            const int g = (tile0 + u) * NT + tid, c0 = 8 * g;
+            const bool act = g < ngroups;
+            float v[8], xh[8], s[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = act ? vv[u][e] : 0.0f;
+            score8v(v, a.dpts, eta, act && has_f, fv[u], xh, s);
+            uint32_t keep;
+            if (a.sel == AS_SEL_NM) {
+                keep = nm_keep_dispatch(s, lane, a.n, a.m);
+            } else if (topk) {
+                if (kk <= 0) keep = 0;
+                else if (kk >= K) keep = 0xFF;
+                else {
+                    uint32_t gt = 0, eq = 0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        uint32_t key = act ? keys[c0 + e] : 0u;
+                        gt |= (uint32_t)(act && key > tau) << e;
+                        eq |= (uint32_t)(act && key == tau) << e;
                     }
-            }
-        } else {
-            keep = 0xFF;
-        }
-        if (!act) continue;
-
-        if (a.bitmask) {
-            uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
-            bm[g] = (uint8_t)keep;
-            if (g == ngroups - 1)
-                for (int b = ngroups; b < words * 4; ++b) bm[b] = 0;
-        }
-        float km[8];
+                    int total;
+                    int before = eq_base + block_excl_scan<NT>(__popc(eq), total, wsum);
+                    eq_base += total;
+                    keep = gt;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) km[e] = ((keep >> e) & 1u) ? xh[e] : 0.0f;
-        if (a.var) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                skm += (double)km[e];
-                skmm += (double)km[e] * (double)km[e];
+                    for (int e = 0; e < 8; ++e)
+                        if ((eq >> e) & 1u) {
+                            keep |= (uint32_t)(before < need) << e;
+                            ++before;
+                        }
+                }
+            } else {
+                keep = 0xFF;
             }
-        }
-        if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
-        if (a.x_compact) {
-            // two 4-blocks per thread, two kept values each (exactly 2:4)
-            float cv[4];
-            uint32_t nib[2];
+            if (act) {
+                if (a.bitmask) {
+                    uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
+                    bm[g] = (uint8_t)keep;
+                    if (g == ngroups - 1)
+                        for (int b = ngroups; b < words * 4; ++b) bm[b] = 0;
+                }
+                float km[8];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t b = (keep >> (4 * h)) & 0xFu;
-                int i0 = __ffs(b) - 1;
-                int i1 = 31 - __clz(b);
-                cv[2 * h] = xh[4 * h + i0];
-                cv[2 * h + 1] = xh[4 * h + i1];
-                nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
-            }
-            __nv_bfloat162 p0 = __floats2bfloat162_rn(cv[0], cv[1]);
-            __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
-            uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1));
-            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) = pk;
-            if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
-        }
+                for (int e = 0; e < 8; ++e) km[e] = ((keep >> e) & 1u) ? xh[e] : 0.0f;
+                if (a.var) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        skm += (double)km[e];
+                        skmm += (double)km[e] * (double)km[e];
+                    }
+                }
+                if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
+                if (a.x_compact) {
+                    // two 4-blocks per thread, two kept values each (exactly 2:4)
+                    float cv[4];
+                    uint32_t nib[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t b = (keep >> (4 * h)) & 0xFu;
+                        int i0 = __ffs(b) - 1;
+                        int i1 = 31 - __clz(b);
+                        cv[2 * h] = xh[4 * h + i0];
+                        cv[2 * h + 1] = xh[4 * h + i1];
+                        nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
+                    }
+                    __nv_bfloat162 p0 = __floats2bfloat162_rn(cv[0], cv[1]);
+                    __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
+                    uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1));
+                    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) = pk;
+                    if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
+                }
+            }  // act
+        }  // u
     }
     if (a.meta24 && tid < 16 * kt - ngroups)  // channel padding of the last 128-channel tile
         *meta_byte(a.meta24, t, 8 * (ngroups + tid), kt) = 0x44;
@@ -291,18 +312,29 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
 }
 
 // ---------------------------------------------------------------- CLACT
+// partial[s][i] = sum over rows [s*rows_per, ...) of x[t, i]^2; a thread
+// owns 8 consecutive channels (16-byte loads), rows unrolled by 8.
 template <typename TX>
-__global__ void k_colsq_rows(const TX *__restrict__ x, int T, int K, int rows_per, double *__restrict__ part)
+__global__ void __launch_bounds__(128) k_colsq_rows(const TX *__restrict__ x, int T, int K, int rows_per,
+                                                    double *__restrict__ part)
 {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x, s = blockIdx.y;
-    if (i >= K) return;
+    const int i8 = blockIdx.x * blockDim.x + threadIdx.x, s = blockIdx.y;
+    if (8 * i8 >= K) return;
     const int t0 = s * rows_per, t1 = min(T, t0 + rows_per);
-    double acc = 0.0;
-    for (int t = t0; t < t1; ++t) {
-        double v = (double)Elem<TX>::to_f32(x[(size_t)t * K + i]);
-        acc += v * v;
+    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int tb = t0; tb < t1; tb += 8) {
+        float v[8][8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            if (tb + r < t1) load8(x + (size_t)(tb + r) * K + 8 * i8, v[r]);
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            if (tb + r < t1)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] += (double)v[r][e] * (double)v[r][e];
     }
-    part[(size_t)s * K + i] = acc;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[(size_t)s * K + 8 * i8 + e] = acc[e];
 }
 
 __global__ void k_colnorm_final(const double *__restrict__ part, int slabs, int K, float *__restrict__ c)
@@ -325,7 +357,7 @@ cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void
 {
     const int slabs = colnorm_slabs(T);
     double *part = static_cast<double *>(ws);
-    dim3 grid((K + 127) / 128, slabs);
+    dim3 grid((K / 8 + 127) / 128, slabs);  // K % 8 == 0
     if (bf16)
         k_colsq_rows<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), T, K, 128, part);
     else

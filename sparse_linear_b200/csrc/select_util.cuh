@@ -60,6 +60,18 @@ __device__ __forceinline__ void score8(const float (&x)[8], bool shift, float et
     }
 }
 
+// Same with the channel factors already in registers (has_f false: f = 1).
+__device__ __forceinline__ void score8v(const float (&x)[8], bool shift, float eta, bool has_f, const float (&fv)[8],
+                                        float (&xh)[8], float (&s)[8])
+{
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        xh[e] = shift ? __fsub_rn(x[e], eta) : x[e];
+        float a = fabsf(xh[e]);
+        s[e] = has_f ? __fmul_rn(a, fv[e]) : a;
+    }
+}
+
 // "j ranks ahead of i": higher score, or equal score and lower index.
 __device__ __forceinline__ int ahead(float sj, int j, float si, int i) { return (sj > si) | ((sj == si) & (j < i)); }
 
