@@ -17,7 +17,7 @@
 //   warps 2-5 epilogue: TMEM -> registers (tcgen05.ld), eta*rowsum or nu
 //            scaling, rounding, stores.  Two accumulator buffers let the
 //            epilogue of one tile overlap the main loop of the next.
-// No cluster multicast is used.  Every mbarrier wait is bounded.
+// No load uses cluster multicast.  Every mbarrier wait is bounded.
 #include <algorithm>
 
 #include "common.cuh"
@@ -273,6 +273,213 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------- sparse, CTA pair (2 SMs)
+// The same 2:4 contraction with two SMs of a cluster working as one
+// 256 x 256 tile (tcgen05.mma.sp.cta_group::2, M = 256, N = 256, K = 32
+// logical per instruction).  Each CTA stages its own 128 rows of A, its own
+// 2:4 positions and half (128 rows) of the weight tile; the leader CTA
+// issues the MMAs, which read both CTAs' shared memory and write each CTA's
+// tensor memory (its 128 rows x 256 columns).  Per SM this halves the
+// weight bytes fetched per multiply-add compared with the 1-SM 128 x 128
+// tile, which is what bounds that kernel (L2 -> SM bandwidth).
+//   warp 0      TMA producer (both CTAs); the leader's full barrier counts
+//               the bytes of both CTAs.
+//   warp 1      tensor-memory allocation (both CTAs, cta_group::2); lane 0
+//               of the leader issues metadata copies and MMAs.
+//   warps 2-9   epilogue: (lane quarter, column half) per warp; the whole
+//               accumulator slice is read into registers and released
+//               before the scaling and the stores, so the next tile's MMAs
+//               overlap the stores.
+// Loads carry no multicast; only tcgen05.commit signals both CTAs.
+constexpr int PAIR_THREADS = 320;
+constexpr int PAIR_BM = 256;  // rows per CTA pair (128 per CTA)
+constexpr int PAIR_BN = 256;  // weight rows per CTA pair (128 per CTA)
+constexpr int PAIR_STAGES = 4;
+constexpr int PAIR_A_BYTES = 128 * 64 * 2;   // kept half of 128 rows x 128 logical K
+constexpr int PAIR_B_BYTES = 128 * 128 * 2;  // 128 weight rows x 128 K, two sub-tiles
+constexpr int PAIR_M_BYTES = 2048;           // 2:4 positions of 128 rows x 128 K
+constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES + PAIR_M_BYTES;
+
+constexpr size_t pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PAIR_STAGE_BYTES + 256; }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
+    k_gemm_sp_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmE, GemmParams p)
+{
+    constexpr int S = PAIR_STAGES;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~uintptr_t(1023));
+    unsigned char *sA = smem;
+    unsigned char *sB = sA + S * PAIR_A_BYTES;
+    unsigned char *sM = sB + S * PAIR_B_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sM + S * PAIR_M_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 1;
+    uint64_t *drain = bars + 2 * S + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 3);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int num_tiles = p.m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
+            mbar_init(&empty[s], 1);  // one commit from the leader's MMA thread
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 16);  // 8 epilogue warps in each CTA (leader's copy is the one used)
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmE);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs initialised before either uses the other's
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = pair; tile < num_tiles && !*(volatile int *)abort_flag; tile += npairs) {
+                int mt, nt;
+                tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
+                const int arow = mt * PAIR_BM + 128 * (int)rank;
+                const int brow = nt * PAIR_BN + 128 * (int)rank;
+                const int echunk = (2 * mt + (int)rank) * p.meta_kt;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
+                    const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
+                    unsigned char *b_dst = sB + stage * PAIR_B_BYTES;
+                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, &tmA, bar, kb * 64, arow);
+                    tma_load_2d_pair(b_dst, &tmB, bar, kb * 128, brow);
+                    tma_load_2d_pair(b_dst + 128 * 128, &tmB, bar, kb * 128 + 64, brow);
+                    tma_load_2d_pair(sM + stage * PAIR_M_BYTES, &tmE, bar, 0, (echunk + kb) * 8);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(PAIR_BM, PAIR_BN, true);
+            const uint32_t meta_tmem = tmem + PAIR_BN;
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int tile = pair; tile < num_tiles && !*(volatile int *)abort_flag; tile += npairs, ++it) {
+                if (!mbar_wait(acc_empty, (it & 1) ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t b_addr = smem_u32(sB + stage * PAIR_B_BYTES);
+                    const uint64_t a_desc = sdesc_kmajor_sw128(smem_u32(sA + stage * PAIR_A_BYTES));
+                    const uint32_t e_tmem = meta_tmem + stage * 4;
+                    tmem_cp_128x128b_pair(e_tmem, sdesc_rows16(smem_u32(sM + stage * PAIR_M_BYTES)));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t a_j = a_desc + (uint64_t)((32 * j) >> 4);
+                        const uint64_t b_j = sdesc_kmajor_sw128(b_addr + (j >> 1) * (128 * 128) + (j & 1) * 64);
+                        mma_sp_bf16_pair(tmem, a_j, b_j, idesc | (uint32_t)(j & 1), e_tmem + (j & ~1),
+                                         (kb | j) != 0);
+                    }
+                    tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) { *(volatile int *)abort_flag = 1; break; }
+                tc_commit_pair_mc(acc_full, 0x3);
+            }
+            tc_commit_pair(drain);
+            mbar_wait(drain, 0);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..9)
+        const int q = warp & 3;           // TMEM lanes 32q..32q+31
+        const int h = (warp - 2) >> 2;    // accumulator columns [128h, 128h+128)
+        const uint32_t acc_empty_leader = mapa_u32(smem_u32(acc_empty), 0);
+        int it = 0;
+        for (int tile = pair; tile < num_tiles && !*(volatile int *)abort_flag; tile += npairs, ++it) {
+            int mt, nt;
+            tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
+            if (!mbar_wait(acc_full, it & 1)) { *(volatile int *)abort_flag = 1; break; }
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + 128 * h + 32 * ch, r[ch]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+
+            const int row = mt * PAIR_BM + 128 * (int)rank + 32 * q + lane;
+            if (row >= p.T) continue;
+            float rscale = 1.0f, reta = 0.0f;
+            if (p.nu) rscale = p.nu[row];
+            if (p.eta) reta = p.eta[row];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                const int col0 = nt * PAIR_BN + 128 * h + 32 * ch;
+                if (col0 >= p.n_out) continue;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float f = __uint_as_float(r[ch][i]);
+                    if (p.nu) f *= rscale;
+                    if (p.eta) {
+                        const int c = min(col0 + i, p.n_out - 1);
+                        f = fmaf(reta, p.rowsum[c], f);
+                    }
+                    v[i] = f;
+                }
+                if (p.out_bf16) {
+                    __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(p.y) + (size_t)row * p.n_out + col0;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        if (col0 + 8 * c8 < p.n_out) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                __nv_bfloat162 hh = __floats2bfloat162_rn(v[8 * c8 + 2 * i], v[8 * c8 + 2 * i + 1]);
+                                w[i] = *reinterpret_cast<uint32_t *>(&hh);
+                            }
+                            *reinterpret_cast<uint4 *>(yr + 8 * c8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                } else {
+                    float *yr = static_cast<float *>(p.y) + (size_t)row * p.n_out + col0;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        if (col0 + 4 * c4 < p.n_out)
+                            *reinterpret_cast<float4 *>(yr + 4 * c4) =
+                                make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+                }
+            }
+        }
+    }
+
+    // Both CTAs' tensor memory stays allocated until the leader's last MMA
+    // has completed and both epilogues have read their accumulators.
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                       const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -303,6 +510,21 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t c
     cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2:4 positions as a 2-D uint32 tensor of 256-byte rows: one 2 KB chunk
+// (128 rows x 128 K of A) is 8 rows, box {64, 8}, no swizzle.
+static bool make_map_meta(CUtensorMap *m, const void *base, uint64_t chunks)
+{
+    PFN_encodeTiled_t enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {64, chunks * 8};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, 8};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -349,8 +571,83 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// Number of 2-CTA clusters of k_gemm_sp_pair that fit on the device at once
+// (0 if the query fails).
+static int pair_clusters(size_t smem)
+{
+    static int cached = -1;
+    if (cached >= 0) return cached;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_sp_pair, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cached = n;
+    return n;
+}
+
+// The pair kernel needs every CTA's 128-row box to hold at least one real
+// row (an even number of 128-row tiles) and a 16-byte-aligned position
+// buffer for its tensor map.
+static bool use_pair(const GemmArgs &a)
+{
+    const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
+    return a.sparse && (mt128 % 2) == 0 && (reinterpret_cast<uintptr_t>(a.meta) & 15) == 0;
+}
+
+static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
+{
+    CUtensorMap mA, mB, mE;
+    const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
+    GemmParams p{};
+    p.meta = a.meta;
+    p.rowsum = a.rowsum;
+    p.eta = a.eta;
+    p.nu = a.nu;
+    p.y = a.y;
+    p.T = a.T;
+    p.K = a.K;
+    p.n_out = a.n_out;
+    p.out_bf16 = a.out_bf16;
+    p.m_tiles = mt128 / 2;
+    p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
+    p.k_blocks = (a.K + 127) / 128;
+    p.meta_kt = (a.K + 127) / 128;
+    if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
+    if (!make_map_meta(&mE, a.meta, (uint64_t)mt128 * p.meta_kt)) return cudaErrorInvalidValue;
+    const size_t smem = pair_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_sp_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int clusters = pair_clusters(smem);
+    if (clusters <= 0) return cudaErrorNotSupported;
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int grid = 2 * std::min(tiles, clusters);
+    k_gemm_sp_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st)
 {
+    if (use_pair(a)) {
+        const size_t smem = pair_smem_bytes();
+        if (cudaFuncSetAttribute(k_gemm_sp_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+                cudaSuccess &&
+            pair_clusters(smem) > 0)
+            return launch_gemm_pair(a, st);
+        cudaGetLastError();
+    }
     return a.sparse ? launch_gemm_t<true>(a, st) : launch_gemm_t<false>(a, st);
 }
 

@@ -181,7 +181,11 @@ def check_select_24(sl, x, bufs, rows):
     return ref_mask
 
 
-@pytest.mark.parametrize("T,K,n_out", [(300, 1024, 520), (128, 14336, 256), (5, 256, 64), (1000, 2048, 1024)])
+# (300, 1024, 520), (128, ...), (5, ...): odd number of 128-row tiles, one SM
+# per tile; the others run on CTA pairs, including a ragged weight tail that
+# leaves the second CTA's weight box wholly outside W (512, 1024, 264).
+@pytest.mark.parametrize("T,K,n_out", [(300, 1024, 520), (128, 14336, 256), (5, 256, 64), (1000, 2048, 1024),
+                                       (256, 512, 200), (512, 1024, 264), (512, 4096, 768)])
 def test_prefill_24(sl, T, K, n_out):
     x, W = synth.random_layer(T, K, n_out, seed=T + K, dist="sqrelu")
     for out in (sl.AS_BF16, sl.AS_F32):
