@@ -252,6 +252,7 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     a.sel = cfg->sel;
     a.n = cfg->n;
     a.m = cfg->m;
+    a.k_keep = cfg->k_keep;
     a.dpts = cfg->dpts;
     a.g = g;
     a.rowsum = rowsum;

@@ -20,6 +20,8 @@
 //   5. reduces row groups in shared memory and split-K partials through the
 //      workspace; the last CTA of a column slice sums the partials in split
 //      order (deterministic), adds eta * rowsum and writes y.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "select_util.cuh"
@@ -351,21 +353,22 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
 // bf16 path: tensor-core decode kernel, D-PTS mean kernel, split-K reduction
 // ============================================================================
 //
-// bf16 decode = three kernels chained by programmatic dependent launch:
-//   k_select (one CTA of 1024 threads per token, select.cu): D-PTS mean,
-//     score, exact N:M or top-k selection -> keep words [T, K/32] and eta;
+// bf16 decode = up to three kernels chained by programmatic dependent launch:
+//   k_select_nm_decode (select.cu, more than 2 tokens): D-PTS mean, score,
+//     exact N:M selection -> keep words [T, K/32] and eta;
 //   k_decode_tc: CTA (slice, split) owns NS = 512 output columns and a range
 //     of up to 1024 channels.  It loads its activation chunk while the
-//     selection finishes, then reads the keep words and eta, compacts the
-//     union over tokens of the kept channels (ascending) with the kept values
-//     split into bf16 hi + lo (xhat = hi + lo to about 2^-16 relative), and
-//     streams those rows of Wt: each of the 8 warps owns 64 output columns
-//     and runs its own cp.async ring over the 128-byte pieces of the kept rows
-//     it multiplies (no block-wide barrier in the loop).  Each staged
-//     16-channel slab goes through ldmatrix.trans into A fragments and the
-//     tensor cores (mma.sync m16n8k16, bf16 in, float32 accumulate; once for
-//     hi, once for lo).  It writes y directly (one split) or its split-K
-//     partial sums;
+//     selection finishes (at most 2 tokens: it computes the means and the
+//     selection itself), turns the chunk in place into the dense kept values
+//     xhat = keep ? x - eta : 0 (bf16 hi, plus lo = xhat - hi for float32
+//     outputs), lists the union over tokens of the kept channels (ascending)
+//     and streams those rows of Wt: each of the 8 warps owns 64 output
+//     columns and runs its own cp.async ring over the 128-byte pieces of the
+//     kept rows (no block-wide barrier in the loop).  Each staged 16-channel
+//     slab goes through ldmatrix.trans into A fragments; the B fragments are
+//     gathered from the dense kept values through the list; the tensor cores
+//     (mma.sync m16n8k16, bf16 in, float32 accumulate) take hi (and lo).  It
+//     writes y directly (one split) or its split-K partial sums;
 //   k_decode_reduce: adds the partials in split order, with eta*rowsum.
 
 constexpr int TC_WARPS = 8;
@@ -376,22 +379,22 @@ constexpr int TC_WROWP = TC_WCOLS * 2 + 16;    // 144-byte padded row piece (ldm
 constexpr int TC_KS = 16;                      // rows per stage = one mma k-step
 constexpr int TC_MAXW = 32;                    // 32-channel words per CTA
 constexpr int TC_MAXL = TC_MAXW * 32;          // 1024 channels
-constexpr int TC_XP = TC_MAXL + 24;            // token-value row stride (bf16): no bank conflicts
+constexpr int TC_XP = TC_MAXL + 24;            // kept-value row stride (bf16): rows 12 banks apart
+constexpr int TC_PAD = TC_MAXL;                // list entry of padding positions: a zero kept value
 
 template <int TP>
 struct TcCfg {
     static constexpr int NS = TC_NS;
     static constexpr int MT = TC_WCOLS / 16;            // 16-output m-tiles per warp
-    static constexpr int STAGES = TP <= 4 ? 4 : 6;
+    static constexpr int STAGES = TP <= 4 ? 4 : 8;
     static constexpr int NT = (TP + 7) / 8;             // 8-token n-tiles
     static constexpr size_t wstage = (size_t)TC_KS * TC_WROWP;
     static constexpr size_t ring = (size_t)TC_WARPS * STAGES * wstage;
-    static constexpr size_t xchunk = (size_t)TP * TC_MAXL * 2;   // bf16 activation chunk; aliases the ring
-    static constexpr size_t red = (size_t)TP * NS * 4;           // aliases the ring
-    static constexpr size_t big = ring > xchunk ? (ring > red ? ring : red) : (xchunk > red ? xchunk : red);
-    static constexpr size_t lists = (size_t)TC_MAXL * 4 + (size_t)2 * TP * TC_XP * 2;
-    static constexpr size_t smem = big + lists;
-    static constexpr int TARGET = TP <= 4 ? 296 : 148;
+    static constexpr size_t red = (size_t)TP * NS * 4;  // after the main loop; aliases the ring
+    static constexpr size_t big = ring > red ? ring : red;
+    static constexpr size_t xrow = (size_t)TP * TC_XP * 2;              // one dense kept-value array
+    static constexpr size_t list = (size_t)(TC_MAXL + TC_KS) * 4;        // channel offsets
+    static constexpr size_t smem(bool lo) { return big + (lo ? 2 : 1) * xrow + list; }
     static constexpr int MINB = TP <= 4 ? 2 : 1;
 };
 
@@ -426,31 +429,59 @@ __device__ __forceinline__ V sum_splits(const V *p, size_t stride, int k_splits)
     return s;
 }
 
-// y = sum of the split-K partials in split order (+ eta*rowsum), 4 columns a thread.
+// y = sum of the split-K partials in split order (+ eta*rowsum).  Partials
+// are [split][column][TP]; a thread owns one column and VW consecutive
+// tokens (one vector load per split).
+template <int TP>
+struct RedVec {
+    static constexpr int VW = TP >= 4 ? 4 : TP;
+    using V = typename std::conditional<VW == 4, float4, typename std::conditional<VW == 2, float2, float>::type>::type;
+};
+template <>
+__device__ __forceinline__ void add_to<float2>(float2 &a, const float2 &b)
+{
+    a.x += b.x; a.y += b.y;
+}
+template <typename V>
+__device__ __forceinline__ float vget(const V &v, int k);
+template <>
+__device__ __forceinline__ float vget<float>(const float &v, int) { return v; }
+template <>
+__device__ __forceinline__ float vget<float2>(const float2 &v, int k) { return k == 0 ? v.x : v.y; }
+template <>
+__device__ __forceinline__ float vget<float4>(const float4 &v, int k)
+{
+    return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+
+template <int TP>
 __global__ void __launch_bounds__(256) k_decode_reduce(const float *__restrict__ partial, int k_splits, int T,
                                                        int n_out, const float *__restrict__ eta,
                                                        const float *__restrict__ rowsum, void *__restrict__ y,
                                                        int out_bf16)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // after the wait: see k_select_nm_decode
+    using R = RedVec<TP>;
+    using V = typename R::V;
+    constexpr int G = TP / R::VW;  // vectors per column
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    const int n4 = T * n_out / 4;
-    if (i >= n4) return;
-    float4 s = sum_splits<float4, 24>(reinterpret_cast<const float4 *>(partial) + i, (size_t)n4, k_splits);
-    const int t = (4 * i) / n_out, o = (4 * i) % n_out;
-    if (eta) {
-        const float e = eta[t];
-        s.x = fmaf(e, rowsum[o], s.x);
-        s.y = fmaf(e, rowsum[o + 1], s.y);
-        s.z = fmaf(e, rowsum[o + 2], s.z);
-        s.w = fmaf(e, rowsum[o + 3], s.w);
-    }
-    if (out_bf16) {
-        __nv_bfloat162 a = __floats2bfloat162_rn(s.x, s.y), b = __floats2bfloat162_rn(s.z, s.w);
-        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(y) + (size_t)t * n_out + o) =
-            make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
-    } else {
-        *reinterpret_cast<float4 *>(static_cast<float *>(y) + (size_t)t * n_out + o) = s;
+    if (i >= n_out * G) return;
+    const int o = i / G, j = i % G;
+    if (R::VW * j >= T) return;
+    const V s = sum_splits<V, 24>(reinterpret_cast<const V *>(partial) + i, (size_t)n_out * G, k_splits);
+    const float rs = eta ? rowsum[o] : 0.0f;
+#pragma unroll
+    for (int k = 0; k < R::VW; ++k) {
+        const int t = R::VW * j + k;
+        if (t < T) {
+            float v = vget(s, k);
+            if (eta) v = fmaf(eta[t], rs, v);
+            if (out_bf16)
+                static_cast<__nv_bfloat16 *>(y)[(size_t)t * n_out + o] = __float2bfloat16_rn(v);
+            else
+                static_cast<float *>(y)[(size_t)t * n_out + o] = v;
+        }
     }
 }
 
@@ -482,24 +513,27 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // FUSED (at most 2 tokens): the kernel computes the means and the selection
 // itself (no select kernel before it).  Otherwise the select kernel precedes
 // it.  With several splits k_decode_reduce follows it in both cases.
-template <int TP, bool FUSED>
+// LO: the kept values enter the tensor cores as bf16 hi + lo (float32 outputs);
+// without it as one bf16 (bf16 outputs, whose own rounding error, up to
+// 2^-9 relative, is as large as that of rounding xhat to bf16).
+// DENSE (not FUSED): the CTA streams every row of its chunk, in order.  Used
+// when the union over tokens of the kept channels is expected to cover
+// nearly all of them; the stream then does not depend on the selection, so
+// the CTA fills its ring before waiting for the select kernel.
+template <int TP, bool FUSED, bool LO, bool DENSE>
 __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     k_decode_tc(DecodeArgs a, int words_per_split)
 {
     using C = TcCfg<TP>;
     extern __shared__ __align__(16) unsigned char smem[];
     unsigned char *ring = smem;
-    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(smem);  // [TP][TC_MAXL] activation chunk
-    float *red = reinterpret_cast<float *>(smem);                  // [TP][NS] after the main loop
-    unsigned char *lists = smem + C::big;
-    int *list_ch = reinterpret_cast<int *>(lists);
-    __nv_bfloat16 *xh_hi = reinterpret_cast<__nv_bfloat16 *>(lists + TC_MAXL * 4);  // [TP][TC_XP]
-    __nv_bfloat16 *xh_lo = xh_hi + TP * TC_XP;
+    float *red = reinterpret_cast<float *>(smem);  // [TP][NS] after the main loop
+    __nv_bfloat16 *xh = reinterpret_cast<__nv_bfloat16 *>(smem + C::big);   // [TP][TC_XP] dense kept values (hi)
+    __nv_bfloat16 *xl = xh + (LO ? TP * TC_XP : 0);                           // [TP][TC_XP] lo parts (LO)
+    int *list_cl = reinterpret_cast<int *>(smem + C::big + (LO ? 2 : 1) * C::xrow);  // [L padded]
 
     __shared__ float s_eta[TP];
     __shared__ uint32_t s_keep[TP][TC_MAXW];
-    __shared__ int s_wbase[TC_MAXW + 1];
-    __shared__ uint32_t s_union[32];
     __shared__ __align__(16) float s_f[FUSED ? TC_MAXL : 4];  // channel factors (16-byte loads)
     __shared__ double s_red[TC_WARPS][TP];
 
@@ -512,12 +546,63 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     const int nw = max(0, w1 - w0);
     const int c_begin = 32 * w0, c_end = min(32 * w1, K);
     const int nch = max(0, c_end - c_begin);  // multiple of 8
+    const int ngc = nch >> 3;                 // 8-channel groups of the chunk
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
 
+    // store 8 kept values (hi, and lo with LO) of token t, channels 8g..8g+7
+    auto put8 = [&](int t, int g, const float (&v)[8], uint32_t keep8, float eta) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float e0 = 0.0f, e1 = 0.0f;
+            if ((keep8 >> (2 * i)) & 1u) e0 = a.dpts ? __fsub_rn(v[2 * i], eta) : v[2 * i];
+            if ((keep8 >> (2 * i + 1)) & 1u) e1 = a.dpts ? __fsub_rn(v[2 * i + 1], eta) : v[2 * i + 1];
+            const __nv_bfloat162 h = __floats2bfloat162_rn(e0, e1);
+            hw[i] = *reinterpret_cast<const uint32_t *>(&h);
+            if constexpr (LO) {
+                const __nv_bfloat162 l =
+                    __floats2bfloat162_rn(e0 - __low2float(h), e1 - __high2float(h));
+                lw[i] = *reinterpret_cast<const uint32_t *>(&l);
+            }
+        }
+        *reinterpret_cast<uint4 *>(xh + t * TC_XP + 8 * g) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        if constexpr (LO) *reinterpret_cast<uint4 *>(xl + t * TC_XP + 8 * g) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    };
+
+    // per-warp cp.async ring: stage st = list positions [16 st, 16 st + 16)
+    // (DENSE: channel offsets), this warp's 64 columns of each row
+    const int col0 = slice * C::NS + warp * TC_WCOLS;
+    const __nv_bfloat16 *wt = static_cast<const __nv_bfloat16 *>(a.Wt) + (size_t)c_begin * n_out;
+    const uint32_t wring = smem_u32(ring) + (uint32_t)(warp * C::STAGES * C::wstage);
+    auto issue = [&](int st) {
+        const uint32_t base = wring + (uint32_t)((st % C::STAGES) * C::wstage);
+#pragma unroll
+        for (int r = 0; r < (TC_KS * TC_WCOLS * 2 / 16) / 32; ++r) {
+            const int id = lane + 32 * r;
+            const int row = id >> 3, c16 = id & 7;
+            const int pos = st * TC_KS + row;
+            const int cl = DENSE ? (pos < nch ? pos : TC_PAD) : list_cl[pos];
+            const int col = col0 + 8 * c16;
+            const bool ok = cl != TC_PAD && col < n_out;
+            const void *src = ok ? (const void *)(wt + (size_t)cl * n_out + col) : (const void *)wt;
+            cp_async16(base + row * TC_WROWP + c16 * 16, src, ok ? 16u : 0u);  // 0 bytes: zero fill
+        }
+    };
+    auto issue_prologue = [&](int nst) {
+#pragma unroll
+        for (int st = 0; st < C::STAGES - 1; ++st) {
+            if (st < nst) issue(st);
+            cp_async_commit();
+        }
+    };
+
     if constexpr (FUSED) {
+        // launched programmatically: wait for the previous kernel in the
+        // stream (which may have written x) before the first load
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         // ---- 1. whole rows (D-PTS mean), own chunk and channel factors,
         // every load issued before any is used
-        const int ng = K >> 3, gc0 = c_begin >> 3, ngc = nch >> 3;
+        const int ng = K >> 3, gc0 = c_begin >> 3;
         uint4 rowv[TP][8];
         float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
         const bool want_g = a.score == AS_SCORE_WEIGHT && tid < (nch >> 2);
@@ -541,65 +626,92 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
                     load8(&rowv[t][r], w);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) sum += (double)w[e];
-                    if (g >= gc0 && g < gc0 + ngc) *reinterpret_cast<uint4 *>(xs + t * TC_MAXL + 8 * (g - gc0)) = rowv[t][r];
+                    if (g >= gc0 && g < gc0 + ngc) *reinterpret_cast<uint4 *>(xh + t * TC_XP + 8 * (g - gc0)) = rowv[t][r];
                 } else if (t >= T && g >= gc0 && g < gc0 + ngc) {
-                    *reinterpret_cast<uint4 *>(xs + t * TC_MAXL + 8 * (g - gc0)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(xh + t * TC_XP + 8 * (g - gc0)) = make_uint4(0, 0, 0, 0);
                 }
             }
             sum = warp_sum_f64(sum);
             if (lane == 0) s_red[warp][t] = sum;
         }
         __syncthreads();
-        if (tid < TP) {
+        // every thread forms the means from the warp sums (same order everywhere)
+        float eta_r[TP];
+#pragma unroll
+        for (int t = 0; t < TP; ++t) {
             double sum = 0.0;
-            for (int w = 0; w < TC_WARPS; ++w) sum += s_red[w][tid];
-            s_eta[tid] = (a.dpts && tid < T) ? (float)(sum / (double)K) : 0.0f;
-            if (a.dpts && slice == 0 && split == 0 && tid < T) {
-                a.eta_in[tid] = s_eta[tid];  // for the split-K reduction kernel
-                if (a.eta_out) a.eta_out[tid] = s_eta[tid];
-            }
+            for (int w = 0; w < TC_WARPS; ++w) sum += s_red[w][t];
+            eta_r[t] = (a.dpts && t < T) ? (float)(sum / (double)K) : 0.0f;
         }
+#pragma unroll
+        for (int t = 0; t < TP; ++t)
+            if (tid == t) {
+                s_eta[t] = eta_r[t];
+                if (a.dpts && slice == 0 && split == 0 && t < T) {
+                    a.eta_in[t] = eta_r[t];  // for the split-K reduction kernel
+                    if (a.eta_out) a.eta_out[t] = eta_r[t];
+                }
+            }
         if (a.score == AS_SCORE_CLACT) {
             for (int i = tid; i < nch; i += TC_THREADS) {
                 double q = 0.0;
                 for (int t = 0; t < T; ++t) {
-                    const double v = (double)__bfloat162float(xs[t * TC_MAXL + i]);
+                    const double v = (double)__bfloat162float(xh[t * TC_XP + i]);
                     q += v * v;
                 }
                 s_f[i] = (float)sqrt(q);
                 if (slice == 0 && a.colnorm_out) a.colnorm_out[c_begin + i] = s_f[i];
             }
+            __syncthreads();
         }
-        __syncthreads();
         // ---- 2. selection: a warp scores a (token, 32-channel word) item, one
-        // channel per lane, ranks each in its M-block; its ballot is the word
-        float *wsc = reinterpret_cast<float *>(smem + (size_t)TP * TC_MAXL * 2) + warp * 32;
+        // channel per lane, ranks each in its M-block; its ballot is the word.
+        // The lane then replaces its activation by the kept value.
+        float *wsc = reinterpret_cast<float *>(ring) + warp * 32;
         for (int item = warp; item < T * nw; item += TC_WARPS) {
             const int t = item / nw, wl = item % nw;
             const int c = 32 * wl + lane;
-            float sc = 0.0f;
+            float eta_t = eta_r[0];  // eta_r[t] without a dynamic register index
+#pragma unroll
+            for (int k = 1; k < TP; ++k)
+                if (t == k) eta_t = eta_r[k];
+            float xv = 0.0f, sc = 0.0f;
             if (c < nch) {
-                const float xv = __bfloat162float(xs[t * TC_MAXL + c]);
-                const float xh = a.dpts ? __fsub_rn(xv, s_eta[t]) : xv;
-                sc = a.score != AS_SCORE_MAG ? __fmul_rn(fabsf(xh), s_f[c]) : fabsf(xh);
+                xv = __bfloat162float(xh[t * TC_XP + c]);
+                const float xs = a.dpts ? __fsub_rn(xv, eta_t) : xv;
+                sc = a.score != AS_SCORE_MAG ? __fmul_rn(fabsf(xs), s_f[c]) : fabsf(xs);
             }
             wsc[lane] = sc;
             __syncwarp();
             const bool keep = c < nch && nm_rank_keep(wsc, lane, a.n, a.m);
             const uint32_t word = __ballot_sync(0xffffffffu, keep);
+            if (c < nch) {
+                const float e = keep ? (a.dpts ? __fsub_rn(xv, eta_t) : xv) : 0.0f;
+                const __nv_bfloat16 h = __float2bfloat16_rn(e);
+                xh[t * TC_XP + c] = h;
+                if constexpr (LO) xl[t * TC_XP + c] = __float2bfloat16_rn(e - __bfloat162float(h));
+            }
             if (lane == 0) {
                 s_keep[t][wl] = word;
                 if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
             }
             __syncwarp();
         }
+        if constexpr (LO) {  // tokens T..TP-1 of the lo array
+            for (int i = tid; i < (TP - T) * ngc; i += TC_THREADS)
+                *reinterpret_cast<uint4 *>(xl + (T + i / ngc) * TC_XP + 8 * (i % ngc)) = make_uint4(0, 0, 0, 0);
+        }
+        if (tid < TP) {
+            xh[tid * TC_XP + TC_PAD] = __float2bfloat16_rn(0.0f);
+            if constexpr (LO) xl[tid * TC_XP + TC_PAD] = __float2bfloat16_rn(0.0f);
+        }
         __syncthreads();
     } else {
         // ---- 1. activation chunk (issued before waiting for the selection
-        // kernel), then the keep words and D-PTS means it wrote
-        const int ngc = nch >> 3;
+        // kernel, which itself waited for the producer of x), then the keep
+        // words and D-PTS means it wrote, then the kept values from registers
         uint4 chv[8];
-    #pragma unroll
+#pragma unroll
         for (int r = 0; r < 8; ++r) {
             const int i = tid + r * TC_THREADS;
             if (i < TP * ngc) {
@@ -608,26 +720,52 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
                                : make_uint4(0, 0, 0, 0);
             }
         }
+        // DENSE: the first stages of the weight stream, also before the wait
+        // (this kernel starts only once the select kernel has passed its own
+        // wait, so everything before that kernel in the stream is complete)
+        if constexpr (DENSE) issue_prologue((nch + TC_KS - 1) / TC_KS);
         asm volatile("griddepcontrol.wait;" ::: "memory");  // selection kernel complete
         if (tid < TP) s_eta[tid] = (a.dpts && tid < T) ? a.eta_in[tid] : 0.0f;
         if (a.eta_out && a.dpts && slice == 0 && split == 0 && tid < T) a.eta_out[tid] = a.eta_in[tid];
-        for (int i = tid; i < T * nw; i += TC_THREADS) {
+        for (int i = tid; i < TP * nw; i += TC_THREADS) {
             const int t = i / nw, wl = i % nw;
-            const uint32_t word = a.mask_in[(size_t)t * nwords + w0 + wl];
+            uint32_t word = 0u;
+            if (t < T) {
+                word = a.mask_in[(size_t)t * nwords + w0 + wl];
+                if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
+            }
             s_keep[t][wl] = word;
-            if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
         }
-    #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int i = tid + r * TC_THREADS;
-            if (i < TP * ngc) *reinterpret_cast<uint4 *>(xs + (i / ngc) * TC_MAXL + 8 * (i % ngc)) = chv[r];
+        if (tid < TP) {
+            xh[tid * TC_XP + TC_PAD] = __float2bfloat16_rn(0.0f);
+            if constexpr (LO) xl[tid * TC_XP + TC_PAD] = __float2bfloat16_rn(0.0f);
         }
         __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = tid + r * TC_THREADS;
+            if (i < TP * ngc) {
+                const int t = i / ngc, g = i % ngc;
+                float v[8];
+                load8(&chv[r], v);
+                put8(t, g, v, (s_keep[t][g >> 2] >> ((g & 3) << 3)) & 0xFFu, s_eta[t]);
+            }
+        }
     }
 
-    // ---- 3. union list (ascending channel order) with the per-token kept
-    // values split into bf16 hi + lo, [token][position]
-    if (warp == 0) {
+    // ---- 3. union list (ascending channel offsets).  Every warp forms the
+    // prefix over the words itself (no barrier), then lists its own words.
+    // DENSE: every channel, in order (no list; the padding columns of the
+    // kept values are zero).
+    int L = nch;
+    if constexpr (DENSE) {
+        const int npad = (nch + TC_KS - 1) / TC_KS * TC_KS - nch;  // multiple of 8
+        for (int i = tid; i < TP * (npad >> 3); i += TC_THREADS) {
+            const int t = i / (npad >> 3), q = i % (npad >> 3);
+            *reinterpret_cast<uint4 *>(xh + t * TC_XP + nch + 8 * q) = make_uint4(0, 0, 0, 0);
+            if constexpr (LO) *reinterpret_cast<uint4 *>(xl + t * TC_XP + nch + 8 * q) = make_uint4(0, 0, 0, 0);
+        }
+    } else {
         uint32_t u = 0;
         if (lane < nw)
             for (int t = 0; t < T; ++t) u |= s_keep[t][lane];
@@ -635,63 +773,22 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         int inc = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xffffffffu, inc, o);
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
             if (lane >= o) inc += v;
         }
-        s_wbase[lane] = inc - cnt;
-        s_union[lane] = u;
-        if (lane == 31) s_wbase[TC_MAXW] = inc;
+        L = __shfl_sync(0xffffffffu, inc, 31);
+        for (int wl = warp; wl < nw; wl += TC_WARPS) {
+            const uint32_t uw = __shfl_sync(0xffffffffu, u, wl);
+            const int base = __shfl_sync(0xffffffffu, inc - cnt, wl);
+            if ((uw >> lane) & 1u) list_cl[base + __popc(uw & ((1u << lane) - 1u))] = 32 * wl + lane;
+        }
     }
-    __syncthreads();
-    const int L = s_wbase[TC_MAXW];
     const int Lp = (L + TC_KS - 1) / TC_KS * TC_KS;
-    for (int wl = warp; wl < nw; wl += TC_WARPS) {
-        const uint32_t u = s_union[wl];
-        if ((u >> lane) & 1u) {
-            const int pos = s_wbase[wl] + __popc(u & ((1u << lane) - 1u));
-            const int cl = 32 * wl + lane;
-            list_ch[pos] = c_begin + cl;
-#pragma unroll
-            for (int t = 0; t < TP; ++t) {
-                float v = 0.0f;
-                if (t < T && ((s_keep[t][wl] >> lane) & 1u)) {
-                    const float xv = __bfloat162float(xs[t * TC_MAXL + cl]);
-                    v = a.dpts ? __fsub_rn(xv, s_eta[t]) : xv;
-                }
-                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-                xh_hi[t * TC_XP + pos] = hi;
-                xh_lo[t * TC_XP + pos] = __float2bfloat16_rn(v - __bfloat162float(hi));
-            }
-        }
-    }
-    for (int i = L + tid; i < Lp; i += TC_THREADS) {  // padding positions of the last k-step
-        list_ch[i] = -1;
-#pragma unroll
-        for (int t = 0; t < TP; ++t) {
-            xh_hi[t * TC_XP + i] = __float2bfloat16_rn(0.0f);
-            xh_lo[t * TC_XP + i] = __float2bfloat16_rn(0.0f);
-        }
-    }
-    __syncthreads();  // the activation chunk is dead: the rings reuse its space
+    if (!DENSE && tid < Lp - L) list_cl[L + tid] = TC_PAD;  // padding positions of the last k-step
+    __syncthreads();
 
     // ---- 4. per-warp cp.async ring over this warp's 64 columns + tensor cores
     const int nst = Lp / TC_KS;
-    const int col0 = slice * C::NS + warp * TC_WCOLS;
-    const __nv_bfloat16 *wt = static_cast<const __nv_bfloat16 *>(a.Wt);
-    const uint32_t wring = smem_u32(ring) + (uint32_t)(warp * C::STAGES * C::wstage);
-    auto issue = [&](int st) {
-        const uint32_t base = wring + (uint32_t)((st % C::STAGES) * C::wstage);
-#pragma unroll
-        for (int r = 0; r < (TC_KS * TC_WCOLS * 2 / 16) / 32; ++r) {
-            const int id = lane + 32 * r;
-            const int row = id >> 3, c16 = id & 7;
-            const int ch = list_ch[st * TC_KS + row];
-            const int col = col0 + 8 * c16;
-            const bool ok = ch >= 0 && col < n_out;
-            const void *src = ok ? (const void *)(wt + (size_t)ch * n_out + col) : (const void *)wt;
-            cp_async16(base + row * TC_WROWP + c16 * 16, src, ok ? 16u : 0u);  // 0 bytes: zero fill
-        }
-    };
     float acc[C::MT][C::NT][4];
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt)
@@ -699,13 +796,14 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
-#pragma unroll
-    for (int st = 0; st < C::STAGES - 1; ++st) {
-        if (st < nst) issue(st);
-        cp_async_commit();
-    }
+    if constexpr (!DENSE) issue_prologue(nst);
     const int g8 = lane >> 2, q4 = lane & 3;
     const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index, row within it
+    auto pack2 = [](const __nv_bfloat16 *row, int c0, int c1) {
+        const uint32_t lo = *reinterpret_cast<const uint16_t *>(row + c0);
+        const uint32_t hi = *reinterpret_cast<const uint16_t *>(row + c1);
+        return lo | (hi << 16);
+    };
     for (int st = 0; st < nst; ++st) {
         cp_async_wait<C::STAGES - 2>();
         __syncwarp();  // every lane's pieces of stage st have landed
@@ -713,17 +811,35 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         cp_async_commit();
         const uint32_t base = wring + (uint32_t)((st % C::STAGES) * C::wstage);
         const int pk = st * TC_KS;
+        // B fragments: kept values of token nt*8+g8 at list positions
+        // pk+2q4, +1 (b0) and pk+2q4+8, +9 (b1), gathered from the dense rows
+        // (DENSE: the positions are the channel offsets, pairs adjacent)
+        int2 ca = make_int2(pk + 2 * q4, pk + 2 * q4 + 1), cb = make_int2(pk + 2 * q4 + 8, pk + 2 * q4 + 9);
+        if constexpr (!DENSE) {
+            ca = *reinterpret_cast<const int2 *>(list_cl + pk + 2 * q4);
+            cb = *reinterpret_cast<const int2 *>(list_cl + pk + 2 * q4 + 8);
+        }
         uint32_t bh[C::NT][2], bl[C::NT][2];
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
             const int t = nt * 8 + g8;
+            bh[nt][0] = bh[nt][1] = bl[nt][0] = bl[nt][1] = 0u;
             if (t < TP) {
-                bh[nt][0] = *reinterpret_cast<const uint32_t *>(xh_hi + t * TC_XP + pk + 2 * q4);
-                bh[nt][1] = *reinterpret_cast<const uint32_t *>(xh_hi + t * TC_XP + pk + 2 * q4 + 8);
-                bl[nt][0] = *reinterpret_cast<const uint32_t *>(xh_lo + t * TC_XP + pk + 2 * q4);
-                bl[nt][1] = *reinterpret_cast<const uint32_t *>(xh_lo + t * TC_XP + pk + 2 * q4 + 8);
-            } else {
-                bh[nt][0] = bh[nt][1] = bl[nt][0] = bl[nt][1] = 0u;
+                if constexpr (DENSE) {
+                    bh[nt][0] = *reinterpret_cast<const uint32_t *>(xh + t * TC_XP + ca.x);
+                    bh[nt][1] = *reinterpret_cast<const uint32_t *>(xh + t * TC_XP + cb.x);
+                    if constexpr (LO) {
+                        bl[nt][0] = *reinterpret_cast<const uint32_t *>(xl + t * TC_XP + ca.x);
+                        bl[nt][1] = *reinterpret_cast<const uint32_t *>(xl + t * TC_XP + cb.x);
+                    }
+                } else {
+                    bh[nt][0] = pack2(xh + t * TC_XP, ca.x, ca.y);
+                    bh[nt][1] = pack2(xh + t * TC_XP, cb.x, cb.y);
+                    if constexpr (LO) {
+                        bl[nt][0] = pack2(xl + t * TC_XP, ca.x, ca.y);
+                        bl[nt][1] = pack2(xl + t * TC_XP, cb.x, cb.y);
+                    }
+                }
             }
         }
 #pragma unroll
@@ -734,14 +850,39 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
 #pragma unroll
             for (int nt = 0; nt < C::NT; ++nt) {
                 mma_16816(acc[mt][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-                mma_16816(acc[mt][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+                if constexpr (LO) mma_16816(acc[mt][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
             }
         }
     }
     cp_async_wait<0>();
-    __syncthreads();  // every warp done with its ring: the space becomes the reduction buffer
 
-    // ---- 5. fragments -> shared [token][column] -> y or split-K partials
+    // ---- 5. split-K partial sums straight from the fragments, layout
+    // [split][column][TP]: a lane holds tokens 2q4, 2q4+1 of columns o and o+8
+    const int k_splits = gridDim.y;
+    if (k_splits > 1) {
+        float *pp = a.partial + (size_t)split * n_out * TP;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < C::NT; ++nt) {
+                const int o = col0 + mt * 16 + g8;
+                const int t = nt * 8 + 2 * q4;
+                if constexpr (TP == 1) {
+                    if (q4 == 0) {
+                        if (o < n_out) pp[o] = acc[mt][nt][0];
+                        if (o + 8 < n_out) pp[o + 8] = acc[mt][nt][2];
+                    }
+                } else if (t < TP) {
+                    if (o < n_out)
+                        *reinterpret_cast<float2 *>(pp + (size_t)o * TP + t) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+                    if (o + 8 < n_out)
+                        *reinterpret_cast<float2 *>(pp + (size_t)(o + 8) * TP + t) =
+                            make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+                }
+            }
+        return;
+    }
+    __syncthreads();  // every warp done with its ring: the space becomes the output staging buffer
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
@@ -758,23 +899,16 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             }
         }
     __syncthreads();
-    const int k_splits = gridDim.y;
     const int ocol0 = slice * C::NS;
-    auto emit = [&](int t, int o, float v) {
+    for (int i = tid; i < T * C::NS; i += TC_THREADS) {
+        const int t = i / C::NS, c = i % C::NS, o = ocol0 + c;
+        if (o >= n_out) continue;
+        float v = red[t * C::NS + c];
         if (a.dpts) v = fmaf(s_eta[t], a.rowsum[o], v);
         if (a.out_bf16)
             static_cast<__nv_bfloat16 *>(a.y)[(size_t)t * n_out + o] = __float2bfloat16_rn(v);
         else
             static_cast<float *>(a.y)[(size_t)t * n_out + o] = v;
-    };
-    for (int i = tid; i < T * C::NS; i += TC_THREADS) {
-        const int t = i / C::NS, c = i % C::NS, o = ocol0 + c;
-        if (o >= n_out) continue;
-        const float v = red[t * C::NS + c];
-        if (k_splits > 1)
-            a.partial[((size_t)split * T + t) * n_out + o] = v;
-        else
-            emit(t, o, v);
     }
 }
 
@@ -789,14 +923,14 @@ static int vec_of(int tp, int bf16)
     return tp <= 8 ? 4 : 2;
 }
 
-static size_t tc_smem(int tp)
+static size_t tc_smem(int tp, bool lo)
 {
     switch (tp) {
-    case 1: return TcCfg<1>::smem;
-    case 2: return TcCfg<2>::smem;
-    case 4: return TcCfg<4>::smem;
-    case 8: return TcCfg<8>::smem;
-    default: return TcCfg<16>::smem;
+    case 1: return TcCfg<1>::smem(lo);
+    case 2: return TcCfg<2>::smem(lo);
+    case 4: return TcCfg<4>::smem(lo);
+    case 8: return TcCfg<8>::smem(lo);
+    default: return TcCfg<16>::smem(lo);
     }
 }
 
@@ -819,11 +953,11 @@ DecodePlan decode_plan(int T, int K, int n_out, int bf16)
     if (wps < 1) wps = 1;
     p.words_per_split = wps;
     p.k_splits = (nwords + wps - 1) / wps;
-    p.partial_bytes = p.k_splits > 1 ? (size_t)p.k_splits * T * n_out * sizeof(float) : 0;
+    p.partial_bytes = p.k_splits > 1 ? (size_t)p.k_splits * p.tpad * n_out * sizeof(float) : 0;
     p.counter_bytes = (size_t)p.n_slices * sizeof(unsigned);
     p.eta_bytes = (size_t)T * sizeof(float);
     if (p.tc) {
-        p.smem_bytes = tc_smem(p.tpad);
+        p.smem_bytes = tc_smem(p.tpad, true);
     } else {
         const int vec = vec_of(p.tpad, bf16);
         const int tpr = DEC_NS / vec, rg = DEC_THREADS / tpr;
@@ -871,42 +1005,61 @@ static void set_pdl(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr)
 // The tensor-core decode follows the select kernel (which wrote the keep
 // words and means) and, for several splits, is followed by the reduction;
 // both links are programmatic.
+// Expected share of channels kept by at least one of the T tokens, if each
+// token keeps a channel with probability f independently.
+static double expected_union(const DecodeArgs &a)
+{
+    double f = 1.0;
+    if (a.sel == AS_SEL_NM) f = (double)a.n / (double)a.m;
+    else if (a.sel == AS_SEL_TOPK) f = a.K > 0 ? (double)a.k_keep / (double)a.K : 0.0;
+    double miss = 1.0;
+    for (int t = 0; t < a.T; ++t) miss *= 1.0 - f;
+    return 1.0 - miss;
+}
+
+// DENSE streaming when the union is expected to reach 97 % of the channels.
+static bool decode_dense(const DecodeArgs &a, int tpad) { return !decode_fused(tpad, a.sel, a.K) && expected_union(a) >= 0.97; }
+
+template <int TP, bool FUSED, bool LO, bool DENSE>
+static cudaError_t launch_tc_one(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
+{
+    const size_t smem = TcCfg<TP>::smem(LO);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_slices, p.k_splits);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    set_pdl(cfg, attr);
+    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<TP, FUSED, LO, DENSE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k_decode_tc<TP, FUSED, LO, DENSE>, a, p.words_per_split);
+    return e;
+}
+
+template <int TP, bool LO>
+static cudaError_t launch_tc_k(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
+{
+    if constexpr (TP <= 2) {
+        if (decode_fused(TP, a.sel, a.K)) return launch_tc_one<TP, true, LO, false>(a, p, st);
+    }
+    if (decode_dense(a, TP)) return launch_tc_one<TP, false, LO, true>(a, p, st);
+    return launch_tc_one<TP, false, LO, false>(a, p, st);
+}
+
 template <int TP>
 static cudaError_t launch_tc(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
 {
-    const size_t smem = TcCfg<TP>::smem;
-    cudaError_t e;
-    bool fused = false;
-    if constexpr (TP <= 2) fused = decode_fused(TP, a.sel, a.K);
-    if (fused) {  // selection inside the decode kernel
-        if constexpr (TP <= 2) {
-            e = cudaFuncSetAttribute(k_decode_tc<TP, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            dim3 grid(p.n_slices, p.k_splits);
-            k_decode_tc<TP, true><<<grid, TC_THREADS, smem, st>>>(a, p.words_per_split);
-            e = cudaGetLastError();
-        }
-    } else {
-        e = cudaFuncSetAttribute(k_decode_tc<TP, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(p.n_slices, p.k_splits);
-        cfg.blockDim = dim3(TC_THREADS);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        set_pdl(cfg, attr);
-        e = cudaLaunchKernelEx(&cfg, k_decode_tc<TP, false>, a, p.words_per_split);
-    }
+    cudaError_t e = a.out_bf16 ? launch_tc_k<TP, false>(a, p, st) : launch_tc_k<TP, true>(a, p, st);
     if (e != cudaSuccess || p.k_splits == 1) return e;
     cudaLaunchConfig_t rc = {};
-    const int n4 = a.T * a.n_out / 4;
-    rc.gridDim = dim3((n4 + 255) / 256);
+    const int nthreads = a.n_out * (TP / RedVec<TP>::VW);
+    rc.gridDim = dim3((nthreads + 255) / 256);
     rc.blockDim = dim3(256);
     rc.stream = st;
     cudaLaunchAttribute rattr[1];
     set_pdl(rc, rattr);
-    return cudaLaunchKernelEx(&rc, k_decode_reduce, (const float *)a.partial, p.k_splits, a.T, a.n_out,
+    return cudaLaunchKernelEx(&rc, k_decode_reduce<TP>, (const float *)a.partial, p.k_splits, a.T, a.n_out,
                               a.dpts ? (const float *)a.eta_in : (const float *)nullptr, a.rowsum, a.y, a.out_bf16);
 }
 

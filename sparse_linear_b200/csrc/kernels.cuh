@@ -40,7 +40,7 @@ struct DecodeArgs {
     const void *Wt;
     int bf16;
     int T, K, n_out;
-    int score, sel, n, m, dpts;
+    int score, sel, n, m, k_keep, dpts;
     const float *g;
     const float *rowsum;
     const uint32_t *mask_in;  // precomputed selection (top-k / all), or nullptr for fused N:M

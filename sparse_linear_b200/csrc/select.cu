@@ -401,6 +401,10 @@ constexpr int SELD_ROWREG = 8;               // row loads held in registers per 
 __global__ void __launch_bounds__(SELD_THREADS) k_select_nm_decode(SelectArgs a)
 {
     using TX = __nv_bfloat16;  // 16-byte row loads hold 8 channels
+    // launched programmatically: the previous kernel in the stream may have
+    // written x.  The decode kernel after this one loads x before its own
+    // wait, so this kernel lets it start only once that wait has returned.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ double red[SELD_THREADS / 32];
     const int t = blockIdx.x, chunk = blockIdx.y;
@@ -464,8 +468,16 @@ cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st)
 {
     dim3 grid(a.T, (a.K + SELD_CHUNK - 1) / SELD_CHUNK);
     if (!a.bf16) return cudaErrorInvalidValue;  // the float32 decode selects inside its kernel
-    k_select_nm_decode<<<grid, SELD_THREADS, 0, st>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(SELD_THREADS);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_select_nm_decode, a);
 }
 
 }  // namespace as
