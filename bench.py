@@ -510,7 +510,8 @@ def main():
                      "frac": d["achieved_gbs"] / peak, "traffic": traffic,
                      "peak_source": f"{pk_src} copy bandwidth (MEASURED_PEAKS.json)" if pk_src == "measured"
                      else "fallback 6650 GB/s",
-                     "kernel": "k_decode", "bytes_per_launch": d["bytes_per_launch"],
+                     "kernel": "k_decode_tc (timed per whole decode call: select, decode and split-K "
+                               "reduction kernels)", "bytes_per_launch": d["bytes_per_launch"],
                      "per_T": {str(T): v for T, v in d["per_t"].items()}},
         "e2e": {"value": d["e2e"], "unit": "tokens/s", "h2d_bytes_per_step": d["h2d"],
                 "d2h_bytes_per_step": d["d2h"]},
