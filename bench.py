@@ -413,6 +413,20 @@ def run_case(args):
         L = SparseLinear(W.to(dev), cfg, alpha=0.5)
         xd = x[:args.T].contiguous().to(dev)
         fn = lambda: L.decode(xd)  # noqa: E731
+    elif args.case in ("select24", "selectclact"):
+        if args.case == "select24":
+            _, x, W = synth.prefill_sqrelu(T=args.T)
+            cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4)
+        else:
+            W = synth.prefill_clact_weight()
+            x = synth.prefill_clact_batch(0)[:args.T].contiguous()
+            cfg = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)
+        L = SparseLinear(W.to(dev), cfg, keep_wt=False)
+        xd = x.to(dev)
+        bufs = L.select_buffers(args.T)
+        run = torch.zeros(args.T, dtype=torch.float32, device=dev)
+        L.select(xd, bufs, running_var=run if cfg.var else None, first_batch=True)
+        fn = lambda: L.select(xd, bufs, running_var=run if cfg.var else None)  # noqa: E731
     elif args.case in ("sqrelu24", "dense"):
         _, x, W = synth.prefill_sqrelu(T=args.T)
         cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4) if args.case == "sqrelu24" else \
@@ -459,7 +473,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--case", default=None, help="profiling case: decode | sqrelu24 | dense")
+    ap.add_argument("--case", default=None,
+                    help="profiling case: decode | sqrelu24 | dense | select24 | selectclact")
     ap.add_argument("--T", type=int, default=1)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

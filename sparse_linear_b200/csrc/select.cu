@@ -14,6 +14,9 @@
 // warp tree, then the eight warps in order), the score is one float32
 // subtraction and one float32 multiply, and the decision compares float32
 // bit patterns (scores are >= 0) with ties to the lower index.
+#include <algorithm>
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "select_util.cuh"
@@ -70,6 +73,16 @@ __device__ __forceinline__ uint8_t *meta_byte(uint32_t *meta, int t, int c0, int
     const int lane = 16 * (p >> 4) + 8 * (q >> 4) + (p & 7);
     const int byte = 2 * ((p & 15) >> 3) + ((q & 15) >> 3);
     return reinterpret_cast<uint8_t *>(meta) + (size_t)tile * 2048 + lane * 16 + j * 4 + byte;
+}
+
+// v[base + i] for i in 0..3 without a dynamic register index.
+__device__ __forceinline__ float pick4(const float (&v)[8], int base, int i)
+{
+    float r = v[base];
+    r = i == 1 ? v[base + 1] : r;
+    r = i == 2 ? v[base + 2] : r;
+    r = i == 3 ? v[base + 3] : r;
+    return r;
 }
 
 template <typename TX>
@@ -279,8 +292,8 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
                         uint32_t b = (keep >> (4 * h)) & 0xFu;
                         int i0 = __ffs(b) - 1;
                         int i1 = 31 - __clz(b);
-                        cv[2 * h] = xh[4 * h + i0];
-                        cv[2 * h + 1] = xh[4 * h + i1];
+                        cv[2 * h] = pick4(xh, 4 * h, i0);
+                        cv[2 * h + 1] = pick4(xh, 4 * h, i1);
                         nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
                     }
                     __nv_bfloat162 p0 = __floats2bfloat162_rn(cv[0], cv[1]);
@@ -307,6 +320,173 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
             if (a.var_dense) a.var_dense[t] = (float)vd;
             if (a.var_kept) a.var_kept[t] = (float)vk;
             if (a.nu) a.nu[t] = (float)sqrt(run / (vk + (double)a.eps));
+        }
+    }
+}
+
+// ---------------------------------------------------------------- N:M rows
+// Prefill N:M (or keep-all) selection, persistent: a CTA takes rows
+// blockIdx.x, blockIdx.x + gridDim.x, ...  Each row arrives in shared
+// memory by 1-D bulk copies into a ring of SR_BUFS row buffers (the next
+// rows are in flight while one is scored), the channel factors once per
+// CTA.  Statistics, score, selection and outputs are those of k_select.
+constexpr int SR_THREADS = 256;
+constexpr int SR_BUFS = 3;
+constexpr uint32_t SR_PIECE = 16384;  // bytes per bulk copy instruction
+
+__device__ __forceinline__ void bulk_load_pieces(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    for (uint32_t o = 0; o < bytes; o += SR_PIECE)
+        bulk_load(static_cast<unsigned char *>(dst) + o, static_cast<const unsigned char *>(src) + o,
+                  min(SR_PIECE, bytes - o), bar);
+}
+
+// M: block size fixed at compile time (0: from the arguments); COMPACT: the
+// 2:4 outputs (compact operand + positions; no masked copy, no VAR).
+template <typename TX, int M, bool COMPACT>
+__global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
+{
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ double red[2][SR_THREADS / 32];
+    __shared__ __align__(8) uint64_t bars[SR_BUFS + 1];
+    const int K = a.K, T = a.T, tid = threadIdx.x, lane = tid & 31;
+    const int ngroups = K >> 3, ntiles = (ngroups + SR_THREADS - 1) / SR_THREADS, kt = (K + 127) >> 7;
+    const int Tpad = a.meta24 ? (T + 127) / 128 * 128 : T;
+    const bool has_f = a.f != nullptr;
+    const uint32_t fbytes = has_f ? (uint32_t)K * 4u : 0u, rowbytes = (uint32_t)K * (uint32_t)sizeof(TX);
+    float *sf = reinterpret_cast<float *>(sm);
+    TX *rows = reinterpret_cast<TX *>(sm + fbytes);
+    const TX *x = static_cast<const TX *>(a.x);
+    const int words = (K + 31) >> 5;
+
+    if (tid == 0) {
+        for (int b = 0; b <= SR_BUFS; ++b) mbar_init(&bars[b], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        if (has_f) {
+            mbar_arrive_expect_tx(&bars[SR_BUFS], fbytes);
+            bulk_load_pieces(sf, a.f, fbytes, &bars[SR_BUFS]);
+        }
+        for (int b = 0; b < SR_BUFS; ++b) {
+            const int t = blockIdx.x + b * gridDim.x;
+            if (t < T) {
+                mbar_arrive_expect_tx(&bars[b], rowbytes);
+                bulk_load_pieces(rows + (size_t)b * K, x + (size_t)t * K, rowbytes, &bars[b]);
+            }
+        }
+    }
+    if (has_f && !mbar_wait(&bars[SR_BUFS], 0)) return;
+
+    int it = 0;
+    for (int t = blockIdx.x; t < Tpad; t += gridDim.x, ++it) {
+        if (t >= T) {  // padding rows of the 2:4 metadata tiles
+            for (int g = tid; g < kt * 16; g += SR_THREADS) *meta_byte(a.meta24, t, 8 * g, kt) = 0x44;
+            continue;
+        }
+        const int buf = it % SR_BUFS;
+        if (!mbar_wait(&bars[buf], (uint32_t)(it / SR_BUFS) & 1u)) return;
+        const TX *xr = rows + (size_t)buf * K;
+
+        // ---- row statistics: sum x, sum x^2 (float64)
+        double sx = 0.0, sxx = 0.0;
+        if (a.dpts || a.var) {
+            for (int g = tid; g < ngroups; g += SR_THREADS) {
+                float v[8];
+                load8(xr + 8 * g, v);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    sx += (double)v[e];
+                    sxx += (double)v[e] * (double)v[e];
+                }
+            }
+            block_sum2<SR_THREADS>(sx, sxx, red);
+        }
+        const float eta = a.dpts ? (float)(sx / (double)K) : 0.0f;
+        if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
+
+        // ---- decisions and outputs, 2048 channels (8 per thread) per tile
+        double skm = 0.0, skmm = 0.0;
+        for (int tile = 0; tile < ntiles; ++tile) {
+            const int g = tile * SR_THREADS + tid, c0 = 8 * g;
+            const bool act = g < ngroups;
+            float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, fv[8] = {1, 1, 1, 1, 1, 1, 1, 1}, xh[8], sc[8];
+            if (act) {
+                load8(xr + c0, v);
+                if (has_f) load8f(sf + c0, fv);
+            }
+            score8v(v, a.dpts, eta, act && has_f, fv, xh, sc);
+            uint32_t keep;
+            if constexpr (COMPACT) keep = keep_2of4(sc);
+            else if constexpr (M == 0) keep = a.sel == AS_SEL_NM ? nm_keep_dispatch(sc, lane, a.n, a.m) : 0xFFu;
+            else if constexpr (M >= 8) keep = nm_keep_sorted<M>(sc, lane, a.n);
+            else keep = nm_keep<M>(sc, lane, a.n);
+            if (act) {
+                if (a.bitmask) {
+                    uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
+                    bm[g] = (uint8_t)keep;
+                    if (g == ngroups - 1)
+                        for (int b = ngroups; b < words * 4; ++b) bm[b] = 0;
+                }
+                if constexpr (!COMPACT) {
+                    float km[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) km[e] = ((keep >> e) & 1u) ? xh[e] : 0.0f;
+                    if (a.var) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            skm += (double)km[e];
+                            skmm += (double)km[e] * (double)km[e];
+                        }
+                    }
+                    if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
+                }
+                if constexpr (COMPACT) {
+                    float cv[4];
+                    uint32_t nib[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t b = (keep >> (4 * h)) & 0xFu;
+                        const int i0 = __ffs(b) - 1, i1 = 31 - __clz(b);
+                        cv[2 * h] = pick4(xh, 4 * h, i0);
+                        cv[2 * h + 1] = pick4(xh, 4 * h, i1);
+                        nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
+                    }
+                    const __nv_bfloat162 p0 = __floats2bfloat162_rn(cv[0], cv[1]);
+                    const __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
+                    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) =
+                        make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
+                    if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
+                }
+            }
+        }
+        if (a.meta24 && tid < 16 * kt - ngroups)  // channel padding of the last 128-channel tile
+            *meta_byte(a.meta24, t, 8 * (ngroups + tid), kt) = 0x44;
+
+        // ---- VAR: variances, running average, scale
+        if (!COMPACT && a.var) {
+            block_sum2<SR_THREADS>(skm, skmm, red);
+            if (tid == 0) {
+                const double Kd = (double)K;
+                const double vd = (sxx - sx * sx / Kd) / (Kd - 1.0);
+                const double vk = (skmm - skm * skm / Kd) / (Kd - 1.0);
+                const double run =
+                    a.first ? vd : (double)a.mom * (double)a.running_var[t] + (1.0 - (double)a.mom) * vd;
+                a.running_var[t] = (float)run;
+                if (a.var_dense) a.var_dense[t] = (float)vd;
+                if (a.var_kept) a.var_kept[t] = (float)vk;
+                if (a.nu) a.nu[t] = (float)sqrt(run / (vk + (double)a.eps));
+            }
+        }
+        // ---- the buffer is free: the row SR_BUFS iterations ahead goes into it
+        __syncthreads();
+        if (tid == 0) {
+            const int tn = t + SR_BUFS * gridDim.x;
+            if (tn < T) {
+                mbar_arrive_expect_tx(&bars[buf], rowbytes);
+                bulk_load_pieces(rows + (size_t)buf * K, x + (size_t)tn * K, rowbytes, &bars[buf]);
+            }
         }
     }
 }
@@ -377,8 +557,54 @@ static cudaError_t launch_select_t(const SelectArgs &a, size_t smem, int grid, c
     return cudaGetLastError();
 }
 
+template <typename TX, int M, bool COMPACT>
+static cudaError_t launch_select_rows_t(const SelectArgs &a, cudaStream_t st)
+{
+    const size_t smem = (a.f ? (size_t)a.K * 4 : 0) + (size_t)SR_BUFS * a.K * sizeof(TX);
+    cudaError_t e = cudaFuncSetAttribute(k_select_rows<TX, M, COMPACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0, dev = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_select_rows<TX, M, COMPACT>, SR_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int rows = a.meta24 ? (a.T + 127) / 128 * 128 : a.T;
+    const int grid = std::min(rows, per_sm * sms);
+    k_select_rows<TX, M, COMPACT><<<grid, SR_THREADS, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename TX>
+static cudaError_t launch_select_rows(const SelectArgs &a, cudaStream_t st)
+{
+    if (a.sel == AS_SEL_NM) {
+        if (a.x_compact) {
+            if constexpr (std::is_same<TX, __nv_bfloat16>::value) return launch_select_rows_t<TX, 4, true>(a, st);
+        }
+        switch (a.m) {
+        case 8: return launch_select_rows_t<TX, 8, false>(a, st);
+        case 16: return launch_select_rows_t<TX, 16, false>(a, st);
+        case 32: return launch_select_rows_t<TX, 32, false>(a, st);
+        default: break;
+        }
+    }
+    return launch_select_rows_t<TX, 0, false>(a, st);
+}
+
+// Shared memory the row kernel needs (channel factors + row ring); the
+// per-token kernel takes over beyond it.
+static bool select_rows_fits(const SelectArgs &a)
+{
+    const size_t elem = a.bf16 ? 2 : 4;
+    return (a.f ? (size_t)a.K * 4 : 0) + (size_t)SR_BUFS * a.K * elem <= 200 * 1024;
+}
+
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st, int wide)
 {
+    if (!wide && a.sel != AS_SEL_TOPK && select_rows_fits(a))
+        return a.bf16 ? launch_select_rows<__nv_bfloat16>(a, st) : launch_select_rows<float>(a, st);
     const bool topk = a.sel == AS_SEL_TOPK && a.k_keep > 0 && a.k_keep < a.K;
     const size_t smem = topk ? (size_t)a.K * sizeof(uint32_t) : 0;
     const int grid = a.meta24 ? ((a.T + 127) / 128) * 128 : a.T;

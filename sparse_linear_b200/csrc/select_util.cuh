@@ -111,15 +111,111 @@ __device__ __forceinline__ uint32_t nm_keep(const float (&s)[8], int lane, int n
     return keep;
 }
 
+// The same decision through the block's n-th largest score theta: keep
+// every score > theta, and of the scores == theta the lowest-indexed ones
+// until n are kept.  That is exactly "rank < n" for the order above (higher
+// score first, equal scores by lower index).  theta comes from a bitonic
+// sort of the M scores (descending) across the M/8 lanes of the block.
+// Requires M >= 8; all 32 lanes must call.
+template <int M>
+__device__ __forceinline__ uint32_t nm_keep_sorted(const float (&s)[8], int lane, int n)
+{
+    constexpr int G = M / 8;  // lanes per block
+    const int q = lane & (G - 1);
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = s[e];
+    // element k = 8 q + e; compare-exchange partners k ^ d, descending where
+    // (k & size) == 0
+#pragma unroll
+    for (int size = 2; size <= M; size <<= 1) {
+#pragma unroll
+        for (int d = size >> 1; d > 0; d >>= 1) {
+            if (d >= 8) {
+                const int ld = d >> 3;  // partner lane distance
+                const bool lower = (q & ld) == 0;
+                const bool desc = ((8 * q) & size) == 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float p = __shfl_xor_sync(0xffffffffu, v[e], ld);
+                    v[e] = (lower == desc) ? fmaxf(v[e], p) : fminf(v[e], p);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int pe = e ^ d;
+                    if (pe > e) {
+                        const bool desc = size >= 8 ? (((8 * q) & size) == 0) : ((e & size) == 0);
+                        const float hi = fmaxf(v[e], v[pe]), lo = fminf(v[e], v[pe]);
+                        v[e] = desc ? hi : lo;
+                        v[pe] = desc ? lo : hi;
+                    }
+                }
+            }
+        }
+    }
+    // theta = sorted[n - 1]: slot (n-1) % 8 of lane (n-1) / 8 of the block
+    const int slot = (n - 1) & 7;
+    float th = v[0];
+#pragma unroll
+    for (int e = 1; e < 8; ++e) th = slot == e ? v[e] : th;
+    th = __shfl_sync(0xffffffffu, th, (lane & ~(G - 1)) + ((n - 1) >> 3));
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        gt |= (uint32_t)(s[e] > th) << e;
+        eq |= (uint32_t)(s[e] == th) << e;
+    }
+    const int neq = __popc(eq);
+    int ngt = __popc(gt), inc = neq;
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) {
+        const int up = __shfl_up_sync(0xffffffffu, inc, o);
+        if (q >= o) inc += up;
+    }
+    int before = inc - neq;  // equal scores in the lower lanes of the block
+    const int room = n - ngt;  // equal scores that still fit
+    uint32_t keep = gt;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        if ((eq >> e) & 1u) {
+            keep |= (uint32_t)(before < room) << e;
+            ++before;
+        }
+    }
+    return keep;
+}
+
+// 2:4 blocks inside the lane: one comparison per pair of the block decides
+// for both (j ahead of i: s_j > s_i, or s_j == s_i and j < i).
+__device__ __forceinline__ uint32_t keep_2of4(const float (&s)[8])
+{
+    uint32_t keep = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float a = s[4 * h], b = s[4 * h + 1], c = s[4 * h + 2], d = s[4 * h + 3];
+        const int ab = b > a, ac = c > a, ad = d > a, bc = c > b, bd = d > b, cd = d > c;
+        const int ra = ab + ac + ad;
+        const int rb = (1 - ab) + bc + bd;
+        const int rc = (1 - ac) + (1 - bc) + cd;
+        const int rd = (1 - ad) + (1 - bd) + (1 - cd);
+        keep |= ((uint32_t)(ra < 2) | ((uint32_t)(rb < 2) << 1) | ((uint32_t)(rc < 2) << 2) | ((uint32_t)(rd < 2) << 3))
+                << (4 * h);
+    }
+    return keep;
+}
+
 __device__ __forceinline__ uint32_t nm_keep_dispatch(const float (&s)[8], int lane, int n, int m)
 {
     switch (m) {
     case 1: return nm_keep<1>(s, lane, n);
     case 2: return nm_keep<2>(s, lane, n);
-    case 4: return nm_keep<4>(s, lane, n);
-    case 8: return nm_keep<8>(s, lane, n);
-    case 16: return nm_keep<16>(s, lane, n);
-    default: return nm_keep<32>(s, lane, n);
+    case 4: return n == 2 ? keep_2of4(s) : nm_keep<4>(s, lane, n);
+    case 8: return nm_keep_sorted<8>(s, lane, n);
+    case 16: return nm_keep_sorted<16>(s, lane, n);
+    default: return nm_keep_sorted<32>(s, lane, n);
     }
 }
 
