@@ -243,6 +243,16 @@ size_t as_meta24_words(int T, int K);
  * the stream itself failed. */
 as_status as_stream_status(cudaStream_t stream);
 
+/* Self-test of the failure path: launches on `stream` one small kernel
+ * whose bounded wait (`polls` polls, 1 .. 1<<20) is on an mbarrier that
+ * nothing signals.  The wait runs out and records AS_ERR_TIMEOUT, and the
+ * kernel returns normally, so the context stays usable.  The next
+ * as_stream_status() reports AS_ERR_TIMEOUT and clears it.  The probe is
+ * the same bounded-wait code every library kernel uses.  Returns
+ * AS_ERR_INVALID_ARG for `polls` out of range, AS_ERR_CUDA if the launch
+ * fails, AS_OK otherwise. */
+as_status as_probe_timeout(unsigned polls, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char *as_status_string(as_status s);
 

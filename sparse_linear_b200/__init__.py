@@ -37,7 +37,7 @@ AS_MAX_DECODE_T = 16
 EXPORTS = [
     "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
-    "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches",
+    "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches", "as_probe_timeout",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -70,6 +70,7 @@ _sig = {
     "as_meta24_words": ([_I, _I], _S),
     "as_decode_launches": ([_I, _I, _I, _I, ctypes.POINTER(as_config)], _I),
     "as_stream_status": ([_P], _I),
+    "as_probe_timeout": ([ctypes.c_uint, _P], _I),
     "as_status_string": ([_I], ctypes.c_char_p),
     "as_abi_version": ([], _I),
 }
@@ -203,3 +204,8 @@ def as_linear_prefill(sel: as_select_out, W, T: int, cfg: as_config, y, rowsum=N
 
 def as_stream_status(stream=None) -> int:
     return _lib.as_stream_status(_stream(stream))
+
+
+def as_probe_timeout(polls: int = 1000, stream=None) -> None:
+    """Runs the failure-path self-test kernel (a bounded wait that runs out)."""
+    _check(_lib.as_probe_timeout(int(polls), _stream(stream)), "as_probe_timeout")

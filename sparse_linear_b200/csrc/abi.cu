@@ -320,6 +320,27 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
     return n + decode_launch_count(a, plan);
 }
 
+namespace {
+// An mbarrier that nothing arrives on: the bounded wait runs out.
+__global__ void k_probe_timeout(unsigned polls)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, polls);
+}
+}  // namespace
+
+as_status as_probe_timeout(unsigned polls, cudaStream_t stream)
+{
+    if (polls < 1 || polls > (1u << 20)) return AS_ERR_INVALID_ARG;
+    k_probe_timeout<<<1, 32, 0, stream>>>(polls);
+    return cuda_status(cudaGetLastError());
+}
+
 as_status as_stream_status(cudaStream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(stream);

@@ -78,10 +78,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false (and records AS_ERR_TIMEOUT) if it does not within AS_SPIN_LIMIT polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+// false (and records AS_ERR_TIMEOUT) if it does not within `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = AS_SPIN_LIMIT)
 {
-    for (uint32_t i = 0; i < AS_SPIN_LIMIT; ++i)
+    for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     record_status(AS_ERR_TIMEOUT);
     return false;

@@ -135,3 +135,9 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         lib.as_linear_decode(x, x, lib.config(), x)
+
+
+def test_timeout_probe_validates_polls(lib):
+    # out-of-range poll counts are refused on the host, before any launch
+    for polls in (0, (1 << 20) + 1):
+        assert lib._lib.as_probe_timeout(polls, None) == lib.AS_ERR_INVALID_ARG
