@@ -406,11 +406,60 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
         const float eta = a.dpts ? (float)(sx / (double)K) : 0.0f;
         if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
 
-        // ---- decisions and outputs, 2048 channels (8 per thread) per tile
+        // ---- decisions and outputs, 8 channels per thread per tile.  The
+        // thread's position-metadata byte moves by a fixed stride per tile
+        // (its channel offset within a 32-channel block is the same in
+        // every tile).
+        uint8_t *mrow = nullptr;
+        if constexpr (COMPACT) mrow = meta_byte(a.meta24, t, 8 * tid, kt);
+        constexpr size_t mstride = (size_t)(8 * SR_THREADS / 128) * 2048;  // bytes per tile
+        const bool plain = !a.dpts && !has_f;  // score = |x|
         double skm = 0.0, skmm = 0.0;
         for (int tile = 0; tile < ntiles; ++tile) {
             const int g = tile * SR_THREADS + tid, c0 = 8 * g;
             const bool act = g < ngroups;
+            if constexpr (COMPACT) {
+                if (plain) {
+                    // score = |x|: compare the bf16 magnitude bits as integers and
+                    // move the kept values as raw 16-bit halves
+                    if (act) {
+                        const uint4 r = *reinterpret_cast<const uint4 *>(xr + c0);
+                        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+                        uint32_t hw[8], mk[8];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            hw[2 * i] = w[i] & 0xFFFFu;
+                            hw[2 * i + 1] = w[i] >> 16;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mk[e] = hw[e] & 0x7FFFu;
+                        const uint32_t keep = keep_2of4(mk);
+                        uint32_t out[2], nib[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            int i0, i1;
+                            pos_2of4((keep >> (4 * h)) & 0xFu, i0, i1);
+                            uint32_t v0 = hw[4 * h], v1 = hw[4 * h + 1];
+                            v0 = i0 == 1 ? hw[4 * h + 1] : v0;
+                            v0 = i0 == 2 ? hw[4 * h + 2] : v0;
+                            v1 = i1 == 2 ? hw[4 * h + 2] : v1;
+                            v1 = i1 == 3 ? hw[4 * h + 3] : v1;
+                            out[h] = v0 | (v1 << 16);
+                            nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
+                        }
+                        if (a.bitmask) {
+                            uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
+                            bm[g] = (uint8_t)keep;
+                            if (g == ngroups - 1)
+                                for (int b = ngroups; b < words * 4; ++b) bm[b] = 0;
+                        }
+                        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) +
+                                                   c0 / 2) = make_uint2(out[0], out[1]);
+                        mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
+                    }
+                    continue;
+                }
+            }
             float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, fv[8] = {1, 1, 1, 1, 1, 1, 1, 1}, xh[8], sc[8];
             if (act) {
                 load8(xr + c0, v);
@@ -447,8 +496,8 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                     uint32_t nib[2];
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint32_t b = (keep >> (4 * h)) & 0xFu;
-                        const int i0 = __ffs(b) - 1, i1 = 31 - __clz(b);
+                        int i0, i1;
+                        pos_2of4((keep >> (4 * h)) & 0xFu, i0, i1);
                         cv[2 * h] = pick4(xh, 4 * h, i0);
                         cv[2 * h + 1] = pick4(xh, 4 * h, i1);
                         nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
@@ -457,7 +506,7 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                     const __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
                     *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) =
                         make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
-                    if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
+                    mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
                 }
             }
         }

@@ -189,8 +189,10 @@ __device__ __forceinline__ uint32_t nm_keep_sorted(const float (&s)[8], int lane
 }
 
 // 2:4 blocks inside the lane: one comparison per pair of the block decides
-// for both (j ahead of i: s_j > s_i, or s_j == s_i and j < i).
-__device__ __forceinline__ uint32_t keep_2of4(const float (&s)[8])
+// for both (j ahead of i: s_j > s_i, or s_j == s_i and j < i).  S is float
+// (scores) or uint32_t (bf16 magnitude bits, which order like the values).
+template <typename S>
+__device__ __forceinline__ uint32_t keep_2of4(const S (&s)[8])
 {
     uint32_t keep = 0;
 #pragma unroll
@@ -205,6 +207,14 @@ __device__ __forceinline__ uint32_t keep_2of4(const float (&s)[8])
                 << (4 * h);
     }
     return keep;
+}
+
+// Positions of the two kept channels of a 2:4 block from its 4-bit keep
+// mask (exactly two bits set), without bit-scan instructions.
+__device__ __forceinline__ void pos_2of4(uint32_t b, int &i0, int &i1)
+{
+    i0 = (b & 1u) ? 0 : ((b & 2u) ? 1 : 2);
+    i1 = (b & 8u) ? 3 : ((b & 4u) ? 2 : 1);
 }
 
 __device__ __forceinline__ uint32_t nm_keep_dispatch(const float (&s)[8], int lane, int n, int m)
