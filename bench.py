@@ -399,6 +399,77 @@ def oracle_decode_sample(budget_s: float):
     return tokens / el, threads, f"{reps} oracle decode steps (T=1,8,16 of the down-projection), {el:.1f} s"
 
 
+def bench_block(sl, dev, reps=200):
+    """The seven layers of a Llama3.1-8B decoder block at one token: per-layer
+    exact top-k (keep fraction and weight-aware exponent seeded per layer),
+    bf16.  The block's weights (436 MB) exceed the L2, so one copy suffices.
+    One graph holds the seven decode calls; returns per-block time and the
+    kept weight bytes it streams."""
+    from sparse_linear_b200.layer import SparseLinear
+    blk = synth.decode_block()
+    layers, calls = [], []
+    kept_bytes = 0
+    stream = torch.cuda.Stream()
+    for ly in blk["layers"]:
+        K, n_out = ly["k"], ly["n_out"]
+        kk = int(math.floor(ly["keep_frac"] * K + 0.5))
+        cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_TOPK, k_keep=kk, out_dtype=sl.AS_BF16)
+        L = SparseLinear(ly["W"].to(dev), cfg, alpha=ly["alpha"], keep_wt=True)
+        x = blk["x"][ly["x_key"]].to(dev)
+        y = torch.empty(1, n_out, dtype=torch.bfloat16, device=dev)
+        layers.append((L, x, y))
+        kept_bytes += kk * n_out * 2 + K * 2 + n_out * 2
+    def run():
+        for L, x, y in layers:
+            L.decode(x, y=y, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            run()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        for _ in range(5):
+            g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize()
+    assert sl.as_stream_status(stream) == sl.AS_OK
+    t = s.elapsed_time(e) / 1e3 / reps
+    return dict(us_per_block=t * 1e6, kept_bytes=kept_bytes, gbs=kept_bytes / t / 1e9,
+                block_tokens_per_s=1.0 / t, launches_per_block=sum(
+                    sl.as_decode_launches(1, L.K, L.n_out, sl.AS_BF16, L.cfg) for L, _, _ in layers))
+
+
+def bench_tiny(sl, dev, reps=500):
+    """The tiny float32 layer (x [4, 256], W [512, 256], 2:4 by magnitude):
+    latency of one decode call, graph-replayed."""
+    from sparse_linear_b200.layer import SparseLinear
+    x, W = synth.tiny_layer()
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, out_dtype=sl.AS_F32)
+    L = SparseLinear(W.to(dev), cfg)
+    xd = x.to(dev)
+    y = torch.empty(x.shape[0], W.shape[0], dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            L.decode(xd, y=y, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            L.decode(xd, y=y, stream=stream)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return dict(us_per_call=s.elapsed_time(e) / reps * 1e3)
+
+
 # ---------------------------------------------------------------- profiling cases
 def run_case(args):
     """A few eager launches of one operation (the small commands the ncu
@@ -498,6 +569,9 @@ def main():
     prefill = None
     if not args.no_prefill and rank == 0:
         prefill = bench_prefill(sl, dev, pk)
+    extra = None
+    if not args.no_prefill and rank == 0:
+        extra = {"decode_block_T1": bench_block(sl, dev), "tiny_fp32_decode": bench_tiny(sl, dev)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         tps, threads, sample = oracle_decode_sample(budget_s=15.0)
@@ -536,6 +610,8 @@ def main():
     }
     if prefill is not None:
         line["prefill"] = prefill
+    if extra is not None:
+        line["configs_extra"] = extra
     print(json.dumps(line), flush=True)
 
 
