@@ -319,6 +319,19 @@ __device__ __forceinline__ void mma_sp_bf16_pair(uint32_t d_tmem, uint64_t a_des
         : "memory");
 }
 
+// Dense MMA over a CTA pair: M = 256 (128 rows of A in each CTA), B's N split
+// between the CTAs, D in each CTA's tensor memory (its 128 rows).
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Each CTA of the pair: 128 rows x 16 bytes of its shared memory -> its TMEM.
 __device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t s_desc)
 {

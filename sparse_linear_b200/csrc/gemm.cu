@@ -480,6 +480,192 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
+// -------------------------------------------------- dense, CTA pair (2 SMs)
+// The masked dense contraction on a CTA pair: 256 x 256 output tile per pair
+// (tcgen05.mma.cta_group::2.kind::f16, M = 256, N = 256, K = 16 per
+// instruction).  Each CTA stages its own 128 rows of A and half (128 rows) of
+// the weight tile per 64-wide K block; the leader issues the MMAs.  Without
+// 2:4 positions two 256-column accumulators fit in tensor memory, so the
+// epilogue of one tile overlaps the main loop of the next.
+constexpr int DP_STAGES = 6;
+constexpr int DP_A_BYTES = 128 * 64 * 2;
+constexpr int DP_B_BYTES = 128 * 64 * 2;
+constexpr int DP_STAGE_BYTES = DP_A_BYTES + DP_B_BYTES;
+
+constexpr size_t dense_pair_smem_bytes() { return 1024 + (size_t)DP_STAGES * DP_STAGE_BYTES + 256; }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
+    k_gemm_dense_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p)
+{
+    constexpr int S = DP_STAGES;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~uintptr_t(1023));
+    unsigned char *sA = smem;
+    unsigned char *sB = sA + S * DP_A_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + S * DP_B_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 2;
+    uint64_t *drain = bars + 2 * S + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int num_tiles = p.m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
+            mbar_init(&empty[s], 1);  // one commit from the leader's MMA thread
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 16);  // 8 epilogue warps in each CTA (the leader's copy is used)
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs initialised before either uses the other's
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = pair; tile < num_tiles && !*(volatile int *)abort_flag; tile += npairs) {
+                int mt, nt;
+                tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
+                const int arow = mt * PAIR_BM + 128 * (int)rank;
+                const int brow = nt * PAIR_BN + 128 * (int)rank;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * DP_STAGE_BYTES);
+                    const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
+                    tma_load_2d_pair(sA + stage * DP_A_BYTES, &tmA, bar, kb * 64, arow);
+                    tma_load_2d_pair(sB + stage * DP_B_BYTES, &tmB, bar, kb * 64, brow);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(PAIR_BM, PAIR_BN, false);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int tile = pair; tile < num_tiles && !*(volatile int *)abort_flag; tile += npairs, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * PAIR_BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t a_desc = sdesc_kmajor_sw128(smem_u32(sA + stage * DP_A_BYTES));
+                    const uint64_t b_desc = sdesc_kmajor_sw128(smem_u32(sB + stage * DP_B_BYTES));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mma_bf16_pair(d_tmem, a_desc + (uint64_t)((32 * j) >> 4), b_desc + (uint64_t)((32 * j) >> 4),
+                                      idesc, (kb | j) != 0);
+                    tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) { *(volatile int *)abort_flag = 1; break; }
+                tc_commit_pair_mc(&acc_full[acc], 0x3);
+            }
+            tc_commit_pair(drain);
+            mbar_wait(drain, 0);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..9)
+        const int q = warp & 3;           // TMEM lanes 32q..32q+31
+        const int h = (warp - 2) >> 2;    // accumulator columns [128h, 128h+128)
+        const uint32_t leader_empty0 = mapa_u32(smem_u32(&acc_empty[0]), 0);
+        int it = 0;
+        for (int tile = pair; tile < num_tiles && !*(volatile int *)abort_flag; tile += npairs, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            int mt, nt;
+            tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
+            if (!mbar_wait(&acc_full[acc], acc_phase)) { *(volatile int *)abort_flag = 1; break; }
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + acc * PAIR_BN + 128 * h + 32 * ch, r[ch]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_empty0 + 8u * (uint32_t)acc);
+
+            const int row = mt * PAIR_BM + 128 * (int)rank + 32 * q + lane;
+            if (row >= p.T) continue;
+            float rscale = 1.0f, reta = 0.0f;
+            if (p.nu) rscale = p.nu[row];
+            if (p.eta) reta = p.eta[row];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                const int col0 = nt * PAIR_BN + 128 * h + 32 * ch;
+                if (col0 >= p.n_out) continue;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float f = __uint_as_float(r[ch][i]);
+                    if (p.nu) f *= rscale;
+                    if (p.eta) {
+                        const int c = min(col0 + i, p.n_out - 1);
+                        f = fmaf(reta, p.rowsum[c], f);
+                    }
+                    v[i] = f;
+                }
+                if (p.out_bf16) {
+                    __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(p.y) + (size_t)row * p.n_out + col0;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        if (col0 + 8 * c8 < p.n_out) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                __nv_bfloat162 hh = __floats2bfloat162_rn(v[8 * c8 + 2 * i], v[8 * c8 + 2 * i + 1]);
+                                w[i] = *reinterpret_cast<uint32_t *>(&hh);
+                            }
+                            *reinterpret_cast<uint4 *>(yr + 8 * c8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                } else {
+                    float *yr = static_cast<float *>(p.y) + (size_t)row * p.n_out + col0;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        if (col0 + 4 * c4 < p.n_out)
+                            *reinterpret_cast<float4 *>(yr + 4 * c4) =
+                                make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+                }
+            }
+        }
+    }
+
+    // Both CTAs' tensor memory stays allocated until the leader's last MMA
+    // has completed and both epilogues have read their accumulators.
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                       const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -573,9 +759,9 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
 
 // Number of 2-CTA clusters of k_gemm_sp_pair that fit on the device at once
 // (0 if the query fails).
-static int pair_clusters(size_t smem)
+template <typename KernelT>
+static int pair_clusters_of(KernelT kernel, size_t smem, int &cached)
 {
-    static int cached = -1;
     if (cached >= 0) return cached;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * 74, 1, 1);
@@ -589,12 +775,25 @@ static int pair_clusters(size_t smem)
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_sp_pair, &cfg) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
         cudaGetLastError();
         n = 0;
     }
     cached = n;
     return n;
+}
+
+static int pair_clusters(size_t smem)
+{
+    static int cached = -1;
+    return pair_clusters_of(k_gemm_sp_pair, smem, cached);
+}
+
+static int dense_pair_clusters(size_t smem)
+{
+    static int cached = -1;
+    return pair_clusters_of(k_gemm_dense_pair, smem, cached);
 }
 
 // The pair kernel needs every CTA's 128-row box to hold at least one real
@@ -603,7 +802,8 @@ static int pair_clusters(size_t smem)
 static bool use_pair(const GemmArgs &a)
 {
     const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
-    return a.sparse && (mt128 % 2) == 0 && (reinterpret_cast<uintptr_t>(a.meta) & 15) == 0;
+    if ((mt128 % 2) != 0) return false;
+    return !a.sparse || (reinterpret_cast<uintptr_t>(a.meta) & 15) == 0;
 }
 
 static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
@@ -638,14 +838,45 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+static cudaError_t launch_gemm_dense_pair(const GemmArgs &a, cudaStream_t st)
+{
+    CUtensorMap mA, mB;
+    const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
+    GemmParams p{};
+    p.rowsum = a.rowsum;
+    p.eta = a.eta;
+    p.nu = a.nu;
+    p.y = a.y;
+    p.T = a.T;
+    p.K = a.K;
+    p.n_out = a.n_out;
+    p.out_bf16 = a.out_bf16;
+    p.m_tiles = mt128 / 2;
+    p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
+    p.k_blocks = (a.K + 63) / 64;
+    if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
+    const size_t smem = dense_pair_smem_bytes();
+    const int clusters = dense_pair_clusters(smem);
+    if (clusters <= 0) return cudaErrorNotSupported;
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int grid = 2 * std::min(tiles, clusters);
+    k_gemm_dense_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st)
 {
     if (use_pair(a)) {
-        const size_t smem = pair_smem_bytes();
-        if (cudaFuncSetAttribute(k_gemm_sp_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
-                cudaSuccess &&
-            pair_clusters(smem) > 0)
-            return launch_gemm_pair(a, st);
+        if (a.sparse) {
+            const size_t smem = pair_smem_bytes();
+            if (cudaFuncSetAttribute(k_gemm_sp_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+                    cudaSuccess &&
+                pair_clusters(smem) > 0)
+                return launch_gemm_pair(a, st);
+        } else if (dense_pair_clusters(dense_pair_smem_bytes()) > 0) {
+            return launch_gemm_dense_pair(a, st);
+        }
         cudaGetLastError();
     }
     return a.sparse ? launch_gemm_t<true>(a, st) : launch_gemm_t<false>(a, st);
