@@ -201,6 +201,24 @@ def test_prefill_24(sl, T, K, n_out):
         assert err <= (TOL_BF16 if out == sl.AS_BF16 else TOL_F32), err
 
 
+def test_prefill_24_partial_wave(sl):
+    """80 CTA-pair tiles on 74 pairs: a partial second wave (the tiles of
+    output columns [2304, 2560) in row blocks 2..7); sampled rows in those
+    blocks and in others, every column."""
+    T, K, n_out = 2048, 512, 2560
+    x, W = synth.random_layer(T, K, n_out, seed=77, dist="sqrelu")
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4)
+    L = layer(sl, W, cfg)
+    y, bufs = L.prefill(dev(x))
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    rows = np.array([3, 255, 600, 1000, 1300, 1790, 2047])
+    mask = check_select_24(sl, x, bufs, rows)
+    ref = oracle.linear(x.float().numpy()[rows], mask, W.float().numpy())
+    assert rel_l2(f32(y)[rows], ref) <= TOL_BF16
+    assert rel_l2(f32(y)[rows][:, 2304:], ref[:, 2304:]) <= TOL_BF16
+
+
 def test_prefill_24_full_size(sl):
     """FFN down-projection at prefill: squared-ReLU activations [4096, 14336],
     2:4 by magnitude on the sparse tensor-core path; sampled rows."""
