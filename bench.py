@@ -484,6 +484,10 @@ def run_case(args):
         L = SparseLinear(W.to(dev), cfg, alpha=0.5)
         xd = x[:args.T].contiguous().to(dev)
         fn = lambda: L.decode(xd)  # noqa: E731
+    elif args.case == "block":
+        res = bench_block(sl, dev, reps=args.reps)
+        print(json.dumps({"case": "block", **res}))
+        return
     elif args.case in ("select24", "selectclact"):
         if args.case == "select24":
             _, x, W = synth.prefill_sqrelu(T=args.T)
@@ -545,7 +549,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--case", default=None,
-                    help="profiling case: decode | sqrelu24 | dense | select24 | selectclact")
+                    help="profiling case: decode | sqrelu24 | dense | select24 | selectclact | block")
     ap.add_argument("--T", type=int, default=1)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

@@ -950,6 +950,9 @@ DecodePlan decode_plan(int T, int K, int n_out, int bf16)
     if (want < 1) want = 1;
     int wps = (nwords + want - 1) / want;
     if (wps > maxw) wps = maxw;
+    // at least 128 channels a CTA: narrow layers would otherwise split K so
+    // finely that summing the partials costs more than streaming the rows
+    if (p.tc && wps < 4) wps = 4;
     if (wps < 1) wps = 1;
     p.words_per_split = wps;
     p.k_splits = (nwords + wps - 1) / wps;

@@ -217,13 +217,18 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
     const int words = (K + 31) >> 5;
     double skm = 0.0, skmm = 0.0;
     int eq_base = 0;
+    // top-k decides from the keys; the activations are reread only when a
+    // value output (masked copy, compact operand, VAR sums) needs them
+    const bool need_vals = !topk || a.x_masked || a.x_compact || a.var;
     for (int tile0 = 0; tile0 < ntiles; tile0 += U) {
         float vv[U][8], fv[U][8];
         const bool has_f = a.f != nullptr;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int g = (tile0 + u) * NT + tid;
-            if (g < ngroups) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) { vv[u][e] = 0.0f; fv[u][e] = 1.0f; }
+            if (g < ngroups && need_vals) {
                 load8(xr + 8 * g, vv[u]);
                 if (has_f) load8f(a.f + 8 * g, fv[u]);
             }
