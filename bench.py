@@ -261,24 +261,106 @@ def bench_decode(sl, dev, steps, warmup, world):
         per_t[T] = timed(lambda j, T=T: per_t_graphs[T].replay(), reps) / (reps * N_ROT)
     t_max = max_over_ranks(t_local, world)
 
-    # end to end through host buffers: pinned host x -> device, decode, y -> pinned host
+    # end to end through host buffers, every step: pinned host x -> device,
+    # decode, y -> pinned host.  Copies run on their own streams (H2D and D2H
+    # use separate copy engines) into double-buffered device x and y, so the
+    # copies of one call overlap the decode of its neighbours; events order
+    # each copy against the decode that reads or writes its buffer.
     xh = {T: [xs[i][:T].cpu().pin_memory() for i in range(N_ROT)] for T in DECODE_TS}
-    xd = {T: torch.empty(T, K_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS}
-    yh = {T: torch.empty(T, N_DOWN, dtype=torch.bfloat16).pin_memory() for T in DECODE_TS}
+    yh = {T: [torch.empty(T, N_DOWN, dtype=torch.bfloat16).pin_memory() for _ in range(2)] for T in DECODE_TS}
+    xdb = [{T: torch.empty(T, K_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS} for _ in range(2)]
+    ydb = [{T: torch.empty(T, N_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS} for _ in range(2)]
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [{T: torch.cuda.Event() for T in DECODE_TS} for _ in range(2)] for k in ("h2d", "dec", "d2h")}
+    for b in range(2):  # every event recorded once before first use
+        for T in DECODE_TS:
+            for k in ev:
+                ev[k][b][T].record(stream)
+    # the layer's fixed arguments are marshalled once per (weight copy, T)
+    calls = {(i, T): sl.DecodeCall(Wts[i], cfg, g=L.g, rowsum=L.rowsum, workspace=wss[T], stream=stream)
+             for i in range(N_ROT) for T in DECODE_TS}
 
     def e2e_step(j):
-        i = j % N_ROT
+        i, b = j % N_ROT, j % 2
         for T in DECODE_TS:
-            xd[T].copy_(xh[T][i], non_blocking=True)
-            sl.as_linear_decode(xd[T], Wts[i], cfg, ys[T], g=L.g, rowsum=L.rowsum, workspace=wss[T],
-                                stream=stream)
-            yh[T].copy_(ys[T], non_blocking=True)
+            with torch.cuda.stream(h2d_s):
+                h2d_s.wait_event(ev["dec"][b][T])  # the decode two steps back has read this buffer
+                xdb[b][T].copy_(xh[T][i], non_blocking=True)
+                ev["h2d"][b][T].record(h2d_s)
+        for T in DECODE_TS:
+            stream.wait_event(ev["h2d"][b][T])
+            stream.wait_event(ev["d2h"][b][T])  # y of two steps back has been read out
+            calls[(i, T)](xdb[b][T], ydb[b][T])
+            ev["dec"][b][T].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev["dec"][b][T])
+                yh[T][b].copy_(ydb[b][T], non_blocking=True)
+                ev["d2h"][b][T].record(d2h_s)
 
-    for j in range(3):
-        with torch.cuda.stream(stream):
+    def timed_e2e(n):
+        barrier(world)
+        torch.cuda.synchronize()
+        s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        h2d_s.wait_event(s0)
+        d2h_s.wait_event(s0)
+        for j in range(n):
             e2e_step(j)
+        for b in range(2):
+            for T in DECODE_TS:
+                stream.wait_event(ev["d2h"][b][T])
+        e0.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return s0.elapsed_time(e0) / 1e3
+
+    timed_e2e(3)
+    t_e2e_eager = max_over_ranks(timed_e2e(steps), world)
+
+    # the same step captured once per rotation index, copies included: the
+    # capture forks the three input copies onto the H2D stream up front and
+    # each output copy onto the D2H stream after its decode, then joins them,
+    # so a replay overlaps copies with decode without host work per call
+    xg = [{T: torch.empty(T, K_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS} for _ in range(N_ROT)]
+    yg = [{T: torch.empty(T, N_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS} for _ in range(N_ROT)]
+    yhg = [{T: torch.empty(T, N_DOWN, dtype=torch.bfloat16).pin_memory() for T in DECODE_TS} for _ in range(N_ROT)]
+
+    def step_forked(i):
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        h2d_s.wait_event(fork)
+        d2h_s.wait_event(fork)
+        e_in = {T: torch.cuda.Event() for T in DECODE_TS}
+        e_out = {T: torch.cuda.Event() for T in DECODE_TS}
+        with torch.cuda.stream(h2d_s):
+            for T in DECODE_TS:
+                xg[i][T].copy_(xh[T][i], non_blocking=True)
+                e_in[T].record(h2d_s)
+        for T in DECODE_TS:
+            stream.wait_event(e_in[T])
+            calls[(i, T)](xg[i][T], yg[i][T])
+            e_out[T].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(e_out[T])
+                yhg[i][T].copy_(yg[i][T], non_blocking=True)
+        j_h, j_d = torch.cuda.Event(), torch.cuda.Event()
+        j_h.record(h2d_s)
+        j_d.record(d2h_s)
+        stream.wait_event(j_h)
+        stream.wait_event(j_d)
+
+    e2e_graphs = []
+    with torch.cuda.stream(stream):
+        for i in range(N_ROT):
+            step_forked(i)  # warm outside capture
+        stream.synchronize()
+        for i in range(N_ROT):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                step_forked(i)
+            e2e_graphs.append(gr)
     torch.cuda.synchronize()
-    t_e2e = max_over_ranks(timed(e2e_step, steps), world)
+    t_e2e = max_over_ranks(timed(lambda j: e2e_graphs[j % N_ROT].replay(), steps), world)
     clk.__exit__(None, None, None)
     h2d = sum(T * K_DOWN * 2 for T in DECODE_TS)
     d2h = sum(T * N_DOWN * 2 for T in DECODE_TS)
@@ -291,7 +373,7 @@ def bench_decode(sl, dev, steps, warmup, world):
     return dict(
         t=t_max, steps=steps, tokens_per_step=tokens,
         value=tokens * steps * world / t_max,
-        e2e=tokens * steps * world / t_e2e, h2d=h2d, d2h=d2h,
+        e2e=tokens * steps * world / t_e2e, e2e_eager=tokens * steps * world / t_e2e_eager, h2d=h2d, d2h=d2h,
         per_t={T: dict(us=per_t[T] * 1e6, gbs=bytes_call[T] / per_t[T] / 1e9, bytes=bytes_call[T])
                for T in DECODE_TS},
         achieved_gbs=step_bytes / kern_time / 1e9, bytes_per_step=step_bytes,
@@ -607,7 +689,12 @@ def main():
                                "reduction kernels)", "bytes_per_launch": d["bytes_per_launch"],
                      "per_T": {str(T): v for T, v in d["per_t"].items()}},
         "e2e": {"value": d["e2e"], "unit": "tokens/s", "h2d_bytes_per_step": d["h2d"],
-                "d2h_bytes_per_step": d["d2h"]},
+                "d2h_bytes_per_step": d["d2h"],
+                "mode": "per step: the pinned x of each call copied in and its y copied out (separate "
+                        "copy streams, overlapping the neighbouring decode calls), the step captured once "
+                        "per rotation index in a CUDA graph through sl.DecodeCall and replayed",
+                "eager_value": d["e2e_eager"],
+                "eager_mode": "the same pipelined step issued eagerly from Python every step"},
         "gpu_launches": d["launches"],
         "clocks": d["clocks"],
         "cpu_baseline": cpu,

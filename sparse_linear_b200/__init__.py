@@ -181,6 +181,32 @@ def as_linear_decode(x, Wt, cfg: as_config, y, g=None, rowsum=None, mask_out=Non
            "as_linear_decode")
 
 
+class DecodeCall:
+    """as_linear_decode with a layer's fixed arguments (Wt, cfg, g, rowsum,
+    workspace, stream) converted once; each call passes x and y.  For
+    decode loops where the per-call marshalling would otherwise cost more
+    host time than the GPU spends."""
+
+    def __init__(self, Wt, cfg: as_config, g=None, rowsum=None, workspace=None, stream=None):
+        self._K, self._n_out = Wt.shape
+        self._dt = _dt(Wt)
+        self._cfg = cfg  # keeps the structure alive
+        self._args = (_ptr(Wt), _ptr(g), _ptr(rowsum), ctypes.byref(cfg))
+        self._ws = _ptr(workspace)
+        self._wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        self._st = _stream(stream)
+        self._fn = _lib.as_linear_decode
+
+    def __call__(self, x, y, mask_out=None, eta_out=None, colnorm_out=None) -> None:
+        if _dt(x) != self._dt:
+            raise TypeError("x must have the weights' dtype")
+        wt, g, rs, cfgp = self._args
+        code = self._fn(_ptr(x), self._dt, x.shape[0], self._K, self._n_out, wt, g, rs, cfgp, _ptr(y),
+                        _ptr(mask_out), _ptr(eta_out), _ptr(colnorm_out), self._ws, self._wsb, self._st)
+        if code != AS_OK:
+            raise ASError(code, "as_linear_decode")
+
+
 def as_linear_decode_noalloc(x, Wt, cfg: as_config, y, g=None, rowsum=None, mask_out=None, eta_out=None,
                              colnorm_out=None, stream=None) -> None:
     """as_linear_decode without a workspace argument: the scratch is the

@@ -338,6 +338,20 @@ __device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t s
     asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
 }
 
+// ------------------------------------------------------------ host helpers
+// Raises a kernel's dynamic shared-memory limit to `smem` once per device
+// (the caller passes a static array of its own, one per kernel instance).
+template <typename Kernel>
+static cudaError_t smem_limit_once(Kernel kernel, size_t smem, int (&done)[64])
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (dev >= 0 && dev < 64 && done[dev] >= (int)smem) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = (int)smem;
+    return e;
+}
+
 // -------------------------------------------------------------- misc
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 

@@ -1034,8 +1034,8 @@ static cudaError_t launch_tc_one(const DecodeArgs &a, const DecodePlan &p, cudaS
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     set_pdl(cfg, attr);
-    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<TP, FUSED, LO, DENSE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int done[64];
+    cudaError_t e = smem_limit_once(k_decode_tc<TP, FUSED, LO, DENSE>, smem, done);
     if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k_decode_tc<TP, FUSED, LO, DENSE>, a, p.words_per_split);
     return e;
 }

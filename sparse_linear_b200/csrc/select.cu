@@ -604,7 +604,8 @@ template <typename TX, int NT>
 static cudaError_t launch_select_t(const SelectArgs &a, size_t smem, int grid, cudaStream_t st)
 {
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_select<TX, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static int done[64];
+        cudaError_t e = smem_limit_once(k_select<TX, NT>, smem, done);
         if (e != cudaSuccess) return e;
     }
     k_select<TX, NT><<<grid, NT, smem, st>>>(a);
@@ -615,8 +616,8 @@ template <typename TX, int M, bool COMPACT>
 static cudaError_t launch_select_rows_t(const SelectArgs &a, cudaStream_t st)
 {
     const size_t smem = (a.f ? (size_t)a.K * 4 : 0) + (size_t)SR_BUFS * a.K * sizeof(TX);
-    cudaError_t e = cudaFuncSetAttribute(k_select_rows<TX, M, COMPACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    static int done[64];
+    cudaError_t e = smem_limit_once(k_select_rows<TX, M, COMPACT>, smem, done);
     if (e != cudaSuccess) return e;
     int per_sm = 0, dev = 0, sms = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_select_rows<TX, M, COMPACT>, SR_THREADS, smem);
