@@ -90,3 +90,23 @@ def test_var_state_checkpoint_and_resume(sl):
     np.testing.assert_array_equal(f32(run2), f32(state_full))
     for a, b in zip(ys[3:], ys2):
         assert torch.equal(a, b)
+
+
+def test_prepared_decode_call_matches(sl):
+    """sl.DecodeCall (fixed arguments marshalled once) gives the bitwise
+    result of as_linear_decode, across calls with different x."""
+    from sparse_linear_b200.layer import SparseLinear, workspace
+    x, W, _ = synth.decode_downproj(8)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
+    L = SparseLinear(dev(W), cfg, alpha=0.5)
+    ws = workspace(sl.as_workspace_size(sl.AS_OP_DECODE, 8, L.K, L.n_out, cfg), "cuda")
+    call = sl.DecodeCall(L.Wt, cfg, g=L.g, rowsum=L.rowsum, workspace=ws)
+    for T in (1, 8):
+        xd = dev(x[:T])
+        y1 = torch.empty(T, L.n_out, dtype=torch.bfloat16, device="cuda")
+        y2 = torch.empty_like(y1)
+        call(xd, y1)
+        sl.as_linear_decode(xd, L.Wt, cfg, y2, g=L.g, rowsum=L.rowsum, workspace=ws)
+        torch.cuda.synchronize()
+        assert sl.as_stream_status() == sl.AS_OK
+        assert torch.equal(y1, y2)
