@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define AS_ABI_VERSION 1
+#define AS_ABI_VERSION 2
 #define AS_MAX_DECODE_T 16
 
 typedef enum as_status {
@@ -69,20 +69,34 @@ typedef enum as_dtype { AS_F32 = 0, AS_BF16 = 1 } as_dtype;
 typedef enum as_score { AS_SCORE_MAG = 0, AS_SCORE_WEIGHT = 1, AS_SCORE_CLACT = 2 } as_score;
 
 /* Selection ([OVW] 2.1; [WIS] 2.2):
- *   AS_SEL_NM:   in every block of m consecutive channels [jm, jm+m) keep the
- *                n largest scores; m in {1,2,4,8,16,32}, 1 <= n <= m, K % m == 0.
- *   AS_SEL_TOPK: keep the k_keep largest scores of each token, 0 <= k_keep <= K.
- *   AS_SEL_ALL:  keep every channel (dense layer, for baselines and checks). */
-typedef enum as_sel { AS_SEL_NM = 0, AS_SEL_TOPK = 1, AS_SEL_ALL = 2 } as_sel;
+ *   AS_SEL_NM:     in every block of m consecutive channels [jm, jm+m) keep the
+ *                  n largest scores; m in {1,2,4,8,16,32}, 1 <= n <= m, K % m == 0.
+ *   AS_SEL_TOPK:   keep the k_keep largest scores of each token, 0 <= k_keep <= K.
+ *   AS_SEL_ALL:    keep every channel (dense layer, for baselines and checks).
+ *   AS_SEL_THRESH: keep every channel whose score is > cfg->tau (a calibrated
+ *                  per-layer threshold: [WIS] 3.1 builds on TEAL's sparse
+ *                  operator, [WIS] 5 tunes its threshold tau); the number
+ *                  kept varies per token. */
+typedef enum as_sel { AS_SEL_NM = 0, AS_SEL_TOPK = 1, AS_SEL_ALL = 2, AS_SEL_THRESH = 3 } as_sel;
+
+/* Token shift ([OVW] 3.1): */
+enum {
+    AS_PTS_OFF = 0,     /* no shift */
+    AS_PTS_DYNAMIC = 1, /* D-PTS: eta_t = mean_i x_ti of the call's token */
+    AS_PTS_STATIC = 2   /* S-PTS: eta_t = cfg->eta_static[t], a calibrated table
+                           ([OVW] 3.1 static version, indexed per token; read here
+                           as one float32 per token row of the call, [T]) */
+};
 
 typedef struct as_config {
     int32_t score;        /* as_score */
     int32_t sel;          /* as_sel */
     int32_t n, m;         /* N:M pattern (AS_SEL_NM) */
     int32_t k_keep;       /* kept channels per token (AS_SEL_TOPK) */
-    int32_t dpts;         /* 1: D-PTS, [OVW] 3.1: score and keep xhat = x - eta_t,
-                             eta_t = mean_i x_ti, and add eta_t * rowsum_o back:
-                             y = (xhat*m) W^T + eta * rowsum(W). */
+    int32_t dpts;         /* token shift, AS_PTS_*, [OVW] 3.1: score and keep
+                             xhat = x - eta_t and add eta_t * rowsum_o back:
+                             y = (xhat*m) W^T + eta * rowsum(W).  1: eta_t =
+                             mean_i x_ti (D-PTS); 2: eta_t = eta_static[t] (S-PTS). */
     int32_t var;          /* 1: VAR, [OVW] 3.2 (prefill only; not with dpts):
                              running_t <- var_dense_t on the first batch, else
                              mom*running_t + (1-mom)*var_dense_t; then
@@ -91,6 +105,9 @@ typedef struct as_config {
     float var_momentum;   /* mom, 0.9 on the page */
     float var_eps;        /* eps, 1e-6 on the page */
     int32_t out_dtype;    /* as_dtype of y */
+    float tau;            /* AS_SEL_THRESH: keep scores > tau */
+    const float *eta_static; /* dpts == AS_PTS_STATIC: device [T] float32 eta table
+                                (16-byte aligned); ignored otherwise */
 } as_config;
 
 /* Outputs of as_select.  Every pointer is optional (NULL = not written) unless

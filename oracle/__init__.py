@@ -19,6 +19,10 @@ Functions and the passages they follow (page title, section):
 * ``score``         overview §2.2.1, §2.2.3, §3.1; WiSparse eq. (4).
 * ``select_nm``     overview §2.1 / §2.2.1 (block top-N).
 * ``select_topk``   WiSparse §2.2 (per-layer keep fraction).
+* ``select_thresh`` WiSparse §3.1 / §5 (TEAL-style threshold tau).
+  S-PTS (overview §3.1, static version) needs no function of its own:
+  ``score`` and ``linear`` take the token shift eta as an input, dynamic
+  (``token_mean``) or a calibrated table.
 * ``var_scale``     overview §3.2.
 * ``linear``        overview §3.1 / §3.2 and the layer definition y = prune(x) W^T.
 * ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
@@ -69,6 +73,7 @@ def _load():
                 "or_score": [P, I, I, P, P, P],
                 "or_select_nm": [P, I, I, I, I, P],
                 "or_select_topk": [P, I, I, I, P],
+                "or_select_thresh": [P, I, I, ctypes.c_float, P],
                 "or_var_scale": [P, P, I, I, P, D, D, P, P, P, P],
                 "or_linear": [P, P, I, I, P, P, I, P, P, P, I, P],
                 "or_compress_nm": [P, P, I, I, I, I, P, P],
@@ -158,6 +163,14 @@ def select_topk(s, kk: int):
     T, k = s.shape
     mask = np.empty((T, k), np.uint8)
     _load().or_select_topk(_ptr(s), T, k, int(kk), _ptr(mask))
+    return mask
+
+
+def select_thresh(s, tau: float):
+    s = np.ascontiguousarray(s, np.float32)
+    T, k = s.shape
+    mask = np.empty((T, k), np.uint8)
+    _load().or_select_thresh(_ptr(s), T, k, ctypes.c_float(tau), _ptr(mask))
     return mask
 
 

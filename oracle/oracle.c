@@ -175,6 +175,16 @@ void or_select_nm(const float *s, int T, int k, int n, int m, uint8_t *mask)
     }
 }
 
+/* Threshold selection (WiSparse page section 3.1 builds on TEAL's sparse
+ * operator; section 5 tunes its threshold tau): keep every channel whose
+ * score is above tau. */
+void or_select_thresh(const float *s, int T, int k, float tau, uint8_t *mask)
+{
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; t++)
+        for (int i = 0; i < k; i++) mask[(size_t)t * k + i] = (uint8_t)(s[(size_t)t * k + i] > tau);
+}
+
 typedef struct { float s; int i; } keyed;
 
 static int cmp_keyed(const void *a, const void *b)

@@ -30,7 +30,8 @@ AS_OK, AS_ERR_INVALID_ARG, AS_ERR_SHAPE, AS_ERR_DTYPE, AS_ERR_ALIGN = 0, 1, 2, 3
 AS_ERR_UNSUPPORTED, AS_ERR_WORKSPACE, AS_ERR_CUDA, AS_ERR_TIMEOUT = 5, 6, 7, 8
 AS_F32, AS_BF16 = 0, 1
 AS_SCORE_MAG, AS_SCORE_WEIGHT, AS_SCORE_CLACT = 0, 1, 2
-AS_SEL_NM, AS_SEL_TOPK, AS_SEL_ALL = 0, 1, 2
+AS_SEL_NM, AS_SEL_TOPK, AS_SEL_ALL, AS_SEL_THRESH = 0, 1, 2, 3
+AS_PTS_OFF, AS_PTS_DYNAMIC, AS_PTS_STATIC = 0, 1, 2
 AS_OP_WEIGHT_PREP, AS_OP_SELECT, AS_OP_DECODE, AS_OP_PREFILL = 0, 1, 2, 3
 AS_MAX_DECODE_T = 16
 
@@ -46,7 +47,8 @@ class as_config(ctypes.Structure):
     _fields_ = [("score", ctypes.c_int32), ("sel", ctypes.c_int32), ("n", ctypes.c_int32),
                 ("m", ctypes.c_int32), ("k_keep", ctypes.c_int32), ("dpts", ctypes.c_int32),
                 ("var", ctypes.c_int32), ("var_momentum", ctypes.c_float),
-                ("var_eps", ctypes.c_float), ("out_dtype", ctypes.c_int32)]
+                ("var_eps", ctypes.c_float), ("out_dtype", ctypes.c_int32),
+                ("tau", ctypes.c_float), ("eta_static", ctypes.c_void_p)]
 
 
 class as_select_out(ctypes.Structure):
@@ -118,9 +120,12 @@ def _stream(stream) -> int | None:
 
 
 def config(score: int = AS_SCORE_MAG, sel: int = AS_SEL_NM, n: int = 2, m: int = 4, k_keep: int = 0,
-           dpts: bool = False, var: bool = False, var_momentum: float = 0.9, var_eps: float = 1e-6,
-           out_dtype: int = AS_BF16) -> as_config:
-    return as_config(score, sel, n, m, k_keep, int(dpts), int(var), var_momentum, var_eps, out_dtype)
+           dpts: int = AS_PTS_OFF, var: bool = False, var_momentum: float = 0.9, var_eps: float = 1e-6,
+           out_dtype: int = AS_BF16, tau: float = 0.0, eta_static=None) -> as_config:
+    """dpts: False/0 off, True/1 D-PTS, 2 S-PTS (eta_static: device [T] float32,
+    kept alive by the caller for as long as the config is used)."""
+    return as_config(score, sel, n, m, k_keep, int(dpts), int(var), var_momentum, var_eps, out_dtype,
+                     float(tau), _ptr(eta_static))
 
 
 def select_out(**bufs) -> as_select_out:

@@ -23,7 +23,10 @@ as_status check_cfg(const as_config *cfg, int K)
 {
     if (!cfg) return AS_ERR_INVALID_ARG;
     if (cfg->score < AS_SCORE_MAG || cfg->score > AS_SCORE_CLACT) return AS_ERR_INVALID_ARG;
-    if (cfg->sel < AS_SEL_NM || cfg->sel > AS_SEL_ALL) return AS_ERR_INVALID_ARG;
+    if (cfg->sel < AS_SEL_NM || cfg->sel > AS_SEL_THRESH) return AS_ERR_INVALID_ARG;
+    if (cfg->dpts < AS_PTS_OFF || cfg->dpts > AS_PTS_STATIC) return AS_ERR_INVALID_ARG;
+    if (cfg->dpts == AS_PTS_STATIC && (!cfg->eta_static || !aligned16(cfg->eta_static))) return AS_ERR_INVALID_ARG;
+    if (cfg->sel == AS_SEL_THRESH && !(cfg->tau == cfg->tau)) return AS_ERR_INVALID_ARG;  // NaN
     if (cfg->out_dtype != AS_F32 && cfg->out_dtype != AS_BF16) return AS_ERR_DTYPE;
     if (cfg->sel == AS_SEL_NM) {
         if (!valid_m(cfg->m)) return AS_ERR_SHAPE;
@@ -162,6 +165,8 @@ as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *c
     a.m = cfg->m;
     a.k_keep = cfg->k_keep;
     a.dpts = cfg->dpts;
+    a.tau = cfg->tau;
+    a.eta_static = cfg->dpts == AS_PTS_STATIC ? cfg->eta_static : nullptr;
     a.var = cfg->var;
     a.first = var_first_batch;
     a.mom = cfg->var_momentum;
@@ -231,6 +236,8 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
         s.m = cfg->m;
         s.k_keep = cfg->k_keep;
         s.dpts = cfg->dpts;
+        s.tau = cfg->tau;
+        s.eta_static = cfg->dpts == AS_PTS_STATIC ? cfg->eta_static : nullptr;
         s.f = f;
         s.bitmask = bm;
         s.eta = cfg->dpts ? eta_ws : nullptr;  // the decode kernel reuses the means the selection used
@@ -254,6 +261,8 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     a.m = cfg->m;
     a.k_keep = cfg->k_keep;
     a.dpts = cfg->dpts;
+    a.tau = cfg->tau;
+    a.eta_static = cfg->dpts == AS_PTS_STATIC ? cfg->eta_static : nullptr;
     a.g = g;
     a.rowsum = rowsum;
     a.mask_in = mask_in;
@@ -312,6 +321,8 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
     a.K = K;
     a.n_out = n_out;
     a.dpts = cfg->dpts;
+    a.tau = cfg->tau;
+    a.eta_static = cfg->dpts == AS_PTS_STATIC ? cfg->eta_static : nullptr;
     a.bf16 = bf16;
     a.sel = cfg->sel;
     int n = 0;

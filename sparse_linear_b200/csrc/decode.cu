@@ -128,8 +128,13 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
     const int nw = max(0, w1 - w0);
     const TW *x = static_cast<const TW *>(a.x);
 
-    // ---- 1. D-PTS mean of every token (float64, identical in every CTA)
-    if (a.dpts) {
+    // ---- 1. D-PTS mean of every token (float64, identical in every CTA);
+    // S-PTS takes the caller's table
+    if (a.dpts == AS_PTS_STATIC) {
+        if (tid < TP) s_eta[tid] = tid < T ? a.eta_static[tid] : 0.0f;
+        __syncthreads();
+        if (a.eta_out && slice == 0 && split == 0 && tid < T) a.eta_out[tid] = s_eta[tid];
+    } else if (a.dpts) {
         double acc[TP];
 #pragma unroll
         for (int t = 0; t < TP; ++t) acc[t] = 0.0;
@@ -204,7 +209,9 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
                 } else {
                     score8(v, a.dpts, s_eta[t], fac, c0, xh, s);
                 }
-                keep = a.sel == AS_SEL_NM ? nm_keep_dispatch(s, lane, a.n, a.m) : 0xFFu;
+                keep = a.sel == AS_SEL_NM       ? nm_keep_dispatch(s, lane, a.n, a.m)
+                       : a.sel == AS_SEL_THRESH ? keep_thresh(s, a.tau)
+                                                : 0xFFu;
                 if (!act) keep = 0;
             }
             // assemble 32-bit words: lanes 4j..4j+3 hold the bytes of word j
@@ -607,12 +614,14 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
         const bool want_g = a.score == AS_SCORE_WEIGHT && tid < (nch >> 2);
         if (want_g) gv = *reinterpret_cast<const float4 *>(a.g + c_begin + 4 * tid);
+        const bool whole = a.dpts == AS_PTS_DYNAMIC;  // whole rows for the mean, else the chunk alone
 #pragma unroll
         for (int t = 0; t < TP; ++t)
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 const int g = tid + r * TC_THREADS;
-                if (t < T && g < ng) rowv[t][r] = *reinterpret_cast<const uint4 *>(x + (size_t)t * K + 8 * g);
+                if (t < T && g < ng && (whole || (g >= gc0 && g < gc0 + ngc)))
+                    rowv[t][r] = *reinterpret_cast<const uint4 *>(x + (size_t)t * K + 8 * g);
             }
         if (want_g) *reinterpret_cast<float4 *>(s_f + 4 * tid) = gv;
 #pragma unroll
@@ -621,11 +630,13 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 const int g = tid + r * TC_THREADS;
-                if (t < T && g < ng) {
-                    float w[8];
-                    load8(&rowv[t][r], w);
+                if (t < T && g < ng && (whole || (g >= gc0 && g < gc0 + ngc))) {
+                    if (whole) {
+                        float w[8];
+                        load8(&rowv[t][r], w);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) sum += (double)w[e];
+                        for (int e = 0; e < 8; ++e) sum += (double)w[e];
+                    }
                     if (g >= gc0 && g < gc0 + ngc) *reinterpret_cast<uint4 *>(xh + t * TC_XP + 8 * (g - gc0)) = rowv[t][r];
                 } else if (t >= T && g >= gc0 && g < gc0 + ngc) {
                     *reinterpret_cast<uint4 *>(xh + t * TC_XP + 8 * (g - gc0)) = make_uint4(0, 0, 0, 0);
@@ -641,7 +652,8 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         for (int t = 0; t < TP; ++t) {
             double sum = 0.0;
             for (int w = 0; w < TC_WARPS; ++w) sum += s_red[w][t];
-            eta_r[t] = (a.dpts && t < T) ? (float)(sum / (double)K) : 0.0f;
+            eta_r[t] = (a.dpts && t < T) ? (a.dpts == AS_PTS_STATIC ? a.eta_static[t] : (float)(sum / (double)K))
+                                         : 0.0f;
         }
 #pragma unroll
         for (int t = 0; t < TP; ++t)
@@ -683,7 +695,8 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             }
             wsc[lane] = sc;
             __syncwarp();
-            const bool keep = c < nch && nm_rank_keep(wsc, lane, a.n, a.m);
+            const bool keep =
+                c < nch && (a.sel == AS_SEL_THRESH ? sc > a.tau : nm_rank_keep(wsc, lane, a.n, a.m));
             const uint32_t word = __ballot_sync(0xffffffffu, keep);
             if (c < nch) {
                 const float e = keep ? (a.dpts ? __fsub_rn(xv, eta_t) : xv) : 0.0f;
@@ -986,7 +999,10 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &p, cudaStream
 }
 
 // whole-row loads for the mean are held in registers: K <= 8 * 256 * 8
-bool decode_fused(int tpad, int sel, int K) { return tpad <= 2 && sel == AS_SEL_NM && K <= 8 * TC_THREADS * 8; }
+bool decode_fused(int tpad, int sel, int K)
+{
+    return tpad <= 2 && (sel == AS_SEL_NM || sel == AS_SEL_THRESH) && K <= 8 * TC_THREADS * 8;
+}
 
 int decode_launch_count(const DecodeArgs &, const DecodePlan &p)
 {
@@ -1012,6 +1028,7 @@ static void set_pdl(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr)
 // token keeps a channel with probability f independently.
 static double expected_union(const DecodeArgs &a)
 {
+    if (a.sel == AS_SEL_THRESH) return 0.0;  // the share kept depends on the data: stream the union
     double f = 1.0;
     if (a.sel == AS_SEL_NM) f = (double)a.n / (double)a.m;
     else if (a.sel == AS_SEL_TOPK) f = a.K > 0 ? (double)a.k_keep / (double)a.K : 0.0;

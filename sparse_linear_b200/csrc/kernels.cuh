@@ -19,6 +19,8 @@ struct SelectArgs {
     int T, K;
     int score, sel, n, m, k_keep, dpts, var, first;
     float mom, eps;
+    float tau;                 // AS_SEL_THRESH
+    const float *eta_static;   // S-PTS table [T], or nullptr
     const float *f;  // channel factor (g or c) or nullptr
     float *running_var;
     uint32_t *bitmask;
@@ -41,6 +43,8 @@ struct DecodeArgs {
     int bf16;
     int T, K, n_out;
     int score, sel, n, m, k_keep, dpts;
+    float tau;                 // AS_SEL_THRESH
+    const float *eta_static;   // S-PTS table [T], or nullptr
     const float *g;
     const float *rowsum;
     const uint32_t *mask_in;  // precomputed selection (top-k / all), or nullptr for fused N:M

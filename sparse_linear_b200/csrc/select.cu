@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
     // ---- row statistics: sum x, sum x^2 (float64)
     constexpr int U = 1;  // tiles whose loads are in flight together (more costs occupancy)
     double sx = 0.0, sxx = 0.0;
-    if (a.dpts || a.var) {
+    if (a.dpts == AS_PTS_DYNAMIC || a.var) {
         for (int g0 = tid; g0 < ngroups; g0 += U * NT) {
             float v[U][8];
 #pragma unroll
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
         }
         block_sum2<NT>(sx, sxx, red);
     }
-    const float eta = a.dpts ? (float)(sx / (double)K) : 0.0f;
+    const float eta = a.dpts == AS_PTS_STATIC ? a.eta_static[t] : (a.dpts ? (float)(sx / (double)K) : 0.0f);
     if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
 
     // ---- top-k: scores to shared memory, then an MSB-first radix select of
@@ -245,6 +245,8 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
             uint32_t keep;
             if (a.sel == AS_SEL_NM) {
                 keep = nm_keep_dispatch(s, lane, a.n, a.m);
+            } else if (a.sel == AS_SEL_THRESH) {
+                keep = keep_thresh(s, a.tau);
             } else if (topk) {
                 if (kk <= 0) keep = 0;
                 else if (kk >= K) keep = 0xFF;
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
 
         // ---- row statistics: sum x, sum x^2 (float64)
         double sx = 0.0, sxx = 0.0;
-        if (a.dpts || a.var) {
+        if (a.dpts == AS_PTS_DYNAMIC || a.var) {
             for (int g = tid; g < ngroups; g += SR_THREADS) {
                 float v[8];
                 load8(xr + 8 * g, v);
@@ -408,7 +410,8 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
             }
             block_sum2<SR_THREADS>(sx, sxx, red);
         }
-        const float eta = a.dpts ? (float)(sx / (double)K) : 0.0f;
+        const float eta =
+            a.dpts == AS_PTS_STATIC ? a.eta_static[t] : (a.dpts ? (float)(sx / (double)K) : 0.0f);
         if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
 
         // ---- decisions and outputs, 8 channels per thread per tile.  The
@@ -473,7 +476,10 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
             score8v(v, a.dpts, eta, act && has_f, fv, xh, sc);
             uint32_t keep;
             if constexpr (COMPACT) keep = keep_2of4(sc);
-            else if constexpr (M == 0) keep = a.sel == AS_SEL_NM ? nm_keep_dispatch(sc, lane, a.n, a.m) : 0xFFu;
+            else if constexpr (M == 0)
+                keep = a.sel == AS_SEL_NM       ? nm_keep_dispatch(sc, lane, a.n, a.m)
+                       : a.sel == AS_SEL_THRESH ? keep_thresh(sc, a.tau)
+                                                : 0xFFu;
             else if constexpr (M >= 8) keep = nm_keep_sorted<M>(sc, lane, a.n);
             else keep = nm_keep<M>(sc, lane, a.n);
             if (act) {
@@ -700,8 +706,9 @@ __global__ void __launch_bounds__(SELD_THREADS) k_select_nm_decode(SelectArgs a)
     if (act) load8(xr + c0, v);
     const bool has_f = a.f != nullptr && act;
     if (has_f) load8f(a.f + c0, f);
-    float eta = 0.0f;
-    if (a.dpts) {
+    float eta = a.dpts == AS_PTS_STATIC ? a.eta_static[t] : 0.0f;
+    if (a.dpts == AS_PTS_STATIC && chunk == 0 && tid == 0 && a.eta) a.eta[t] = eta;
+    if (a.dpts == AS_PTS_DYNAMIC) {
         uint4 raw[SELD_ROWREG];
 #pragma unroll
         for (int r = 0; r < SELD_ROWREG; ++r) {
@@ -736,7 +743,7 @@ __global__ void __launch_bounds__(SELD_THREADS) k_select_nm_decode(SelectArgs a)
     }
     float xh[8], sc[8];
     score8(v, a.dpts, eta, has_f ? f : nullptr, 0, xh, sc);
-    uint32_t keep = nm_keep_dispatch(sc, lane, a.n, a.m);
+    uint32_t keep = a.sel == AS_SEL_THRESH ? keep_thresh(sc, a.tau) : nm_keep_dispatch(sc, lane, a.n, a.m);
     if (!act) keep = 0;
     uint32_t word = keep << (8 * (lane & 3));
     word |= __shfl_xor_sync(0xffffffffu, word, 1);

@@ -217,6 +217,15 @@ __device__ __forceinline__ void pos_2of4(uint32_t b, int &i0, int &i1)
     i1 = (b & 8u) ? 3 : ((b & 4u) ? 2 : 1);
 }
 
+// Threshold selection: keep the channels whose score is above tau.
+__device__ __forceinline__ uint32_t keep_thresh(const float (&s)[8], float tau)
+{
+    uint32_t keep = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) keep |= (uint32_t)(s[e] > tau) << e;
+    return keep;
+}
+
 __device__ __forceinline__ uint32_t nm_keep_dispatch(const float (&s)[8], int lane, int n, int m)
 {
     switch (m) {

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(lib):
     for n in declared():
         assert hasattr(raw, n), n
     assert set(lib.EXPORTS) == set(declared())
-    assert lib.as_abi_version() == 1
+    assert lib.as_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -141,3 +141,14 @@ def test_timeout_probe_validates_polls(lib):
     # out-of-range poll counts are refused on the host, before any launch
     for polls in (0, (1 << 20) + 1):
         assert lib._lib.as_probe_timeout(polls, None) == lib.AS_ERR_INVALID_ARG
+
+
+def test_threshold_and_static_pts_validation(lib):
+    # S-PTS without its table, an unknown shift mode, and a NaN threshold are
+    # refused on the host (workspace sizing validates the config too)
+    bad = [lib.config(dpts=lib.AS_PTS_STATIC), lib.config(dpts=3),
+           lib.config(sel=lib.AS_SEL_THRESH, tau=float("nan"))]
+    for cfg in bad:
+        assert lib._lib.as_workspace_size(lib.AS_OP_DECODE, 1, 64, 64, ctypes.byref(cfg)) == ctypes.c_size_t(-1).value
+    ok = lib.config(sel=lib.AS_SEL_THRESH, tau=0.5)
+    assert lib._lib.as_workspace_size(lib.AS_OP_DECODE, 1, 64, 64, ctypes.byref(ok)) != ctypes.c_size_t(-1).value

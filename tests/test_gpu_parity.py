@@ -48,7 +48,17 @@ def test_weight_prep(sl, alpha):
 
 
 # ---------------------------------------------------------------- decode
-def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None):
+def ref_selection(sl, s, cfg):
+    if cfg.sel == sl.AS_SEL_NM:
+        return oracle.select_nm(s, cfg.n, cfg.m)
+    if cfg.sel == sl.AS_SEL_TOPK:
+        return oracle.select_topk(s, cfg.k_keep)
+    if cfg.sel == sl.AS_SEL_THRESH:
+        return oracle.select_thresh(s, cfg.tau)
+    return np.ones_like(s, np.uint8)
+
+
+def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None, eta_static=None):
     """Runs as_linear_decode; checks eta, mask (bit-exact) and y."""
     T, K = x.shape
     L = layer(sl, W, cfg, alpha)
@@ -63,7 +73,11 @@ def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None):
     xf = x.float().numpy()
     eta32 = None
     eta64 = None
-    if cfg.dpts:
+    if cfg.dpts == sl.AS_PTS_STATIC:  # S-PTS: the table itself, bit for bit
+        eta32 = f32(eta_d)
+        np.testing.assert_array_equal(eta32, f32(eta_static))
+        eta64 = eta32.astype(np.float64)
+    elif cfg.dpts:
         eta64 = oracle.token_mean(xf)
         eta32 = f32(eta_d)
         assert (np.abs(eta32 - eta64) <= 1e-6 * np.abs(xf).mean(1)).all()
@@ -75,12 +89,7 @@ def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None):
     else:
         f = None
     s = oracle.score(xf, eta=eta32, f=f)
-    if cfg.sel == sl.AS_SEL_NM:
-        ref_mask = oracle.select_nm(s, cfg.n, cfg.m)
-    elif cfg.sel == sl.AS_SEL_TOPK:
-        ref_mask = oracle.select_topk(s, cfg.k_keep)
-    else:
-        ref_mask = np.ones_like(s, np.uint8)
+    ref_mask = ref_selection(sl, s, cfg)
     got = unpack_bitmask(mask_d, K)
     np.testing.assert_array_equal(got, ref_mask)
     _, rs = oracle.weight_prep(W.float().numpy(), 1.0)
@@ -241,7 +250,7 @@ def test_prefill_24_full_size(sl):
     assert abs(dropped - (4 * p ** 3 * (1 - p) + 2 * p ** 4) / (4 * p)) < 2e-4
 
 
-def check_prefill_masked(sl, xs, W, cfg, alpha=0.0, rows=None):
+def check_prefill_masked(sl, xs, W, cfg, alpha=0.0, rows=None, eta_static=None):
     """Runs select + prefill over a list of batches (VAR running state
     carried); checks statistics, masks and outputs on `rows`."""
     L = layer(sl, W, cfg, alpha)
@@ -262,13 +271,15 @@ def check_prefill_masked(sl, xs, W, cfg, alpha=0.0, rows=None):
         else:
             f = None
         eta32 = f32(bufs["eta"])[rows] if cfg.dpts else None
-        eta64 = oracle.token_mean(xf[rows]) if cfg.dpts else None
-        if cfg.dpts:
-            assert (np.abs(eta32 - eta64) <= 1e-6 * np.abs(xf[rows]).mean(1)).all()
+        if cfg.dpts == sl.AS_PTS_STATIC:
+            np.testing.assert_array_equal(eta32, f32(eta_static)[rows])
+            eta64 = eta32.astype(np.float64)
+        else:
+            eta64 = oracle.token_mean(xf[rows]) if cfg.dpts else None
+            if cfg.dpts:
+                assert (np.abs(eta32 - eta64) <= 1e-6 * np.abs(xf[rows]).mean(1)).all()
         s = oracle.score(xf[rows], eta=eta32, f=f)
-        ref_mask = (oracle.select_nm(s, cfg.n, cfg.m) if cfg.sel == sl.AS_SEL_NM
-                    else oracle.select_topk(s, cfg.k_keep) if cfg.sel == sl.AS_SEL_TOPK
-                    else np.ones_like(s, np.uint8))
+        ref_mask = ref_selection(sl, s, cfg)
         np.testing.assert_array_equal(unpack_bitmask(bufs["bitmask"], K)[rows], ref_mask)
         nu = None
         if cfg.var:
@@ -323,3 +334,53 @@ def test_prefill_clact_var_full_size(sl):
     cfg = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)
     rows = np.array([0, 127, 128, 4097, 8190, 8191])
     check_prefill_masked(sl, xs, W, cfg, rows=rows)
+
+
+# ---------------------------------------------------------------- threshold and S-PTS
+def _tau_for_share(sl, x, W, alpha, share, eta=None):
+    """A threshold that keeps about `share` of the scores (a calibration
+    stand-in: the quantile of the scores of this input)."""
+    from sparse_linear_b200.layer import SparseLinear
+    g = f32(SparseLinear(dev(W), sl.config(), alpha=alpha).g)
+    s = oracle.score(x.float().numpy(), eta=eta, f=g)
+    return float(np.quantile(s, 1.0 - share))
+
+
+@pytest.mark.parametrize("T,dpts", [(1, 1), (2, 0), (8, 1), (13, 0)])
+def test_decode_thresh(sl, T, dpts):
+    x, W, _ = synth.decode_downproj(T)
+    eta = oracle.token_mean(x.float().numpy()).astype(np.float32) if dpts else None
+    tau = _tau_for_share(sl, x, W, 0.5, 0.5, eta)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_THRESH, tau=tau, dpts=dpts)
+    y, got = check_decode(sl, x, W, cfg, alpha=0.5)
+    assert 0.3 < got.mean() < 0.7
+
+
+def test_decode_thresh_fp32_weights(sl):
+    x, W = synth.random_layer(3, 1024, 264, seed=31, dtype=torch.float32)
+    cfg = sl.config(sel=sl.AS_SEL_THRESH, tau=0.4, out_dtype=sl.AS_F32)
+    check_decode(sl, x, W, cfg)
+
+
+@pytest.mark.parametrize("T", [1, 2, 8, 16])
+def test_decode_static_pts(sl, T):
+    """S-PTS: eta from a calibrated table (here: the means of another batch
+    of the same distribution), 8:16 weight-aware."""
+    x, W, _ = synth.decode_downproj(T)
+    calib = synth.decode_downproj(T, seed=91, with_weight=False)[0]
+    eta_static = dev(torch.from_numpy(oracle.token_mean(calib.float().numpy()).astype(np.float32)))
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=sl.AS_PTS_STATIC,
+                    eta_static=eta_static)
+    check_decode(sl, x, W, cfg, alpha=0.5, eta_static=eta_static)
+
+
+def test_prefill_thresh_and_static_pts(sl):
+    T, K, n_out = 200, 2048, 392
+    x, W = synth.random_layer(T, K, n_out, seed=57, dist="laplace")
+    eta_static = dev(torch.from_numpy((0.01 * np.sin(np.arange(T))).astype(np.float32)))
+    cfg = sl.config(sel=sl.AS_SEL_THRESH, tau=0.25, dpts=sl.AS_PTS_STATIC, eta_static=eta_static,
+                    out_dtype=sl.AS_F32)
+    check_prefill_masked(sl, [x], W, cfg, eta_static=eta_static)
+    cfg2 = sl.config(sel=sl.AS_SEL_NM, n=8, m=16, dpts=sl.AS_PTS_STATIC, eta_static=eta_static,
+                     out_dtype=sl.AS_F32)
+    check_prefill_masked(sl, [x], W, cfg2, eta_static=eta_static)

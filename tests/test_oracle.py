@@ -338,3 +338,41 @@ def test_sqrelu_sparsity_closed_form(oracle_lib):
     d = np.maximum(blocks - 2, 0)
     sig = math.sqrt(np.var(d - expect * blocks) / len(blocks)) / (4 * p)
     assert abs(dropped - expect) < 5 * sig, (dropped, expect, sig)
+
+
+# ---------------------------------------------------------------- threshold selection
+def test_thresh_extremes_reduce_to_dense_and_empty(oracle_lib):
+    """tau below every score keeps all (y = x W^T, the dense product); tau at
+    or above the largest score keeps none (y = eta * rowsum with the shift)."""
+    import synth
+    x, W = synth.random_layer(3, 64, 16, seed=41)
+    xf, Wf = x.float().numpy(), W.float().numpy()
+    s = oracle_lib.score(xf)
+    assert oracle_lib.select_thresh(s, -1.0).all()
+    y = oracle_lib.linear(xf, oracle_lib.select_thresh(s, -1.0), Wf)
+    np.testing.assert_allclose(y, xf.astype(np.float64) @ Wf.astype(np.float64).T, rtol=1e-12, atol=1e-12)
+    eta = oracle_lib.token_mean(xf)
+    s_sh = oracle_lib.score(xf, eta=eta.astype(np.float32))
+    none = oracle_lib.select_thresh(s_sh, float(s_sh.max()))
+    assert not none.any()
+    _, rs = oracle_lib.weight_prep(Wf, 1.0)
+    y0 = oracle_lib.linear(xf, none, Wf, eta=eta, rowsum=rs)
+    np.testing.assert_allclose(y0, np.outer(eta, rs), rtol=1e-12, atol=1e-15)
+
+
+def test_thresh_kept_share_matches_laplace_tail(oracle_lib):
+    """|x| for x ~ Laplace(0, b) exceeds tau with probability exp(-tau/b):
+    the kept share over 4 x 2^16 channels lies within 5 sigma of it."""
+    rng = np.random.default_rng(5)
+    b, tau = 0.3, 0.2
+    x = rng.laplace(0.0, b, size=(4, 1 << 16)).astype(np.float32)
+    kept = oracle_lib.select_thresh(oracle_lib.score(x), tau).mean()
+    p = math.exp(-tau / b)
+    assert abs(kept - p) < 5 * math.sqrt(p * (1 - p) / x.size)
+
+
+def test_thresh_is_monotone(oracle_lib):
+    rng = np.random.default_rng(6)
+    s = oracle_lib.score(rng.standard_normal((8, 256)).astype(np.float32))
+    lo, hi = oracle_lib.select_thresh(s, 0.3), oracle_lib.select_thresh(s, 0.9)
+    assert ((hi == 1) <= (lo == 1)).all() and hi.sum() < lo.sum()
