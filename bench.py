@@ -266,6 +266,30 @@ def bench_decode(sl, dev, steps, warmup, world):
         per_t[T] = timed(lambda j, T=T: per_t_graphs[T].replay(), reps) / (reps * N_ROT)
     t_max = max_over_ranks(t_local, world)
 
+    # the same calls with S-PTS: eta from a calibrated table (the token means
+    # of a separate calibration batch) instead of each token's own mean
+    calib = synth.decode_downproj(16, seed=4242, with_weight=False)[0].float()
+    eta_tab = calib.mean(dim=1).to(dev)
+    per_t_spts = {}
+    with torch.cuda.stream(stream):
+        for T in DECODE_TS:
+            tab = eta_tab[:T].contiguous()  # kept alive with the graph below
+            cfg_s = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=sl.AS_PTS_STATIC,
+                              eta_static=tab, out_dtype=sl.AS_BF16)
+
+            def call_s(i, T=T, cfg_s=cfg_s):
+                sl.as_linear_decode(xs[i][:T], Wts[i], cfg_s, ys[T], g=L.g, rowsum=L.rowsum, workspace=wss[T],
+                                    stream=stream)
+            for i in range(N_ROT):
+                call_s(i)
+            stream.synchronize()
+            g_s = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_s, stream=stream):
+                for i in range(N_ROT):
+                    call_s(i)
+            per_t_spts[T] = (timed(lambda j, g_s=g_s: g_s.replay(), reps) / (reps * N_ROT), tab, cfg_s, g_s)
+    per_t_spts = {T: v[0] for T, v in per_t_spts.items()}
+
     # end to end through host buffers, every step: pinned host x -> device,
     # decode, y -> pinned host.  Copies run on their own streams (H2D and D2H
     # use separate copy engines) into double-buffered device x and y, so the
@@ -381,6 +405,7 @@ def bench_decode(sl, dev, steps, warmup, world):
         e2e=tokens * steps * world / t_e2e, e2e_eager=tokens * steps * world / t_e2e_eager, h2d=h2d, d2h=d2h,
         per_t={T: dict(us=per_t[T] * 1e6, gbs=bytes_call[T] / per_t[T] / 1e9, bytes=bytes_call[T])
                for T in DECODE_TS},
+        per_t_spts={T: dict(us=per_t_spts[T] * 1e6, tokens_per_s=T / per_t_spts[T]) for T in DECODE_TS},
         achieved_gbs=step_bytes / kern_time / 1e9, bytes_per_step=step_bytes,
         bytes_per_launch=step_bytes / len(DECODE_TS),
         clocks=clk.summary(), launches=steps * launches_per_step)
@@ -706,8 +731,13 @@ def main():
     }
     if prefill is not None:
         line["prefill"] = prefill
-    if extra is not None:
-        line["configs_extra"] = extra
+    if extra is None:
+        extra = {}
+    extra["decode_downproj_static_pts"] = {
+        "note": "the same decode calls with S-PTS (eta from a calibration table) instead of D-PTS",
+        "per_T": {str(T): v for T, v in d["per_t_spts"].items()},
+        "step_us": sum(v["us"] for v in d["per_t_spts"].values())}
+    line["configs_extra"] = extra
     print(json.dumps(line), flush=True)
 
 
