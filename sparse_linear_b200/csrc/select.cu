@@ -422,27 +422,36 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
         if constexpr (COMPACT) mrow = meta_byte(a.meta24, t, 8 * tid, kt);
         constexpr size_t mstride = (size_t)(8 * SR_THREADS / 128) * 2048;  // bytes per tile
         const bool plain = !a.dpts && !has_f;  // score = |x|
-        double skm = 0.0, skmm = 0.0;
-        for (int tile = 0; tile < ntiles; ++tile) {
-            const int g = tile * SR_THREADS + tid, c0 = 8 * g;
-            const bool act = g < ngroups;
-            if constexpr (COMPACT) {
-                if (plain) {
-                    // score = |x|: compare the bf16 magnitude bits as integers and
-                    // move the kept values as raw 16-bit halves
-                    if (act) {
-                        const uint4 r = *reinterpret_cast<const uint4 *>(xr + c0);
-                        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        if constexpr (COMPACT) {
+            if (plain) {
+                // score = |x|: a thread takes 16 channels (two 2:4 byte groups
+                // whose metadata bytes are adjacent), compares the bf16
+                // magnitude bits as integers and moves the kept values as raw
+                // 16-bit halves: one 16-byte compact store per thread
+                const int ng16 = K >> 4;
+                uint8_t *m16 = meta_byte(a.meta24, t, 16 * tid, kt);
+                constexpr size_t mst16 = (size_t)(16 * SR_THREADS / 128) * 2048;
+                uint8_t *bmr = a.bitmask ? reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words) : nullptr;
+                for (int tile = 0; tile * SR_THREADS < ng16; ++tile) {
+                    const int g16 = tile * SR_THREADS + tid;
+                    if (g16 >= ng16) continue;
+                    const int c0 = 16 * g16;
+                    const uint4 r0 = *reinterpret_cast<const uint4 *>(xr + c0);
+                    const uint4 r1 = *reinterpret_cast<const uint4 *>(xr + c0 + 8);
+                    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                    uint32_t out[4], keepbits = 0, metab = 0;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
                         uint32_t hw[8], mk[8];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            hw[2 * i] = w[i] & 0xFFFFu;
-                            hw[2 * i + 1] = w[i] >> 16;
+                            hw[2 * i] = w[4 * q + i] & 0xFFFFu;
+                            hw[2 * i + 1] = w[4 * q + i] >> 16;
                         }
 #pragma unroll
                         for (int e = 0; e < 8; ++e) mk[e] = hw[e] & 0x7FFFu;
                         const uint32_t keep = keep_2of4(mk);
-                        uint32_t out[2], nib[2];
+                        keepbits |= keep << (8 * q);
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             int i0, i1;
@@ -452,21 +461,27 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                             v0 = i0 == 2 ? hw[4 * h + 2] : v0;
                             v1 = i1 == 2 ? hw[4 * h + 2] : v1;
                             v1 = i1 == 3 ? hw[4 * h + 3] : v1;
-                            out[h] = v0 | (v1 << 16);
-                            nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
+                            out[2 * q + h] = v0 | (v1 << 16);
+                            metab |= ((uint32_t)i0 | ((uint32_t)i1 << 2)) << (8 * q + 4 * h);
                         }
-                        if (a.bitmask) {
-                            uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
-                            bm[g] = (uint8_t)keep;
-                            if (g == ngroups - 1)
-                                for (int b = ngroups; b < words * 4; ++b) bm[b] = 0;
-                        }
-                        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) +
-                                                   c0 / 2) = make_uint2(out[0], out[1]);
-                        mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
                     }
-                    continue;
+                    if (bmr) {
+                        *reinterpret_cast<uint16_t *>(bmr + 2 * g16) = (uint16_t)keepbits;
+                        if (g16 == ng16 - 1)
+                            for (int b = 2 * ng16; b < words * 4; ++b) bmr[b] = 0;
+                    }
+                    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) =
+                        make_uint4(out[0], out[1], out[2], out[3]);
+                    *reinterpret_cast<uint16_t *>(m16 + tile * mst16) = (uint16_t)metab;
                 }
+            }
+        }
+        double skm = 0.0, skmm = 0.0;
+        for (int tile = 0; tile < ntiles; ++tile) {
+            const int g = tile * SR_THREADS + tid, c0 = 8 * g;
+            const bool act = g < ngroups;
+            if constexpr (COMPACT) {
+                if (plain) break;  // done by the 16-channel loop above
             }
             float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, fv[8] = {1, 1, 1, 1, 1, 1, 1, 1}, xh[8], sc[8];
             if (act) {
