@@ -13,6 +13,7 @@ Functions and the passages they follow (page title, section):
 
 * ``weight_prep``   WiSparse page §2.1 eq. (4) (g) and activation-sparsity
                     overview §3.1 (rowsum for the mean shift).
+* ``amber``         overview §2.2.2 (Amber-Pruner channel importance).
 * ``token_mean``    overview §3.1 (D-PTS eta).
 * ``token_var``     overview §3.2 (VAR, unbiased variance).
 * ``channel_energy``/``clact_full``  overview §2.2.3 (CLACT).
@@ -66,6 +67,7 @@ def _load():
             D = ctypes.c_double
             sig = {
                 "or_weight_prep": [P, I, I, D, P, P],
+                "or_amber": [P, I, I, D, D, D, P, P, P],
                 "or_token_mean": [P, I, I, P],
                 "or_token_var": [P, I, I, P],
                 "or_channel_energy": [P, I, I, P],
@@ -103,6 +105,18 @@ def weight_prep(W, alpha: float):
     rs = np.empty(n_out, np.float64)
     _load().or_weight_prep(_ptr(W), n_out, k, float(alpha), _ptr(g), _ptr(rs))
     return g, rs
+
+
+def amber(W, alpha: float = 1.0, lo_pct: float = 0.5, hi_pct: float = 99.5):
+    """Amber-Pruner importance g [k] (float64) and the two percentile values."""
+    W = _f32(W)
+    n_out, k = W.shape
+    g = np.empty(k, np.float64)
+    lo = ctypes.c_double()
+    hi = ctypes.c_double()
+    _load().or_amber(_ptr(W), n_out, k, float(alpha), float(lo_pct), float(hi_pct), _ptr(g),
+                     ctypes.addressof(lo), ctypes.addressof(hi))
+    return g, lo.value, hi.value
 
 
 def token_mean(x):

@@ -16,7 +16,7 @@
  *   [OVW]  "激活稀疏化技术：提升LLM推理效率的动态剪枝方法"
  *          (activation-sparsity overview): section 2.1 N:M patterns,
  *          2.2.1 magnitude pruning, 2.2.3 CLACT score, 3.1 D-PTS,
- *          3.2 VAR variance correction.
+ *          3.2 VAR variance correction, 2.2.2 Amber-Pruner channel importance.
  *   [WIS]  "大模型推理优化：WiSparse激活稀疏化技术解析": section 2.1, eq. (4),
  *          weight-aware score s_i = |x_i| * ||W[:,i]||_2^alpha; section 2.2
  *          per-layer keep fraction (top-k).
@@ -33,6 +33,11 @@
  * VAR: unbiased variances, running variance initialised to the first batch's
  * dense variance and updated with momentum before the scale is formed, scale
  * = sqrt(running / (Var[x*m] + eps)), applied to the whole output row.
+ * Amber-Pruner: a percentile is the order statistic of ascending rank
+ * floor(q (N-1)) of all N weights; weights outside [lo, hi] (inclusive ends)
+ * are dropped and contribute nothing; z uses the population mean and standard
+ * deviation of the kept weights; the exponent alpha of [WIS] eq. (4) also
+ * applies (alpha = 1 gives the plain norm).
  */
 #include <math.h>
 #include <stdint.h>
@@ -68,6 +73,61 @@ void or_weight_prep(const float *W, int n_out, int k, double alpha,
             rowsum[o] = s;
         }
     }
+}
+
+/* ---------------------------------------------------------------------------
+ * Amber-Pruner channel importance.  [OVW] section 2.2.2: remove the weights
+ * beyond the lo/hi percentiles (0.5 and 99.5 on the page), z-score the rest,
+ * and score each input channel by the l2 norm of its standardised weights:
+ *   v_lo, v_hi  = sorted(W)[floor(q (N-1))], q = lo_pct/100, hi_pct/100
+ *   kept        = { W[o,i] : v_lo <= W[o,i] <= v_hi }
+ *   mu, sigma   = mean and population standard deviation of the kept weights
+ *   z[o,i]      = (W[o,i] - mu) / sigma for kept weights, 0 for dropped ones
+ *   g_i         = (sqrt(sum_o z[o,i]^2))^alpha
+ * sigma == 0 (all kept weights equal) gives z = 0 everywhere.
+ * ------------------------------------------------------------------------- */
+static int cmp_float(const void *a, const void *b)
+{
+    float x = *(const float *)a, y = *(const float *)b;
+    return (x > y) - (x < y);
+}
+
+void or_amber(const float *W, int n_out, int k, double alpha, double lo_pct, double hi_pct,
+              double *g, double *v_lo_out, double *v_hi_out)
+{
+    size_t N = (size_t)n_out * k;
+    float *sorted = (float *)malloc(N * sizeof(float));
+    memcpy(sorted, W, N * sizeof(float));
+    qsort(sorted, N, sizeof(float), cmp_float);
+    float v_lo = sorted[(size_t)floor(lo_pct / 100.0 * (double)(N - 1))];
+    float v_hi = sorted[(size_t)floor(hi_pct / 100.0 * (double)(N - 1))];
+    free(sorted);
+
+    double count = 0.0, sum = 0.0;
+    for (size_t j = 0; j < N; j++)
+        if (W[j] >= v_lo && W[j] <= v_hi) {
+            count += 1.0;
+            sum += (double)W[j];
+        }
+    double mu = count > 0.0 ? sum / count : 0.0;
+    double ss = 0.0;
+    for (size_t j = 0; j < N; j++)
+        if (W[j] >= v_lo && W[j] <= v_hi) ss += ((double)W[j] - mu) * ((double)W[j] - mu);
+    double sigma = count > 0.0 ? sqrt(ss / count) : 0.0;
+
+    for (int i = 0; i < k; i++) {
+        double zz = 0.0;
+        for (int o = 0; o < n_out; o++) {
+            float w = W[(size_t)o * k + i];
+            if (w >= v_lo && w <= v_hi && sigma > 0.0) {
+                double z = ((double)w - mu) / sigma;
+                zz += z * z;
+            }
+        }
+        g[i] = pow(sqrt(zz), alpha);
+    }
+    if (v_lo_out) *v_lo_out = (double)v_lo;
+    if (v_hi_out) *v_hi_out = (double)v_hi;
 }
 
 /* [OVW] section 3.1: eta_t = mean over the channels of token t. */

@@ -27,6 +27,11 @@ no model weights or datasets are used):
                       W bf16 [4096, 14336] ~ N(0, 0.02^2), seed 3.
 * ``prefill_clact``   x bf16 [8192, 8192] ~ 0.5 * Student-t(3) per batch
                       (8 batches), W bf16 [8192, 8192] ~ N(0, 0.02^2), seed 4.
+* ``outlier_weight``  W [n_out, k], a two-component mixture: each weight is
+                      N(-0.02, 0.01^2) or N(+0.02, 0.01^2) with probability
+                      1/2 (a bimodal layer), and a seeded 0.2% of the entries
+                      replaced by +-U[0.5, 1.0] (outliers), seed 5.  Default
+                      shape: the v-projection [1024, 4096].
 """
 from __future__ import annotations
 
@@ -36,7 +41,7 @@ import torch
 __all__ = [
     "streams", "to_dtype", "tiny_layer", "decode_downproj", "decode_block",
     "prefill_sqrelu", "prefill_clact_weight", "prefill_clact_batch",
-    "random_layer", "BLOCK_LAYERS",
+    "random_layer", "BLOCK_LAYERS", "outlier_weight",
 ]
 
 
@@ -168,3 +173,17 @@ def random_layer(T: int, k: int, n_out: int, seed: int, dtype=torch.bfloat16,
     x = to_dtype(x64, dtype)
     w = to_dtype(rw.normal(0.0, 0.02, size=(n_out, k)), dtype)
     return x, w
+
+
+def outlier_weight(seed: int = 5, n_out: int = 1024, k: int = 4096, dtype=torch.bfloat16,
+                   outlier_frac: float = 0.002):
+    """Bimodal weight with a few large outliers (see the module recipe)."""
+    rm, rn, ro, rs, rv = streams(seed, 5)
+    mode = np.where(rm.random(size=(n_out, k)) < 0.5, -0.02, 0.02)
+    w = mode + rn.normal(0.0, 0.01, size=(n_out, k))
+    n_o = int(round(outlier_frac * n_out * k))
+    if n_o:
+        idx = ro.choice(n_out * k, size=n_o, replace=False)
+        sign = np.where(rs.random(size=n_o) < 0.5, -1.0, 1.0)
+        w.reshape(-1)[idx] = sign * rv.uniform(0.5, 1.0, size=n_o)
+    return to_dtype(w, dtype)

@@ -376,3 +376,98 @@ def test_thresh_is_monotone(oracle_lib):
     s = oracle_lib.score(rng.standard_normal((8, 256)).astype(np.float32))
     lo, hi = oracle_lib.select_thresh(s, 0.3), oracle_lib.select_thresh(s, 0.9)
     assert ((hi == 1) <= (lo == 1)).all() and hi.sum() < lo.sum()
+
+
+# ---------------------------------------------------------------- Amber-Pruner importance
+def test_amber_2x2_closed_form(oracle_lib):
+    """W = [[1, 2], [3, 4]], all kept: mean 2.5, population variance 1.25,
+    each column's z = +-(1.5, 0.5)/sqrt(1.25), so sum z^2 = 2 per column."""
+    W = np.array([[1, 2], [3, 4]], np.float32)
+    for alpha, want in ((1.0, math.sqrt(2.0)), (2.0, 2.0), (0.5, 2.0 ** 0.25)):
+        g, lo, hi = oracle_lib.amber(W, alpha, 0.0, 100.0)
+        np.testing.assert_allclose(g, [want, want], rtol=1e-14)
+        assert (lo, hi) == (1.0, 4.0)
+
+
+def test_amber_keep_all_is_standardised_column_norm(oracle_lib):
+    """0th..100th percentile keeps every weight; the importance is then the
+    column norm of numpy's population z-score (np.std, ddof=0)."""
+    import synth
+    W = synth.outlier_weight(seed=7, n_out=96, k=40, dtype=torch.float32).numpy()
+    W64 = W.astype(np.float64)
+    Z = (W64 - W64.mean()) / W64.std()
+    for alpha in (1.0, 0.5):
+        g, _, _ = oracle_lib.amber(W, alpha, 0.0, 100.0)
+        np.testing.assert_allclose(g, np.linalg.norm(Z, axis=0) ** alpha, rtol=1e-12)
+
+
+def test_amber_percentiles_are_numpy_lower_order_statistics(oracle_lib):
+    """The clip values equal numpy's percentile with method='lower' (the
+    order statistic of rank floor(q (N-1))) for several q and sizes."""
+    import synth
+    for (n_out, k, seed) in ((100, 37, 8), (256, 512, 9), (1, 7, 10)):
+        W = synth.outlier_weight(seed=seed, n_out=n_out, k=k, dtype=torch.float32).numpy()
+        for lo_p, hi_p in ((0.5, 99.5), (0.0, 100.0), (10.0, 90.0), (37.3, 62.9)):
+            _, lo, hi = oracle_lib.amber(W, 1.0, lo_p, hi_p)
+            assert lo == float(np.percentile(W, lo_p, method="lower"))
+            assert hi == float(np.percentile(W, hi_p, method="lower"))
+
+
+def test_amber_sum_of_squared_importance_counts_kept_weights(oracle_lib):
+    """With alpha = 1, sum_i g_i^2 = sum of z^2 over the kept weights = the
+    number of kept weights (population variance); a sample variance, a
+    missing mean subtraction or clipping in place of dropping breaks it."""
+    import synth
+    W = synth.outlier_weight(seed=11, n_out=200, k=64, dtype=torch.float32).numpy()
+    g, lo, hi = oracle_lib.amber(W, 1.0, 0.5, 99.5)
+    kept = int(((W >= lo) & (W <= hi)).sum())
+    assert kept < W.size
+    np.testing.assert_allclose((g ** 2).sum(), kept, rtol=1e-12)
+
+
+def test_amber_drops_outliers(oracle_lib):
+    """One far outlier beyond the 99.5th percentile leaves the importance as
+    it was without it, except in its own column and the column of the weight
+    at the new clip edge; kept in (0..100 window) it would swamp sigma."""
+    rng = np.random.default_rng(12)
+    W = rng.normal(0.0, 0.02, size=(400, 50)).astype(np.float32)
+    g0, _, _ = oracle_lib.amber(W, 1.0, 0.0, 99.5)
+    W2 = W.copy()
+    W2[3, 7] = 100.0
+    g2, _, hi2 = oracle_lib.amber(W2, 1.0, 0.0, 99.5)
+    assert hi2 < 1.0
+    rel = np.abs(g2 - g0) / g0
+    assert (rel > 1e-3).sum() <= 2 and rel.max() < 2e-2
+    g_all, _, _ = oracle_lib.amber(W2, 1.0, 0.0, 100.0)
+    assert (g_all[np.arange(50) != 7] < 0.1 * g0[np.arange(50) != 7]).all()
+
+
+def test_amber_affine_invariance(oracle_lib):
+    """z-scores are unchanged by W -> a W + b with a > 0 (the percentiles
+    move with W, the kept set is the same).  Weights on a 1/64 grid keep
+    a = 4, b = 3 exact in float32."""
+    rng = np.random.default_rng(13)
+    W = (rng.integers(-64, 65, size=(60, 30)) / 64.0).astype(np.float32)
+    g, lo, hi = oracle_lib.amber(W, 1.0, 0.5, 99.5)
+    g2, lo2, hi2 = oracle_lib.amber((4.0 * W + 3.0).astype(np.float32), 1.0, 0.5, 99.5)
+    assert (lo2, hi2) == (4 * lo + 3, 4 * hi + 3)
+    np.testing.assert_allclose(g2, g, rtol=1e-12)
+    # a < 0 mirrors the distribution: the kept set changes only at the ends.
+    perm = rng.permutation(30)
+    g3, _, _ = oracle_lib.amber(W[:, perm], 1.0, 0.5, 99.5)
+    np.testing.assert_allclose(g3, g[perm], rtol=1e-12)
+
+
+def test_amber_ties_at_the_clip_values_are_kept(oracle_lib):
+    """Values equal to a clip value are kept (inclusive ends); a 50..50
+    window keeps only the median value, so sigma = 0 and g = 0."""
+    W = np.array([[0, 1, 1, 2], [2, 2, 1, 0], [1, 2, 2, 2]], np.float32)
+    g, lo, hi = oracle_lib.amber(W, 1.0, 20.0, 80.0)
+    # sorted: 0 0 1 1 1 1 2 2 2 2 2 2; ranks floor(.2*11)=2 -> 1, floor(.8*11)=8 -> 2
+    assert (lo, hi) == (1.0, 2.0)
+    kept = W[W >= 1].astype(np.float64)
+    mu, sd = kept.mean(), kept.std()
+    Z = np.where(W >= 1, (W - mu) / sd, 0.0)
+    np.testing.assert_allclose(g, np.linalg.norm(Z, axis=0), rtol=1e-12)
+    g0, lo0, hi0 = oracle_lib.amber(W, 1.0, 50.0, 50.0)
+    assert lo0 == hi0 == 1.0 and not g0.any()
