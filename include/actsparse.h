@@ -150,6 +150,32 @@ as_status as_weight_prep(const void *W, as_dtype dt, int n_out, int K, float alp
                          void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Amber-Pruner channel importance, once per layer ([OVW] 2.2.2): the weights
+ * outside the lo/hi percentiles are dropped, the rest standardised by their
+ * own mean and standard deviation, and each input channel scored by the l2
+ * norm of its standardised weights.  Feed g as the chan_factor of
+ * AS_SCORE_WEIGHT (score s_ti = |x_ti| * g_i).
+ *   W       [n_out, K] in `dt` (input); finite values.
+ *   lo_pct, hi_pct: percentiles in [0, 100], lo_pct <= hi_pct (0.5 and 99.5
+ *           on the page).  A percentile is the value of ascending rank
+ *           floor(pct/100 * (N-1)) among all N = n_out*K weights (exact
+ *           order statistic; -0 and +0 are equal); N < 2^32.
+ *   kept:   v_lo <= W[o,i] <= v_hi (both ends inclusive).  mu and sigma are
+ *           the mean and population standard deviation of the kept weights
+ *           (float64); z[o,i] = (W[o,i] - mu) / sigma for kept weights, 0 for
+ *           dropped ones, and 0 everywhere when sigma == 0.
+ *   g       [K] float32 (output): (sqrt(sum_o z[o,i]^2))^alpha.
+ *   bounds  [2] float32 (output, optional): v_lo, v_hi.
+ *   Workspace: as_workspace_size(AS_OP_AMBER, 0, K, n_out, NULL); no
+ *   zero-fill needed.  Deterministic (fixed reduction order).
+ *   AS_ERR_INVALID_ARG for a NULL W or g, or percentiles out of range;
+ *   AS_ERR_SHAPE when N >= 2^32.
+ * ------------------------------------------------------------------------ */
+as_status as_weight_prep_amber(const void *W, as_dtype dt, int n_out, int K, float alpha,
+                               double lo_pct, double hi_pct, float *g, float *bounds,
+                               void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
  * Score + selection + compensation statistics for T tokens (prefill side, or
  * to inspect a decode selection).  x [T, K] in `dt`.
  *   chan_factor: g [K] for AS_SCORE_WEIGHT (required); ignored otherwise
@@ -241,7 +267,7 @@ as_status as_linear_decode_noalloc(const void *x, as_dtype dt, int T, int K, int
                                    float *eta_out, float *colnorm_out, cudaStream_t stream);
 
 /* Which operation a workspace size is asked for. */
-enum { AS_OP_WEIGHT_PREP = 0, AS_OP_SELECT = 1, AS_OP_DECODE = 2, AS_OP_PREFILL = 3 };
+enum { AS_OP_WEIGHT_PREP = 0, AS_OP_SELECT = 1, AS_OP_DECODE = 2, AS_OP_PREFILL = 3, AS_OP_AMBER = 4 };
 
 /* Bytes of workspace the operation needs (0 if none); (size_t)-1 if the
  * arguments are invalid. */

@@ -32,13 +32,14 @@ AS_F32, AS_BF16 = 0, 1
 AS_SCORE_MAG, AS_SCORE_WEIGHT, AS_SCORE_CLACT = 0, 1, 2
 AS_SEL_NM, AS_SEL_TOPK, AS_SEL_ALL, AS_SEL_THRESH = 0, 1, 2, 3
 AS_PTS_OFF, AS_PTS_DYNAMIC, AS_PTS_STATIC = 0, 1, 2
-AS_OP_WEIGHT_PREP, AS_OP_SELECT, AS_OP_DECODE, AS_OP_PREFILL = 0, 1, 2, 3
+AS_OP_WEIGHT_PREP, AS_OP_SELECT, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_AMBER = 0, 1, 2, 3, 4
 AS_MAX_DECODE_T = 16
 
 EXPORTS = [
     "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
     "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches", "as_probe_timeout",
+    "as_weight_prep_amber",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -60,6 +61,7 @@ class as_select_out(ctypes.Structure):
 _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _sig = {
     "as_weight_prep": ([_P, _I, _I, _I, _F, _P, _P, _P, _P, _S, _P], _I),
+    "as_weight_prep_amber": ([_P, _I, _I, _I, _F, ctypes.c_double, ctypes.c_double, _P, _P, _P, _S, _P], _I),
     "as_select": ([_P, _I, _I, _I, ctypes.POINTER(as_config), _P, _P, _I,
                    ctypes.POINTER(as_select_out), _P, _S, _P], _I),
     "as_linear_decode": ([_P, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(as_config), _P, _P, _P, _P,
@@ -164,6 +166,15 @@ def as_weight_prep(W, alpha: float, Wt=None, g=None, rowsum=None, workspace=None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_lib.as_weight_prep(_ptr(W), _dt(W), n_out, K, float(alpha), _ptr(Wt), _ptr(g), _ptr(rowsum),
                                _ptr(workspace), ws_bytes, _stream(stream)), "as_weight_prep")
+
+
+def as_weight_prep_amber(W, g, alpha: float = 1.0, lo_pct: float = 0.5, hi_pct: float = 99.5,
+                         bounds=None, workspace=None, stream=None) -> None:
+    n_out, K = W.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_weight_prep_amber(_ptr(W), _dt(W), n_out, K, float(alpha), float(lo_pct), float(hi_pct),
+                                     _ptr(g), _ptr(bounds), _ptr(workspace), ws_bytes, _stream(stream)),
+           "as_weight_prep_amber")
 
 
 def as_select(x, cfg: as_config, out: as_select_out, chan_factor=None, running_var=None,

@@ -106,6 +106,9 @@ size_t as_workspace_size(int op, int T, int K, int n_out, const as_config *cfg)
     case AS_OP_PREFILL:
         if (T <= 0 || n_out <= 0 || check_cfg(cfg, K) != AS_OK) return (size_t)-1;
         return 0;
+    case AS_OP_AMBER:
+        if (n_out <= 0) return (size_t)-1;
+        return amber_workspace(n_out, K);
     }
     return (size_t)-1;
 }
@@ -121,6 +124,24 @@ as_status as_weight_prep(const void *W, as_dtype dt, int n_out, int K, float alp
         if (!aligned16(workspace)) return AS_ERR_ALIGN;
     }
     return cuda_status(launch_weight_prep(W, dt == AS_BF16, n_out, K, alpha, Wt, g, rowsum, workspace, stream));
+}
+
+as_status as_weight_prep_amber(const void *W, as_dtype dt, int n_out, int K, float alpha, double lo_pct,
+                               double hi_pct, float *g, float *bounds, void *workspace, size_t ws_bytes,
+                               cudaStream_t stream)
+{
+    if (!W || !g || n_out <= 0 || K <= 0) return AS_ERR_INVALID_ARG;
+    if (!(lo_pct >= 0.0 && lo_pct <= hi_pct && hi_pct <= 100.0)) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    const uint64_t N = (uint64_t)n_out * (uint64_t)K;
+    if (N >= (1ull << 32)) return AS_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(g) || !aligned16(bounds)) return AS_ERR_ALIGN;
+    if (!workspace || ws_bytes < amber_workspace(n_out, K)) return AS_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return AS_ERR_ALIGN;
+    // Ascending ranks of the two percentile values among the N weights.
+    const uint32_t r_lo = (uint32_t)floor(lo_pct / 100.0 * (double)(N - 1));
+    const uint32_t r_hi = (uint32_t)floor(hi_pct / 100.0 * (double)(N - 1));
+    return cuda_status(launch_amber(W, dt == AS_BF16, n_out, K, alpha, r_lo, r_hi, g, bounds, workspace, stream));
 }
 
 as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *cfg, const float *chan_factor,

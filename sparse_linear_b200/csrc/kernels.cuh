@@ -11,6 +11,10 @@ namespace as {
 size_t weight_prep_workspace(int n_out, int k);
 cudaError_t launch_weight_prep(const void *W, int bf16, int n_out, int k, float alpha, void *Wt, float *g,
                                float *rowsum, void *ws, cudaStream_t st);
+// Amber-Pruner importance: ranks of the two percentile weights (ascending).
+size_t amber_workspace(int n_out, int k);
+cudaError_t launch_amber(const void *W, int bf16, int n_out, int k, float alpha, uint32_t rank_lo, uint32_t rank_hi,
+                         float *g, float *bounds, void *ws, cudaStream_t st);
 
 // ------------------------------------------------------------ select
 struct SelectArgs {

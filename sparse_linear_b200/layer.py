@@ -9,9 +9,10 @@ from __future__ import annotations
 
 import torch
 
-from . import (AS_BF16, AS_F32, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_SELECT, AS_OP_WEIGHT_PREP,
-               AS_SCORE_CLACT, AS_SEL_NM, as_linear_decode, as_linear_prefill, as_meta24_words,
-               as_select, as_weight_prep, as_workspace_size, select_out)
+from . import (AS_BF16, AS_F32, AS_OP_AMBER, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_SELECT,
+               AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SEL_NM, as_linear_decode, as_linear_prefill,
+               as_meta24_words, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size,
+               select_out)
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -25,9 +26,15 @@ class SparseLinear:
     W: [n_out, K] bf16 or f32 CUDA tensor (PyTorch Linear layout).
     cfg: ``as_config``; ``alpha`` is the weight-aware exponent.
     ``keep_wt`` builds the channel-major copy needed by the decode path.
+    ``importance`` picks the channel factor g of the weight-aware score:
+    ``"norm"`` (column norm of W) or ``"amber"`` (Amber-Pruner: column norm
+    of the standardised weights inside the ``amber_pct`` percentiles).
     """
 
-    def __init__(self, W: torch.Tensor, cfg, alpha: float = 0.0, keep_wt: bool = True):
+    def __init__(self, W: torch.Tensor, cfg, alpha: float = 0.0, keep_wt: bool = True,
+                 importance: str = "norm", amber_pct: tuple[float, float] = (0.5, 99.5)):
+        if importance not in ("norm", "amber"):
+            raise ValueError(f"unknown importance {importance!r}")
         self.W = W.contiguous()
         self.cfg = cfg
         self.alpha = float(alpha)
@@ -37,7 +44,15 @@ class SparseLinear:
         self.rowsum = torch.empty(self.n_out, dtype=torch.float32, device=dev)
         self.Wt = torch.empty(self.K, self.n_out, dtype=W.dtype, device=dev) if keep_wt else None
         ws = workspace(as_workspace_size(AS_OP_WEIGHT_PREP, 0, self.K, self.n_out, None), dev)
-        as_weight_prep(self.W, self.alpha, Wt=self.Wt, g=self.g, rowsum=self.rowsum, workspace=ws)
+        amber = importance == "amber"
+        as_weight_prep(self.W, self.alpha, Wt=self.Wt, g=None if amber else self.g, rowsum=self.rowsum,
+                       workspace=ws)
+        self.amber_bounds = None
+        if amber:
+            self.amber_bounds = torch.empty(4, dtype=torch.float32, device=dev)
+            ws = workspace(as_workspace_size(AS_OP_AMBER, 0, self.K, self.n_out, None), dev)
+            as_weight_prep_amber(self.W, self.g, self.alpha, amber_pct[0], amber_pct[1],
+                                 bounds=self.amber_bounds, workspace=ws)
         self._ws = {}
 
     def _workspace(self, op: int, T: int) -> torch.Tensor:

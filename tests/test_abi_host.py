@@ -152,3 +152,28 @@ def test_threshold_and_static_pts_validation(lib):
         assert lib._lib.as_workspace_size(lib.AS_OP_DECODE, 1, 64, 64, ctypes.byref(cfg)) == ctypes.c_size_t(-1).value
     ok = lib.config(sel=lib.AS_SEL_THRESH, tau=0.5)
     assert lib._lib.as_workspace_size(lib.AS_OP_DECODE, 1, 64, 64, ctypes.byref(ok)) != ctypes.c_size_t(-1).value
+
+
+def test_amber_validation_launches_nothing(lib):
+    """Percentiles out of [0, 100] or reversed, NULL outputs, too many
+    weights and a short workspace are refused on the host (fake addresses:
+    any launch would fail here without a GPU)."""
+    fake = 1 << 20
+    f = lib._lib.as_weight_prep_amber
+    ws = lib.as_workspace_size(lib.AS_OP_AMBER, 0, 4096, 1024, None)
+    assert ws == 4096 + 296 * 16 + 4 * 4096 * 8
+
+    def call(W=fake, n_out=1024, K=4096, lo=0.5, hi=99.5, g=fake, b=None, w=fake, wb=ws, dt=lib.AS_BF16):
+        return f(W, dt, n_out, K, 1.0, lo, hi, g, b, w, wb, None)
+
+    assert call(lo=-0.1) == lib.AS_ERR_INVALID_ARG
+    assert call(hi=100.5) == lib.AS_ERR_INVALID_ARG
+    assert call(lo=60.0, hi=40.0) == lib.AS_ERR_INVALID_ARG
+    assert call(lo=float("nan")) == lib.AS_ERR_INVALID_ARG
+    assert call(W=None) == lib.AS_ERR_INVALID_ARG
+    assert call(g=None) == lib.AS_ERR_INVALID_ARG
+    assert call(n_out=65536, K=65536) == lib.AS_ERR_SHAPE
+    assert call(dt=5) == lib.AS_ERR_DTYPE
+    assert call(b=fake + 8) == lib.AS_ERR_ALIGN
+    assert call(w=None) == lib.AS_ERR_WORKSPACE
+    assert call(wb=ws - 1) == lib.AS_ERR_WORKSPACE

@@ -30,9 +30,9 @@ def dev(t):
     return t.cuda().contiguous()
 
 
-def layer(sl, W, cfg, alpha=0.0):
+def layer(sl, W, cfg, alpha=0.0, importance="norm"):
     from sparse_linear_b200.layer import SparseLinear
-    return SparseLinear(dev(W), cfg, alpha=alpha)
+    return SparseLinear(dev(W), cfg, alpha=alpha, importance=importance)
 
 
 # ---------------------------------------------------------------- weight prep
@@ -47,6 +47,57 @@ def test_weight_prep(sl, alpha):
     assert torch.equal(L.Wt.cpu(), W.t().contiguous())
 
 
+# ---------------------------------------------------------------- Amber-Pruner importance
+@pytest.mark.parametrize("n_out,K,lo,hi,alpha,dtype", [
+    (1024, 4096, 0.5, 99.5, 1.0, torch.bfloat16),   # v-projection shape
+    (4096, 11008, 0.5, 99.5, 0.5, torch.bfloat16),  # down-projection, full size
+    (37, 250, 0.5, 99.5, 1.0, torch.float32),       # ragged
+    (300, 1000, 10.0, 90.0, 0.5, torch.bfloat16),
+    (1, 7, 0.0, 100.0, 1.0, torch.float32),         # one row, keep all
+    (64, 64, 50.0, 50.0, 1.0, torch.bfloat16),      # one value kept: sigma 0, g 0
+])
+def test_amber_importance(sl, n_out, K, lo, hi, alpha, dtype):
+    """Clip values are the exact order statistics; g within float32 rounding
+    of the float64 oracle.  The workspace starts as 0xFF bytes: no zero-fill
+    is needed."""
+    W = synth.outlier_weight(seed=31, n_out=n_out, k=K, dtype=dtype)
+    g = torch.empty(K, dtype=torch.float32, device="cuda")
+    b = torch.empty(4, dtype=torch.float32, device="cuda")
+    ws = torch.full((sl.as_workspace_size(sl.AS_OP_AMBER, 0, K, n_out, None),), 255, dtype=torch.uint8,
+                    device="cuda")
+    sl.as_weight_prep_amber(dev(W), g, alpha, lo, hi, bounds=b, workspace=ws)
+    torch.cuda.synchronize()
+    g_ref, v_lo, v_hi = oracle.amber(W.float().numpy(), alpha, lo, hi)
+    bb = f32(b)
+    assert (bb[0], bb[1]) == (v_lo, v_hi)
+    np.testing.assert_allclose(f32(g), g_ref, rtol=1e-6, atol=0)
+
+
+def test_amber_deterministic(sl):
+    W = dev(synth.outlier_weight(seed=32))
+    out = []
+    for _ in range(2):
+        g = torch.empty(W.shape[1], dtype=torch.float32, device="cuda")
+        ws = torch.empty(sl.as_workspace_size(sl.AS_OP_AMBER, 0, W.shape[1], W.shape[0], None),
+                         dtype=torch.uint8, device="cuda")
+        sl.as_weight_prep_amber(W, g, workspace=ws)
+        out.append(g)
+    assert torch.equal(out[0], out[1])
+
+
+def test_decode_amber_importance(sl):
+    """Weight-aware 8:16 decode with D-PTS on the Amber-Pruner channel
+    factors of a bimodal weight with outliers (the layer's g is checked
+    against the oracle first, then used as the score factor)."""
+    x, _, _ = synth.decode_downproj(T=4, k=4096, with_weight=False)
+    W = synth.outlier_weight(seed=33, n_out=1024, k=4096)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
+    L = layer(sl, W, cfg, 1.0, "amber")
+    g_ref, _, _ = oracle.amber(W.float().numpy(), 1.0)
+    np.testing.assert_allclose(f32(L.g), g_ref, rtol=1e-6)
+    check_decode(sl, x, W, cfg, alpha=1.0, importance="amber")
+
+
 # ---------------------------------------------------------------- decode
 def ref_selection(sl, s, cfg):
     if cfg.sel == sl.AS_SEL_NM:
@@ -58,10 +109,10 @@ def ref_selection(sl, s, cfg):
     return np.ones_like(s, np.uint8)
 
 
-def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None, eta_static=None):
+def check_decode(sl, x, W, cfg, alpha=0.0, tol=None, f_override=None, eta_static=None, importance="norm"):
     """Runs as_linear_decode; checks eta, mask (bit-exact) and y."""
     T, K = x.shape
-    L = layer(sl, W, cfg, alpha)
+    L = layer(sl, W, cfg, alpha, importance)
     xd = dev(x)
     words = (K + 31) // 32
     mask_d = torch.zeros(T, words, dtype=torch.int32, device="cuda")
