@@ -27,6 +27,10 @@ Functions and the passages they follow (page title, section):
 * ``var_scale``     overview §3.2.
 * ``linear``        overview §3.1 / §3.2 and the layer definition y = prune(x) W^T.
 * ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
+* ``e4m3_encode``/``e4m3_decode``, ``quant_rows_fp8``, ``sqrelu24_fp8``,
+  ``linear_fp8``    2:4 + Squared-ReLU page §3.1 (fused Squared-ReLU + 2:4 +
+                    FP8 producer, FP8 row-scaled GEMM) and §5.3 (sparsify
+                    before quantising).
 """
 from __future__ import annotations
 
@@ -79,11 +83,17 @@ def _load():
                 "or_var_scale": [P, P, I, I, P, D, D, P, P, P, P],
                 "or_linear": [P, P, I, I, P, P, I, P, P, P, I, P],
                 "or_compress_nm": [P, P, I, I, I, I, P, P],
+                "or_quant_rows_fp8": [P, I, I, P, P],
+                "or_sqrelu24_fp8": [P, I, I, P, P, P, P, P],
             }
             for name, args in sig.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
                 fn.restype = None
+            lib.or_e4m3_encode.argtypes = [D]
+            lib.or_e4m3_encode.restype = ctypes.c_uint8
+            lib.or_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.or_e4m3_decode.restype = D
             _lib = lib
     return _lib
 
@@ -231,3 +241,78 @@ def compress_nm(v, mask, n: int, m: int):
     pos = np.empty((T, kc), np.uint8)
     _load().or_compress_nm(_ptr(v), _ptr(mask), T, k, int(n), int(m), _ptr(vals), _ptr(pos))
     return vals, pos
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """E4M3 codes (uint8) of float64 values: nearest, ties to even, clamp at 448."""
+    lib = _load()
+    v = np.asarray(v, np.float64)
+    return np.array([lib.or_e4m3_encode(float(a)) for a in v.reshape(-1)], np.uint8).reshape(v.shape)
+
+
+def e4m3_decode(c) -> np.ndarray:
+    """float64 values of E4M3 codes."""
+    lib = _load()
+    c = np.asarray(c, np.uint8)
+    return np.array([lib.or_e4m3_decode(int(a)) for a in c.reshape(-1)], np.float64).reshape(c.shape)
+
+
+def quant_rows_fp8(W):
+    """W [n_out, k] -> (codes uint8 [n_out, k], scale float32 [n_out])."""
+    W = _f32(W)
+    n_out, k = W.shape
+    codes = np.empty((n_out, k), np.uint8)
+    scale = np.empty(n_out, np.float32)
+    _load().or_quant_rows_fp8(_ptr(W), n_out, k, _ptr(codes), _ptr(scale))
+    return codes, scale
+
+
+def sqrelu24_fp8(z):
+    """Fused producer from bf16 z [T, k] (torch tensor or uint16 bit array).
+
+    Returns dict mask [T, k], codes [T, k/2], pos [T, k/2], scale [T], x [T, k].
+    """
+    if hasattr(z, "view") and not isinstance(z, np.ndarray):
+        import torch
+        z = z.contiguous().view(torch.int16).numpy().view(np.uint16)
+    z = np.ascontiguousarray(z, np.uint16)
+    T, k = z.shape
+    if k % 4:
+        raise ValueError("k must be a multiple of 4")
+    out = dict(mask=np.empty((T, k), np.uint8), codes=np.empty((T, k // 2), np.uint8),
+               pos=np.empty((T, k // 2), np.uint8), scale=np.empty(T, np.float32),
+               x=np.empty((T, k), np.float32))
+    _load().or_sqrelu24_fp8(_ptr(z), T, k, _ptr(out["mask"]), _ptr(out["codes"]), _ptr(out["pos"]),
+                            _ptr(out["scale"]), _ptr(out["x"]))
+    return out
+
+
+_E4M3 = None
+
+
+def _e4m3_table():
+    global _E4M3
+    if _E4M3 is None:
+        _E4M3 = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return _E4M3
+
+
+def dequant_fp8(codes, scale):
+    """float64 codes * row scale."""
+    return _e4m3_table()[np.asarray(codes, np.uint8)] * np.asarray(scale, np.float64).reshape(-1, 1)
+
+
+def linear_fp8(x_codes, x_pos, x_scale, w_codes, w_scale, rows=None):
+    """float64 y [T, n_out] of the FP8 2:4 GEMM: the kept values (codes at
+    their block positions, times the token's scale) against the dequantised
+    weight (codes times the output row's scale), summed in float64."""
+    x_codes = np.asarray(x_codes, np.uint8)
+    x_pos = np.asarray(x_pos, np.uint8)
+    if rows is not None:
+        x_codes, x_pos, x_scale = x_codes[rows], x_pos[rows], np.asarray(x_scale)[rows]
+    T, kc = x_codes.shape
+    k = 2 * kc
+    xd = np.zeros((T, k), np.float64)
+    col = (np.arange(kc) // 2) * 4 + x_pos.astype(np.int64)
+    np.put_along_axis(xd, col, dequant_fp8(x_codes, x_scale), axis=1)
+    return xd @ dequant_fp8(w_codes, w_scale).T

@@ -22,7 +22,9 @@
  *          per-layer keep fraction (top-k).
  *   [SQR]  "利用2:4稀疏性与Squared-ReLU加速Transformer训练与推理": section 2.1
  *          2:4 pattern, 2.3 dropping the smallest of a 3-nonzero block,
- *          3.3 compressed layout with the kept values stored contiguously.
+ *          3.3 compressed layout with the kept values stored contiguously,
+ *          3.1 fused Squared-ReLU + 2:4 + FP8 producer and the FP8
+ *          row-scaled 2:4 GEMM, 5.3 sparsify before quantising.
  *
  * Readings where the pages are silent or disagree (all listed in the design
  * notes): exactly N per M-block (or exactly k per token), equal float32
@@ -38,11 +40,19 @@
  * are dropped and contribute nothing; z uses the population mean and standard
  * deviation of the kept weights; the exponent alpha of [WIS] eq. (4) also
  * applies (alpha = 1 gives the plain norm).
+ * FP8 ([SQR] 3.1 names FP8 and row scaling but no format or scale rule):
+ * E4M3 with round-to-nearest-even and saturation at 448; one float32 scale
+ * per row (token row of the activation, output row of the weight),
+ * scale = amax / 448 over the row's kept values (1 for an all-zero row),
+ * code = E4M3(fl32(v / scale)); the activation is sparsified first ([SQR]
+ * 5.3), so its amax runs over the kept values only.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+
+void or_select_nm(const float *s, int T, int k, int n, int m, uint8_t *mask);
 
 /* ---------------------------------------------------------------------------
  * Weight preparation.  [WIS] section 2.1, eq. (4): g_i = (||W[:,i]||_2)^alpha,
@@ -73,6 +83,104 @@ void or_weight_prep(const float *W, int n_out, int k, double alpha,
             rowsum[o] = s;
         }
     }
+}
+
+/* ---------------------------------------------------------------------------
+ * FP8 E4M3 (the OCP 8-bit float, "fn" variant): sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits; no infinities; exponent field 15 with mantissa 7
+ * is NaN, so the largest finite value is 1.75 * 2^8 = 448; subnormals are
+ * m * 2^-9, m = 1..7.  Encoding rounds to the nearest representable value,
+ * ties to an even mantissa, and clamps finite magnitudes above 448 to 448.
+ * ------------------------------------------------------------------------- */
+uint8_t or_e4m3_encode(double v)
+{
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {                    /* subnormal range: step 2^-9 */
+        double m = nearbyint(a / ldexp(1.0, -9)); /* ties to even */
+        return sign | (uint8_t)m;                /* m == 8 is 2^-6: field 1, mantissa 0 */
+    }
+    int E;
+    frexp(a, &E);                                /* a = f 2^E, f in [0.5, 1) */
+    int e = E - 1;                               /* 2^e <= a < 2^(e+1) */
+    double m = nearbyint(a / ldexp(1.0, e - 3)); /* 8 <= m <= 16 */
+    if (m == 16.0) { m = 8.0; e += 1; }
+    return sign | (uint8_t)((e + 7) << 3) | (uint8_t)(m - 8.0);
+}
+
+double or_e4m3_decode(uint8_t c)
+{
+    int ef = (c >> 3) & 15, mf = c & 7;
+    double s = (c & 0x80) ? -1.0 : 1.0;
+    if (ef == 15 && mf == 7) return NAN;
+    if (ef == 0) return s * ldexp((double)mf, -9);
+    return s * ldexp((double)(8 + mf), ef - 10);
+}
+
+/* One row of float32 values to E4M3 codes with its float32 scale. */
+static float quant_row(const float *v, const uint8_t *keep, int n, uint8_t *codes)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; i++)
+        if (!keep || keep[i]) {
+            float a = fabsf(v[i]);
+            if (a > amax) amax = a;
+        }
+    float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int i = 0; i < n; i++) {
+        float q = v[i] / scale;
+        codes[i] = (!keep || keep[i]) ? or_e4m3_encode((double)q) : 0;
+    }
+    return scale;
+}
+
+/* Weight side of the FP8 GEMM: W [n_out, k] float32 -> codes [n_out, k] and
+ * one scale per output row. */
+void or_quant_rows_fp8(const float *W, int n_out, int k, uint8_t *codes, float *scale)
+{
+    for (int o = 0; o < n_out; o++)
+        scale[o] = quant_row(W + (size_t)o * k, NULL, k, codes + (size_t)o * k);
+}
+
+/* [SQR] 3.1 fused producer for one layer input, from the pre-activation z
+ * (bfloat16 bit patterns, [T, k]):
+ *   x = r * r with r = max(0, z) in float32 (one rounding),
+ *   2:4 selection on |x| = x (exactly two per block of four, ties to the
+ *   lower index), then the kept values to E4M3 with the row scale.
+ * Outputs: mask [T, k], codes of the kept values [T, k/2] in channel order,
+ * their positions in the block [T, k/2], scale [T], and x itself [T, k]. */
+void or_sqrelu24_fp8(const uint16_t *z, int T, int k, uint8_t *mask, uint8_t *codes,
+                     uint8_t *pos, float *scale, float *x)
+{
+    size_t kc = (size_t)k / 2;
+    for (int t = 0; t < T; t++) {
+        float *xt = x + (size_t)t * k;
+        for (int i = 0; i < k; i++) {
+            uint32_t bits = (uint32_t)z[(size_t)t * k + i] << 16;
+            float zf;
+            memcpy(&zf, &bits, 4);
+            float r = zf > 0.0f ? zf : 0.0f;
+            xt[i] = r * r;
+        }
+    }
+    or_select_nm(x, T, k, 2, 4, mask);
+    uint8_t *row_codes = (uint8_t *)malloc((size_t)k);
+    for (int t = 0; t < T; t++) {
+        const float *xt = x + (size_t)t * k;
+        const uint8_t *mt = mask + (size_t)t * k;
+        scale[t] = quant_row(xt, mt, k, row_codes);
+        size_t w = 0;
+        for (int b = 0; b < k; b += 4)
+            for (int i = b; i < b + 4; i++)
+                if (mt[i]) {
+                    codes[(size_t)t * kc + w] = row_codes[i];
+                    pos[(size_t)t * kc + w] = (uint8_t)(i - b);
+                    w++;
+                }
+    }
+    free(row_codes);
 }
 
 /* ---------------------------------------------------------------------------

@@ -471,3 +471,113 @@ def test_amber_ties_at_the_clip_values_are_kept(oracle_lib):
     np.testing.assert_allclose(g, np.linalg.norm(Z, axis=0), rtol=1e-12)
     g0, lo0, hi0 = oracle_lib.amber(W, 1.0, 50.0, 50.0)
     assert lo0 == hi0 == 1.0 and not g0.any()
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) producer and GEMM
+def _e4m3_positive_values():
+    import oracle as o
+    return o.e4m3_decode(np.arange(0x7F, dtype=np.uint8))  # 0 .. 448, ascending
+
+
+def test_e4m3_code_table(oracle_lib):
+    """Codes fixed by the format: bias 7, 3 mantissa bits, 448 the largest
+    finite value, 2^-9 the smallest subnormal, 0x7F NaN."""
+    cases = {448.0: 0x7E, 1.0: 0x38, 2.0 ** -9: 0x01, 2.0 ** -6: 0x08, 7 * 2.0 ** -9: 0x07,
+             -2.0: 0xC0, 240.0: 0x77, 0.0: 0x00, 1.125: 0x39, 256.0: 0x78, 3.0: 0x44}
+    for v, c in cases.items():
+        assert int(oracle_lib.e4m3_encode([v])[0]) == c, v
+        assert oracle_lib.e4m3_decode([c])[0] == v
+    assert int(oracle_lib.e4m3_encode([-0.0])[0]) == 0x80
+    assert np.isnan(oracle_lib.e4m3_decode([0x7F])[0]) and np.isnan(oracle_lib.e4m3_decode([0xFF])[0])
+    # every finite code round-trips; saturation clamps at 448
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    np.testing.assert_array_equal(oracle_lib.e4m3_encode(oracle_lib.e4m3_decode(codes)), codes)
+    np.testing.assert_array_equal(oracle_lib.e4m3_encode([449.0, 464.0, 1e9, -500.0]), [0x7E, 0x7E, 0x7E, 0xFE])
+    assert int(oracle_lib.e4m3_encode([float("nan")])[0]) == 0x7F
+
+
+def test_e4m3_matches_torch_cast_on_ties_and_random(oracle_lib):
+    """In range, nearest-even rounding equals torch's float8_e4m3fn cast on
+    every midpoint between neighbours, one float32 step either side of it,
+    and random values over the whole range."""
+    pos = _e4m3_positive_values()
+    mid = (pos[:-1] + pos[1:]) / 2
+    m32 = mid.astype(np.float32)
+    near = np.concatenate([m32, np.nextafter(m32, np.float32(0)), np.nextafter(m32, np.float32(1e9))])
+    rnd = (np.random.default_rng(14).uniform(-448, 448, 100000)).astype(np.float32)
+    small = (np.random.default_rng(15).uniform(-2.0 ** -5, 2.0 ** -5, 20000)).astype(np.float32)
+    v = np.concatenate([near, -near, rnd, small, pos.astype(np.float32)])
+    got = oracle_lib.e4m3_encode(v.astype(np.float64))
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(got, want)
+
+
+def test_quant_rows_fp8_bounds(oracle_lib):
+    """Per-row scale amax/448: the largest magnitude of every nonzero row
+    codes to +-448; relative error at most 2^-4 in the normal range and
+    absolute error at most 2^-10 * scale below it; an all-zero row gets
+    scale 1 and zero codes."""
+    r = np.random.default_rng(16)
+    W = r.normal(0, 0.02, size=(33, 200)).astype(np.float32)
+    W[5] = 0.0
+    codes, scale = oracle_lib.quant_rows_fp8(W)
+    assert scale[5] == 1.0 and not codes[5].any()
+    for o in range(33):
+        if o == 5:
+            continue
+        assert (codes[o] & 0x7F).max() == 0x7E
+        assert scale[o] == np.float32(np.abs(W[o]).max()) / np.float32(448.0)
+    deq = oracle_lib.dequant_fp8(codes, scale)
+    q = np.abs(W.astype(np.float64)) / scale.astype(np.float64)[:, None]
+    err = np.abs(deq - W)
+    normal = q >= 2.0 ** -6
+    assert (err[normal] <= 2.0 ** -4 * np.abs(W[normal]) * (1 + 1e-6)).all()
+    assert (err[~normal] <= 2.0 ** -10 * np.broadcast_to(scale[:, None], W.shape)[~normal] * (1 + 1e-6)).all()
+
+
+def _bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_sqrelu24_fp8_worked_row(oracle_lib):
+    """z = [1 -2 3 .5 | 0 0 0 0 | 2 2 -1 2]: x = [1 0 9 .25 | 0 0 0 0 | 4 4 0 4];
+    kept (0, 2), (0, 1) (all equal: the lower indices), (0, 1); amax 9,
+    scale fl32(9/448); codes 9 -> 448 (0x7E), 1 -> 48 (0x64), 4 -> 192 (0x74)."""
+    z = _bf16_bits([[1, -2, 3, 0.5, 0, 0, 0, 0, 2, 2, -1, 2]])
+    out = oracle_lib.sqrelu24_fp8(z)
+    np.testing.assert_array_equal(out["x"][0], [1, 0, 9, 0.25, 0, 0, 0, 0, 4, 4, 0, 4])
+    np.testing.assert_array_equal(out["mask"][0], [1, 0, 1, 0, 1, 1, 0, 0, 1, 1, 0, 0])
+    np.testing.assert_array_equal(out["pos"][0], [0, 2, 0, 1, 0, 1])
+    assert out["scale"][0] == np.float32(9.0) / np.float32(448.0)
+    np.testing.assert_array_equal(out["codes"][0], [0x64, 0x7E, 0, 0, 0x74, 0x74])
+    zero = oracle_lib.sqrelu24_fp8(_bf16_bits([[-1.0] * 8]))
+    assert zero["scale"][0] == 1.0 and not zero["codes"].any()
+
+
+def test_sqrelu24_fp8_matches_generator_and_selection(oracle_lib):
+    """x equals the Squared-ReLU input generator's x before its bf16 rounding;
+    the mask is the plain 2:4 magnitude selection of x; every row's largest
+    kept value codes to 448."""
+    import synth
+    z, xb, _ = synth.prefill_sqrelu(T=16, k=256, with_weight=False)
+    out = oracle_lib.sqrelu24_fp8(z)
+    np.testing.assert_array_equal(torch.from_numpy(out["x"]).to(torch.bfloat16).float().numpy(), xb.float().numpy())
+    np.testing.assert_array_equal(out["mask"], oracle_lib.select_nm(oracle_lib.score(out["x"]), 2, 4))
+    for t in range(16):
+        if out["x"][t][out["mask"][t] == 1].max() > 0:
+            assert out["codes"][t].max() == 0x7E
+
+
+def test_linear_fp8_integer_case(oracle_lib):
+    """Scales 1 and small integer codes: the FP8 GEMM is an exact integer
+    matmul of the scattered kept values against the weight."""
+    r = np.random.default_rng(17)
+    T, k, n_out = 5, 32, 7
+    xv = r.integers(0, 9, size=(T, k)).astype(np.float64)
+    mask = oracle_lib.select_nm(oracle_lib.score(xv.astype(np.float32)), 2, 4)
+    xk = np.where(mask == 1, xv, 0.0)
+    codes = oracle_lib.e4m3_encode(xk[mask == 1].reshape(T, k // 2))
+    pos = np.tile(np.arange(4), (T, k // 4))[mask == 1].reshape(T, k // 2).astype(np.uint8)
+    w = r.integers(-8, 9, size=(n_out, k)).astype(np.float64)
+    y = oracle_lib.linear_fp8(codes, pos, np.ones(T, np.float32), oracle_lib.e4m3_encode(w), np.ones(n_out, np.float32))
+    np.testing.assert_array_equal(y, xk @ w.T)
