@@ -454,6 +454,38 @@ def bench_prefill(sl, dev, pk):
     del x, W, L, bufs, y
     torch.cuda.empty_cache()
 
+    # FP8 2:4: fused Squared-ReLU + 2:4 + E4M3 producer from z, then the
+    # kind::f8f6f4 sparse GEMM; peak = measured bf16 x 2 (nominal fp8/bf16
+    # ratio) x 2 (2:4)
+    z, _, W = synth.prefill_sqrelu()
+    z, W = z.to(dev), W.to(dev)
+    T, K = z.shape
+    n_out = W.shape[0]
+    Wq = torch.empty(n_out, K, dtype=torch.uint8, device=dev)
+    ws = torch.empty(n_out, dtype=torch.float32, device=dev)
+    sl.as_weight_quant_fp8(W, Wq, ws)
+    x8 = torch.empty(T, K // 2, dtype=torch.uint8, device=dev)
+    meta8 = torch.empty(sl.as_meta8_words(T, K), dtype=torch.int32, device=dev)
+    xs = torch.empty(T, dtype=torch.float32, device=dev)
+    y = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
+    prod = lambda: sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)  # noqa: E731
+    gemm = lambda: sl.as_linear_prefill_fp8(x8, meta8, xs, Wq, ws, y)  # noqa: E731
+    for _ in range(3):
+        prod()
+        gemm()
+    t_prod = ev_time(prod, 10)
+    t_gemm = ev_time(gemm, 10)
+    dense_eq = 2.0 * T * n_out * K
+    sp_peak8 = 4.0 * pk["bf16_tflops"]
+    prod_bytes = T * K * 2 + T * K // 2 + T * K // 8 + T * 4
+    out["sqrelu_2of4_fp8"] = dict(
+        shape=[T, K, n_out], producer_us=t_prod * 1e6, producer_gbs=prod_bytes / t_prod / 1e9,
+        gemm_us=t_gemm * 1e6, gemm_dense_equiv_tflops=dense_eq / t_gemm / 1e12,
+        frac_of_sparse_fp8_peak=dense_eq / t_gemm / 1e12 / sp_peak8,
+        speedup_vs_bf16_2of4_gemm=out["sqrelu_2of4"]["gemm_us"] / (t_gemm * 1e6))
+    del z, W, Wq, x8, meta8, y
+    torch.cuda.empty_cache()
+
     # CLACT + VAR at 16:32: masked dense tensor-core GEMM
     W = synth.prefill_clact_weight().to(dev)
     x = synth.prefill_clact_batch(0).to(dev)
@@ -614,6 +646,22 @@ def run_case(args):
         run = torch.zeros(args.T, dtype=torch.float32, device=dev)
         L.select(xd, bufs, running_var=run if cfg.var else None, first_batch=True)
         fn = lambda: L.select(xd, bufs, running_var=run if cfg.var else None)  # noqa: E731
+    elif args.case == "sqrelu24_fp8":
+        z, _, W = synth.prefill_sqrelu(T=args.T)
+        z, W = z.to(dev), W.to(dev)
+        K, n_out = z.shape[1], W.shape[0]
+        Wq = torch.empty(n_out, K, dtype=torch.uint8, device=dev)
+        ws = torch.empty(n_out, dtype=torch.float32, device=dev)
+        sl.as_weight_quant_fp8(W, Wq, ws)
+        x8 = torch.empty(args.T, K // 2, dtype=torch.uint8, device=dev)
+        meta8 = torch.empty(sl.as_meta8_words(args.T, K), dtype=torch.int32, device=dev)
+        xs = torch.empty(args.T, dtype=torch.float32, device=dev)
+        y = torch.empty(args.T, n_out, dtype=torch.bfloat16, device=dev)
+        sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)
+
+        def fn():
+            sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)
+            sl.as_linear_prefill_fp8(x8, meta8, xs, Wq, ws, y)
     elif args.case in ("sqrelu24", "dense"):
         _, x, W = synth.prefill_sqrelu(T=args.T)
         cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4) if args.case == "sqrelu24" else \
@@ -661,7 +709,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--case", default=None,
-                    help="profiling case: decode | sqrelu24 | dense | select24 | selectclact | block")
+                    help="profiling case: decode | sqrelu24 | sqrelu24_fp8 | dense | select24 | selectclact | block")
     ap.add_argument("--T", type=int, default=1)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

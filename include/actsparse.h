@@ -281,6 +281,55 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
 /* Number of 32-bit metadata words of a 2:4 selection of T tokens x K channels. */
 size_t as_meta24_words(int T, int K);
 
+/* --------------------------------------------------------------------------
+ * FP8 2:4 prefill ([SQR] 3.1: a fused Squared-ReLU + 2:4 + FP8 producer and
+ * a 2:4 GEMM on FP8 operands with row scaling; [SQR] 5.3: sparsify before
+ * quantising).  FP8 is E4M3 (largest finite 448, no infinities), converted
+ * with round-to-nearest-even and saturation.  Every row carries one float32
+ * scale: scale = amax / 448 over the row's (kept) values, 1 for an all-zero
+ * row; code = E4M3(fl32(v / scale)); the value a code stands for is
+ * E4M3value(code) * scale.
+ * ------------------------------------------------------------------------ */
+
+/* Number of 32-bit words of FP8 2:4 positions for T tokens x K channels:
+ * ceil(T/256)*2 tiles of 128 tokens by ceil(K/256) tiles of 256 channels,
+ * 1024 words each.  Tile (r, c) starts at word (r * ceil(K/256) + c) * 1024
+ * and holds two 512-word halves (channels 0..127 and 128..255 of the tile);
+ * in a half, word p*4 + j holds channels 32j..32j+31 of the half for token
+ * p of the tile, with the 4-block at channel q in bits [4*((q%32)/4), +4):
+ * i0 | i1 << 2, i0 < i1 the kept positions.  Channels past K and tokens past
+ * T (up to the next multiple of 256) hold positions (0, 1). */
+size_t as_meta8_words(int T, int K);
+
+/* Weight side, once per layer: W [n_out, K] in `dt` -> Wq [n_out, K] E4M3
+ * codes and w_scale [n_out] (amax over the output row).  K % 16 == 0;
+ * pointers 16-byte aligned. */
+as_status as_weight_quant_fp8(const void *W, as_dtype dt, int n_out, int K, uint8_t *Wq, float *w_scale,
+                              cudaStream_t stream);
+
+/* Activation side, the fused producer.  z [T, K] bf16 pre-activations:
+ *   x = fl32(max(0, z))^2 (computed in registers, never written);
+ *   in every block of 4 channels keep the 2 largest x (ties to the lower
+ *   channel);
+ *   x_scale[t] = amax of the kept x of token t / 448 (1 if all are zero);
+ *   x8 [T, K/2] codes of the kept values, in channel order;
+ *   meta8 [as_meta8_words(T, K)] their positions (layout above);
+ *   bitmask [T, K/32] (optional): bit i%32 of word i/32 set if kept.
+ * K % 64 == 0; pointers 16-byte aligned. */
+as_status as_select_sqrelu24_fp8(const void *z, int T, int K, uint8_t *x8, uint32_t *meta8, float *x_scale,
+                                 uint32_t *bitmask, cudaStream_t stream);
+
+/* The FP8 2:4 GEMM on CTA pairs (tcgen05.mma.sp kind::f8f6f4, float32
+ * accumulation in tensor memory):
+ *   y[t, o] = fl32(fl32(acc[t, o] * x_scale[t]) * w_scale[o]),
+ *   acc[t, o] = sum over the kept channels i of E4M3value(x8) * E4M3value(Wq[o, i]).
+ * y [T, n_out] in out_dtype (AS_BF16 or AS_F32).  K % 64 == 0,
+ * n_out % 8 == 0.  AS_ERR_UNSUPPORTED if the device cannot co-schedule the
+ * CTA pairs. */
+as_status as_linear_prefill_fp8(const uint8_t *x8, const uint32_t *meta8, const float *x_scale, int T, int K,
+                                int n_out, const uint8_t *Wq, const float *w_scale, as_dtype out_dtype, void *y,
+                                cudaStream_t stream);
+
 /* Synchronises `stream`, then reports (and clears) a device-side error such
  * as AS_ERR_TIMEOUT recorded by a kernel of this library, or AS_ERR_CUDA if
  * the stream itself failed. */

@@ -39,7 +39,8 @@ EXPORTS = [
     "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
     "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches", "as_probe_timeout",
-    "as_weight_prep_amber",
+    "as_weight_prep_amber", "as_meta8_words", "as_weight_quant_fp8", "as_select_sqrelu24_fp8",
+    "as_linear_prefill_fp8",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -62,6 +63,10 @@ _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _sig = {
     "as_weight_prep": ([_P, _I, _I, _I, _F, _P, _P, _P, _P, _S, _P], _I),
     "as_weight_prep_amber": ([_P, _I, _I, _I, _F, ctypes.c_double, ctypes.c_double, _P, _P, _P, _S, _P], _I),
+    "as_meta8_words": ([_I, _I], _S),
+    "as_weight_quant_fp8": ([_P, _I, _I, _I, _P, _P, _P], _I),
+    "as_select_sqrelu24_fp8": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
+    "as_linear_prefill_fp8": ([_P, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P], _I),
     "as_select": ([_P, _I, _I, _I, ctypes.POINTER(as_config), _P, _P, _I,
                    ctypes.POINTER(as_select_out), _P, _S, _P], _I),
     "as_linear_decode": ([_P, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(as_config), _P, _P, _P, _P,
@@ -175,6 +180,30 @@ def as_weight_prep_amber(W, g, alpha: float = 1.0, lo_pct: float = 0.5, hi_pct: 
     _check(_lib.as_weight_prep_amber(_ptr(W), _dt(W), n_out, K, float(alpha), float(lo_pct), float(hi_pct),
                                      _ptr(g), _ptr(bounds), _ptr(workspace), ws_bytes, _stream(stream)),
            "as_weight_prep_amber")
+
+
+def as_meta8_words(T: int, K: int) -> int:
+    return _lib.as_meta8_words(T, K)
+
+
+def as_weight_quant_fp8(W, Wq, w_scale, stream=None) -> None:
+    n_out, K = W.shape
+    _check(_lib.as_weight_quant_fp8(_ptr(W), _dt(W), n_out, K, _ptr(Wq), _ptr(w_scale), _stream(stream)),
+           "as_weight_quant_fp8")
+
+
+def as_select_sqrelu24_fp8(z, x8, meta8, x_scale, bitmask=None, stream=None) -> None:
+    T, K = z.shape
+    _check(_lib.as_select_sqrelu24_fp8(_ptr(z), T, K, _ptr(x8), _ptr(meta8), _ptr(x_scale), _ptr(bitmask),
+                                       _stream(stream)), "as_select_sqrelu24_fp8")
+
+
+def as_linear_prefill_fp8(x8, meta8, x_scale, Wq, w_scale, y, stream=None) -> None:
+    T = x8.shape[0]
+    n_out, K = Wq.shape
+    out = AS_BF16 if y.dtype == torch.bfloat16 else AS_F32
+    _check(_lib.as_linear_prefill_fp8(_ptr(x8), _ptr(meta8), _ptr(x_scale), T, K, n_out, _ptr(Wq), _ptr(w_scale),
+                                      out, _ptr(y), _stream(stream)), "as_linear_prefill_fp8")
 
 
 def as_select(x, cfg: as_config, out: as_select_out, chan_factor=None, running_var=None,

@@ -144,6 +144,58 @@ as_status as_weight_prep_amber(const void *W, as_dtype dt, int n_out, int K, flo
     return cuda_status(launch_amber(W, dt == AS_BF16, n_out, K, alpha, r_lo, r_hi, g, bounds, workspace, stream));
 }
 
+size_t as_meta8_words(int T, int K)
+{
+    if (T <= 0 || K <= 0) return 0;
+    return meta8_words(T, K);
+}
+
+as_status as_weight_quant_fp8(const void *W, as_dtype dt, int n_out, int K, uint8_t *Wq, float *w_scale,
+                              cudaStream_t stream)
+{
+    if (!W || !Wq || !w_scale || n_out <= 0 || K <= 0) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    if (K % 16 != 0) return AS_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(Wq) || !aligned16(w_scale)) return AS_ERR_ALIGN;
+    return cuda_status(launch_quant_rows_fp8(W, dt == AS_BF16, n_out, K, Wq, w_scale, stream));
+}
+
+as_status as_select_sqrelu24_fp8(const void *z, int T, int K, uint8_t *x8, uint32_t *meta8, float *x_scale,
+                                 uint32_t *bitmask, cudaStream_t stream)
+{
+    if (!z || !x8 || !meta8 || !x_scale || T <= 0 || K <= 0) return AS_ERR_INVALID_ARG;
+    if (K % 64 != 0) return AS_ERR_SHAPE;
+    if (!aligned16(z) || !aligned16(x8) || !aligned16(meta8) || !aligned16(x_scale) || !aligned16(bitmask))
+        return AS_ERR_ALIGN;
+    return cuda_status(launch_sqrelu24_fp8(z, T, K, x8, meta8, x_scale, bitmask, stream));
+}
+
+as_status as_linear_prefill_fp8(const uint8_t *x8, const uint32_t *meta8, const float *x_scale, int T, int K,
+                                int n_out, const uint8_t *Wq, const float *w_scale, as_dtype out_dtype, void *y,
+                                cudaStream_t stream)
+{
+    if (!x8 || !meta8 || !x_scale || !Wq || !w_scale || !y || T <= 0 || K <= 0 || n_out <= 0)
+        return AS_ERR_INVALID_ARG;
+    if (out_dtype != AS_F32 && out_dtype != AS_BF16) return AS_ERR_DTYPE;
+    if (K % 64 != 0 || n_out % 8 != 0) return AS_ERR_SHAPE;
+    for (const void *q : {(const void *)x8, (const void *)meta8, (const void *)x_scale, (const void *)Wq,
+                          (const void *)w_scale, (const void *)y})
+        if (!aligned16(q)) return AS_ERR_ALIGN;
+    Fp8GemmArgs a{};
+    a.x8 = x8;
+    a.meta8 = meta8;
+    a.x_scale = x_scale;
+    a.Wq = Wq;
+    a.w_scale = w_scale;
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.y = y;
+    a.out_bf16 = out_dtype == AS_BF16;
+    const cudaError_t e = launch_gemm_fp8(a, stream);
+    return e == cudaErrorNotSupported ? AS_ERR_UNSUPPORTED : cuda_status(e);
+}
+
 as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *cfg, const float *chan_factor,
                     float *running_var, int var_first_batch, const as_select_out *out, void *workspace,
                     size_t ws_bytes, cudaStream_t stream)

@@ -4,5 +4,6 @@
 #include "select.cu"
 #include "decode.cu"
 #include "gemm.cu"
+#include "fp8.cu"
 #include "abi.cu"
 #include "noalloc.cu"

@@ -236,6 +236,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool sparse)
            ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0
+// in [7,10) and [10,13)), f32 D, both K-major; otherwise as idesc_bf16.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool sparse)
+{
+    return (sparse ? (1u << 2) : 0u) | (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // ------------------------------------------------ CTA pairs (cta_group::2)
 // Rank of this CTA in its cluster and the shared::cluster address of the
 // same shared-memory offset in CTA `rank` of the cluster.
@@ -315,6 +322,19 @@ __device__ __forceinline__ void mma_sp_bf16_pair(uint32_t d_tmem, uint64_t a_des
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+        : "memory");
+}
+
+// Sparse E4M3 MMA over a CTA pair (kind::f8f6f4, K = 64 logical): 64 bits of
+// positions per row in two TMEM columns at e_tmem (row = lane), selector 0.
+__device__ __forceinline__ void mma_sp_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t e_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
         : "memory");
 }

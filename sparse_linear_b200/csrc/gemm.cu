@@ -64,6 +64,7 @@ constexpr size_t gemm_smem_bytes()
 struct GemmParams {
     const uint32_t *meta;
     const float *rowsum, *eta, *nu;
+    const float *xscale, *wscale;  // FP8 row scales (tokens, output rows)
     void *y;
     int T, K, n_out, out_bf16;
     int m_tiles, n_tiles, k_blocks, meta_kt;
@@ -291,22 +292,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //               before the scaling and the stores, so the next tile's MMAs
 //               overlap the stores.
 // Loads carry no multicast; only tcgen05.commit signals both CTAs.
+//
+// FP8 variant (2:4 + Squared-ReLU page section 3.1, FP8 row-scaled 2:4 GEMM):
+// tcgen05.mma.sp kind::f8f6f4 with E4M3 A and B, K = 64 (logical) per
+// instruction.  A stage holds the same bytes (128 compact codes per row =
+// 256 logical K; B two 128-byte sub-tiles) and twice the positions: each
+// instruction reads 64 position bits per row from two TMEM columns (row =
+// lane).  The epilogue multiplies by the token's and the output row's scale.
 constexpr int PAIR_THREADS = 320;
 constexpr int PAIR_BM = 256;  // rows per CTA pair (128 per CTA)
 constexpr int PAIR_BN = 256;  // weight rows per CTA pair (128 per CTA)
 constexpr int PAIR_STAGES = 4;
-constexpr int PAIR_A_BYTES = 128 * 64 * 2;   // kept half of 128 rows x 128 logical K
-constexpr int PAIR_B_BYTES = 128 * 128 * 2;  // 128 weight rows x 128 K, two sub-tiles
-constexpr int PAIR_M_BYTES = 2048;           // 2:4 positions of 128 rows x 128 K
-constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES + PAIR_M_BYTES;
+constexpr int PAIR_A_BYTES = 128 * 128;      // kept half of 128 rows: 128 bytes per row
+constexpr int PAIR_B_BYTES = 128 * 256;      // 128 weight rows x 256 bytes, two sub-tiles
 
-constexpr size_t pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PAIR_STAGE_BYTES + 256; }
+template <bool FP8>
+struct PairCfg {
+    static constexpr int M_BYTES = FP8 ? 4096 : 2048;  // positions of 128 rows x one K block
+    static constexpr int STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES + M_BYTES;
+    static constexpr int KB = FP8 ? 256 : 128;         // logical K per stage
+    static constexpr int KA = KB / 2;                  // compact A elements per stage
+    static constexpr int BSUB = FP8 ? 128 : 64;        // B elements per 128-byte sub-tile
+    static constexpr int META_COLS = FP8 ? 8 : 4;      // TMEM columns of positions per stage
+};
 
+template <bool FP8>
+constexpr size_t pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PairCfg<FP8>::STAGE_BYTES + 256; }
+
+template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     k_gemm_sp_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmE, GemmParams p)
 {
+    using C = PairCfg<FP8>;
     constexpr int S = PAIR_STAGES;
+    constexpr int PAIR_M_BYTES = C::M_BYTES;
+    constexpr int PAIR_STAGE_BYTES = C::STAGE_BYTES;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                             ~uintptr_t(1023));
@@ -363,10 +384,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
                     const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
                     unsigned char *b_dst = sB + stage * PAIR_B_BYTES;
-                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, &tmA, bar, kb * 64, arow);
-                    tma_load_2d_pair(b_dst, &tmB, bar, kb * 128, brow);
-                    tma_load_2d_pair(b_dst + 128 * 128, &tmB, bar, kb * 128 + 64, brow);
-                    tma_load_2d_pair(sM + stage * PAIR_M_BYTES, &tmE, bar, 0, (echunk + kb) * 8);
+                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, &tmA, bar, kb * C::KA, arow);
+                    tma_load_2d_pair(b_dst, &tmB, bar, kb * C::KB, brow);
+                    tma_load_2d_pair(b_dst + 128 * 128, &tmB, bar, kb * C::KB + C::BSUB, brow);
+                    tma_load_2d_pair(sM + stage * PAIR_M_BYTES, &tmE, bar, 0, (echunk + kb) * (PAIR_M_BYTES / 256));
+                    if constexpr (FP8)
+                        tma_load_2d_pair(sM + stage * PAIR_M_BYTES + 2048, &tmE, bar, 0,
+                                         (echunk + kb) * (PAIR_M_BYTES / 256) + 8);
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
@@ -374,7 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader only)
         if (rank == 0 && lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(PAIR_BM, PAIR_BN, true);
+            constexpr uint32_t idesc = FP8 ? idesc_e4m3(PAIR_BM, PAIR_BN, true) : idesc_bf16(PAIR_BM, PAIR_BN, true);
             const uint32_t meta_tmem = tmem + PAIR_BN;
             int stage = 0;
             uint32_t phase = 0;
@@ -388,14 +412,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     tc_fence_after();
                     const uint32_t b_addr = smem_u32(sB + stage * PAIR_B_BYTES);
                     const uint64_t a_desc = sdesc_kmajor_sw128(smem_u32(sA + stage * PAIR_A_BYTES));
-                    const uint32_t e_tmem = meta_tmem + stage * 4;
+                    const uint32_t e_tmem = meta_tmem + stage * C::META_COLS;
                     tmem_cp_128x128b_pair(e_tmem, sdesc_rows16(smem_u32(sM + stage * PAIR_M_BYTES)));
+                    if constexpr (FP8)
+                        tmem_cp_128x128b_pair(e_tmem + 4, sdesc_rows16(smem_u32(sM + stage * PAIR_M_BYTES + 2048)));
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint64_t a_j = a_desc + (uint64_t)((32 * j) >> 4);
                         const uint64_t b_j = sdesc_kmajor_sw128(b_addr + (j >> 1) * (128 * 128) + (j & 1) * 64);
-                        mma_sp_bf16_pair(tmem, a_j, b_j, idesc | (uint32_t)(j & 1), e_tmem + (j & ~1),
-                                         (kb | j) != 0);
+                        if constexpr (FP8)
+                            mma_sp_e4m3_pair(tmem, a_j, b_j, idesc, e_tmem + 2 * j, (kb | j) != 0);
+                        else
+                            mma_sp_bf16_pair(tmem, a_j, b_j, idesc | (uint32_t)(j & 1), e_tmem + (j & ~1),
+                                             (kb | j) != 0);
                     }
                     tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
                     if (++stage == S) { stage = 0; phase ^= 1; }
@@ -428,13 +457,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 
             const int row = mt * PAIR_BM + 128 * (int)rank + 32 * q + lane;
             if (row >= p.T) continue;
-            float rscale = 1.0f, reta = 0.0f;
+            float rscale = 1.0f, reta = 0.0f, xs = 1.0f;
             if (p.nu) rscale = p.nu[row];
             if (p.eta) reta = p.eta[row];
+            if (FP8) xs = p.xscale[row];
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 const int col0 = nt * PAIR_BN + 128 * h + 32 * ch;
                 if (col0 >= p.n_out) continue;
+                if constexpr (FP8) {
+                    // n_out % 8 == 0: every 4-column group past col0 starts in range
+                    // or is clamped to the last one (its values are not stored)
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const int c = min(col0 + 4 * c4, p.n_out - 4);
+                        const float4 w4 = *reinterpret_cast<const float4 *>(p.wscale + c);
+                        const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            r[ch][4 * c4 + i] = __float_as_uint((__uint_as_float(r[ch][4 * c4 + i]) * xs) * ws[i]);
+                    }
+                }
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -714,6 +757,20 @@ static bool make_map_meta(CUtensorMap *m, const void *base, uint64_t chunks)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// E4M3 codes as a 2-D uint8 tensor, 128-byte (128-element) boxes, 128-byte swizzle.
+static bool make_map_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    PFN_encodeTiled_t enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int sm_count()
 {
     static int n = 0;
@@ -787,7 +844,13 @@ static int pair_clusters_of(KernelT kernel, size_t smem, int &cached)
 static int pair_clusters(size_t smem)
 {
     static int cached = -1;
-    return pair_clusters_of(k_gemm_sp_pair, smem, cached);
+    return pair_clusters_of(k_gemm_sp_pair<false>, smem, cached);
+}
+
+static int pair_clusters_fp8(size_t smem)
+{
+    static int cached = -1;
+    return pair_clusters_of(k_gemm_sp_pair<true>, smem, cached);
 }
 
 static int dense_pair_clusters(size_t smem)
@@ -827,14 +890,14 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map_meta(&mE, a.meta, (uint64_t)mt128 * p.meta_kt)) return cudaErrorInvalidValue;
-    const size_t smem = pair_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_sp_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = pair_smem_bytes<false>();
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_sp_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int clusters = pair_clusters(smem);
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_sp_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, p);
+    k_gemm_sp_pair<false><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, p);
     return cudaGetLastError();
 }
 
@@ -865,12 +928,45 @@ static cudaError_t launch_gemm_dense_pair(const GemmArgs &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// FP8 2:4 GEMM on CTA pairs.  The metadata buffer covers an even number of
+// 128-row tiles (meta8_words), so an odd tile count runs its last pair with
+// a second CTA whose rows all lie past T (zero-filled by TMA, not stored).
+cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st)
+{
+    CUtensorMap mA, mB, mE;
+    const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
+    GemmParams p{};
+    p.xscale = a.x_scale;
+    p.wscale = a.w_scale;
+    p.y = a.y;
+    p.T = a.T;
+    p.K = a.K;
+    p.n_out = a.n_out;
+    p.out_bf16 = a.out_bf16;
+    p.m_tiles = (mt128 + 1) / 2;
+    p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
+    p.k_blocks = (a.K + 255) / 256;
+    p.meta_kt = p.k_blocks;
+    if (!make_map_u8(&mA, a.x8, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
+    if (!make_map_u8(&mB, a.Wq, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
+    if (!make_map_meta(&mE, a.meta8, (uint64_t)p.m_tiles * 2 * p.meta_kt * 2)) return cudaErrorInvalidValue;
+    const size_t smem = pair_smem_bytes<true>();
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_sp_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int clusters = pair_clusters_fp8(smem);
+    if (clusters <= 0) return cudaErrorNotSupported;
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int grid = 2 * std::min(tiles, clusters);
+    k_gemm_sp_pair<true><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st)
 {
     if (use_pair(a)) {
         if (a.sparse) {
-            const size_t smem = pair_smem_bytes();
-            if (cudaFuncSetAttribute(k_gemm_sp_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+            const size_t smem = pair_smem_bytes<false>();
+            if (cudaFuncSetAttribute(k_gemm_sp_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
                     cudaSuccess &&
                 pair_clusters(smem) > 0)
                 return launch_gemm_pair(a, st);

@@ -84,4 +84,23 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 
+// FP8 2:4 prefill (fp8.cu, gemm.cu).
+struct Fp8GemmArgs {
+    const uint8_t *x8;       // E4M3 codes of the kept values [T, K/2]
+    const uint32_t *meta8;   // positions, meta8_words(T, K) words
+    const float *x_scale;    // [T]
+    const uint8_t *Wq;       // E4M3 [n_out, K]
+    const float *w_scale;    // [n_out]
+    int T, K, n_out;
+    void *y;
+    int out_bf16;
+};
+cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st);
+int meta8_kt(int K);
+size_t meta8_words(int T, int K);
+cudaError_t launch_sqrelu24_fp8(const void *z, int T, int K, uint8_t *x8, uint32_t *meta8, float *x_scale,
+                                uint32_t *bitmask, cudaStream_t st);
+cudaError_t launch_quant_rows_fp8(const void *W, int bf16, int n_out, int K, uint8_t *Wq, float *w_scale,
+                                  cudaStream_t st);
+
 }  // namespace as

@@ -41,3 +41,22 @@ def decode_meta24(meta: torch.Tensor, T: int, K: int):
 
 def f32(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
+
+
+def decode_meta8(meta: torch.Tensor, T: int, K: int, T_pad: int | None = None):
+    """FP8 2:4 position words (layout documented in include/actsparse.h) ->
+    [T_pad or T, ceil(K/256)*64, 2] positions i0, i1 per 4-block, padding
+    blocks included."""
+    m = meta.cpu().numpy().view(np.uint32)
+    kt = (K + 255) // 256
+    rows = T if T_pad is None else T_pad
+    t = np.arange(rows)[:, None]
+    c = (np.arange(kt * 64) * 4)[None, :]
+    p = t % 128
+    tile = (t // 128) * kt + c // 256
+    q = c % 256
+    j = q // 32
+    word = m[tile * 1024 + (j // 4) * 512 + p * 4 + (j % 4)]
+    shift = (4 * ((q % 32) // 4)).astype(np.uint32)
+    nib = (word >> shift) & 0xF
+    return np.stack([nib & 3, nib >> 2], axis=-1).astype(np.int64)

@@ -177,3 +177,26 @@ def test_amber_validation_launches_nothing(lib):
     assert call(b=fake + 8) == lib.AS_ERR_ALIGN
     assert call(w=None) == lib.AS_ERR_WORKSPACE
     assert call(wb=ws - 1) == lib.AS_ERR_WORKSPACE
+
+
+def test_fp8_validation_launches_nothing(lib):
+    """Shape, dtype, alignment and NULL checks of the FP8 entry points run on
+    the host (fake addresses: a launch would fail without a GPU)."""
+    fake = 1 << 20
+    L = lib._lib
+    assert lib.as_meta8_words(4096, 14336) == 16 * 2 * 56 * 1024
+    assert lib.as_meta8_words(1, 64) == 2 * 1 * 1024
+    assert L.as_weight_quant_fp8(fake, lib.AS_BF16, 64, 40, fake, fake, None) == lib.AS_ERR_SHAPE
+    assert L.as_weight_quant_fp8(fake, 9, 64, 64, fake, fake, None) == lib.AS_ERR_DTYPE
+    assert L.as_weight_quant_fp8(None, lib.AS_BF16, 64, 64, fake, fake, None) == lib.AS_ERR_INVALID_ARG
+    assert L.as_weight_quant_fp8(fake, lib.AS_BF16, 64, 64, fake + 1, fake, None) == lib.AS_ERR_ALIGN
+    assert L.as_select_sqrelu24_fp8(fake, 8, 96, fake, fake, fake, None, None) == lib.AS_ERR_SHAPE
+    assert L.as_select_sqrelu24_fp8(fake, 0, 128, fake, fake, fake, None, None) == lib.AS_ERR_INVALID_ARG
+    assert L.as_select_sqrelu24_fp8(fake, 8, 128, fake, None, fake, None, None) == lib.AS_ERR_INVALID_ARG
+    assert L.as_select_sqrelu24_fp8(fake, 8, 128, fake, fake, fake, fake + 4, None) == lib.AS_ERR_ALIGN
+    f = L.as_linear_prefill_fp8
+    assert f(fake, fake, fake, 8, 96, 64, fake, fake, lib.AS_BF16, fake, None) == lib.AS_ERR_SHAPE
+    assert f(fake, fake, fake, 8, 128, 60, fake, fake, lib.AS_BF16, fake, None) == lib.AS_ERR_SHAPE
+    assert f(fake, fake, fake, 8, 128, 64, fake, fake, 5, fake, None) == lib.AS_ERR_DTYPE
+    assert f(fake, None, fake, 8, 128, 64, fake, fake, lib.AS_BF16, fake, None) == lib.AS_ERR_INVALID_ARG
+    assert f(fake, fake, fake, 8, 128, 64, fake, fake + 8, lib.AS_BF16, fake, None) == lib.AS_ERR_ALIGN

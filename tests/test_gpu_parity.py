@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import decode_meta24, f32, rel_l2, unpack_bitmask
+from gpu_util import decode_meta8, decode_meta24, f32, rel_l2, unpack_bitmask
 
 pytestmark = pytest.mark.gpu
 
@@ -435,3 +435,94 @@ def test_prefill_thresh_and_static_pts(sl):
     cfg2 = sl.config(sel=sl.AS_SEL_NM, n=8, m=16, dpts=sl.AS_PTS_STATIC, eta_static=eta_static,
                      out_dtype=sl.AS_F32)
     check_prefill_masked(sl, [x], W, cfg2, eta_static=eta_static)
+
+
+# ---------------------------------------------------------------- FP8 2:4 prefill
+def _fp8_weight(sl, W):
+    n_out, K = W.shape
+    Wq = torch.empty(n_out, K, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(n_out, dtype=torch.float32, device="cuda")
+    sl.as_weight_quant_fp8(dev(W), Wq, ws)
+    return Wq, ws
+
+
+def _fp8_produce(sl, z):
+    T, K = z.shape
+    x8 = torch.empty(T, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.full((sl.as_meta8_words(T, K),), 0x7777, dtype=torch.int32, device="cuda")
+    xs = torch.empty(T, dtype=torch.float32, device="cuda")
+    bm = torch.empty(T, K // 32, dtype=torch.int32, device="cuda")
+    sl.as_select_sqrelu24_fp8(dev(z), x8, meta, xs, bitmask=bm)
+    return x8, meta, xs, bm
+
+
+@pytest.mark.parametrize("n_out,K,dtype", [(264, 1024, torch.bfloat16), (64, 272, torch.float32),
+                                           (4096, 14336, torch.bfloat16)])
+def test_fp8_weight_quant(sl, n_out, K, dtype):
+    """Codes and row scales bit-exact against the oracle (one IEEE division
+    and one round-to-nearest-even conversion on both sides)."""
+    _, W = synth.random_layer(1, K, n_out, seed=51, dtype=dtype)
+    W[3] = 0  # an all-zero row: scale 1, zero codes
+    Wq, ws = _fp8_weight(sl, W)
+    torch.cuda.synchronize()
+    codes, scale = oracle.quant_rows_fp8(W.float().numpy())
+    np.testing.assert_array_equal(ws.cpu().numpy(), scale)
+    np.testing.assert_array_equal(Wq.cpu().numpy(), codes)
+
+
+@pytest.mark.parametrize("T,K", [(1, 64), (300, 1024), (129, 832)])
+def test_fp8_producer(sl, T, K):
+    """Fused Squared-ReLU + 2:4 + FP8: codes, scales, bitmask and positions
+    bit-exact; padding blocks (channels past K, tokens past T up to the pair
+    tile) hold positions (0, 1)."""
+    z, _, _ = synth.prefill_sqrelu(T=T, k=K, with_weight=False)
+    z[0, :8] = torch.tensor([1, -2, 3, 0.5, 2, 2, -1, 2], dtype=torch.bfloat16)
+    if T > 2:
+        z[2] = -1  # all-zero row
+    x8, meta, xs, bm = _fp8_produce(sl, z)
+    torch.cuda.synchronize()
+    ref = oracle.sqrelu24_fp8(z)
+    np.testing.assert_array_equal(xs.cpu().numpy(), ref["scale"])
+    np.testing.assert_array_equal(x8.cpu().numpy(), ref["codes"])
+    np.testing.assert_array_equal(unpack_bitmask(bm, K), ref["mask"])
+    T_pad = (T + 255) // 256 * 256
+    pos = decode_meta8(meta, T, K, T_pad)
+    want = ref["pos"].reshape(T, K // 4, 2).astype(np.int64)
+    np.testing.assert_array_equal(pos[:T, :K // 4], want)
+    assert (pos[:, K // 4:] == [0, 1]).all() and (pos[T:] == [0, 1]).all()
+
+
+def check_fp8_gemm(sl, T, K, n_out, out_dtype, seed=52, rows=None):
+    z, _, W = synth.prefill_sqrelu(T=T, k=K, n_out=n_out, seed=seed)
+    x8, meta, xs, _ = _fp8_produce(sl, z)
+    Wq, ws = _fp8_weight(sl, W)
+    y = torch.empty(T, n_out, dtype=out_dtype, device="cuda")
+    sl.as_linear_prefill_fp8(x8, meta, xs, Wq, ws, y)
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    ref_x = oracle.sqrelu24_fp8(z if rows is None else z[rows])
+    np.testing.assert_array_equal(x8.cpu().numpy()[rows] if rows is not None else x8.cpu().numpy(), ref_x["codes"])
+    codes_w, scale_w = oracle.quant_rows_fp8(W.float().numpy())
+    ref = oracle.linear_fp8(ref_x["codes"], ref_x["pos"], ref_x["scale"], codes_w, scale_w)
+    got = f32(y) if rows is None else f32(y)[rows]
+    tol = TOL_BF16 if out_dtype == torch.bfloat16 else TOL_F32
+    err = rel_l2(got, ref)
+    assert err <= tol, err
+    return err
+
+
+@pytest.mark.parametrize("T,K,n_out,out", [
+    (256, 512, 256, torch.float32),     # one pair tile, two K blocks
+    (300, 1024, 264, torch.bfloat16),   # ragged T and n_out
+    (384, 832, 512, torch.float32),     # odd number of 128-row tiles, ragged last K block
+    (512, 4096, 768, torch.bfloat16),   # several tiles per CTA pair
+])
+def test_fp8_gemm(sl, T, K, n_out, out):
+    check_fp8_gemm(sl, T, K, n_out, out)
+
+
+def test_fp8_gemm_full_size(sl):
+    """The Squared-ReLU down-projection at full size (T 4096, K 14336,
+    n_out 4096), checked on sampled rows spread over every row tile."""
+    rows = np.arange(5, 4096, 61)
+    check_fp8_gemm(sl, 4096, 14336, 4096, torch.bfloat16, seed=3, rows=rows)
