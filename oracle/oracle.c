@@ -43,8 +43,9 @@
  * FP8 ([SQR] 3.1 names FP8 and row scaling but no format or scale rule):
  * E4M3 with round-to-nearest-even and saturation at 448; one float32 scale
  * per row (token row of the activation, output row of the weight),
- * scale = amax / 448 over the row's kept values (1 for an all-zero row),
- * code = E4M3(fl32(v / scale)); the activation is sparsified first ([SQR]
+ * scale = fl32(amax / 448) over the row's kept values, and the codes are
+ * E4M3(fl32(v * inv)) with the reciprocal scale inv = fl32(448 / amax)
+ * (scale = inv = 1 for an all-zero row); the activation is sparsified first ([SQR]
  * 5.3), so its amax runs over the kept values only.
  */
 #include <math.h>
@@ -129,8 +130,9 @@ static float quant_row(const float *v, const uint8_t *keep, int n, uint8_t *code
             if (a > amax) amax = a;
         }
     float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
     for (int i = 0; i < n; i++) {
-        float q = v[i] / scale;
+        float q = v[i] * inv;
         codes[i] = (!keep || keep[i]) ? or_e4m3_encode((double)q) : 0;
     }
     return scale;
