@@ -646,7 +646,7 @@ def run_case(args):
         run = torch.zeros(args.T, dtype=torch.float32, device=dev)
         L.select(xd, bufs, running_var=run if cfg.var else None, first_batch=True)
         fn = lambda: L.select(xd, bufs, running_var=run if cfg.var else None)  # noqa: E731
-    elif args.case == "sqrelu24_fp8":
+    elif args.case in ("sqrelu24_fp8", "sqrelu24_fp8_producer"):
         z, _, W = synth.prefill_sqrelu(T=args.T)
         z, W = z.to(dev), W.to(dev)
         K, n_out = z.shape[1], W.shape[0]
@@ -658,10 +658,10 @@ def run_case(args):
         xs = torch.empty(args.T, dtype=torch.float32, device=dev)
         y = torch.empty(args.T, n_out, dtype=torch.bfloat16, device=dev)
         sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)
-
-        def fn():
-            sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)
-            sl.as_linear_prefill_fp8(x8, meta8, xs, Wq, ws, y)
+        if args.case == "sqrelu24_fp8":
+            fn = lambda: sl.as_linear_prefill_fp8(x8, meta8, xs, Wq, ws, y)  # noqa: E731
+        else:
+            fn = lambda: sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)  # noqa: E731
     elif args.case in ("sqrelu24", "dense"):
         _, x, W = synth.prefill_sqrelu(T=args.T)
         cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4) if args.case == "sqrelu24" else \
@@ -709,7 +709,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--case", default=None,
-                    help="profiling case: decode | sqrelu24 | sqrelu24_fp8 | dense | select24 | selectclact | block")
+                    help="profiling case: decode | sqrelu24 | sqrelu24_fp8 | sqrelu24_fp8_producer | dense | select24 | selectclact | block")
     ap.add_argument("--T", type=int, default=1)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

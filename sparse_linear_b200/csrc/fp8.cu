@@ -5,15 +5,16 @@
 // before quantising).
 //
 // Format: E4M3 ("fn": largest finite 448, no infinities), round to nearest
-// even, saturating.  One float32 scale per row: scale = amax / 448 over the
-// row's kept values (1 for an all-zero row), code = E4M3(fl32(v / scale)).
+// even, saturating.  One float32 scale per row: scale = fl32(amax / 448) over
+// the row's kept values, codes E4M3(fl32(v * inv)) with inv = fl32(448 / amax)
+// (scale = inv = 1 for an all-zero row).
 //
 // k_sqrelu24_fp8     one CTA per token row: x = fl32(max(0, z))^2 from the
 //                    bf16 pre-activation, 2:4 by magnitude (ties to the lower
 //                    index), the row amax, then the kept values' codes, their
 //                    positions in the FP8 sparse-MMA metadata layout and the
-//                    optional bitmask.  x is never written.  The row is read
-//                    twice (amax pass, code pass); the second read hits L2.
+//                    optional bitmask.  x is never written; rows up to 16384
+//                    channels are read once and held in registers.
 // k_quant_rows_fp8   one CTA per weight row: amax, then codes.
 #include <cuda_fp8.h>
 
@@ -25,11 +26,6 @@ namespace as {
 
 constexpr int F8_THREADS = 256;
 constexpr uint8_t F8_PAD_META = 0x44;  // positions (0, 1) in both 4-blocks of a byte
-
-__device__ __forceinline__ uint8_t e4m3_rn_sat(float v)
-{
-    return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
-}
 
 __device__ __forceinline__ float block_max(float v, float *red)
 {
@@ -45,9 +41,8 @@ __device__ __forceinline__ float block_max(float v, float *red)
 }
 
 // Eight consecutive bf16 pre-activations -> x = max(0, z)^2 in float32.
-__device__ __forceinline__ void sqrelu8(const __nv_bfloat16 *z, float (&x)[8])
+__device__ __forceinline__ void sqrelu8(const uint4 u, float (&x)[8])
 {
-    const uint4 u = *reinterpret_cast<const uint4 *>(z);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -72,6 +67,51 @@ __device__ __forceinline__ size_t meta8_byte(int t, int c, int kt)
     return word * 4 + (c & 3);
 }
 
+// E4M3 codes of two values, a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b)
+{
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Codes (4 bytes, channel order) and positions (one byte) of the kept values
+// of one 8-channel chunk (two 4-blocks); `keep` gets the 8 keep bits.
+__device__ __forceinline__ void chunk_codes(const float (&x)[8], float inv, uint32_t &codes, uint32_t &meta,
+                                            uint32_t &keep)
+{
+    keep = keep_2of4<float>(x);
+    const uint32_t lo = e4m3x2(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv)) |
+                            (e4m3x2(__fmul_rn(x[2], inv), __fmul_rn(x[3], inv)) << 16);
+    const uint32_t hi = e4m3x2(__fmul_rn(x[4], inv), __fmul_rn(x[5], inv)) |
+                            (e4m3x2(__fmul_rn(x[6], inv), __fmul_rn(x[7], inv)) << 16);
+    int a0, a1, b0, b1;
+    pos_2of4(keep & 15u, a0, a1);
+    pos_2of4((keep >> 4) & 15u, b0, b1);
+    // byte permutes: bytes a0, a1 of lo, then bytes b0, b1 of hi (selector 4..7)
+    codes = __byte_perm(lo, hi, (uint32_t)a0 | ((uint32_t)a1 << 4) | ((uint32_t)(b0 + 4) << 8) |
+                                    ((uint32_t)(b1 + 4) << 12));
+    meta = (uint32_t)(a0 | (a1 << 2)) | ((uint32_t)(b0 | (b1 << 2)) << 4);
+}
+
+// Largest of eight bf16 values (as float32).
+__device__ __forceinline__ float max8_bf16(const uint4 u)
+{
+    __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+    a = __hmax2(a, *reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    a = __hmax2(a, *reinterpret_cast<const __nv_bfloat162 *>(&u.z));
+    a = __hmax2(a, *reinterpret_cast<const __nv_bfloat162 *>(&u.w));
+    return fmaxf(__low2float(a), __high2float(a));
+}
+
+// A row of up to F8_HELD * 8 * F8_THREADS channels is loaded once, with all
+// of a thread's loads in flight together, and kept in registers between the
+// amax pass and the code pass; longer rows are processed in slices of that
+// size and read again (from L2) for the codes.
+constexpr int F8_HELD = 8;
+
+// The amax over the kept values equals the amax over all of x: the largest
+// value of every 4-block is among its two kept ones.  x = r * r is exact for
+// a bf16 r (at most 16 significant bits) and increasing in r >= 0, so the
+// amax is the square of the largest positive z.
 __global__ void __launch_bounds__(F8_THREADS) k_sqrelu24_fp8(const __nv_bfloat16 *__restrict__ z, int T, int K,
                                                              uint8_t *__restrict__ x8, uint8_t *__restrict__ meta8,
                                                              float *__restrict__ x_scale,
@@ -81,47 +121,55 @@ __global__ void __launch_bounds__(F8_THREADS) k_sqrelu24_fp8(const __nv_bfloat16
     const int t = blockIdx.x;
     const int nch = K / 8;          // real 8-channel chunks
     const int nch_pad = kt * 32;    // chunks the metadata tiles cover
+    const int tid = threadIdx.x;
+    for (int c = nch + tid; c < nch_pad; c += F8_THREADS) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
     if (t >= T) {                   // padding rows of the last 256-row pair tile
-        for (int c = threadIdx.x; c < nch_pad; c += F8_THREADS) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
+        for (int c = tid; c < nch; c += F8_THREADS) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
         return;
     }
     const __nv_bfloat16 *zr = z + (size_t)t * K;
-    float amax = 0.0f;
-    for (int c = threadIdx.x; c < nch; c += F8_THREADS) {
-        float x[8];
-        sqrelu8(zr + 8 * c, x);
-        const uint32_t keep = keep_2of4<float>(x);
+    constexpr int SLICE = F8_HELD * F8_THREADS;  // chunks per slice
+    uint4 held[F8_HELD];
+    float zmax = 0.0f;
+    for (int base = 0; base < nch; base += SLICE) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if ((keep >> e) & 1u) amax = fmaxf(amax, x[e]);
+        for (int r = 0; r < F8_HELD; ++r) {
+            const int c = base + tid + r * F8_THREADS;
+            held[r] = c < nch ? *reinterpret_cast<const uint4 *>(zr + 8 * c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int r = 0; r < F8_HELD; ++r) zmax = fmaxf(zmax, max8_bf16(held[r]));
     }
-    amax = block_max(amax, red);
+    zmax = block_max(zmax, red);
+    const float amax = __fmul_rn(zmax, zmax);
     const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    if (threadIdx.x == 0) x_scale[t] = scale;
+    const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+    if (tid == 0) x_scale[t] = scale;
 
     uint8_t *xr = x8 + (size_t)t * (K / 2);
-    for (int c = threadIdx.x; c < nch_pad; c += F8_THREADS) {
-        if (c >= nch) {
-            meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
-            continue;
-        }
-        float x[8];
-        sqrelu8(zr + 8 * c, x);
-        const uint32_t keep = keep_2of4<float>(x);
-        uint32_t codes = 0, meta = 0;
+    const size_t bm_row = (size_t)t * ((K + 31) / 32) * 4;
+    for (int base = 0; base < nch; base += SLICE) {
+        if (nch > SLICE) {  // several slices: `held` has the last one, read each again
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            int i0, i1;
-            pos_2of4((keep >> (4 * h)) & 15u, i0, i1);
-            const float v0 = h ? (i0 == 0 ? x[4] : i0 == 1 ? x[5] : x[6]) : (i0 == 0 ? x[0] : i0 == 1 ? x[1] : x[2]);
-            const float v1 = h ? (i1 == 3 ? x[7] : i1 == 2 ? x[6] : x[5]) : (i1 == 3 ? x[3] : i1 == 2 ? x[2] : x[1]);
-            codes |= ((uint32_t)e4m3_rn_sat(__fdiv_rn(v0, scale)) | ((uint32_t)e4m3_rn_sat(__fdiv_rn(v1, scale)) << 8))
-                     << (16 * h);
-            meta |= (uint32_t)(i0 | (i1 << 2)) << (4 * h);
+            for (int r = 0; r < F8_HELD; ++r) {
+                const int c = base + tid + r * F8_THREADS;
+                held[r] = c < nch ? *reinterpret_cast<const uint4 *>(zr + 8 * c) : make_uint4(0, 0, 0, 0);
+            }
         }
-        *reinterpret_cast<uint32_t *>(xr + 4 * c) = codes;
-        meta8[meta8_byte(t, c, kt)] = (uint8_t)meta;
-        if (bitmask) bitmask[(size_t)t * ((K + 31) / 32) * 4 + c] = (uint8_t)keep;
+        // chunks c and c + F8_THREADS lie 8 metadata tiles (32 KB) apart
+        const size_t mb0 = meta8_byte(t, base + tid, kt);
+#pragma unroll
+        for (int r = 0; r < F8_HELD; ++r) {
+            const int c = base + tid + r * F8_THREADS;
+            if (c >= nch) break;
+            float x[8];
+            sqrelu8(held[r], x);
+            uint32_t codes, meta, keep;
+            chunk_codes(x, inv, codes, meta, keep);
+            *reinterpret_cast<uint32_t *>(xr + 4 * c) = codes;
+            meta8[mb0 + (size_t)r * (F8_THREADS / 32) * 4096] = (uint8_t)meta;
+            if (bitmask) bitmask[bm_row + c] = (uint8_t)keep;
+        }
     }
 }
 
@@ -163,17 +211,16 @@ __global__ void __launch_bounds__(F8_THREADS) k_quant_rows_fp8(const TW *__restr
     }
     amax = block_max(amax, red);
     const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
     if (threadIdx.x == 0) w_scale[o] = scale;
     uint8_t *qr = Wq + (size_t)o * K;
     for (int c = threadIdx.x; c < nch; c += F8_THREADS) {
         float v[8];
         load8<TW>(wr + 8 * c, v);
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            lo |= (uint32_t)e4m3_rn_sat(__fdiv_rn(v[e], scale)) << (8 * e);
-            hi |= (uint32_t)e4m3_rn_sat(__fdiv_rn(v[4 + e], scale)) << (8 * e);
-        }
+        const uint32_t lo = e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
+                                (e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
+        const uint32_t hi = e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv)) |
+                                (e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv)) << 16);
         *reinterpret_cast<uint2 *>(qr + 8 * c) = make_uint2(lo, hi);
     }
 }
