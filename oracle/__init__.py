@@ -26,6 +26,8 @@ Functions and the passages they follow (page title, section):
   (``token_mean``) or a calibrated table.
 * ``var_scale``     overview §3.2.
 * ``linear``        overview §3.1 / §3.2 and the layer definition y = prune(x) W^T.
+* ``rsparse``, ``rsparse_factors``  overview §3.3 (R-Sparse low-rank compensation;
+                    the factors from a truncated SVD, numpy's).
 * ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
 * ``e4m3_encode``/``e4m3_decode``, ``quant_rows_fp8``, ``sqrelu24_fp8``,
   ``linear_fp8``    2:4 + Squared-ReLU page §3.1 (fused Squared-ReLU + 2:4 +
@@ -84,6 +86,7 @@ def _load():
                 "or_linear": [P, P, I, I, P, P, I, P, P, P, I, P],
                 "or_compress_nm": [P, P, I, I, I, I, P, P],
                 "or_quant_rows_fp8": [P, I, I, P, P],
+                "or_rsparse": [P, P, I, I, P, P, P, I, I, P],
                 "or_sqrelu24_fp8": [P, I, I, P, P, P, P, P],
             }
             for name, args in sig.items():
@@ -316,3 +319,27 @@ def linear_fp8(x_codes, x_pos, x_scale, w_codes, w_scale, rows=None):
     col = (np.arange(kc) // 2) * 4 + x_pos.astype(np.int64)
     np.put_along_axis(xd, col, dequant_fp8(x_codes, x_scale), axis=1)
     return xd @ dequant_fp8(w_codes, w_scale).T
+
+
+def rsparse_factors(W, r: int):
+    """A_r = U_r diag(S_r) [n_out, r] and B_r = V_r [k, r] from numpy's SVD of
+    W [n_out, k] in float64 (overview page §3.3)."""
+    W64 = np.asarray(W.float().numpy() if hasattr(W, "numpy") and not isinstance(W, np.ndarray) else W,
+                     np.float64)
+    U, S, Vh = np.linalg.svd(W64, full_matrices=False)
+    return U[:, :r] * S[:r], Vh[:r, :].T.copy()
+
+
+def rsparse(x, mask, B, A, eta=None):
+    """float64 compensation [T, n_out] = (xhat * (1 - mask)) B A^T."""
+    x = _f32(x)
+    T, k = x.shape
+    B = _f32(B)
+    A = _f32(A)
+    r = B.shape[1]
+    n_out = A.shape[0]
+    mask = np.ascontiguousarray(mask, np.uint8)
+    e = None if eta is None else np.ascontiguousarray(eta, np.float64)
+    comp = np.empty((T, n_out), np.float64)
+    _load().or_rsparse(_ptr(x), _ptr(mask), T, k, _ptr(e), _ptr(B), _ptr(A), n_out, r, _ptr(comp))
+    return comp

@@ -16,7 +16,8 @@
  *   [OVW]  "激活稀疏化技术：提升LLM推理效率的动态剪枝方法"
  *          (activation-sparsity overview): section 2.1 N:M patterns,
  *          2.2.1 magnitude pruning, 2.2.3 CLACT score, 3.1 D-PTS,
- *          3.2 VAR variance correction, 2.2.2 Amber-Pruner channel importance.
+ *          3.2 VAR variance correction, 2.2.2 Amber-Pruner channel importance,
+ *          3.3 R-Sparse low-rank compensation.
  *   [WIS]  "大模型推理优化：WiSparse激活稀疏化技术解析": section 2.1, eq. (4),
  *          weight-aware score s_i = |x_i| * ||W[:,i]||_2^alpha; section 2.2
  *          per-layer keep fraction (top-k).
@@ -455,6 +456,36 @@ void or_linear(const float *x, const uint8_t *mask, int T, int k,
         }
         free(xv);
     }
+}
+
+/* ---------------------------------------------------------------------------
+ * R-Sparse low-rank compensation ([OVW] section 3.3): W ~ W_sparse + A_r B_r^T
+ * with A_r = U_r diag(S_r) [n_out, r] and B_r = V_r [k, r] from a truncated
+ * SVD of W.  Reading: the kept channels go through W itself and the dropped
+ * ones through the rank-r factors, so the layer adds
+ *   comp[t,o] = sum_j ( sum_i xhat_ti (1 - m_ti) B[i,j] ) A[o,j]
+ * to y (xhat = x - eta with D-PTS, else x).  Computed in float64 in the
+ * order written: first u = xhat_dropped B_r, then u A_r^T.
+ * ------------------------------------------------------------------------- */
+void or_rsparse(const float *x, const uint8_t *mask, int T, int k, const double *eta,
+                const float *B, const float *A, int n_out, int r, double *comp)
+{
+    double *u = (double *)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1));
+    for (int t = 0; t < T; t++) {
+        for (int j = 0; j < r; j++) u[j] = 0.0;
+        for (int i = 0; i < k; i++) {
+            if (mask[(size_t)t * k + i]) continue;
+            double v = (double)x[(size_t)t * k + i];
+            if (eta) v -= eta[t];
+            for (int j = 0; j < r; j++) u[j] += v * (double)B[(size_t)i * r + j];
+        }
+        for (int o = 0; o < n_out; o++) {
+            double acc = 0.0;
+            for (int j = 0; j < r; j++) acc += u[j] * (double)A[(size_t)o * r + j];
+            comp[(size_t)t * n_out + o] = acc;
+        }
+    }
+    free(u);
 }
 
 /* [SQR] section 3.3: compressed N:M layout, the kept values of every block

@@ -581,3 +581,61 @@ def test_linear_fp8_integer_case(oracle_lib):
     w = r.integers(-8, 9, size=(n_out, k)).astype(np.float64)
     y = oracle_lib.linear_fp8(codes, pos, np.ones(T, np.float32), oracle_lib.e4m3_encode(w), np.ones(n_out, np.float32))
     np.testing.assert_array_equal(y, xk @ w.T)
+
+
+# ---------------------------------------------------------------- R-Sparse low-rank compensation
+def test_rsparse_full_rank_restores_dense(oracle_lib):
+    """With every singular vector kept (r = min(n_out, k)), A B^T = W, so the
+    pruned product plus the compensation is the dense product (with and
+    without D-PTS, whose eta * rowsum term restores the shift)."""
+    import synth
+    x, W = synth.random_layer(3, 48, 40, seed=61, dtype=torch.float32)
+    xf, Wf = x.numpy(), W.numpy()
+    A, B = oracle_lib.rsparse_factors(Wf, 40)
+    mask = oracle_lib.select_nm(oracle_lib.score(xf), 8, 16)
+    dense = xf.astype(np.float64) @ Wf.astype(np.float64).T
+    for use_eta in (False, True):
+        eta = oracle_lib.token_mean(xf) if use_eta else None
+        _, rs = oracle_lib.weight_prep(Wf, 1.0)
+        y = oracle_lib.linear(xf, mask, Wf, eta=eta, rowsum=rs if use_eta else None)
+        comp = oracle_lib.rsparse(xf, mask, B.astype(np.float32), A.astype(np.float32), eta=eta)
+        # A, B rounded to float32: the identity holds to float32 precision of the factors
+        np.testing.assert_allclose(y + comp, dense, rtol=0, atol=2e-6 * np.abs(dense).max())
+
+
+def test_rsparse_exact_low_rank_weight(oracle_lib):
+    """W = P Q^T of rank 4 with P, Q on a coarse grid (exact in float32):
+    rank-4 compensation with A = P, B = Q is exact, and keep-all adds 0."""
+    r = np.random.default_rng(62)
+    P = (r.integers(-4, 5, size=(24, 4)) / 4).astype(np.float32)
+    Q = (r.integers(-4, 5, size=(32, 4)) / 4).astype(np.float32)
+    W = (P.astype(np.float64) @ Q.T.astype(np.float64)).astype(np.float32)
+    x = (r.integers(-8, 9, size=(5, 32)) / 8).astype(np.float32)
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    y = oracle_lib.linear(x, mask, W) + oracle_lib.rsparse(x, mask, Q, P)
+    np.testing.assert_array_equal(y, x.astype(np.float64) @ W.astype(np.float64).T)
+    assert not oracle_lib.rsparse(x, np.ones_like(mask), Q, P).any()
+    # the factors of an exactly rank-4 W from the SVD reproduce it
+    A, B = oracle_lib.rsparse_factors(W, 4)
+    np.testing.assert_allclose(A @ B.T, W, atol=1e-12)
+
+
+def test_rsparse_truncation_error_is_the_tail(oracle_lib):
+    """The compensation's error against the dense product is the dropped
+    part times the discarded singular directions: it shrinks as r grows and
+    vanishes at full rank (Eckart-Young ordering of the SVD)."""
+    import synth
+    x, W = synth.random_layer(2, 64, 48, seed=63, dtype=torch.float32)
+    xf, Wf = x.numpy(), W.numpy()
+    mask = oracle_lib.select_nm(oracle_lib.score(xf), 2, 4)
+    dense = xf.astype(np.float64) @ Wf.astype(np.float64).T
+    base = oracle_lib.linear(xf, mask, Wf)
+    errs = []
+    for rank in (0, 8, 24, 48):
+        if rank:
+            A, B = oracle_lib.rsparse_factors(Wf, rank)
+            y = base + oracle_lib.rsparse(xf, mask, B.astype(np.float32), A.astype(np.float32))
+        else:
+            y = base
+        errs.append(np.linalg.norm(y - dense))
+    assert errs[0] > errs[1] > errs[2] > errs[3] and errs[3] < 1e-5 * errs[0]
