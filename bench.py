@@ -290,6 +290,46 @@ def bench_decode(sl, dev, steps, warmup, world):
             per_t_spts[T] = (timed(lambda j, g_s=g_s: g_s.replay(), reps) / (reps * N_ROT), tab, cfg_s, g_s)
     per_t_spts = {T: v[0] for T, v in per_t_spts.items()}
 
+    # the same calls with R-Sparse compensation (rank 64, float32 output): the
+    # decode exports its mask and eta, then the dropped channels go through
+    # the low-rank factors (random bf16 factors: only the time is measured)
+    rng = np.random.default_rng(4343)
+    A_rs = torch.from_numpy(rng.normal(0, 0.05, (N_DOWN, 64)).astype(np.float32)).to(torch.bfloat16).to(dev)
+    B_rs = torch.from_numpy(rng.normal(0, 0.02, (K_DOWN, 64)).astype(np.float32)).to(torch.bfloat16).to(dev)
+    cfg_r = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True, out_dtype=sl.AS_F32)
+    per_t_rs = {}
+    with torch.cuda.stream(stream):
+        for T in DECODE_TS:
+            bufs_r = dict(y=torch.empty(T, N_DOWN, dtype=torch.float32, device=dev),
+                          m=torch.empty(T, words, dtype=torch.int32, device=dev),
+                          e=torch.empty(T, dtype=torch.float32, device=dev),
+                          ws=workspace(sl.as_workspace_size(sl.AS_OP_DECODE, T, K_DOWN, N_DOWN, cfg_r), dev),
+                          wr=workspace(sl.as_rsparse_workspace(T, K_DOWN, 64), dev))
+
+            def call_r(i, T=T, b=bufs_r):
+                sl.as_linear_decode(xs[i][:T], Wts[i], cfg_r, b["y"], g=L.g, rowsum=L.rowsum, mask_out=b["m"],
+                                    eta_out=b["e"], workspace=b["ws"], stream=stream)
+                sl.as_rsparse_decode(xs[i][:T], b["m"], B_rs, A_rs, b["y"], eta=b["e"], workspace=b["wr"],
+                                     stream=stream)
+            def call_f(i, T=T, b=bufs_r):
+                sl.as_linear_decode(xs[i][:T], Wts[i], cfg_r, b["y"], g=L.g, rowsum=L.rowsum, mask_out=b["m"],
+                                    eta_out=b["e"], workspace=b["ws"], stream=stream)
+            for i in range(N_ROT):
+                call_r(i)
+            stream.synchronize()
+            g_r = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_r, stream=stream):
+                for i in range(N_ROT):
+                    call_r(i)
+            g_f = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_f, stream=stream):
+                for i in range(N_ROT):
+                    call_f(i)
+            per_t_rs[T] = (timed(lambda j, g_r=g_r: g_r.replay(), reps) / (reps * N_ROT),
+                           timed(lambda j, g_f=g_f: g_f.replay(), reps) / (reps * N_ROT), bufs_r, g_r, g_f)
+    per_t_f32 = {T: v[1] for T, v in per_t_rs.items()}
+    per_t_rs = {T: v[0] for T, v in per_t_rs.items()}
+
     # end to end through host buffers, every step: pinned host x -> device,
     # decode, y -> pinned host.  Copies run on their own streams (H2D and D2H
     # use separate copy engines) into double-buffered device x and y, so the
@@ -406,6 +446,8 @@ def bench_decode(sl, dev, steps, warmup, world):
         per_t={T: dict(us=per_t[T] * 1e6, gbs=bytes_call[T] / per_t[T] / 1e9, bytes=bytes_call[T])
                for T in DECODE_TS},
         per_t_spts={T: dict(us=per_t_spts[T] * 1e6, tokens_per_s=T / per_t_spts[T]) for T in DECODE_TS},
+        per_t_rs={T: dict(us=per_t_rs[T] * 1e6, tokens_per_s=T / per_t_rs[T],
+                          decode_only_f32_out_us=per_t_f32[T] * 1e6) for T in DECODE_TS},
         achieved_gbs=step_bytes / kern_time / 1e9, bytes_per_step=step_bytes,
         bytes_per_launch=step_bytes / len(DECODE_TS),
         clocks=clk.summary(), launches=steps * launches_per_step)
@@ -785,6 +827,12 @@ def main():
         "note": "the same decode calls with S-PTS (eta from a calibration table) instead of D-PTS",
         "per_T": {str(T): v for T, v in d["per_t_spts"].items()},
         "step_us": sum(v["us"] for v in d["per_t_spts"].values())}
+    extra["decode_downproj_rsparse_r64"] = {
+        "note": "the same decode calls with float32 output plus the R-Sparse rank-64 compensation of the "
+                "dropped channels (two more kernels per call; random bf16 factors); decode_only_f32_out_us "
+                "times the float32-output decode calls without it",
+        "per_T": {str(T): v for T, v in d["per_t_rs"].items()},
+        "step_us": sum(v["us"] for v in d["per_t_rs"].values())}
     line["configs_extra"] = extra
     print(json.dumps(line), flush=True)
 

@@ -278,6 +278,29 @@ size_t as_workspace_size(int op, int T, int K, int n_out, const as_config *cfg);
  * invalid.  Host-only. */
 int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cfg);
 
+/* --------------------------------------------------------------------------
+ * R-Sparse low-rank compensation of a decode call ([OVW] 3.3).  The weight
+ * is approximated as W ~ W_sparse + A_r B_r^T with A_r = U_r diag(S_r)
+ * [n_out, r] and B_r = V_r [K, r] from a truncated SVD of W (computed
+ * offline by the caller; the page uses r = 64).  The kept channels already
+ * went through W in the call; this adds the dropped ones through the
+ * factors:
+ *   u[t, j]  = sum over channels i with mask bit (t, i) clear of xhat[t, i] B[i, j]
+ *   y[t, o] += sum_j u[t, j] A[o, j]
+ * with xhat = fl32(x - eta[t]) when eta is given (D-PTS or S-PTS: pass the
+ * call's eta_out or table) and x otherwise.
+ *   x      [T, K] in `dt`, the call's input, 1 <= T <= 16.
+ *   mask   [T, ceil(K/32)] uint32, the call's mask_out (bit i%32 of word i/32 = kept).
+ *   B, A   bf16 [K, r] and [n_out, r]; r in {32, 64, 128}; A 16-byte aligned.
+ *   y      [T, n_out] float32, in/out (the call with out_dtype AS_F32).
+ * Float32 accumulation in a fixed order (deterministic); two kernels.
+ * Workspace: as_rsparse_workspace(T, K, r) bytes, no zero-fill needed.
+ * ------------------------------------------------------------------------ */
+size_t as_rsparse_workspace(int T, int K, int r);
+as_status as_rsparse_decode(const void *x, as_dtype dt, int T, int K, int n_out, int r, const uint32_t *mask,
+                            const float *eta, const void *B, const void *A, float *y, void *workspace,
+                            size_t ws_bytes, cudaStream_t stream);
+
 /* Number of 32-bit metadata words of a 2:4 selection of T tokens x K channels. */
 size_t as_meta24_words(int T, int K);
 

@@ -40,7 +40,7 @@ EXPORTS = [
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
     "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches", "as_probe_timeout",
     "as_weight_prep_amber", "as_meta8_words", "as_weight_quant_fp8", "as_select_sqrelu24_fp8",
-    "as_linear_prefill_fp8",
+    "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -64,6 +64,8 @@ _sig = {
     "as_weight_prep": ([_P, _I, _I, _I, _F, _P, _P, _P, _P, _S, _P], _I),
     "as_weight_prep_amber": ([_P, _I, _I, _I, _F, ctypes.c_double, ctypes.c_double, _P, _P, _P, _S, _P], _I),
     "as_meta8_words": ([_I, _I], _S),
+    "as_rsparse_workspace": ([_I, _I, _I], _S),
+    "as_rsparse_decode": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P], _I),
     "as_weight_quant_fp8": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "as_select_sqrelu24_fp8": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
     "as_linear_prefill_fp8": ([_P, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P], _I),
@@ -180,6 +182,22 @@ def as_weight_prep_amber(W, g, alpha: float = 1.0, lo_pct: float = 0.5, hi_pct: 
     _check(_lib.as_weight_prep_amber(_ptr(W), _dt(W), n_out, K, float(alpha), float(lo_pct), float(hi_pct),
                                      _ptr(g), _ptr(bounds), _ptr(workspace), ws_bytes, _stream(stream)),
            "as_weight_prep_amber")
+
+
+def as_rsparse_workspace(T: int, K: int, r: int) -> int:
+    n = _lib.as_rsparse_workspace(T, K, r)
+    if n == ctypes.c_size_t(-1).value:
+        raise ASError(AS_ERR_SHAPE, "as_rsparse_workspace")
+    return n
+
+
+def as_rsparse_decode(x, mask, B, A, y, eta=None, workspace=None, stream=None) -> None:
+    """y (float32, in/out) += R-Sparse compensation of the dropped channels."""
+    T, K = x.shape
+    n_out, r = A.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_rsparse_decode(_ptr(x), _dt(x), T, K, n_out, r, _ptr(mask), _ptr(eta), _ptr(B), _ptr(A),
+                                  _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "as_rsparse_decode")
 
 
 def as_meta8_words(T: int, K: int) -> int:

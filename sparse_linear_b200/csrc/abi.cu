@@ -144,6 +144,39 @@ as_status as_weight_prep_amber(const void *W, as_dtype dt, int n_out, int K, flo
     return cuda_status(launch_amber(W, dt == AS_BF16, n_out, K, alpha, r_lo, r_hi, g, bounds, workspace, stream));
 }
 
+static bool rsparse_rank_ok(int r) { return r == 32 || r == 64 || r == 128; }
+
+size_t as_rsparse_workspace(int T, int K, int r)
+{
+    if (T < 1 || T > AS_MAX_DECODE_T || K <= 0 || !rsparse_rank_ok(r)) return (size_t)-1;
+    return rsparse_workspace(T, K, r);
+}
+
+as_status as_rsparse_decode(const void *x, as_dtype dt, int T, int K, int n_out, int r, const uint32_t *mask,
+                            const float *eta, const void *B, const void *A, float *y, void *workspace,
+                            size_t ws_bytes, cudaStream_t stream)
+{
+    if (!x || !mask || !B || !A || !y || K <= 0 || n_out <= 0) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    if (T < 1 || T > AS_MAX_DECODE_T || !rsparse_rank_ok(r)) return AS_ERR_SHAPE;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(workspace)) return AS_ERR_ALIGN;
+    if (!workspace || ws_bytes < rsparse_workspace(T, K, r)) return AS_ERR_WORKSPACE;
+    RsparseArgs a{};
+    a.x = x;
+    a.bf16 = dt == AS_BF16;
+    a.mask = mask;
+    a.eta = eta;
+    a.B = B;
+    a.A = A;
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.r = r;
+    a.y = y;
+    a.workspace = workspace;
+    return cuda_status(launch_rsparse(a, stream));
+}
+
 size_t as_meta8_words(int T, int K)
 {
     if (T <= 0 || K <= 0) return 0;

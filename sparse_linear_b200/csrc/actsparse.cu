@@ -5,5 +5,6 @@
 #include "decode.cu"
 #include "gemm.cu"
 #include "fp8.cu"
+#include "rsparse.cu"
 #include "abi.cu"
 #include "noalloc.cu"

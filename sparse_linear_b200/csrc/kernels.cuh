@@ -96,6 +96,20 @@ struct Fp8GemmArgs {
     int out_bf16;
 };
 cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st);
+
+// R-Sparse decode compensation (rsparse.cu).
+struct RsparseArgs {
+    const void *x;          // [T, K] in the call's dtype
+    int bf16;
+    const uint32_t *mask;   // [T, ceil(K/32)], bit set = kept
+    const float *eta;       // [T] or NULL
+    const void *B, *A;      // bf16 [K, r], [n_out, r]
+    int T, K, n_out, r;
+    float *y;               // [T, n_out], in/out
+    void *workspace;
+};
+size_t rsparse_workspace(int T, int K, int r);
+cudaError_t launch_rsparse(const RsparseArgs &a, cudaStream_t st);
 int meta8_kt(int K);
 size_t meta8_words(int T, int K);
 cudaError_t launch_sqrelu24_fp8(const void *z, int T, int K, uint8_t *x8, uint32_t *meta8, float *x_scale,

@@ -200,3 +200,23 @@ def test_fp8_validation_launches_nothing(lib):
     assert f(fake, fake, fake, 8, 128, 64, fake, fake, 5, fake, None) == lib.AS_ERR_DTYPE
     assert f(fake, None, fake, 8, 128, 64, fake, fake, lib.AS_BF16, fake, None) == lib.AS_ERR_INVALID_ARG
     assert f(fake, fake, fake, 8, 128, 64, fake, fake + 8, lib.AS_BF16, fake, None) == lib.AS_ERR_ALIGN
+
+
+def test_rsparse_validation_launches_nothing(lib):
+    fake = 1 << 20
+    f = lib._lib.as_rsparse_decode
+    ws = lib.as_rsparse_workspace(16, 11008, 64)
+    assert ws == 86 * 16 * 64 * 4
+    for r in (0, 8, 16, 48, 256):
+        with pytest.raises(lib.ASError):
+            lib.as_rsparse_workspace(1, 64, r)
+
+    def call(T=1, K=64, n_out=64, r=64, x=fake, A=fake, wb=1 << 20, dt=lib.AS_BF16):
+        return f(x, dt, T, K, n_out, r, fake, None, fake, A, fake, fake, wb, None)
+
+    assert call(T=0) == lib.AS_ERR_SHAPE and call(T=17) == lib.AS_ERR_SHAPE
+    assert call(r=48) == lib.AS_ERR_SHAPE
+    assert call(x=None) == lib.AS_ERR_INVALID_ARG
+    assert call(dt=3) == lib.AS_ERR_DTYPE
+    assert call(A=fake + 2) == lib.AS_ERR_ALIGN
+    assert call(wb=0) == lib.AS_ERR_WORKSPACE

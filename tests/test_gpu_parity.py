@@ -526,3 +526,68 @@ def test_fp8_gemm_full_size(sl):
     n_out 4096), checked on sampled rows spread over every row tile."""
     rows = np.arange(5, 4096, 61)
     check_fp8_gemm(sl, 4096, 14336, 4096, torch.bfloat16, seed=3, rows=rows)
+
+
+# ---------------------------------------------------------------- R-Sparse compensation (decode)
+def _bf16r(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("T,K,n_out,r,dpts,svd", [
+    (1, 1024, 512, 64, True, True),
+    (5, 1008, 264, 32, False, True),
+    (16, 2048, 1024, 128, True, True),
+    (8, 11008, 4096, 64, True, False),   # the down-projection, random factors
+])
+def test_rsparse_decode(sl, T, K, n_out, r, dpts, svd):
+    """The decode call (float32 out) followed by the compensation against the
+    oracle's pruned product plus its float64 compensation, on the same
+    bf16-rounded factors (from numpy's SVD of W, or random at full size)."""
+    x, W = synth.random_layer(T, K, n_out, seed=71)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=dpts, out_dtype=sl.AS_F32)
+    L = layer(sl, W, cfg, 0.5)
+    if svd:
+        U, S, Vh = np.linalg.svd(W.double().numpy(), full_matrices=False)
+        A, B = _bf16r(U[:, :r] * S[:r]), _bf16r(Vh[:r, :].T)
+    else:
+        rng = np.random.default_rng(72)
+        A, B = _bf16r(rng.normal(0, 0.05, (n_out, r))), _bf16r(rng.normal(0, 0.02, (K, r)))
+    xd = dev(x)
+    mask_d = torch.zeros(T, (K + 31) // 32, dtype=torch.int32, device="cuda")
+    eta_d = torch.zeros(T, dtype=torch.float32, device="cuda")
+    y = L.decode(xd, mask_out=mask_d, eta_out=eta_d)
+    ws = torch.empty(sl.as_rsparse_workspace(T, K, r), dtype=torch.uint8, device="cuda")
+    sl.as_rsparse_decode(xd, mask_d, dev(B), dev(A), y, eta=eta_d if dpts else None, workspace=ws)
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    xf, Wf = x.float().numpy(), W.float().numpy()
+    mask = unpack_bitmask(mask_d, K)
+    eta32 = f32(eta_d) if dpts else None
+    s = oracle.score(xf, eta=eta32, f=f32(L.g))
+    np.testing.assert_array_equal(mask, oracle.select_nm(s, 8, 16))
+    eta64 = oracle.token_mean(xf) if dpts else None
+    _, rs = oracle.weight_prep(Wf, 1.0)
+    ref = oracle.linear(xf, mask, Wf, eta=eta64, rowsum=rs if dpts else None)
+    comp = oracle.rsparse(xf, mask, B.float().numpy(), A.float().numpy(), eta=eta64)
+    assert rel_l2(f32(y), ref + comp) <= TOL_F32
+    # the compensation itself, isolated from the pruned product
+    y2 = L.decode(xd)
+    y0 = y2.clone()
+    sl.as_rsparse_decode(xd, mask_d, dev(B), dev(A), y2, eta=eta_d if dpts else None, workspace=ws)
+    torch.cuda.synchronize()
+    assert rel_l2(f32(y2) - f32(y0), comp) <= TOL_F32
+
+
+def test_rsparse_keep_all_adds_nothing(sl):
+    """A mask with every bit set (nothing dropped) leaves y unchanged, bit for bit."""
+    T, K, n_out, r = 4, 512, 256, 32
+    x, _ = synth.random_layer(T, K, n_out, seed=73)
+    rng = np.random.default_rng(74)
+    A, B = _bf16r(rng.normal(0, 0.05, (n_out, r))), _bf16r(rng.normal(0, 0.02, (K, r)))
+    y = torch.randn(T, n_out, device="cuda")
+    y0 = y.clone()
+    full = torch.full((T, K // 32), -1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(sl.as_rsparse_workspace(T, K, r), dtype=torch.uint8, device="cuda")
+    sl.as_rsparse_decode(dev(x), full, dev(B), dev(A), y, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0)
