@@ -26,6 +26,8 @@ Functions and the passages they follow (page title, section):
   (``token_mean``) or a calibrated table.
 * ``var_scale``     overview §3.2.
 * ``linear``        overview §3.1 / §3.2 and the layer definition y = prune(x) W^T.
+* ``block_nnz``, ``pick_dense``, ``hybrid_mode``, ``hybrid_mask``  2:4 +
+                    Squared-ReLU page §3.2-3.3 (sparse/dense split, mode switch).
 * ``rsparse``, ``rsparse_factors``  overview §3.3 (R-Sparse low-rank compensation;
                     the factors from a truncated SVD, numpy's).
 * ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
@@ -87,12 +89,15 @@ def _load():
                 "or_compress_nm": [P, P, I, I, I, I, P, P],
                 "or_quant_rows_fp8": [P, I, I, P, P],
                 "or_rsparse": [P, P, I, I, P, P, P, I, I, P],
+                "or_pick_dense": [P, I, I, P],
                 "or_sqrelu24_fp8": [P, I, I, P, P, P, P, P],
             }
             for name, args in sig.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
                 fn.restype = None
+            lib.or_block_nnz.argtypes = [P, I, I, P]
+            lib.or_block_nnz.restype = ctypes.c_longlong
             lib.or_e4m3_encode.argtypes = [D]
             lib.or_e4m3_encode.restype = ctypes.c_uint8
             lib.or_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -343,3 +348,43 @@ def rsparse(x, mask, B, A, eta=None):
     comp = np.empty((T, n_out), np.float64)
     _load().or_rsparse(_ptr(x), _ptr(mask), T, k, _ptr(e), _ptr(B), _ptr(A), n_out, r, _ptr(comp))
     return comp
+
+
+def block_nnz(x):
+    """Nonzeros per 4-channel block over all tokens [k/4] and the total."""
+    x = _f32(x)
+    T, k = x.shape
+    nnz = np.empty(k // 4, np.int32)
+    total = _load().or_block_nnz(_ptr(x), T, k, _ptr(nnz))
+    return nnz, int(total)
+
+
+def pick_dense(nnz, n_dense: int):
+    """Block indices (ascending) of the n_dense blocks with the most nonzeros."""
+    nnz = np.ascontiguousarray(nnz, np.int32)
+    idx = np.empty(n_dense, np.int32)
+    _load().or_pick_dense(_ptr(nnz), len(nnz), int(n_dense), _ptr(idx))
+    return idx
+
+
+def hybrid_mode(sparsity: float) -> str:
+    """The 2:4 + Squared-ReLU page §3.3: above 95 % pure 2:4, 90-95 % split,
+    below 90 % dense."""
+    if sparsity > 0.95:
+        return "2:4"
+    if sparsity >= 0.90:
+        return "split"
+    return "dense"
+
+
+def hybrid_mask(x, n_dense: int):
+    """Mask of the split: all channels of the dense blocks, 2:4 by magnitude
+    elsewhere; returns (mask, dense block indices, sparsity)."""
+    x = _f32(x)
+    T, k = x.shape
+    nnz, total = block_nnz(x)
+    idx = pick_dense(nnz, n_dense)
+    mask = select_nm(score(x), 2, 4)
+    for b in idx:
+        mask[:, 4 * b:4 * b + 4] = 1
+    return mask, idx, 1.0 - total / float(T * k)

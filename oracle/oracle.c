@@ -24,6 +24,7 @@
  *   [SQR]  "利用2:4稀疏性与Squared-ReLU加速Transformer训练与推理": section 2.1
  *          2:4 pattern, 2.3 dropping the smallest of a 3-nonzero block,
  *          3.3 compressed layout with the kept values stored contiguously,
+ *          3.2-3.3 sparse/dense feature split and the sparsity-driven mode,
  *          3.1 fused Squared-ReLU + 2:4 + FP8 producer and the FP8
  *          row-scaled 2:4 GEMM, 5.3 sparsify before quantising.
  *
@@ -486,6 +487,47 @@ void or_rsparse(const float *x, const uint8_t *mask, int T, int k, const double 
         }
     }
     free(u);
+}
+
+/* ---------------------------------------------------------------------------
+ * Hybrid 2:4 for inference ([SQR] sections 3.2 and 3.3): the layer's measured
+ * sparsity picks the mode (above 95 %: pure 2:4; 90-95 %: split; below
+ * 90 %: dense), and the split computes the densest features densely and
+ * the rest with 2:4.  Readings: features are taken in 4-channel blocks so
+ * the 2:4 part stays block-aligned; the dense set is the n_dense blocks
+ * with the most nonzeros over the T tokens (ties to the lower block index);
+ * the result is the masked product with mask = 1 on the dense blocks and
+ * the 2:4 magnitude selection elsewhere.
+ * nnz[b] = number of nonzero x[t, 4b..4b+3] over all t; total returned.
+ * ------------------------------------------------------------------------- */
+long long or_block_nnz(const float *x, int T, int k, int *nnz)
+{
+    long long total = 0;
+    for (int b = 0; b < k / 4; b++) nnz[b] = 0;
+    for (int t = 0; t < T; t++)
+        for (int i = 0; i < k; i++)
+            if (x[(size_t)t * k + i] != 0.0f) {
+                nnz[i / 4]++;
+                total++;
+            }
+    return total;
+}
+
+/* The n_dense blocks ranked first by (more nonzeros, then lower index),
+ * returned in ascending block order. */
+void or_pick_dense(const int *nnz, int nblocks, int n_dense, int *idx)
+{
+    uint8_t *taken = (uint8_t *)calloc((size_t)nblocks, 1);
+    for (int b = 0; b < nblocks; b++) {
+        int rank = 0;
+        for (int c = 0; c < nblocks; c++)
+            if (nnz[c] > nnz[b] || (nnz[c] == nnz[b] && c < b)) rank++;
+        taken[b] = (uint8_t)(rank < n_dense);
+    }
+    int w = 0;
+    for (int b = 0; b < nblocks; b++)
+        if (taken[b]) idx[w++] = b;
+    free(taken);
 }
 
 /* [SQR] section 3.3: compressed N:M layout, the kept values of every block

@@ -639,3 +639,64 @@ def test_rsparse_truncation_error_is_the_tail(oracle_lib):
             y = base
         errs.append(np.linalg.norm(y - dense))
     assert errs[0] > errs[1] > errs[2] > errs[3] and errs[3] < 1e-5 * errs[0]
+
+
+# ---------------------------------------------------------------- hybrid 2:4 (sparse/dense split)
+def test_hybrid_mode_thresholds(oracle_lib):
+    """The page's inference rule: > 95 % pure 2:4, 90-95 % split, < 90 % dense."""
+    assert [oracle_lib.hybrid_mode(s) for s in (0.99, 0.951, 0.95, 0.92, 0.90, 0.899, 0.5)] == \
+        ["2:4", "2:4", "split", "split", "split", "dense", "dense"]
+
+
+def test_pick_dense_ranks_by_nonzeros_then_index(oracle_lib):
+    """Hand case with ties, checked against a stable sort (numpy lexsort)."""
+    nnz = np.array([3, 9, 9, 0, 5, 9, 5, 1], np.int32)
+    np.testing.assert_array_equal(oracle_lib.pick_dense(nnz, 3), [1, 2, 5])
+    np.testing.assert_array_equal(oracle_lib.pick_dense(nnz, 5), [1, 2, 4, 5, 6])
+    r = np.random.default_rng(81)
+    for _ in range(20):
+        v = r.integers(0, 6, size=50).astype(np.int32)
+        n = int(r.integers(0, 51))
+        order = np.lexsort((np.arange(50), -v.astype(np.int64)))
+        np.testing.assert_array_equal(oracle_lib.pick_dense(v, n), np.sort(order[:n]))
+
+
+def test_block_nnz_counts(oracle_lib):
+    x = np.array([[0, 1, 0, 2, 0, 0, 0, 0], [3, 0, 0, 0, 0, 0, -1, 0]], np.float32)
+    nnz, total = oracle_lib.block_nnz(x)
+    np.testing.assert_array_equal(nnz, [3, 1])
+    assert total == 4
+
+
+def test_hybrid_extremes_are_pure_24_and_dense(oracle_lib):
+    """No dense blocks: the pure 2:4 product; every block dense: x W^T."""
+    import synth
+    x, W = synth.random_layer(6, 64, 24, seed=82, dtype=torch.float32, dist="sqrelu")
+    xf, Wf = x.numpy(), W.numpy()
+    m0, idx0, s = oracle_lib.hybrid_mask(xf, 0)
+    assert len(idx0) == 0 and 0.0 <= s <= 1.0
+    np.testing.assert_array_equal(m0, oracle_lib.select_nm(oracle_lib.score(xf), 2, 4))
+    mall, idx, _ = oracle_lib.hybrid_mask(xf, 16)
+    np.testing.assert_array_equal(idx, np.arange(16))
+    y = oracle_lib.linear(xf, mall, Wf)
+    np.testing.assert_allclose(y, xf.astype(np.float64) @ Wf.astype(np.float64).T, rtol=1e-12, atol=1e-14)
+
+
+def test_hybrid_recovers_dropped_nonzeros_of_dense_blocks(oracle_lib):
+    """Blocks with more than two nonzeros lose values under 2:4; making the
+    busiest blocks dense keeps all of theirs: the dropped nonzeros never grow
+    with the dense set, the dense blocks drop none, and with every block
+    dense the product is exact."""
+    import synth
+    x, W = synth.random_layer(16, 128, 32, seed=83, dtype=torch.float32, dist="sqrelu")
+    xf, Wf = x.numpy(), W.numpy()
+    dense = xf.astype(np.float64) @ Wf.astype(np.float64).T
+    dropped = []
+    for nd in (0, 4, 8, 16, 32):
+        mask, idx, _ = oracle_lib.hybrid_mask(xf, nd)
+        lost = (xf != 0) & (mask == 0)
+        dropped.append(int(lost.sum()))
+        for b in idx:
+            assert not lost[:, 4 * b:4 * b + 4].any()
+    assert dropped[0] > 0 and all(a >= b for a, b in zip(dropped, dropped[1:])) and dropped[-1] == 0
+    np.testing.assert_allclose(oracle_lib.linear(xf, mask, Wf), dense, rtol=1e-12, atol=1e-14)
