@@ -528,6 +528,35 @@ def bench_prefill(sl, dev, pk):
     del z, W, Wq, x8, meta8, y
     torch.cuda.empty_cache()
 
+    # hybrid 2:4 on activations with hot channels (~94 % zeros: the page's
+    # split regime): 2:4 GEMM alone vs the split with 192 dense blocks
+    # (768 channels), each against the dense product for the error it leaves
+    _, x, W, _ = synth.prefill_sqrelu_hot()
+    x, W = x.to(dev), W.to(dev)
+    T, K = x.shape
+    n_out = W.shape[0]
+    L = SparseLinear(W, sl.config(sel=sl.AS_SEL_NM, n=2, m=4), keep_wt=False)
+    bufs = L.select_buffers(T)
+    y24 = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
+    yh = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
+    sp = torch.empty(1, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        L.select(x, bufs)
+        L.prefill_from(bufs, T, y24)
+        L.prefill_hybrid_from(x, bufs, 192, y=yh, sparsity=sp)
+    t_sel = ev_time(lambda: L.select(x, bufs), 10)
+    t_24 = ev_time(lambda: L.prefill_from(bufs, T, y24), 10)
+    t_h = ev_time(lambda: L.prefill_hybrid_from(x, bufs, 192, y=yh, sparsity=sp), 10)
+    t_dense = ev_time(lambda: torch.matmul(x, W.t()), 10)
+    yd = torch.matmul(x.float(), W.float().t())
+    err = lambda yy: float(torch.linalg.norm(yy.float() - yd) / torch.linalg.norm(yd))  # noqa: E731
+    out["hybrid_split_hot_channels"] = dict(
+        shape=[T, K, n_out], sparsity=float(sp.item()), dense_blocks=192, select_us=t_sel * 1e6,
+        gemm_24_us=t_24 * 1e6, hybrid_us=t_h * 1e6, cublas_dense_us=t_dense * 1e6,
+        rel_err_vs_dense_24=err(y24), rel_err_vs_dense_hybrid=err(yh))
+    del x, W, L, bufs, y24, yh, yd
+    torch.cuda.empty_cache()
+
     # CLACT + VAR at 16:32: masked dense tensor-core GEMM
     W = synth.prefill_clact_weight().to(dev)
     x = synth.prefill_clact_batch(0).to(dev)
@@ -704,6 +733,13 @@ def run_case(args):
             fn = lambda: sl.as_linear_prefill_fp8(x8, meta8, xs, Wq, ws, y)  # noqa: E731
         else:
             fn = lambda: sl.as_select_sqrelu24_fp8(z, x8, meta8, xs)  # noqa: E731
+    elif args.case == "hybrid":
+        _, x, W, _ = synth.prefill_sqrelu_hot(T=args.T)
+        L = SparseLinear(W.to(dev), sl.config(sel=sl.AS_SEL_NM, n=2, m=4), keep_wt=False)
+        xd = x.to(dev)
+        bufs = L.select_buffers(args.T)
+        L.select(xd, bufs)
+        fn = lambda: L.prefill_hybrid_from(xd, bufs, 192)  # noqa: E731
     elif args.case in ("sqrelu24", "dense"):
         _, x, W = synth.prefill_sqrelu(T=args.T)
         cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4) if args.case == "sqrelu24" else \
@@ -751,7 +787,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--case", default=None,
-                    help="profiling case: decode | sqrelu24 | sqrelu24_fp8 | sqrelu24_fp8_producer | dense | select24 | selectclact | block")
+                    help="profiling case: decode | sqrelu24 | sqrelu24_fp8 | sqrelu24_fp8_producer | hybrid | dense | select24 | selectclact | block")
     ap.add_argument("--T", type=int, default=1)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()

@@ -279,6 +279,38 @@ size_t as_workspace_size(int op, int T, int K, int n_out, const as_config *cfg);
 int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cfg);
 
 /* --------------------------------------------------------------------------
+ * Hybrid 2:4 prefill ([SQR] 3.2: the densest features are computed densely
+ * and the rest with 2:4; [SQR] 3.3: the layer's sparsity picks the mode,
+ * above 95 %: pure 2:4, 90-95 %: the split, below 90 %: dense).  Features
+ * are 4-channel blocks.  The dense set D is the n_dense blocks with the most
+ * nonzeros of x over the T tokens, ties to the lower block index; the result
+ * is the masked product with D's blocks kept whole and 2:4 elsewhere:
+ *   y = (x (.) m) W^T + (x (.) (1 - m))[:, D] W[:, D]^T,
+ * m the 2:4 magnitude selection of x.  The second term is a dense tcgen05
+ * GEMM over the 4*n_dense gathered channels (float32) that the 2:4 GEMM adds
+ * in its epilogue.
+ *   sel      the as_select outputs of x with sel = AS_SEL_NM, n = 2, m = 4,
+ *            score AS_SCORE_MAG, no token shift or VAR: bitmask, x_compact
+ *            and meta24 are required.
+ *   x, W     bf16 [T, K] (the same x) and [n_out, K]; K % 64 == 0,
+ *            K <= 32768, n_out % 8 == 0, T < 2^22.
+ *   n_dense  0 <= n_dense <= K/4, a multiple of 16 (0: pure 2:4).
+ *   y        [T, n_out] in out_dtype.
+ *   dense_idx [n_dense] int32 (optional): D in ascending block order.
+ *   sparsity [1] float32 (optional): 1 - nnz(x) / (T*K).
+ * Workspace: as_hybrid_workspace(T, K, n_out, n_dense) bytes, no zero-fill
+ * needed.  as_block_sparsity runs only the counting (and, with n_dense > 0,
+ * the choice of D) for the mode decision; its workspace is
+ * as_hybrid_workspace(T, K, 0, 0).
+ * ------------------------------------------------------------------------ */
+size_t as_hybrid_workspace(int T, int K, int n_out, int n_dense);
+as_status as_linear_prefill_hybrid(const as_select_out *sel, const void *x, int T, int K, const void *W, int n_out,
+                                   int n_dense, as_dtype out_dtype, void *y, int32_t *dense_idx, float *sparsity,
+                                   void *workspace, size_t ws_bytes, cudaStream_t stream);
+as_status as_block_sparsity(const void *x, int T, int K, int n_dense, int32_t *dense_idx, float *sparsity,
+                            void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
  * R-Sparse low-rank compensation of a decode call ([OVW] 3.3).  The weight
  * is approximated as W ~ W_sparse + A_r B_r^T with A_r = U_r diag(S_r)
  * [n_out, r] and B_r = V_r [K, r] from a truncated SVD of W (computed

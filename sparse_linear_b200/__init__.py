@@ -40,7 +40,8 @@ EXPORTS = [
     "as_workspace_size", "as_meta24_words", "as_stream_status", "as_status_string",
     "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches", "as_probe_timeout",
     "as_weight_prep_amber", "as_meta8_words", "as_weight_quant_fp8", "as_select_sqrelu24_fp8",
-    "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode",
+    "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode", "as_hybrid_workspace",
+    "as_linear_prefill_hybrid", "as_block_sparsity",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -65,6 +66,10 @@ _sig = {
     "as_weight_prep_amber": ([_P, _I, _I, _I, _F, ctypes.c_double, ctypes.c_double, _P, _P, _P, _S, _P], _I),
     "as_meta8_words": ([_I, _I], _S),
     "as_rsparse_workspace": ([_I, _I, _I], _S),
+    "as_hybrid_workspace": ([_I, _I, _I, _I], _S),
+    "as_linear_prefill_hybrid": ([ctypes.POINTER(as_select_out), _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, _S,
+                                  _P], _I),
+    "as_block_sparsity": ([_P, _I, _I, _I, _P, _P, _P, _S, _P], _I),
     "as_rsparse_decode": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P], _I),
     "as_weight_quant_fp8": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "as_select_sqrelu24_fp8": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
@@ -182,6 +187,31 @@ def as_weight_prep_amber(W, g, alpha: float = 1.0, lo_pct: float = 0.5, hi_pct: 
     _check(_lib.as_weight_prep_amber(_ptr(W), _dt(W), n_out, K, float(alpha), float(lo_pct), float(hi_pct),
                                      _ptr(g), _ptr(bounds), _ptr(workspace), ws_bytes, _stream(stream)),
            "as_weight_prep_amber")
+
+
+def as_hybrid_workspace(T: int, K: int, n_out: int, n_dense: int) -> int:
+    n = _lib.as_hybrid_workspace(T, K, n_out, n_dense)
+    if n == ctypes.c_size_t(-1).value:
+        raise ASError(AS_ERR_SHAPE, "as_hybrid_workspace")
+    return n
+
+
+def as_linear_prefill_hybrid(out: as_select_out, x, W, y, n_dense: int, dense_idx=None, sparsity=None,
+                             workspace=None, stream=None) -> None:
+    T, K = x.shape
+    n_out = W.shape[0]
+    odt = AS_BF16 if y.dtype == torch.bfloat16 else AS_F32
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_linear_prefill_hybrid(ctypes.byref(out), _ptr(x), T, K, _ptr(W), n_out, int(n_dense), odt,
+                                         _ptr(y), _ptr(dense_idx), _ptr(sparsity), _ptr(workspace), ws_bytes,
+                                         _stream(stream)), "as_linear_prefill_hybrid")
+
+
+def as_block_sparsity(x, sparsity, n_dense: int = 0, dense_idx=None, workspace=None, stream=None) -> None:
+    T, K = x.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_block_sparsity(_ptr(x), T, K, int(n_dense), _ptr(dense_idx), _ptr(sparsity), _ptr(workspace),
+                                  ws_bytes, _stream(stream)), "as_block_sparsity")
 
 
 def as_rsparse_workspace(T: int, K: int, r: int) -> int:

@@ -144,6 +144,63 @@ as_status as_weight_prep_amber(const void *W, as_dtype dt, int n_out, int K, flo
     return cuda_status(launch_amber(W, dt == AS_BF16, n_out, K, alpha, r_lo, r_hi, g, bounds, workspace, stream));
 }
 
+static as_status hybrid_shape(int T, int K, int n_out, int n_dense)
+{
+    if (T <= 0 || K <= 0 || n_out < 0) return AS_ERR_INVALID_ARG;
+    if (K % 64 != 0 || K > 32768 || n_out % 8 != 0) return AS_ERR_SHAPE;
+    if (T >= (1 << 22)) return AS_ERR_SHAPE;  // block counts (4 per token) stay below 2^24
+    if (n_dense < 0 || n_dense > K / 4 || n_dense % 16 != 0) return AS_ERR_SHAPE;
+    return AS_OK;
+}
+
+size_t as_hybrid_workspace(int T, int K, int n_out, int n_dense)
+{
+    if (hybrid_shape(T, K, n_out, n_dense) != AS_OK) return (size_t)-1;
+    return hybrid_layout(T, K, n_out, n_dense).bytes;
+}
+
+as_status as_block_sparsity(const void *x, int T, int K, int n_dense, int32_t *dense_idx, float *sparsity,
+                            void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!x || !sparsity || (n_dense > 0 && !dense_idx)) return AS_ERR_INVALID_ARG;
+    as_status st = hybrid_shape(T, K, 0, n_dense);
+    if (st != AS_OK) return st;
+    if (!aligned16(x) || !aligned16(workspace)) return AS_ERR_ALIGN;
+    if (!workspace || ws_bytes < hybrid_layout(T, K, 0, 0).bytes) return AS_ERR_WORKSPACE;
+    return cuda_status(launch_block_sparsity(x, T, K, n_dense, dense_idx, sparsity, workspace, stream));
+}
+
+as_status as_linear_prefill_hybrid(const as_select_out *sel, const void *x, int T, int K, const void *W, int n_out,
+                                   int n_dense, as_dtype out_dtype, void *y, int32_t *dense_idx, float *sparsity,
+                                   void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!sel || !x || !W || !y || !sel->bitmask || !sel->x_compact || !sel->meta24) return AS_ERR_INVALID_ARG;
+    if (n_out <= 0) return AS_ERR_INVALID_ARG;
+    as_status st = hybrid_shape(T, K, n_out, n_dense);
+    if (st != AS_OK) return st;
+    if (out_dtype != AS_F32 && out_dtype != AS_BF16) return AS_ERR_DTYPE;
+    for (const void *q : {x, W, (const void *)y, (const void *)sel->bitmask, (const void *)sel->x_compact,
+                          (const void *)sel->meta24, (const void *)workspace})
+        if (!aligned16(q)) return AS_ERR_ALIGN;
+    if (!workspace || ws_bytes < hybrid_layout(T, K, n_out, n_dense).bytes) return AS_ERR_WORKSPACE;
+    HybridArgs a{};
+    a.x = x;
+    a.bitmask = sel->bitmask;
+    a.x_compact = sel->x_compact;
+    a.meta24 = sel->meta24;
+    a.W = W;
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.n_dense = n_dense;
+    a.y = y;
+    a.out_bf16 = out_dtype == AS_BF16;
+    a.idx_out = dense_idx;
+    a.sparsity_out = sparsity;
+    a.workspace = workspace;
+    return cuda_status(launch_hybrid(a, stream));
+}
+
 static bool rsparse_rank_ok(int r) { return r == 32 || r == 64 || r == 128; }
 
 size_t as_rsparse_workspace(int T, int K, int r)

@@ -6,5 +6,6 @@
 #include "gemm.cu"
 #include "fp8.cu"
 #include "rsparse.cu"
+#include "hybrid.cu"
 #include "abi.cu"
 #include "noalloc.cu"

@@ -81,6 +81,7 @@ struct GemmArgs {
     const float *rowsum, *eta, *nu;  // epilogue terms (optional)
     void *y;
     int out_bf16;
+    const float *addend = nullptr;  // float32 [T, n_out] added to the accumulator (2:4 only)
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 
@@ -108,6 +109,27 @@ struct RsparseArgs {
     float *y;               // [T, n_out], in/out
     void *workspace;
 };
+// Hybrid 2:4 prefill (hybrid.cu).
+struct HybridArgs {
+    const void *x;            // bf16 [T, K]
+    const uint32_t *bitmask;  // 2:4 selection of x, [T, ceil(K/32)]
+    const void *x_compact;    // its kept values
+    const uint32_t *meta24;   // and positions
+    const void *W;            // bf16 [n_out, K]
+    int T, K, n_out, n_dense;
+    void *y;
+    int out_bf16;
+    int *idx_out;             // [n_dense] or NULL
+    float *sparsity_out;      // [1] or NULL
+    void *workspace;
+};
+struct HybridLayout {
+    size_t nnz, total, idx, xr, wd, yd, bytes;
+};
+HybridLayout hybrid_layout(int T, int K, int n_out, int n_dense);
+cudaError_t launch_block_sparsity(const void *x, int T, int K, int n_dense, int *idx, float *sparsity, void *ws,
+                                  cudaStream_t st);
+cudaError_t launch_hybrid(const HybridArgs &a, cudaStream_t st);
 size_t rsparse_workspace(int T, int K, int r);
 cudaError_t launch_rsparse(const RsparseArgs &a, cudaStream_t st);
 int meta8_kt(int K);

@@ -10,8 +10,9 @@ from __future__ import annotations
 import torch
 
 from . import (AS_BF16, AS_F32, AS_OP_AMBER, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_SELECT,
-               AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SEL_NM, as_linear_decode, as_linear_prefill,
-               as_meta24_words, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size,
+               AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SCORE_MAG, AS_SEL_ALL, AS_SEL_NM, as_block_sparsity,
+               as_hybrid_workspace, as_linear_decode, as_linear_prefill, as_linear_prefill_hybrid,
+               as_meta24_words, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size, config,
                select_out)
 
 
@@ -109,6 +110,59 @@ class SparseLinear:
                           self.W, T, self.cfg, y, rowsum=self.rowsum, eta=bufs.get("eta"),
                           nu=bufs.get("nu"), workspace=self._workspace(AS_OP_PREFILL, T), stream=stream)
         return y
+
+    # ---------------------------------------------------------------- hybrid 2:4
+    def prefill_hybrid_from(self, x: torch.Tensor, bufs: dict, n_dense: int, y: torch.Tensor | None = None,
+                            dense_idx=None, sparsity=None, stream=None) -> torch.Tensor:
+        """The split of the 2:4 + Squared-ReLU page (section 3.2): the n_dense
+        busiest 4-channel blocks dense, 2:4 elsewhere.  `bufs` holds this
+        layer's 2:4 selection of x (cfg: 2:4 by magnitude)."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=x.device)
+        key = ("hybrid", T, n_dense)
+        if key not in self._ws:
+            self._ws[key] = workspace(as_hybrid_workspace(T, self.K, self.n_out, n_dense), x.device)
+        sel = select_out(**{k: v for k, v in bufs.items() if k in ("bitmask", "x_compact", "meta24")})
+        as_linear_prefill_hybrid(sel, x, self.W, y, n_dense, dense_idx=dense_idx, sparsity=sparsity,
+                                 workspace=self._ws[key], stream=stream)
+        return y
+
+    def prefill_auto(self, x: torch.Tensor, dense_frac: float = 0.05, stream=None):
+        """Mode chosen by the measured sparsity of x (2:4 + Squared-ReLU page,
+        section 3.3): above 95 % pure 2:4, 90-95 % the split with the
+        ceil(dense_frac * K/4 / 16) * 16 busiest blocks dense, below 90 %
+        the dense product.  Reads the sparsity back to the host (one
+        synchronisation).  Returns (y, mode, sparsity)."""
+        if not (self.cfg.sel == AS_SEL_NM and self.cfg.n == 2 and self.cfg.m == 4
+                and self.cfg.score == AS_SCORE_MAG and not self.cfg.dpts and not self.cfg.var):
+            raise ValueError("prefill_auto needs a 2:4 magnitude configuration")
+        T = x.shape[0]
+        key = ("sparsity", T)
+        if key not in self._ws:
+            self._ws[key] = workspace(as_hybrid_workspace(T, self.K, 0, 0), x.device)
+        sp = torch.empty(1, dtype=torch.float32, device=x.device)
+        as_block_sparsity(x, sp, workspace=self._ws[key], stream=stream)
+        s = float(sp.item())
+        if s > 0.95:
+            mode = "2:4"
+        elif s >= 0.90:
+            mode = "split"
+        else:
+            mode = "dense"
+        if mode == "dense":
+            cfg_all = config(sel=AS_SEL_ALL, out_dtype=self.cfg.out_dtype)
+            y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=x.device)
+            as_linear_prefill(select_out(x_masked=x), self.W, T, cfg_all, y,
+                              workspace=self._workspace(AS_OP_PREFILL, T), stream=stream)
+            return y, mode, s
+        bufs = self.select_buffers(T, x.device)
+        self.select(x, bufs, stream=stream)
+        if mode == "2:4":
+            return self.prefill_from(bufs, T, stream=stream), mode, s
+        n_dense = int(-(-dense_frac * (self.K // 4) // 16)) * 16
+        n_dense = max(16, min(n_dense, self.K // 4 // 16 * 16))
+        return self.prefill_hybrid_from(x, bufs, n_dense, stream=stream), mode, s
 
     def prefill(self, x: torch.Tensor, running_var=None, first_batch: bool = False, stream=None):
         bufs = self.select_buffers(x.shape[0], x.device)

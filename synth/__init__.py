@@ -27,6 +27,10 @@ no model weights or datasets are used):
                       W bf16 [4096, 14336] ~ N(0, 0.02^2), seed 3.
 * ``prefill_clact``   x bf16 [8192, 8192] ~ 0.5 * Student-t(3) per batch
                       (8 batches), W bf16 [8192, 8192] ~ N(0, 0.02^2), seed 4.
+* ``prefill_sqrelu_hot`` Squared-ReLU input with feature-dependent sparsity:
+                      a seeded 5% of channels ("hot") have z ~ N(0, 1), the
+                      rest z ~ N(-1.8, 1); x = bf16(fp32(max(0,z))^2), about
+                      94% zeros overall; W bf16 ~ N(0, 0.02^2), seed 6.
 * ``outlier_weight``  W [n_out, k], a two-component mixture: each weight is
                       N(-0.02, 0.01^2) or N(+0.02, 0.01^2) with probability
                       1/2 (a bimodal layer), and a seeded 0.2% of the entries
@@ -41,7 +45,7 @@ import torch
 __all__ = [
     "streams", "to_dtype", "tiny_layer", "decode_downproj", "decode_block",
     "prefill_sqrelu", "prefill_clact_weight", "prefill_clact_batch",
-    "random_layer", "BLOCK_LAYERS", "outlier_weight",
+    "random_layer", "BLOCK_LAYERS", "outlier_weight", "prefill_sqrelu_hot",
 ]
 
 
@@ -187,3 +191,18 @@ def outlier_weight(seed: int = 5, n_out: int = 1024, k: int = 4096, dtype=torch.
         sign = np.where(rs.random(size=n_o) < 0.5, -1.0, 1.0)
         w.reshape(-1)[idx] = sign * rv.uniform(0.5, 1.0, size=n_o)
     return to_dtype(w, dtype)
+
+
+def prefill_sqrelu_hot(T: int = 4096, seed: int = 6, k: int = 14336, n_out: int = 4096, hot_frac: float = 0.05,
+                       mu_cold: float = -1.8, mu_hot: float = 0.0, with_weight: bool = True):
+    """Squared-ReLU activations whose sparsity differs by channel (see the
+    module recipe).  Returns ``(z, x, W, hot_channels)``."""
+    rz, rw, rh = streams(seed, 3)
+    hot = np.sort(rh.choice(k, size=max(1, round(hot_frac * k)), replace=False))
+    mu = np.full(k, mu_cold)
+    mu[hot] = mu_hot
+    z = to_dtype(rz.normal(0.0, 1.0, size=(T, k)) + mu[None, :], torch.bfloat16)
+    zf = z.float()
+    x = (torch.clamp_min(zf, 0.0) * torch.clamp_min(zf, 0.0)).to(torch.bfloat16)
+    w = _normal(rw, (n_out, k), 0.02, torch.bfloat16) if with_weight else None
+    return z, x, w, torch.from_numpy(hot)

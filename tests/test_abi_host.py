@@ -220,3 +220,19 @@ def test_rsparse_validation_launches_nothing(lib):
     assert call(dt=3) == lib.AS_ERR_DTYPE
     assert call(A=fake + 2) == lib.AS_ERR_ALIGN
     assert call(wb=0) == lib.AS_ERR_WORKSPACE
+
+
+def test_hybrid_validation_launches_nothing(lib):
+    fake = 1 << 20
+    assert lib.as_hybrid_workspace(4096, 14336, 4096, 192) > 4096 * 4096 * 4
+    for bad in ((4096, 14300, 4096, 16), (4096, 14336, 4096, 17), (4096, 14336, 4096, 14336 // 4 + 16),
+                (16, 65536, 64, 16), (16, 1024, 60, 16)):
+        with pytest.raises(lib.ASError):
+            lib.as_hybrid_workspace(*bad)
+    sel = lib.select_out(bitmask=None)
+    f = lib._lib.as_linear_prefill_hybrid
+    assert f(ctypes.byref(sel), fake, 16, 1024, fake, 64, 16, lib.AS_BF16, fake, None, None, fake, 1 << 30,
+             None) == lib.AS_ERR_INVALID_ARG  # no 2:4 outputs
+    assert lib._lib.as_block_sparsity(fake, 16, 1000, 0, None, fake, fake, 1 << 20, None) == lib.AS_ERR_SHAPE
+    assert lib._lib.as_block_sparsity(fake, 16, 1024, 16, None, fake, fake, 1 << 20, None) == lib.AS_ERR_INVALID_ARG
+    assert lib._lib.as_block_sparsity(fake, 16, 1024, 0, None, fake, fake, 0, None) == lib.AS_ERR_WORKSPACE

@@ -591,3 +591,80 @@ def test_rsparse_keep_all_adds_nothing(sl):
     sl.as_rsparse_decode(dev(x), full, dev(B), dev(A), y, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(y, y0)
+
+
+# ---------------------------------------------------------------- hybrid 2:4 (sparse/dense split)
+def check_hybrid(sl, T, K, n_out, n_dense, out_dtype, rows=None, seed=91):
+    _, x, W, _ = synth.prefill_sqrelu_hot(T=T, k=K, n_out=n_out, seed=seed)
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, out_dtype=sl.AS_BF16 if out_dtype == torch.bfloat16 else sl.AS_F32)
+    L = layer(sl, W, cfg)
+    xd = dev(x)
+    bufs = L.select_buffers(T)
+    L.select(xd, bufs)
+    idx = torch.full((max(n_dense, 1),), -1, dtype=torch.int32, device="cuda")
+    sp = torch.empty(1, dtype=torch.float32, device="cuda")
+    y = L.prefill_hybrid_from(xd, bufs, n_dense, dense_idx=idx, sparsity=sp)
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    xf, Wf = x.float().numpy(), W.float().numpy()
+    mask_h, idx_ref, s_ref = oracle.hybrid_mask(xf, n_dense)
+    if n_dense:
+        np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref)
+    assert sp.item() == np.float32(s_ref)
+    ref = oracle.linear(xf, mask_h, Wf, rows=rows)
+    got = f32(y) if rows is None else f32(y)[rows]
+    tol = TOL_BF16 if out_dtype == torch.bfloat16 else TOL_F32
+    assert rel_l2(got, ref) <= tol
+    return L, xd, bufs, y
+
+
+@pytest.mark.parametrize("T,K,n_out,n_dense,out", [
+    (256, 1024, 256, 16, torch.bfloat16),     # pair kernels
+    (384, 2048, 264, 32, torch.float32),      # odd number of 128-row tiles: one-SM kernels, ragged n_out
+    (512, 4096, 512, 48, torch.bfloat16),
+])
+def test_hybrid_split(sl, T, K, n_out, n_dense, out):
+    check_hybrid(sl, T, K, n_out, n_dense, out)
+
+
+def test_hybrid_without_dense_blocks_is_the_24_prefill(sl):
+    """n_dense = 0 runs the 2:4 GEMM alone: bitwise the plain 2:4 prefill."""
+    L, xd, bufs, y = check_hybrid(sl, 256, 1024, 256, 0, torch.bfloat16)
+    y0 = L.prefill_from(bufs, 256)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0)
+
+
+def test_hybrid_full_size(sl):
+    """The down-projection shape with hot channels (T 4096, K 14336, n_out
+    4096, 192 dense blocks = 768 channels), sampled rows of every tile."""
+    check_hybrid(sl, 4096, 14336, 4096, 192, torch.bfloat16, rows=np.arange(3, 4096, 67))
+
+
+def test_prefill_auto_modes(sl):
+    """The page's mode rule on three activation mixes: hot channels (~94 %
+    zeros: split), all cold (~96 %: pure 2:4), plain N(-1.2, 1) (~88 %: dense);
+    each result against the oracle for that mode."""
+    from sparse_linear_b200.layer import SparseLinear
+    T, K, n_out = 256, 2048, 256
+    cases = [synth.prefill_sqrelu_hot(T=T, k=K, n_out=n_out, seed=92)[1:3],
+             synth.prefill_sqrelu_hot(T=T, k=K, n_out=n_out, seed=93, hot_frac=0.0005, mu_hot=-1.8)[1:3],
+             synth.prefill_sqrelu(T=T, k=K, n_out=n_out, seed=94)[1:3]]
+    modes = []
+    for x, W in cases:
+        L = SparseLinear(dev(W), sl.config(sel=sl.AS_SEL_NM, n=2, m=4, out_dtype=sl.AS_F32), keep_wt=False)
+        y, mode, s = L.prefill_auto(dev(x))
+        torch.cuda.synchronize()
+        xf, Wf = x.float().numpy(), W.float().numpy()
+        _, total = oracle.block_nnz(xf)
+        s_ref = 1.0 - total / float(T * K)
+        assert s == np.float32(s_ref) and mode == oracle.hybrid_mode(s_ref)
+        if mode == "dense":
+            mask = np.ones_like(xf, np.uint8)
+        elif mode == "2:4":
+            mask = oracle.select_nm(oracle.score(xf), 2, 4)
+        else:
+            mask = oracle.hybrid_mask(xf, 32)[0]   # ceil(0.05 * 512 / 16) * 16 = 32 blocks
+        assert rel_l2(f32(y), oracle.linear(xf, mask, Wf)) <= TOL_F32
+        modes.append(mode)
+    assert modes == ["split", "2:4", "dense"]
