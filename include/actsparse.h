@@ -20,8 +20,11 @@
  *   - Every call is asynchronous and ordered on `stream` (0 = legacy default
  *     stream).  Scratch memory is passed in as `workspace`, sized with
  *     as_workspace_size().  Workspace must be zero-filled once before its
- *     first use; every call leaves it zero-filled again.  Calls that share a
- *     workspace must not run concurrently.
+ *     first use; every call leaves it zero-filled again.  The exceptions
+ *     are as_weight_prep_amber, as_rsparse_decode, as_linear_prefill_hybrid
+ *     and as_block_sparsity: they need no zero-fill and leave their
+ *     workspace in an unspecified state (do not share it with the other
+ *     calls).  Calls that share a workspace must not run concurrently.
  *   - Errors are returned, never raised: arguments are validated on the host
  *     and an invalid call launches nothing.  A kernel that gives up a bounded
  *     wait records AS_ERR_TIMEOUT in a device status word that
