@@ -7,6 +7,8 @@ points.  It performs no arithmetic of its own.
 """
 from __future__ import annotations
 
+import math
+
 import torch
 
 from . import (AS_BF16, AS_F32, AS_OP_AMBER, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_SELECT,
@@ -14,6 +16,26 @@ from . import (AS_BF16, AS_F32, AS_OP_AMBER, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_
                as_hybrid_workspace, as_linear_decode, as_linear_prefill, as_linear_prefill_hybrid,
                as_meta24_words, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size, config,
                select_out)
+
+
+def hybrid_mode(sparsity: float) -> str:
+    """Mode by a layer's measured sparsity (2:4 + Squared-ReLU page, section
+    3.3): above 95 % pure 2:4, 90-95 % the sparse/dense split, below 90 %
+    dense."""
+    if sparsity > 0.95:
+        return "2:4"
+    if sparsity >= 0.90:
+        return "split"
+    return "dense"
+
+
+def dense_blocks_for(K: int, dense_frac: float) -> int:
+    """Dense 4-channel blocks of the split: dense_frac of the K/4 blocks,
+    rounded up to a multiple of 16 (64 channels), at least 16 and at most
+    the whole multiple-of-16 part of K/4."""
+    nb = K // 4
+    n = math.ceil(dense_frac * nb / 16) * 16
+    return max(16, min(n, nb // 16 * 16))
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -144,12 +166,7 @@ class SparseLinear:
         sp = torch.empty(1, dtype=torch.float32, device=x.device)
         as_block_sparsity(x, sp, workspace=self._ws[key], stream=stream)
         s = float(sp.item())
-        if s > 0.95:
-            mode = "2:4"
-        elif s >= 0.90:
-            mode = "split"
-        else:
-            mode = "dense"
+        mode = hybrid_mode(s)
         if mode == "dense":
             cfg_all = config(sel=AS_SEL_ALL, out_dtype=self.cfg.out_dtype)
             y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=x.device)
@@ -160,9 +177,7 @@ class SparseLinear:
         self.select(x, bufs, stream=stream)
         if mode == "2:4":
             return self.prefill_from(bufs, T, stream=stream), mode, s
-        n_dense = int(-(-dense_frac * (self.K // 4) // 16)) * 16
-        n_dense = max(16, min(n_dense, self.K // 4 // 16 * 16))
-        return self.prefill_hybrid_from(x, bufs, n_dense, stream=stream), mode, s
+        return self.prefill_hybrid_from(x, bufs, dense_blocks_for(self.K, dense_frac), stream=stream), mode, s
 
     def prefill(self, x: torch.Tensor, running_var=None, first_batch: bool = False, stream=None):
         bufs = self.select_buffers(x.shape[0], x.device)
@@ -170,4 +185,4 @@ class SparseLinear:
         return self.prefill_from(bufs, x.shape[0], stream=stream), bufs
 
 
-__all__ = ["SparseLinear", "workspace", "AS_F32", "AS_BF16"]
+__all__ = ["SparseLinear", "workspace", "hybrid_mode", "dense_blocks_for", "AS_F32", "AS_BF16"]

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -236,3 +237,22 @@ def test_hybrid_validation_launches_nothing(lib):
     assert lib._lib.as_block_sparsity(fake, 16, 1000, 0, None, fake, fake, 1 << 20, None) == lib.AS_ERR_SHAPE
     assert lib._lib.as_block_sparsity(fake, 16, 1024, 16, None, fake, fake, 1 << 20, None) == lib.AS_ERR_INVALID_ARG
     assert lib._lib.as_block_sparsity(fake, 16, 1024, 0, None, fake, fake, 0, None) == lib.AS_ERR_WORKSPACE
+
+
+def test_hybrid_mode_rule_and_dense_block_count(lib):
+    """The product's mode rule equals the oracle's reading of the page's
+    thresholds; the dense-block count is 5 % of the blocks rounded up to
+    64 channels, within [16, K/4]."""
+    import oracle
+    from sparse_linear_b200.layer import dense_blocks_for, hybrid_mode
+    for s in np.linspace(0.0, 1.0, 2001):
+        assert hybrid_mode(float(s)) == oracle.hybrid_mode(float(s))
+    for s in (0.95, 0.90, 0.9500001, 0.8999999):
+        assert hybrid_mode(s) == oracle.hybrid_mode(s)
+    assert dense_blocks_for(14336, 0.05) == 192      # 179.2 blocks -> 12 x 16
+    assert dense_blocks_for(2048, 0.05) == 32        # 25.6 -> 2 x 16
+    assert dense_blocks_for(256, 0.05) == 16         # at least 16
+    assert dense_blocks_for(1024, 1.0) == 256        # at most K/4
+    for K in range(64, 32769, 64):
+        n = dense_blocks_for(K, 0.05)
+        assert n % 16 == 0 and 16 <= n <= max(16, K // 4 // 16 * 16)
