@@ -296,7 +296,7 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
  *            score AS_SCORE_MAG, no token shift or VAR: bitmask, x_compact
  *            and meta24 are required.
  *   x, W     bf16 [T, K] (the same x) and [n_out, K]; K % 64 == 0,
- *            K <= 32768, n_out % 8 == 0, T < 2^22.
+ *            K <= 32768, n_out % 8 == 0, T + n_out <= 65535.
  *   n_dense  0 <= n_dense <= K/4, a multiple of 16 (0: pure 2:4).
  *   y        [T, n_out] in out_dtype.
  *   dense_idx [n_dense] int32 (optional): D in ascending block order.

@@ -148,7 +148,7 @@ static as_status hybrid_shape(int T, int K, int n_out, int n_dense)
 {
     if (T <= 0 || K <= 0 || n_out < 0) return AS_ERR_INVALID_ARG;
     if (K % 64 != 0 || K > 32768 || n_out % 8 != 0) return AS_ERR_SHAPE;
-    if (T >= (1 << 22)) return AS_ERR_SHAPE;  // block counts (4 per token) stay below 2^24
+    if (T + n_out > 65535) return AS_ERR_SHAPE;  // one gather row per token and weight row (grid y)
     if (n_dense < 0 || n_dense > K / 4 || n_dense % 16 != 0) return AS_ERR_SHAPE;
     return AS_OK;
 }

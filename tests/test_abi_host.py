@@ -227,7 +227,7 @@ def test_hybrid_validation_launches_nothing(lib):
     fake = 1 << 20
     assert lib.as_hybrid_workspace(4096, 14336, 4096, 192) > 4096 * 4096 * 4
     for bad in ((4096, 14300, 4096, 16), (4096, 14336, 4096, 17), (4096, 14336, 4096, 14336 // 4 + 16),
-                (16, 65536, 64, 16), (16, 1024, 60, 16)):
+                (16, 65536, 64, 16), (16, 1024, 60, 16), (60000, 1024, 8192, 16)):
         with pytest.raises(lib.ASError):
             lib.as_hybrid_workspace(*bad)
     sel = lib.select_out(bitmask=None)
