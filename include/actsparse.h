@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define AS_ABI_VERSION 2
+#define AS_ABI_VERSION 3
 #define AS_MAX_DECODE_T 16
 
 typedef enum as_status {
@@ -137,6 +137,15 @@ typedef struct as_select_out {
                             32-channel step): bits [16*((p%16)/8) + 4*((q%16)/4),
                             +4) of that word hold the 4-block's two positions
                             i0 | i1 << 2, i0 < i1.  Padding blocks hold 0x4. */
+    void *x_masked_lo;   /* bf16 x only, [T, K] bf16: bf16(xhat*m - x_masked), the
+                            part of the kept values that rounding to bf16 lost.
+                            With a token shift the kept values xhat = x - eta
+                            are float32 numbers, not bf16 ones; for float32
+                            output as_linear_prefill adds x_masked_lo W^T in a
+                            second pass over K (hi + lo keeps xhat to about
+                            2^-17 relative).  Needs x_masked. */
+    void *x_compact_lo;  /* 2:4 only, bf16 [T, K/2]: the same residual of
+                            x_compact (zeros when no shift).  Needs x_compact. */
 } as_select_out;
 
 /* --------------------------------------------------------------------------
@@ -229,6 +238,12 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out,
  *   W [n_out, K] bf16 (K-major, the PyTorch layout).  Epilogue:
  *   y = nu_t * acc (cfg->var, nu from as_select) or acc + eta_t * rowsum_o
  *   (cfg->dpts), then rounding to the output dtype.
+ *   Residual operand: when sel->x_masked_lo (dense path) or
+ *   sel->x_compact_lo (2:4 path) is given, a second pass over K adds its
+ *   product with the same W blocks (and 2:4 positions) to the accumulator,
+ *   so acc = (hi + lo) W^T.  Use it for float32 output with a token shift
+ *   (twice the tensor-core work); with bf16 output the output's own
+ *   rounding is as large as the kept values' and one pass suffices.
  *   Requires K % 8 == 0 (K % 16 == 0 for 2:4) and n_out % 8 == 0.
  *   Workspace: as_workspace_size(AS_OP_PREFILL, T, K, n_out, cfg) (zero).
  * ------------------------------------------------------------------------ */
@@ -256,7 +271,12 @@ as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int 
  *     exceeds AS_NOALLOC_SCRATCH_BYTES return AS_ERR_WORKSPACE and launch nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  The cached address is
+ *     valid for the life of the device's context: after cudaDeviceReset the
+ *     library's device code is loaded again and the array may move, so do
+ *     not call this entry point again in that process.
+ *   - Every argument is checked before the array is touched: a refused call
+ *     (any error status) enqueues nothing on `stream`.
  *   - All calls share the array and it keeps the last call's contents.  The
  *     part that must start at zero is cleared on `stream` at every call.
  *     Calls whose executions overlap on the GPU (different streams without
@@ -296,7 +316,7 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
  *            score AS_SCORE_MAG, no token shift or VAR: bitmask, x_compact
  *            and meta24 are required.
  *   x, W     bf16 [T, K] (the same x) and [n_out, K]; K % 64 == 0,
- *            K <= 32768, n_out % 8 == 0, T + n_out <= 65535.
+ *            K <= 32768, n_out % 8 == 0, T < 2^22.
  *   n_dense  0 <= n_dense <= K/4, a multiple of 16 (0: pure 2:4).
  *   y        [T, n_out] in out_dtype.
  *   dense_idx [n_dense] int32 (optional): D in ascending block order.
@@ -312,6 +332,23 @@ as_status as_linear_prefill_hybrid(const as_select_out *sel, const void *x, int 
                                    void *workspace, size_t ws_bytes, cudaStream_t stream);
 as_status as_block_sparsity(const void *x, int T, int K, int n_dense, int32_t *dense_idx, float *sparsity,
                             void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* The inference mode switch ([SQR] 3.3), host-only.  The page keys the mode
+ * on the layer's measured activation sparsity (as_block_sparsity's output):
+ * above 95 %: pure 2:4; from 90 % to 95 % (both ends included): the split;
+ * below 90 %: the dense product.  The page's snippet lost its comparison
+ * signs, so the two thresholds themselves are read as "split".  Returns an
+ * as_mode; a NaN sparsity returns AS_MODE_DENSE. */
+typedef enum as_mode { AS_MODE_24 = 0, AS_MODE_SPLIT = 1, AS_MODE_DENSE = 2 } as_mode;
+int as_prefill_mode(double sparsity);
+
+/* Number of dense 4-channel blocks of the split ([SQR] 3.2 keeps about 5 %
+ * of the features dense): dense_frac of the K/4 blocks rounded up to a
+ * multiple of 16 (64 channels, the dense GEMM's K step), at least 16 and at
+ * most the multiple-of-16 part of K/4 (as_linear_prefill_hybrid's bounds).
+ * Host-only; -1 for K not a positive multiple of 64 or dense_frac outside
+ * [0, 1]. */
+int as_hybrid_dense_blocks(int K, double dense_frac);
 
 /* --------------------------------------------------------------------------
  * R-Sparse low-rank compensation of a decode call ([OVW] 3.3).  The weight
@@ -344,9 +381,10 @@ size_t as_meta24_words(int T, int K);
  * a 2:4 GEMM on FP8 operands with row scaling; [SQR] 5.3: sparsify before
  * quantising).  FP8 is E4M3 (largest finite 448, no infinities), converted
  * with round-to-nearest-even and saturation.  Every row carries one float32
- * scale: scale = amax / 448 over the row's (kept) values, 1 for an all-zero
- * row; code = E4M3(fl32(v / scale)); the value a code stands for is
- * E4M3value(code) * scale.
+ * scale: scale = fl32(amax / 448) over the row's (kept) values, 1 for an
+ * all-zero row.  The codes use the reciprocal, one multiply per value:
+ * code = E4M3(fl32(v * r)) with r = fl32(448 / amax) (r = 1 for an all-zero
+ * row); the value a code stands for is E4M3value(code) * scale.
  * ------------------------------------------------------------------------ */
 
 /* Number of 32-bit words of FP8 2:4 positions for T tokens x K channels:

@@ -34,6 +34,7 @@ AS_SEL_NM, AS_SEL_TOPK, AS_SEL_ALL, AS_SEL_THRESH = 0, 1, 2, 3
 AS_PTS_OFF, AS_PTS_DYNAMIC, AS_PTS_STATIC = 0, 1, 2
 AS_OP_WEIGHT_PREP, AS_OP_SELECT, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_AMBER = 0, 1, 2, 3, 4
 AS_MAX_DECODE_T = 16
+AS_MODE_24, AS_MODE_SPLIT, AS_MODE_DENSE = 0, 1, 2
 
 EXPORTS = [
     "as_weight_prep", "as_select", "as_linear_decode", "as_linear_prefill",
@@ -41,7 +42,7 @@ EXPORTS = [
     "as_abi_version", "as_linear_decode_noalloc", "as_decode_launches", "as_probe_timeout",
     "as_weight_prep_amber", "as_meta8_words", "as_weight_quant_fp8", "as_select_sqrelu24_fp8",
     "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode", "as_hybrid_workspace",
-    "as_linear_prefill_hybrid", "as_block_sparsity",
+    "as_linear_prefill_hybrid", "as_block_sparsity", "as_prefill_mode", "as_hybrid_dense_blocks",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -57,7 +58,7 @@ class as_config(ctypes.Structure):
 class as_select_out(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in (
         "bitmask", "eta", "colnorm", "var_dense", "var_kept", "nu", "x_masked",
-        "x_compact", "meta24")]
+        "x_compact", "meta24", "x_masked_lo", "x_compact_lo")]
 
 
 _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -89,6 +90,8 @@ _sig = {
     "as_probe_timeout": ([ctypes.c_uint, _P], _I),
     "as_status_string": ([_I], ctypes.c_char_p),
     "as_abi_version": ([], _I),
+    "as_prefill_mode": ([ctypes.c_double], _I),
+    "as_hybrid_dense_blocks": ([_I, ctypes.c_double], _I),
 }
 for _name, (_args, _res) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -212,6 +215,19 @@ def as_block_sparsity(x, sparsity, n_dense: int = 0, dense_idx=None, workspace=N
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_lib.as_block_sparsity(_ptr(x), T, K, int(n_dense), _ptr(dense_idx), _ptr(sparsity), _ptr(workspace),
                                   ws_bytes, _stream(stream)), "as_block_sparsity")
+
+
+def as_prefill_mode(sparsity: float) -> int:
+    """The mode switch of the 2:4 + Squared-ReLU page (section 3.3), run in
+    the library: AS_MODE_24, AS_MODE_SPLIT or AS_MODE_DENSE."""
+    return _lib.as_prefill_mode(float(sparsity))
+
+
+def as_hybrid_dense_blocks(K: int, dense_frac: float) -> int:
+    n = _lib.as_hybrid_dense_blocks(int(K), float(dense_frac))
+    if n < 0:
+        raise ASError(AS_ERR_SHAPE, "as_hybrid_dense_blocks")
+    return n
 
 
 def as_rsparse_workspace(T: int, K: int, r: int) -> int:

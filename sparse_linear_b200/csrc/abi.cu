@@ -148,7 +148,7 @@ static as_status hybrid_shape(int T, int K, int n_out, int n_dense)
 {
     if (T <= 0 || K <= 0 || n_out < 0) return AS_ERR_INVALID_ARG;
     if (K % 64 != 0 || K > 32768 || n_out % 8 != 0) return AS_ERR_SHAPE;
-    if (T + n_out > 65535) return AS_ERR_SHAPE;  // one gather row per token and weight row (grid y)
+    if (T >= (1 << 22)) return AS_ERR_SHAPE;  // a block's count (<= 4 T) must stay below 2^24
     if (n_dense < 0 || n_dense > K / 4 || n_dense % 16 != 0) return AS_ERR_SHAPE;
     return AS_OK;
 }
@@ -199,6 +199,22 @@ as_status as_linear_prefill_hybrid(const as_select_out *sel, const void *x, int 
     a.sparsity_out = sparsity;
     a.workspace = workspace;
     return cuda_status(launch_hybrid(a, stream));
+}
+
+int as_prefill_mode(double sparsity)
+{
+    if (sparsity > 0.95) return AS_MODE_24;
+    if (sparsity >= 0.90) return AS_MODE_SPLIT;
+    return AS_MODE_DENSE;  // also NaN
+}
+
+int as_hybrid_dense_blocks(int K, double dense_frac)
+{
+    if (K <= 0 || K % 64 != 0 || !(dense_frac >= 0.0 && dense_frac <= 1.0)) return -1;
+    const int nb = K / 4;
+    const int n = (int)ceil(dense_frac * (double)nb / 16.0) * 16;
+    const int hi = nb / 16 * 16;
+    return n < 16 ? 16 : (n > hi ? hi : n);
 }
 
 static bool rsparse_rank_ok(int r) { return r == 32 || r == 64 || r == 128; }
@@ -299,8 +315,11 @@ as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *c
     if (cfg->var && !running_var) return AS_ERR_INVALID_ARG;
     if ((out->x_compact || out->meta24) && (!is24(cfg) || dt != AS_BF16 || K % 16 != 0)) return AS_ERR_UNSUPPORTED;
     if ((out->x_compact == nullptr) != (out->meta24 == nullptr)) return AS_ERR_INVALID_ARG;
+    if ((out->x_masked_lo && (!out->x_masked || dt != AS_BF16)) || (out->x_compact_lo && !out->x_compact))
+        return AS_ERR_INVALID_ARG;
     const void *ptrs[] = {x, chan_factor, running_var, out->bitmask, out->eta, out->colnorm, out->var_dense,
-                          out->var_kept, out->nu, out->x_masked, out->x_compact, out->meta24, workspace};
+                          out->var_kept, out->nu, out->x_masked, out->x_compact, out->meta24, workspace,
+                          out->x_masked_lo, out->x_compact_lo};
     for (const void *p : ptrs)
         if (!aligned16(p)) return AS_ERR_ALIGN;
     if (cfg->sel == AS_SEL_TOPK && cfg->k_keep > 0 && cfg->k_keep < K && (size_t)K * 4 > 200 * 1024)
@@ -344,12 +363,19 @@ as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *c
     a.x_masked = out->x_masked;
     a.x_compact = out->x_compact;
     a.meta24 = out->meta24;
+    a.x_masked_lo = out->x_masked_lo;
+    a.x_compact_lo = out->x_compact_lo;
     return cuda_status(launch_select(a, stream));
 }
 
-as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, const void *Wt, const float *g,
-                           const float *rowsum, const as_config *cfg, void *y, uint32_t *mask_out, float *eta_out,
-                           float *colnorm_out, void *workspace, size_t ws_bytes, cudaStream_t stream)
+}  // extern "C"
+
+// Every check of a decode call except the workspace's (shared with the
+// entry point that takes no workspace, which must refuse a bad call before
+// it touches its scratch).
+as_status decode_check_args(const void *x, as_dtype dt, int T, int K, int n_out, const void *Wt, const float *g,
+                            const float *rowsum, const as_config *cfg, const void *y, const uint32_t *mask_out,
+                            const float *eta_out, const float *colnorm_out)
 {
     if (!x || !Wt || !y) return AS_ERR_INVALID_ARG;
     if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
@@ -360,9 +386,23 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     if (K % 8 != 0 || n_out % 8 != 0) return AS_ERR_SHAPE;
     if (cfg->score == AS_SCORE_WEIGHT && !g) return AS_ERR_INVALID_ARG;
     if (cfg->dpts && !rowsum) return AS_ERR_INVALID_ARG;
-    const void *ptrs[] = {x, Wt, g, rowsum, y, mask_out, eta_out, colnorm_out, workspace};
+    if (cfg->sel == AS_SEL_TOPK && (size_t)K * 4 > 200 * 1024 && cfg->k_keep > 0 && cfg->k_keep < K)
+        return AS_ERR_SHAPE;  // top-k keeps the row's scores in shared memory
+    const void *ptrs[] = {x, Wt, g, rowsum, y, mask_out, eta_out, colnorm_out};
     for (const void *p : ptrs)
         if (!aligned16(p)) return AS_ERR_ALIGN;
+    return AS_OK;
+}
+
+extern "C" {
+
+as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, const void *Wt, const float *g,
+                           const float *rowsum, const as_config *cfg, void *y, uint32_t *mask_out, float *eta_out,
+                           float *colnorm_out, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    as_status st = decode_check_args(x, dt, T, K, n_out, Wt, g, rowsum, cfg, y, mask_out, eta_out, colnorm_out);
+    if (st != AS_OK) return st;
+    if (!aligned16(workspace)) return AS_ERR_ALIGN;
     const int bf16 = dt == AS_BF16;
     const size_t need = decode_ws(T, K, n_out, cfg, bf16);
     if (!workspace || ws_bytes < need) return AS_ERR_WORKSPACE;
@@ -404,8 +444,6 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
         s.f = f;
         s.bitmask = bm;
         s.eta = cfg->dpts ? eta_ws : nullptr;  // the decode kernel reuses the means the selection used
-        if (cfg->sel == AS_SEL_TOPK && (size_t)K * 4 > 200 * 1024 && cfg->k_keep > 0 && cfg->k_keep < K)
-            return AS_ERR_SHAPE;
         const cudaError_t se = (cfg->sel == AS_SEL_NM) ? launch_select_nm_decode(s, stream)
                                                        : launch_select(s, stream, /*wide=*/1);
         if (se != cudaSuccess) return AS_ERR_CUDA;
@@ -455,11 +493,13 @@ as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int 
     if (!sparse && !sel->x_masked) return AS_ERR_INVALID_ARG;
     if (cfg->dpts && (!rowsum || !eta)) return AS_ERR_INVALID_ARG;
     if (cfg->var && !nu) return AS_ERR_INVALID_ARG;
-    const void *ptrs[] = {W, rowsum, eta, nu, y, sel->x_compact, sel->meta24, sel->x_masked};
+    const void *ptrs[] = {W, rowsum, eta, nu, y, sel->x_compact, sel->meta24, sel->x_masked, sel->x_masked_lo,
+                          sel->x_compact_lo};
     for (const void *p : ptrs)
         if (!aligned16(p)) return AS_ERR_ALIGN;
     GemmArgs a{};
     a.A = sparse ? sel->x_compact : sel->x_masked;
+    a.A_lo = sparse ? sel->x_compact_lo : sel->x_masked_lo;
     a.meta = sparse ? sel->meta24 : nullptr;
     a.W = W;
     a.T = T;

@@ -69,6 +69,7 @@ struct GemmParams {
     void *y;
     int T, K, n_out, out_bf16;
     int m_tiles, n_tiles, k_blocks, meta_kt;
+    int kb_pass;  // K blocks of one pass over K; k_blocks = 2 kb_pass when a residual A operand follows
 };
 
 // Adds row `row`, columns col0 .. col0+31 of a float32 [T, n_out] term to 32
@@ -98,7 +99,8 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
 
 template <bool SPARSE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmA2, GemmParams p)
 {
     using C = GemmCfg<SPARSE>;
     constexpr int BN = C::BN, S = C::STAGES;
@@ -131,6 +133,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         fence_mbar_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmA2);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -152,16 +155,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
                     mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + C::M_BYTES);
+                    // second pass over K: the residual operand against the same W blocks
+                    const bool lo = kb >= p.kb_pass;
+                    const int kk = lo ? kb - p.kb_pass : kb;
                     unsigned char *a_dst = sA + stage * C::A_BYTES;
                     unsigned char *b_dst = sB + stage * C::B_BYTES;
-                    tma_load_2d(a_dst, &tmA, &full[stage], kb * 64, mt * GEMM_BM);
+                    tma_load_2d(a_dst, lo ? &tmA2 : &tmA, &full[stage], kk * 64, mt * GEMM_BM);
                     if constexpr (SPARSE) {
-                        tma_load_2d(b_dst, &tmB, &full[stage], kb * 128, nt * BN);
-                        tma_load_2d(b_dst + BN * 128, &tmB, &full[stage], kb * 128 + 64, nt * BN);
-                        const uint32_t *src = p.meta + ((size_t)mt * p.meta_kt + kb) * 512;
+                        tma_load_2d(b_dst, &tmB, &full[stage], kk * 128, nt * BN);
+                        tma_load_2d(b_dst + BN * 128, &tmB, &full[stage], kk * 128 + 64, nt * BN);
+                        const uint32_t *src = p.meta + ((size_t)mt * p.meta_kt + kk) * 512;
                         bulk_load(sM + stage * C::M_BYTES, src, C::M_BYTES, &full[stage]);
                     } else {
-                        tma_load_2d(b_dst, &tmB, &full[stage], kb * 64, nt * BN);
+                        tma_load_2d(b_dst, &tmB, &full[stage], kk * 64, nt * BN);
                     }
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
@@ -340,7 +346,7 @@ constexpr size_t pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PairCfg
 template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     k_gemm_sp_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmE, GemmParams p)
+                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmA2, GemmParams p)
 {
     using C = PairCfg<FP8>;
     constexpr int S = PAIR_STAGES;
@@ -376,6 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmE);
+        prefetch_tensormap(&tmA2);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, 512);
@@ -401,14 +408,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
                     const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
+                    // second pass over K: the residual operand, same positions and W blocks
+                    const bool lo = kb >= p.kb_pass;
+                    const int kk = lo ? kb - p.kb_pass : kb;
                     unsigned char *b_dst = sB + stage * PAIR_B_BYTES;
-                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, &tmA, bar, kb * C::KA, arow);
-                    tma_load_2d_pair(b_dst, &tmB, bar, kb * C::KB, brow);
-                    tma_load_2d_pair(b_dst + 128 * 128, &tmB, bar, kb * C::KB + C::BSUB, brow);
-                    tma_load_2d_pair(sM + stage * PAIR_M_BYTES, &tmE, bar, 0, (echunk + kb) * (PAIR_M_BYTES / 256));
+                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, lo ? &tmA2 : &tmA, bar, kk * C::KA, arow);
+                    tma_load_2d_pair(b_dst, &tmB, bar, kk * C::KB, brow);
+                    tma_load_2d_pair(b_dst + 128 * 128, &tmB, bar, kk * C::KB + C::BSUB, brow);
+                    tma_load_2d_pair(sM + stage * PAIR_M_BYTES, &tmE, bar, 0, (echunk + kk) * (PAIR_M_BYTES / 256));
                     if constexpr (FP8)
                         tma_load_2d_pair(sM + stage * PAIR_M_BYTES + 2048, &tmE, bar, 0,
-                                         (echunk + kb) * (PAIR_M_BYTES / 256) + 8);
+                                         (echunk + kk) * (PAIR_M_BYTES / 256) + 8);
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
@@ -557,7 +567,8 @@ constexpr int DP_STAGE_BYTES = DP_A_BYTES + DP_B_BYTES;
 constexpr size_t dense_pair_smem_bytes() { return 1024 + (size_t)DP_STAGES * DP_STAGE_BYTES + 256; }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
-    k_gemm_dense_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p)
+    k_gemm_dense_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmA2, GemmParams p)
 {
     constexpr int S = DP_STAGES;
     extern __shared__ unsigned char smem_raw[];
@@ -590,6 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
         fence_mbar_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmA2);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, 512);
@@ -614,8 +626,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * DP_STAGE_BYTES);
                     const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
-                    tma_load_2d_pair(sA + stage * DP_A_BYTES, &tmA, bar, kb * 64, arow);
-                    tma_load_2d_pair(sB + stage * DP_B_BYTES, &tmB, bar, kb * 64, brow);
+                    // second pass over K: the residual operand against the same W blocks
+                    const bool lo = kb >= p.kb_pass;
+                    const int kk = lo ? kb - p.kb_pass : kb;
+                    tma_load_2d_pair(sA + stage * DP_A_BYTES, lo ? &tmA2 : &tmA, bar, kk * 64, arow);
+                    tma_load_2d_pair(sB + stage * DP_B_BYTES, &tmB, bar, kk * 64, brow);
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
@@ -806,10 +821,11 @@ template <bool SPARSE>
 static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
 {
     using C = GemmCfg<SPARSE>;
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mA2;
     const uint64_t ka = SPARSE ? (uint64_t)a.K / 2 : (uint64_t)a.K;
     if (!make_map(&mA, a.A, (uint64_t)a.T, ka, GEMM_BM)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, C::BN)) return cudaErrorInvalidValue;
+    if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, ka, GEMM_BM)) return cudaErrorInvalidValue;
     GemmParams p{};
     p.meta = a.meta;
     p.rowsum = a.rowsum;
@@ -823,14 +839,15 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     p.out_bf16 = a.out_bf16;
     p.m_tiles = (a.T + GEMM_BM - 1) / GEMM_BM;
     p.n_tiles = (a.n_out + C::BN - 1) / C::BN;
-    p.k_blocks = (a.K + C::KB - 1) / C::KB;
+    p.kb_pass = (a.K + C::KB - 1) / C::KB;
+    p.k_blocks = p.kb_pass * (a.A_lo ? 2 : 1);
     p.meta_kt = (a.K + 127) / 128;
     const size_t smem = gemm_smem_bytes<SPARSE>();
     cudaError_t e = cudaFuncSetAttribute(k_gemm<SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = std::min(tiles, sm_count());
-    k_gemm<SPARSE><<<grid, GEMM_THREADS, smem, st>>>(mA, mB, p);
+    k_gemm<SPARSE><<<grid, GEMM_THREADS, smem, st>>>(mA, mB, mA2, p);
     return cudaGetLastError();
 }
 
@@ -891,7 +908,7 @@ static bool use_pair(const GemmArgs &a)
 
 static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
 {
-    CUtensorMap mA, mB, mE;
+    CUtensorMap mA, mB, mE, mA2;
     const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
     GemmParams p{};
     p.meta = a.meta;
@@ -906,9 +923,11 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     p.out_bf16 = a.out_bf16;
     p.m_tiles = mt128 / 2;
     p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
-    p.k_blocks = (a.K + 127) / 128;
+    p.kb_pass = (a.K + 127) / 128;
+    p.k_blocks = p.kb_pass * (a.A_lo ? 2 : 1);
     p.meta_kt = (a.K + 127) / 128;
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map_meta(&mE, a.meta, (uint64_t)mt128 * p.meta_kt)) return cudaErrorInvalidValue;
     const size_t smem = pair_smem_bytes<false>();
@@ -918,13 +937,13 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_sp_pair<false><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, p);
+    k_gemm_sp_pair<false><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, mA2, p);
     return cudaGetLastError();
 }
 
 static cudaError_t launch_gemm_dense_pair(const GemmArgs &a, cudaStream_t st)
 {
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mA2;
     const int mt128 = (a.T + GEMM_BM - 1) / GEMM_BM;
     GemmParams p{};
     p.rowsum = a.rowsum;
@@ -937,15 +956,17 @@ static cudaError_t launch_gemm_dense_pair(const GemmArgs &a, cudaStream_t st)
     p.out_bf16 = a.out_bf16;
     p.m_tiles = mt128 / 2;
     p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
-    p.k_blocks = (a.K + 63) / 64;
+    p.kb_pass = (a.K + 63) / 64;
+    p.k_blocks = p.kb_pass * (a.A_lo ? 2 : 1);
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     const size_t smem = dense_pair_smem_bytes();
     const int clusters = dense_pair_clusters(smem);
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_dense_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, p);
+    k_gemm_dense_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mA2, p);
     return cudaGetLastError();
 }
 
@@ -967,6 +988,7 @@ cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st)
     p.m_tiles = (mt128 + 1) / 2;
     p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
     p.k_blocks = (a.K + 255) / 256;
+    p.kb_pass = p.k_blocks;
     p.meta_kt = p.k_blocks;
     if (!make_map_u8(&mA, a.x8, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map_u8(&mB, a.Wq, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
@@ -978,7 +1000,7 @@ cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st)
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_sp_pair<true><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, p);
+    k_gemm_sp_pair<true><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, mA, p);
     return cudaGetLastError();
 }
 

@@ -169,7 +169,11 @@ __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *
 }
 
 // Rows 0..T-1: the dropped values of the dense blocks; rows T..T+n_out-1:
-// the weight columns of the dense blocks.  One thread per (row, block).
+// the weight columns of the dense blocks.  One thread per (row, block); the
+// rows are strided over gridDim.y (at most HY_GATHER_ROWS CTAs), so any
+// T + n_out fits the launch.
+constexpr int HY_GATHER_ROWS = 16384;
+
 __global__ void __launch_bounds__(HY_THREADS) k_gather_dense(const __nv_bfloat16 *__restrict__ x,
                                                              const uint32_t *__restrict__ bitmask,
                                                              const __nv_bfloat16 *__restrict__ W, int T, int K,
@@ -178,22 +182,24 @@ __global__ void __launch_bounds__(HY_THREADS) k_gather_dense(const __nv_bfloat16
                                                              __nv_bfloat16 *__restrict__ wd)
 {
     const int q = blockIdx.x * HY_THREADS + threadIdx.x;
-    const int row = blockIdx.y;
     if (q >= n_dense) return;
     const int b = idx[q];
-    if (row < T) {
-        uint2 v = *reinterpret_cast<const uint2 *>(x + (size_t)row * K + 4 * b);
-        const uint32_t m = (bitmask[(size_t)row * ((K + 31) / 32) + (b >> 3)] >> (4 * (b & 7))) & 15u;
-        // keep the dropped values (mask bit clear), zero the kept ones
-        if (m & 1u) v.x &= 0xffff0000u;
-        if (m & 2u) v.x &= 0x0000ffffu;
-        if (m & 4u) v.y &= 0xffff0000u;
-        if (m & 8u) v.y &= 0x0000ffffu;
-        *reinterpret_cast<uint2 *>(xr + (size_t)row * (4 * n_dense) + 4 * q) = v;
-    } else {
-        const int o = row - T;
-        *reinterpret_cast<uint2 *>(wd + (size_t)o * (4 * n_dense) + 4 * q) =
-            *reinterpret_cast<const uint2 *>(W + (size_t)o * K + 4 * b);
+    const long long rows = (long long)T + n_out;
+    for (long long r = blockIdx.y; r < rows; r += gridDim.y) {
+        if (r < T) {
+            uint2 v = *reinterpret_cast<const uint2 *>(x + (size_t)r * K + 4 * b);
+            const uint32_t m = (bitmask[(size_t)r * ((K + 31) / 32) + (b >> 3)] >> (4 * (b & 7))) & 15u;
+            // keep the dropped values (mask bit clear), zero the kept ones
+            if (m & 1u) v.x &= 0xffff0000u;
+            if (m & 2u) v.x &= 0x0000ffffu;
+            if (m & 4u) v.y &= 0xffff0000u;
+            if (m & 8u) v.y &= 0x0000ffffu;
+            *reinterpret_cast<uint2 *>(xr + (size_t)r * (4 * n_dense) + 4 * q) = v;
+        } else {
+            const size_t o = (size_t)(r - T);
+            *reinterpret_cast<uint2 *>(wd + o * (4 * n_dense) + 4 * q) =
+                *reinterpret_cast<const uint2 *>(W + o * K + 4 * b);
+        }
     }
 }
 
@@ -240,7 +246,8 @@ cudaError_t launch_hybrid(const HybridArgs &a, cudaStream_t st)
         __nv_bfloat16 *xr = reinterpret_cast<__nv_bfloat16 *>(base + L.xr);
         __nv_bfloat16 *wd = reinterpret_cast<__nv_bfloat16 *>(base + L.wd);
         float *yd = reinterpret_cast<float *>(base + L.yd);
-        dim3 g((a.n_dense + HY_THREADS - 1) / HY_THREADS, a.T + a.n_out);
+        const long long rows = (long long)a.T + a.n_out;
+        dim3 g((a.n_dense + HY_THREADS - 1) / HY_THREADS, (unsigned)(rows < HY_GATHER_ROWS ? rows : HY_GATHER_ROWS));
         k_gather_dense<<<g, HY_THREADS, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.x), a.bitmask,
                                                  static_cast<const __nv_bfloat16 *>(a.W), a.T, a.K, a.n_out, idx,
                                                  a.n_dense, xr, wd);

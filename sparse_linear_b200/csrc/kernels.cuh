@@ -32,6 +32,8 @@ struct SelectArgs {
     void *x_masked;
     void *x_compact;
     uint32_t *meta24;
+    void *x_masked_lo;   // bf16 residuals of x_masked (float32-output GEMM operand), or nullptr
+    void *x_compact_lo;  // bf16 residuals of x_compact, or nullptr
 };
 // CLACT column energy c_j = sqrt(sum_t x_tj^2), float64 partials in ws.
 size_t colnorm_workspace(int T, int K);
@@ -74,6 +76,7 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &p, cudaStream_t
 // ------------------------------------------------------------ prefill GEMM
 struct GemmArgs {
     const void *A;        // bf16 [T, Ka] K-major (x_masked, x or x_compact)
+    const void *A_lo = nullptr;  // bf16 residual of A (same layout): a second pass over K adds A_lo W^T
     const uint32_t *meta; // 2:4 metadata (sparse only)
     const void *W;        // bf16 [n_out, K] K-major
     int T, K, n_out;

@@ -14,7 +14,10 @@
 // array is only a host-side handle, not a device address, so the device
 // address is fetched once per device with cudaGetSymbolAddress (with that
 // device current) and cached; the first call on each device does this
-// set-up, so it should be made before any stream capture.  All calls share
+// set-up, so it should be made before any stream capture.  The cached
+// address belongs to the device's context: after cudaDeviceReset the
+// module is loaded again and the array may move, so this entry point must
+// not be called again in that process.  All calls share
 // the array and it keeps the last call's contents: the part that must start
 // at zero (the arrival counters) is cleared on the stream at every call, and
 // calls whose executions overlap on the GPU race on the array.
@@ -56,13 +59,15 @@ extern "C" as_status as_linear_decode_noalloc(const void *x, as_dtype dt, int T,
                                               uint32_t *mask_out, float *eta_out, float *colnorm_out,
                                               cudaStream_t stream)
 {
+    // every argument is checked before the shared scratch is touched: a
+    // refused call enqueues nothing on the stream
+    as_status st = decode_check_args(x, dt, T, K, n_out, Wt, g, rowsum, cfg, y, mask_out, eta_out, colnorm_out);
+    if (st != AS_OK) return st;
     const size_t need = as_workspace_size(AS_OP_DECODE, T, K, n_out, cfg);
-    if (need == (size_t)-1)  // invalid shape or config: the regular validation reports which
-        return as_linear_decode(x, dt, T, K, n_out, Wt, g, rowsum, cfg, y, mask_out, eta_out, colnorm_out,
-                                nullptr, 0, stream);
+    if (need == (size_t)-1) return AS_ERR_SHAPE;
     if (need > (size_t)AS_NOALLOC_SCRATCH_BYTES) return AS_ERR_WORKSPACE;
     void *scratch = nullptr;
-    as_status st = noalloc_scratch(&scratch);
+    st = noalloc_scratch(&scratch);
     if (st != AS_OK) return st;
     // the arrival counters lead the scratch layout and must start at zero
     const as::DecodePlan plan = as::decode_plan(T, K, n_out, dt == AS_BF16);

@@ -107,6 +107,32 @@ __device__ __forceinline__ void store8<float>(float *p, const float (&v)[8])
     *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// Residuals of rounding 8 float32 values to bf16: lo = bf16(v - bf16(v)).
+// hi + lo keeps v to about 2^-17 relative, which the float32-output GEMM
+// needs when the kept values were shifted (D-PTS / S-PTS) and so are no
+// longer bf16 numbers.
+__device__ __forceinline__ void store8_lo(__nv_bfloat16 *p, const float (&v)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(v[2 * i] - __low2float(h), v[2 * i + 1] - __high2float(h));
+        w[i] = *reinterpret_cast<const uint32_t *>(&l);
+    }
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The same for 4 values (two 2:4 blocks of the compact operand).
+__device__ __forceinline__ uint2 lo4(const float (&cv)[4])
+{
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(cv[0], cv[1]);
+    const __nv_bfloat162 h1 = __floats2bfloat162_rn(cv[2], cv[3]);
+    const __nv_bfloat162 l0 = __floats2bfloat162_rn(cv[0] - __low2float(h0), cv[1] - __high2float(h0));
+    const __nv_bfloat162 l1 = __floats2bfloat162_rn(cv[2] - __low2float(h1), cv[3] - __high2float(h1));
+    return make_uint2(*reinterpret_cast<const uint32_t *>(&l0), *reinterpret_cast<const uint32_t *>(&l1));
+}
+
 // NT threads per token row: 256 for prefill batches, 1024 for the few rows
 // of a decode call (fewer rounds of loads per row).
 template <typename TX, int NT>
@@ -290,6 +316,7 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
                     }
                 }
                 if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
+                if (a.x_masked_lo) store8_lo(static_cast<__nv_bfloat16 *>(a.x_masked_lo) + (size_t)t * K + c0, km);
                 if (a.x_compact) {
                     // two 4-blocks per thread, two kept values each (exactly 2:4)
                     float cv[4];
@@ -307,6 +334,9 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
                     __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
                     uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1));
                     *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) = pk;
+                    if (a.x_compact_lo)
+                        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
+                                                   c0 / 2) = lo4(cv);
                     if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
                 }
             }  // act
@@ -472,6 +502,9 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                     }
                     *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) =
                         make_uint4(out[0], out[1], out[2], out[3]);
+                    if (a.x_compact_lo)  // unshifted bf16 values: nothing is lost in rounding
+                        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
+                                                   c0 / 2) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint16_t *>(m16 + tile * mst16) = (uint16_t)metab;
                 }
             }
@@ -516,6 +549,8 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                         }
                     }
                     if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
+                    if (a.x_masked_lo)
+                        store8_lo(static_cast<__nv_bfloat16 *>(a.x_masked_lo) + (size_t)t * K + c0, km);
                 }
                 if constexpr (COMPACT) {
                     float cv[4];
@@ -532,6 +567,9 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                     const __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
                     *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) + c0 / 2) =
                         make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
+                    if (a.x_compact_lo)
+                        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
+                                                   c0 / 2) = lo4(cv);
                     mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
                 }
             }

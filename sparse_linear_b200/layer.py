@@ -7,35 +7,27 @@ points.  It performs no arithmetic of its own.
 """
 from __future__ import annotations
 
-import math
-
 import torch
 
-from . import (AS_BF16, AS_F32, AS_OP_AMBER, AS_OP_DECODE, AS_OP_PREFILL, AS_OP_SELECT,
-               AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SCORE_MAG, AS_SEL_ALL, AS_SEL_NM, as_block_sparsity,
-               as_hybrid_workspace, as_linear_decode, as_linear_prefill, as_linear_prefill_hybrid,
-               as_meta24_words, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size, config,
-               select_out)
+from . import (AS_BF16, AS_F32, AS_MODE_24, AS_MODE_DENSE, AS_MODE_SPLIT, AS_OP_AMBER, AS_OP_DECODE,
+               AS_OP_PREFILL, AS_OP_SELECT, AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SCORE_MAG, AS_SEL_ALL, AS_SEL_NM,
+               as_block_sparsity, as_hybrid_dense_blocks, as_hybrid_workspace, as_linear_decode, as_linear_prefill,
+               as_linear_prefill_hybrid, as_meta24_words, as_prefill_mode, as_select, as_weight_prep,
+               as_weight_prep_amber, as_workspace_size, config, select_out)
+
+
+_MODE_NAMES = {AS_MODE_24: "2:4", AS_MODE_SPLIT: "split", AS_MODE_DENSE: "dense"}
 
 
 def hybrid_mode(sparsity: float) -> str:
-    """Mode by a layer's measured sparsity (2:4 + Squared-ReLU page, section
-    3.3): above 95 % pure 2:4, 90-95 % the sparse/dense split, below 90 %
-    dense."""
-    if sparsity > 0.95:
-        return "2:4"
-    if sparsity >= 0.90:
-        return "split"
-    return "dense"
+    """Name of the mode the library's switch (as_prefill_mode) picks for a
+    layer's measured sparsity."""
+    return _MODE_NAMES[as_prefill_mode(sparsity)]
 
 
 def dense_blocks_for(K: int, dense_frac: float) -> int:
-    """Dense 4-channel blocks of the split: dense_frac of the K/4 blocks,
-    rounded up to a multiple of 16 (64 channels), at least 16 and at most
-    the whole multiple-of-16 part of K/4."""
-    nb = K // 4
-    n = math.ceil(dense_frac * nb / 16) * 16
-    return max(16, min(n, nb // 16 * 16))
+    """Dense 4-channel blocks of the split (as_hybrid_dense_blocks)."""
+    return as_hybrid_dense_blocks(K, dense_frac)
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -110,11 +102,18 @@ class SparseLinear:
         if c.var:
             for k in ("var_dense", "var_kept", "nu"):
                 b[k] = torch.empty(T, dtype=torch.float32, device=dev)
+        # float32 output with a token shift: the kept values also go in as
+        # their bf16 residuals (a second pass of the GEMM over K)
+        lo = c.out_dtype == AS_F32 and bool(c.dpts) and self.W.dtype == torch.bfloat16
         if c.sel == AS_SEL_NM and c.n == 2 and c.m == 4 and self.W.dtype == torch.bfloat16:
             b["x_compact"] = torch.empty(T, K // 2, dtype=torch.bfloat16, device=dev)
             b["meta24"] = torch.empty(as_meta24_words(T, K), dtype=torch.int32, device=dev)
+            if lo:
+                b["x_compact_lo"] = torch.empty(T, K // 2, dtype=torch.bfloat16, device=dev)
         else:
             b["x_masked"] = torch.empty(T, K, dtype=self.W.dtype, device=dev)
+            if lo:
+                b["x_masked_lo"] = torch.empty(T, K, dtype=torch.bfloat16, device=dev)
         return b
 
     def select(self, x: torch.Tensor, bufs: dict, running_var=None, first_batch: bool = False,
@@ -128,7 +127,8 @@ class SparseLinear:
         if y is None:
             y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=self.W.device)
         as_linear_prefill(select_out(**{k: v for k, v in bufs.items()
-                                        if k in ("x_masked", "x_compact", "meta24")}),
+                                        if k in ("x_masked", "x_compact", "meta24", "x_masked_lo",
+                                                 "x_compact_lo")}),
                           self.W, T, self.cfg, y, rowsum=self.rowsum, eta=bufs.get("eta"),
                           nu=bufs.get("nu"), workspace=self._workspace(AS_OP_PREFILL, T), stream=stream)
         return y
@@ -151,10 +151,9 @@ class SparseLinear:
         return y
 
     def prefill_auto(self, x: torch.Tensor, dense_frac: float = 0.05, stream=None):
-        """Mode chosen by the measured sparsity of x (2:4 + Squared-ReLU page,
-        section 3.3): above 95 % pure 2:4, 90-95 % the split with the
-        ceil(dense_frac * K/4 / 16) * 16 busiest blocks dense, below 90 %
-        the dense product.  Reads the sparsity back to the host (one
+        """Mode chosen by the library's switch (as_prefill_mode) on the
+        measured sparsity of x, with as_hybrid_dense_blocks(K, dense_frac)
+        dense blocks for the split.  Reads the sparsity back to the host (one
         synchronisation).  Returns (y, mode, sparsity)."""
         if not (self.cfg.sel == AS_SEL_NM and self.cfg.n == 2 and self.cfg.m == 4
                 and self.cfg.score == AS_SCORE_MAG and not self.cfg.dpts and not self.cfg.var):
@@ -166,8 +165,9 @@ class SparseLinear:
         sp = torch.empty(1, dtype=torch.float32, device=x.device)
         as_block_sparsity(x, sp, workspace=self._ws[key], stream=stream)
         s = float(sp.item())
-        mode = hybrid_mode(s)
-        if mode == "dense":
+        code = as_prefill_mode(s)
+        mode = _MODE_NAMES[code]
+        if code == AS_MODE_DENSE:
             cfg_all = config(sel=AS_SEL_ALL, out_dtype=self.cfg.out_dtype)
             y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=x.device)
             as_linear_prefill(select_out(x_masked=x), self.W, T, cfg_all, y,
@@ -175,9 +175,9 @@ class SparseLinear:
             return y, mode, s
         bufs = self.select_buffers(T, x.device)
         self.select(x, bufs, stream=stream)
-        if mode == "2:4":
+        if code == AS_MODE_24:
             return self.prefill_from(bufs, T, stream=stream), mode, s
-        return self.prefill_hybrid_from(x, bufs, dense_blocks_for(self.K, dense_frac), stream=stream), mode, s
+        return self.prefill_hybrid_from(x, bufs, as_hybrid_dense_blocks(self.K, dense_frac), stream=stream), mode, s
 
     def prefill(self, x: torch.Tensor, running_var=None, first_batch: bool = False, stream=None):
         bufs = self.select_buffers(x.shape[0], x.device)

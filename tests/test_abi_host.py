@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
     for n in declared():
         assert hasattr(raw, n), n
     assert set(lib.EXPORTS) == set(declared())
-    assert lib.as_abi_version() == 2
+    assert lib.as_abi_version() == 3
 
 
 def test_status_strings(lib):
@@ -117,6 +117,21 @@ def test_select_and_prefill_validation(lib):
     clact = lib.config(score=lib.AS_SCORE_CLACT, n=16, m=32)
     assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(clact), None, None, 0, ctypes.byref(lib.as_select_out()),
                None, 0, None) == lib.AS_ERR_WORKSPACE
+    # residual operands need their main operand (and bf16 x for the masked one)
+    lo = lib.as_select_out()
+    lo.x_masked_lo = fake
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(cfg816), None, None, 0, ctypes.byref(lo), None, 0,
+               None) == lib.AS_ERR_INVALID_ARG
+    lo.x_masked = fake
+    assert sel(fake, lib.AS_F32, 4, 64, ctypes.byref(cfg816), None, None, 0, ctypes.byref(lo), None, 0,
+               None) == lib.AS_ERR_INVALID_ARG
+    lo2 = lib.as_select_out()
+    lo2.x_compact_lo = fake
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(cfg24), None, None, 0, ctypes.byref(lo2), None, 0,
+               None) == lib.AS_ERR_INVALID_ARG
+    lo.x_masked_lo = fake + 4
+    assert sel(fake, lib.AS_BF16, 4, 64, ctypes.byref(cfg816), None, None, 0, ctypes.byref(lo), None, 0,
+               None) == lib.AS_ERR_ALIGN
     pre = lib._lib.as_linear_prefill
     empty = lib.as_select_out()
     assert pre(ctypes.byref(empty), fake, 4, 64, 64, None, None, None, ctypes.byref(cfg816), fake, None, 0,
@@ -227,9 +242,13 @@ def test_hybrid_validation_launches_nothing(lib):
     fake = 1 << 20
     assert lib.as_hybrid_workspace(4096, 14336, 4096, 192) > 4096 * 4096 * 4
     for bad in ((4096, 14300, 4096, 16), (4096, 14336, 4096, 17), (4096, 14336, 4096, 14336 // 4 + 16),
-                (16, 65536, 64, 16), (16, 1024, 60, 16), (60000, 1024, 8192, 16)):
+                (16, 65536, 64, 16), (16, 1024, 60, 16), (1 << 22, 1024, 64, 16)):
         with pytest.raises(lib.ASError):
             lib.as_hybrid_workspace(*bad)
+    # the gather rows are strided over the grid: no limit on T + n_out
+    assert lib.as_hybrid_workspace(60000, 1024, 8192, 16) > 0
+    assert lib.as_hybrid_workspace(8192, 1024, 57344, 16) > 0
+    assert lib.as_hybrid_workspace(70000, 1024, 0, 0) > 0
     sel = lib.select_out(bitmask=None)
     f = lib._lib.as_linear_prefill_hybrid
     assert f(ctypes.byref(sel), fake, 16, 1024, fake, 64, 16, lib.AS_BF16, fake, None, None, fake, 1 << 30,
@@ -237,18 +256,28 @@ def test_hybrid_validation_launches_nothing(lib):
     assert lib._lib.as_block_sparsity(fake, 16, 1000, 0, None, fake, fake, 1 << 20, None) == lib.AS_ERR_SHAPE
     assert lib._lib.as_block_sparsity(fake, 16, 1024, 16, None, fake, fake, 1 << 20, None) == lib.AS_ERR_INVALID_ARG
     assert lib._lib.as_block_sparsity(fake, 16, 1024, 0, None, fake, fake, 0, None) == lib.AS_ERR_WORKSPACE
+    # T = 70000 passes validation (without a GPU the accepted call then fails
+    # at its first CUDA call, never with a shape error)
+    ws = lib.as_hybrid_workspace(70000, 1024, 0, 0)
+    assert lib._lib.as_block_sparsity(fake, 70000, 1024, 0, None, fake, fake, ws, None) not in (
+        lib.AS_ERR_SHAPE, lib.AS_ERR_INVALID_ARG, lib.AS_ERR_WORKSPACE, lib.AS_OK)
 
 
 def test_hybrid_mode_rule_and_dense_block_count(lib):
-    """The product's mode rule equals the oracle's reading of the page's
-    thresholds; the dense-block count is 5 % of the blocks rounded up to
-    64 channels, within [16, K/4]."""
+    """The library's mode switch (a C entry point) equals the oracle's
+    reading of the page's thresholds; the dense-block count is 5 % of the
+    blocks rounded up to 64 channels, within [16, K/4]."""
     import oracle
     from sparse_linear_b200.layer import dense_blocks_for, hybrid_mode
+    names = {lib.AS_MODE_24: "2:4", lib.AS_MODE_SPLIT: "split", lib.AS_MODE_DENSE: "dense"}
     for s in np.linspace(0.0, 1.0, 2001):
+        assert names[lib._lib.as_prefill_mode(float(s))] == oracle.hybrid_mode(float(s))
         assert hybrid_mode(float(s)) == oracle.hybrid_mode(float(s))
-    for s in (0.95, 0.90, 0.9500001, 0.8999999):
+    for s in (0.95, 0.90, 0.9500001, 0.8999999, float(np.float32(0.95)), float(np.float32(0.9))):
         assert hybrid_mode(s) == oracle.hybrid_mode(s)
+    assert lib._lib.as_prefill_mode(float("nan")) == lib.AS_MODE_DENSE
+    for K, f in ((1000, 0.05), (0, 0.05), (1024, -0.1), (1024, 1.5), (1024, float("nan"))):
+        assert lib._lib.as_hybrid_dense_blocks(K, f) == -1
     assert dense_blocks_for(14336, 0.05) == 192      # 179.2 blocks -> 12 x 16
     assert dense_blocks_for(2048, 0.05) == 32        # 25.6 -> 2 x 16
     assert dense_blocks_for(256, 0.05) == 16         # at least 16
@@ -256,3 +285,29 @@ def test_hybrid_mode_rule_and_dense_block_count(lib):
     for K in range(64, 32769, 64):
         n = dense_blocks_for(K, 0.05)
         assert n % 16 == 0 and 16 <= n <= max(16, K // 4 // 16 * 16)
+
+
+def test_noalloc_refusals_enqueue_nothing(lib):
+    """as_linear_decode_noalloc checks every argument before it touches its
+    shared scratch: each invalid call returns its own status (fake,
+    never-dereferenced addresses; any launch or memset would fail here
+    without a GPU, with AS_ERR_CUDA)."""
+    fake = 1 << 20
+    f = lib._lib.as_linear_decode_noalloc
+    ok = lib.config(sel=lib.AS_SEL_NM, n=2, m=4)
+
+    def call(x=fake, dt=lib.AS_BF16, T=1, K=1024, n_out=64, wt=fake, g=None, rs=None, cfg=ok, y=fake, mask=None):
+        return f(x, dt, T, K, n_out, wt, g, rs, ctypes.byref(cfg), y, mask, None, None, None)
+
+    assert call(x=None) == lib.AS_ERR_INVALID_ARG
+    assert call(y=None) == lib.AS_ERR_INVALID_ARG
+    assert call(dt=7) == lib.AS_ERR_DTYPE
+    assert call(T=0) == lib.AS_ERR_SHAPE and call(T=17) == lib.AS_ERR_SHAPE
+    assert call(K=1002) == lib.AS_ERR_SHAPE
+    assert call(n_out=60) == lib.AS_ERR_SHAPE
+    assert call(cfg=lib.config(var=True)) == lib.AS_ERR_UNSUPPORTED
+    assert call(cfg=lib.config(dpts=True)) == lib.AS_ERR_INVALID_ARG          # no rowsum
+    assert call(cfg=lib.config(score=lib.AS_SCORE_WEIGHT)) == lib.AS_ERR_INVALID_ARG  # no g
+    assert call(x=fake + 4) == lib.AS_ERR_ALIGN
+    assert call(mask=fake + 8) == lib.AS_ERR_ALIGN
+    assert call(T=16, K=11008, n_out=16384, cfg=lib.config(sel=lib.AS_SEL_NM, n=8, m=16)) == lib.AS_ERR_WORKSPACE

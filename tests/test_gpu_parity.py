@@ -348,8 +348,6 @@ def check_prefill_masked(sl, xs, W, cfg, alpha=0.0, rows=None, eta_static=None):
         ref = oracle.linear(xf[rows], ref_mask, W.float().numpy(), eta=eta64,
                             rowsum=rs if cfg.dpts else None, nu=nu)
         tol = TOL_BF16 if cfg.out_dtype == sl.AS_BF16 else TOL_F32
-        if cfg.dpts:
-            tol = max(tol, TOL_BF16)  # the shifted kept values enter the tensor cores as bf16
         err = rel_l2(f32(y)[rows], ref)
         assert err <= tol, (b, err)
 
@@ -375,6 +373,71 @@ def test_prefill_topk_and_all(sl):
     x, W = synth.random_layer(T, K, n_out, seed=3)
     check_prefill_masked(sl, [x], W, sl.config(sel=sl.AS_SEL_TOPK, k_keep=600))
     check_prefill_masked(sl, [x], W, sl.config(sel=sl.AS_SEL_ALL, out_dtype=sl.AS_F32))
+
+
+def test_prefill_clact_var_eight_batches(sl):
+    """The CLACT + VAR 16:32 chain over all eight seeded batches (momentum
+    0.9) on a smaller problem of the same distributions, x [512, 2048] and W
+    [1024, 2048]: every batch's masks, variances, running variance, nu and y
+    against the oracle, whose running state is carried through its own
+    chain (float64), not taken from the GPU."""
+    W = synth.prefill_clact_weight(k=2048, n_out=1024)
+    xs = [synth.prefill_clact_batch(b, T=512, k=2048) for b in range(8)]
+    cfg = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)
+    check_prefill_masked(sl, xs, W, cfg)
+    cfg32 = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True, out_dtype=sl.AS_F32)
+    check_prefill_masked(sl, xs, W, cfg32)
+
+
+# T = 256: an even number of 128-row tiles (CTA-pair kernels); T = 300: odd
+# (one-SM kernels)
+@pytest.mark.parametrize("T,case", [(256, "2:4 D-PTS"), (300, "2:4 D-PTS"), (256, "8:16 D-PTS"),
+                                    (300, "8:16 D-PTS"), (256, "2:4 S-PTS"), (300, "top-k D-PTS")])
+def test_prefill_shift_float32_residual_pass(sl, T, case):
+    """Float32 output with a token shift: the shifted kept values are not
+    bf16 numbers, so they enter the tensor cores as bf16 hi + lo (a second
+    pass over K with the residual operand) and y holds the float32
+    tolerance against the oracle."""
+    K, n_out = 1024, 264
+    x, W = synth.random_layer(T, K, n_out, seed=T + len(case), dist="sqrelu" if "2:4" in case else "laplace")
+    eta_static = None
+    if case == "2:4 D-PTS":
+        cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, dpts=True, out_dtype=sl.AS_F32)
+    elif case == "8:16 D-PTS":
+        cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True, out_dtype=sl.AS_F32)
+    elif case == "2:4 S-PTS":
+        eta_static = dev(torch.from_numpy((0.05 + 0.01 * np.cos(np.arange(T))).astype(np.float32)))
+        cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, dpts=sl.AS_PTS_STATIC, eta_static=eta_static,
+                        out_dtype=sl.AS_F32)
+    else:
+        cfg = sl.config(sel=sl.AS_SEL_TOPK, k_keep=400, dpts=True, out_dtype=sl.AS_F32)
+    check_prefill_masked(sl, [x], W, cfg, alpha=0.5, eta_static=eta_static)
+
+
+def test_prefill_residual_pass_is_used(sl):
+    """The float32 D-PTS prefill with the residual operand is closer to the
+    oracle than the same call without it (one bf16 pass), which shows the
+    second pass adds the residual rather than leaving it out."""
+    T, K, n_out = 256, 2048, 392
+    x, W = synth.random_layer(T, K, n_out, seed=5, dist="laplace")
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=8, m=16, dpts=True, out_dtype=sl.AS_F32)
+    L = layer(sl, W, cfg)
+    xd = dev(x)
+    bufs = L.select_buffers(T)
+    assert "x_masked_lo" in bufs
+    L.select(xd, bufs)
+    y2 = L.prefill_from(bufs, T)
+    one = {k: v for k, v in bufs.items() if k != "x_masked_lo"}
+    y1 = L.prefill_from(one, T)
+    torch.cuda.synchronize()
+    xf = x.float().numpy()
+    eta64 = oracle.token_mean(xf)
+    s = oracle.score(xf, eta=f32(bufs["eta"]))
+    mask = oracle.select_nm(s, 8, 16)
+    _, rs = oracle.weight_prep(W.float().numpy(), 1.0)
+    ref = oracle.linear(xf, mask, W.float().numpy(), eta=eta64, rowsum=rs)
+    e2, e1 = rel_l2(f32(y2), ref), rel_l2(f32(y1), ref)
+    assert e2 <= TOL_F32 and e2 < 0.25 * e1, (e2, e1)
 
 
 def test_prefill_clact_var_full_size(sl):
