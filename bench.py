@@ -330,6 +330,26 @@ def bench_decode(sl, dev, steps, warmup, world):
     per_t_f32 = {T: v[1] for T, v in per_t_rs.items()}
     per_t_rs = {T: v[0] for T, v in per_t_rs.items()}
 
+    # dense baseline on the same shapes and rotation: torch.matmul (cuBLAS)
+    # of x [T, 11008] by the channel-major weight copy Wt [11008, 4096], 8
+    # calls per graph over the 8 weight copies
+    per_t_dense = {}
+    yd = {T: torch.empty(T, N_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS}
+    with torch.cuda.stream(stream):
+        for T in DECODE_TS:
+            def call_d(i, T=T):
+                torch.matmul(xs[i][:T], Wts[i], out=yd[T])
+            for i in range(N_ROT):
+                call_d(i)
+            stream.synchronize()
+            g_d = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_d, stream=stream):
+                for i in range(N_ROT):
+                    call_d(i)
+            per_t_dense[T] = (timed(lambda j, g_d=g_d: g_d.replay(), reps) / (reps * N_ROT), g_d)
+    per_t_dense = {T: v[0] for T, v in per_t_dense.items()}
+    dense_bytes = {T: K_DOWN * N_DOWN * 2 + T * K_DOWN * 2 + T * N_DOWN * 2 for T in DECODE_TS}
+
     # end to end through host buffers, every step: pinned host x -> device,
     # decode, y -> pinned host.  Copies run on their own streams (H2D and D2H
     # use separate copy engines) into double-buffered device x and y, so the
@@ -443,8 +463,14 @@ def bench_decode(sl, dev, steps, warmup, world):
         t=t_max, steps=steps, tokens_per_step=tokens,
         value=tokens * steps * world / t_max,
         e2e=tokens * steps * world / t_e2e, e2e_eager=tokens * steps * world / t_e2e_eager, h2d=h2d, d2h=d2h,
-        per_t={T: dict(us=per_t[T] * 1e6, gbs=bytes_call[T] / per_t[T] / 1e9, bytes=bytes_call[T])
+        per_t={T: dict(us=per_t[T] * 1e6, gbs=bytes_call[T] / per_t[T] / 1e9, bytes=bytes_call[T],
+                       metadata_to_kept_bytes=(T * words * 4) / (bytes_call[T] - T * K_DOWN * 2 - T * N_DOWN * 2
+                                                                 - K_DOWN * 4 - N_DOWN * 4),
+                       dense_cublas_us=per_t_dense[T] * 1e6,
+                       dense_cublas_gbs=dense_bytes[T] / per_t_dense[T] / 1e9,
+                       speedup_vs_dense=per_t_dense[T] / per_t[T])
                for T in DECODE_TS},
+        dense_step_us=sum(per_t_dense.values()) * 1e6,
         per_t_spts={T: dict(us=per_t_spts[T] * 1e6, tokens_per_s=T / per_t_spts[T]) for T in DECODE_TS},
         per_t_rs={T: dict(us=per_t_rs[T] * 1e6, tokens_per_s=T / per_t_rs[T],
                           decode_only_f32_out_us=per_t_f32[T] * 1e6) for T in DECODE_TS},
@@ -454,19 +480,30 @@ def bench_decode(sl, dev, steps, warmup, world):
 
 
 # ---------------------------------------------------------------- prefill
+PREFILL_REPS = 50
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
 def bench_prefill(sl, dev, pk):
     from sparse_linear_b200.layer import SparseLinear
     out = {}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def ev_time(fn, reps):
-        torch.cuda.synchronize()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        for _ in range(reps):
+    def ev_time(fn, reps=PREFILL_REPS, warm=3):
+        """Median over `reps` launches of fn's CUDA-event time, each launch
+        after a write of a buffer twice the L2 (so no operand starts in L2)."""
+        for _ in range(warm):
             fn()
-        e.record()
-        torch.cuda.synchronize()
-        return s.elapsed_time(e) / 1e3 / reps
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(s.elapsed_time(e) / 1e3)
+        return statistics.median(ts)
 
     # 2:4 on squared-ReLU activations, sparse tensor-core path
     _, x, W = synth.prefill_sqrelu()
@@ -482,12 +519,15 @@ def bench_prefill(sl, dev, pk):
         L.prefill_from(bufs, T, y)
     for _ in range(3):
         torch.matmul(x, W.t())  # cuBLAS handle, workspace and heuristics outside the timing
-    t_sel = ev_time(lambda: L.select(x, bufs), 10)
-    t_gemm = ev_time(lambda: L.prefill_from(bufs, T, y), 10)
-    t_dense = ev_time(lambda: torch.matmul(x, W.t()), 10)
+    t_sel = ev_time(lambda: L.select(x, bufs))
+    t_gemm = ev_time(lambda: L.prefill_from(bufs, T, y))
+    t_dense = ev_time(lambda: torch.matmul(x, W.t()))
     dense_eq = 2.0 * T * n_out * K
     sp_peak = 2.0 * pk["bf16_tflops"]
+    sel_bytes = T * K * 2 + T * K + sl.as_meta24_words(T, K) * 4 + T * ((K + 31) // 32) * 4
     out["sqrelu_2of4"] = dict(
+        select_gbs=sel_bytes / t_sel / 1e9, select_frac_of_hbm=sel_bytes / t_sel / 1e9 / pk["hbm_gbs"],
+        metadata_to_kept_bytes=sl.as_meta24_words(T, K) * 4 / (T * K // 2 * 2),
         shape=[T, K, n_out], select_us=t_sel * 1e6, gemm_us=t_gemm * 1e6,
         gemm_dense_equiv_tflops=dense_eq / t_gemm / 1e12, useful_tflops=dense_eq / 2 / t_gemm / 1e12,
         frac_of_sparse_peak=dense_eq / t_gemm / 1e12 / sp_peak,
@@ -515,13 +555,15 @@ def bench_prefill(sl, dev, pk):
     for _ in range(3):
         prod()
         gemm()
-    t_prod = ev_time(prod, 10)
-    t_gemm = ev_time(gemm, 10)
+    t_prod = ev_time(prod)
+    t_gemm = ev_time(gemm)
     dense_eq = 2.0 * T * n_out * K
     sp_peak8 = 4.0 * pk["bf16_tflops"]
     prod_bytes = T * K * 2 + T * K // 2 + T * K // 8 + T * 4
     out["sqrelu_2of4_fp8"] = dict(
         shape=[T, K, n_out], producer_us=t_prod * 1e6, producer_gbs=prod_bytes / t_prod / 1e9,
+        producer_frac_of_hbm=prod_bytes / t_prod / 1e9 / pk["hbm_gbs"],
+        metadata_to_kept_bytes=sl.as_meta8_words(T, K) * 4 / (T * K // 2),
         gemm_us=t_gemm * 1e6, gemm_dense_equiv_tflops=dense_eq / t_gemm / 1e12,
         frac_of_sparse_fp8_peak=dense_eq / t_gemm / 1e12 / sp_peak8,
         speedup_vs_bf16_2of4_gemm=out["sqrelu_2of4"]["gemm_us"] / (t_gemm * 1e6))
@@ -544,10 +586,10 @@ def bench_prefill(sl, dev, pk):
         L.select(x, bufs)
         L.prefill_from(bufs, T, y24)
         L.prefill_hybrid_from(x, bufs, 192, y=yh, sparsity=sp)
-    t_sel = ev_time(lambda: L.select(x, bufs), 10)
-    t_24 = ev_time(lambda: L.prefill_from(bufs, T, y24), 10)
-    t_h = ev_time(lambda: L.prefill_hybrid_from(x, bufs, 192, y=yh, sparsity=sp), 10)
-    t_dense = ev_time(lambda: torch.matmul(x, W.t()), 10)
+    t_sel = ev_time(lambda: L.select(x, bufs))
+    t_24 = ev_time(lambda: L.prefill_from(bufs, T, y24))
+    t_h = ev_time(lambda: L.prefill_hybrid_from(x, bufs, 192, y=yh, sparsity=sp))
+    t_dense = ev_time(lambda: torch.matmul(x, W.t()))
     yd = torch.matmul(x.float(), W.float().t())
     err = lambda yy: float(torch.linalg.norm(yy.float() - yd) / torch.linalg.norm(yd))  # noqa: E731
     out["hybrid_split_hot_channels"] = dict(
@@ -557,9 +599,11 @@ def bench_prefill(sl, dev, pk):
     del x, W, L, bufs, y24, yh, yd
     torch.cuda.empty_cache()
 
-    # CLACT + VAR at 16:32: masked dense tensor-core GEMM
+    # CLACT + VAR at 16:32: masked dense tensor-core GEMM, over the eight
+    # seeded batches (running variance carried from batch to batch)
     W = synth.prefill_clact_weight().to(dev)
-    x = synth.prefill_clact_batch(0).to(dev)
+    xs = [synth.prefill_clact_batch(b).to(dev) for b in range(8)]
+    x = xs[0]
     T, K = x.shape
     n_out = W.shape[0]
     cfg = sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)
@@ -568,20 +612,39 @@ def bench_prefill(sl, dev, pk):
     run = torch.zeros(T, dtype=torch.float32, device=dev)
     y = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
     L.select(x, bufs, running_var=run, first_batch=True)
-    for _ in range(2):
-        L.select(x, bufs, running_var=run)
+    t_sel = ev_time(lambda: L.select(x, bufs, running_var=run))
+    t_gemm = ev_time(lambda: L.prefill_from(bufs, T, y))
+    t_dense = ev_time(lambda: torch.matmul(x, W.t()))
+    # the eight batches back to back, select + GEMM each (one CUDA-event span)
+    for b in range(8):
+        L.select(xs[b], bufs, running_var=run, first_batch=(b == 0))
         L.prefill_from(bufs, T, y)
-    for _ in range(3):
-        torch.matmul(x, W.t())
-    t_sel = ev_time(lambda: L.select(x, bufs, running_var=run), 5)
-    t_gemm = ev_time(lambda: L.prefill_from(bufs, T, y), 5)
-    t_dense = ev_time(lambda: torch.matmul(x, W.t()), 5)
+    per_batch = []
+    for rep in range(3):
+        flush.zero_()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for b in range(8):
+            L.select(xs[b], bufs, running_var=run, first_batch=(b == 0))
+            L.prefill_from(bufs, T, y)
+        e.record()
+        torch.cuda.synchronize()
+        per_batch.append(s.elapsed_time(e) / 1e3 / 8)
     flops = 2.0 * T * n_out * K
+    sel_bytes = 2 * T * K * 2 + T * K * 2 + T * (K // 32) * 4  # colnorm read, select read, masked write, mask
     out["clact_var_16of32"] = dict(
         shape=[T, K, n_out], select_us=t_sel * 1e6, gemm_us=t_gemm * 1e6,
+        select_gbs=sel_bytes / t_sel / 1e9, select_frac_of_hbm=sel_bytes / t_sel / 1e9 / pk["hbm_gbs"],
         gemm_tflops=flops / t_gemm / 1e12, frac_of_dense_peak=flops / t_gemm / 1e12 / pk["bf16_tflops"],
-        cublas_dense_us=t_dense * 1e6, cublas_dense_tflops=flops / t_dense / 1e12)
+        cublas_dense_us=t_dense * 1e6, cublas_dense_tflops=flops / t_dense / 1e12,
+        eight_batches_us_per_batch=statistics.median(per_batch) * 1e6,
+        eight_batches_vs_cublas_dense=statistics.median(per_batch) / t_dense)
+    del xs, x
+    torch.cuda.empty_cache()
     assert sl.as_stream_status() == sl.AS_OK
+    out["timing"] = (f"median of {PREFILL_REPS} launches, CUDA events, each after writing a "
+                     f"{L2_FLUSH_BYTES >> 20} MB buffer (L2 flushed)")
     return out
 
 
@@ -612,6 +675,16 @@ def oracle_decode_sample(budget_s: float):
             break
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return tokens / el, threads, f"{reps} oracle decode steps (T=1,8,16 of the down-projection), {el:.1f} s"
+
+
+def oracle_one_thread(budget_s: float):
+    """The same oracle sample in a child process held to one OpenMP thread."""
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-sample", str(budget_s)],
+                       env=env, capture_output=True, text=True, timeout=600)
+    if r.returncode != 0:
+        return None
+    return json.loads(r.stdout.strip().splitlines()[-1])
 
 
 def bench_block(sl, dev, reps=200):
@@ -790,7 +863,12 @@ def main():
                     help="profiling case: decode | sqrelu24 | sqrelu24_fp8 | sqrelu24_fp8_producer | hybrid | dense | select24 | selectclact | block")
     ap.add_argument("--T", type=int, default=1)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--oracle-sample", type=float, default=None, help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.oracle_sample is not None:  # child of oracle_one_thread
+        tps, threads, sample = oracle_decode_sample(budget_s=args.oracle_sample)
+        print(json.dumps({"value": tps, "threads": threads, "sample": sample}))
+        return
     if args.case:
         run_case(args)
         return
@@ -818,6 +896,9 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         tps, threads, sample = oracle_decode_sample(budget_s=15.0)
         cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
+        one = oracle_one_thread(8.0)
+        if one is not None:
+            cpu["one_thread"] = {"value": one["value"], "unit": "tokens/s", "cores": 1, "sample": one["sample"]}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -837,12 +918,17 @@ def main():
                    "tokens_per_step": d["tokens_per_step"], "parallelism": f"replicas x{world}",
                    "l2": f"{N_ROT} rotating weight copies ({N_ROT * 90} MB) and activation sets per step cycle",
                    "timing": "CUDA graphs of one step replayed; CUDA events on the launching stream"},
+        "dense_baseline": {"what": "torch.matmul (cuBLAS) x [T, 11008] @ Wt [11008, 4096] bf16, same rotation",
+                           "step_us": d["dense_step_us"],
+                           "tokens_per_s": d["tokens_per_step"] / (d["dense_step_us"] * 1e-6),
+                           "speedup_of_sparse_step": d["dense_step_us"] / sum(v["us"] for v in d["per_t"].values())},
         "roofline": {"bound": "hbm", "achieved": d["achieved_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": d["achieved_gbs"] / peak, "traffic": traffic,
                      "peak_source": f"{pk_src} copy bandwidth (MEASURED_PEAKS.json)" if pk_src == "measured"
                      else "fallback 6650 GB/s",
                      "kernel": "k_decode_tc (timed per whole decode call: select, decode and split-K "
-                               "reduction kernels)", "bytes_per_launch": d["bytes_per_launch"],
+                               "reduction kernels)",
+                     "bytes_per_launch": d["bytes_per_launch"],
                      "per_T": {str(T): v for T, v in d["per_t"].items()}},
         "e2e": {"value": d["e2e"], "unit": "tokens/s", "h2d_bytes_per_step": d["h2d"],
                 "d2h_bytes_per_step": d["d2h"],

@@ -373,6 +373,31 @@ as_status as_rsparse_decode(const void *x, as_dtype dt, int T, int K, int n_out,
                             const float *eta, const void *B, const void *A, float *y, void *workspace,
                             size_t ws_bytes, cudaStream_t stream);
 
+/* --------------------------------------------------------------------------
+ * R-Sparse compensation of a prefill call ([OVW] 3.3): as_linear_prefill
+ * plus the dropped channels through the rank-r factors of W (the same
+ * factors as as_rsparse_decode):
+ *   y = epilogue((xhat (.) m) W^T + U A^T),  U = (xhat (.) (1 - m)) B,
+ * with xhat = fl32(x - eta_t) under a token shift (cfg->dpts, eta the
+ * as_select output), x otherwise, and m the selection (sel->bitmask).  U is
+ * computed first ([T, r], float32 accumulation in a fixed order, the dropped
+ * values entering the tensor cores as bf16 hi + lo) and stored as bf16 hi
+ * and lo; the prefill GEMM then runs 2 r/64 more K blocks whose A operand is
+ * U and whose B operand is A, into the same accumulator.
+ *   sel, W, T, K, n_out, rowsum, eta, cfg, y: as as_linear_prefill (sel
+ *            must also hold the bitmask); cfg->var is not supported
+ *            (AS_ERR_UNSUPPORTED: the pages define no VAR scale of the
+ *            compensation).
+ *   x        bf16 [T, K], the call's input.
+ *   B, A     bf16 [K, r] and [n_out, r]; r in {64, 128}.
+ * Workspace: as_rsparse_prefill_workspace(T, K, r) bytes, no zero-fill.
+ * ------------------------------------------------------------------------ */
+size_t as_rsparse_prefill_workspace(int T, int K, int r);
+as_status as_linear_prefill_rsparse(const as_select_out *sel, const void *x, const void *W, int T, int K, int n_out,
+                                    const float *rowsum, const float *eta, const as_config *cfg, int r,
+                                    const void *B, const void *A, void *y, void *workspace, size_t ws_bytes,
+                                    cudaStream_t stream);
+
 /* Number of 32-bit metadata words of a 2:4 selection of T tokens x K channels. */
 size_t as_meta24_words(int T, int K);
 

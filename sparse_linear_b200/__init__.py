@@ -43,6 +43,7 @@ EXPORTS = [
     "as_weight_prep_amber", "as_meta8_words", "as_weight_quant_fp8", "as_select_sqrelu24_fp8",
     "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode", "as_hybrid_workspace",
     "as_linear_prefill_hybrid", "as_block_sparsity", "as_prefill_mode", "as_hybrid_dense_blocks",
+    "as_rsparse_prefill_workspace", "as_linear_prefill_rsparse",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -91,6 +92,9 @@ _sig = {
     "as_status_string": ([_I], ctypes.c_char_p),
     "as_abi_version": ([], _I),
     "as_prefill_mode": ([ctypes.c_double], _I),
+    "as_rsparse_prefill_workspace": ([_I, _I, _I], _S),
+    "as_linear_prefill_rsparse": ([ctypes.POINTER(as_select_out), _P, _P, _I, _I, _I, _P, _P,
+                                   ctypes.POINTER(as_config), _I, _P, _P, _P, _P, _S, _P], _I),
     "as_hybrid_dense_blocks": ([_I, ctypes.c_double], _I),
 }
 for _name, (_args, _res) in _sig.items():
@@ -335,6 +339,26 @@ def as_linear_prefill(sel: as_select_out, W, T: int, cfg: as_config, y, rowsum=N
     _check(_lib.as_linear_prefill(ctypes.byref(sel), _ptr(W), T, K, n_out, _ptr(rowsum), _ptr(eta), _ptr(nu),
                                   ctypes.byref(cfg), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "as_linear_prefill")
+
+
+def as_rsparse_prefill_workspace(T: int, K: int, r: int) -> int:
+    n = _lib.as_rsparse_prefill_workspace(T, K, r)
+    if n == ctypes.c_size_t(-1).value:
+        raise ASError(AS_ERR_SHAPE, "as_rsparse_prefill_workspace")
+    return n
+
+
+def as_linear_prefill_rsparse(sel: as_select_out, x, W, cfg: as_config, y, B, A, rowsum=None, eta=None,
+                              workspace=None, stream=None) -> None:
+    """as_linear_prefill plus the R-Sparse compensation of the dropped
+    channels through the rank-r factors B [K, r] and A [n_out, r]."""
+    T, K = x.shape
+    n_out = W.shape[0]
+    r = A.shape[1]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_linear_prefill_rsparse(ctypes.byref(sel), _ptr(x), _ptr(W), T, K, n_out, _ptr(rowsum), _ptr(eta),
+                                          ctypes.byref(cfg), r, _ptr(B), _ptr(A), _ptr(y), _ptr(workspace), ws_bytes,
+                                          _stream(stream)), "as_linear_prefill_rsparse")
 
 
 def as_stream_status(stream=None) -> int:

@@ -48,9 +48,8 @@ size_t decode_ws(int T, int K, int n_out, const as_config *cfg, int bf16)
 {
     DecodePlan p = decode_plan(T, K, n_out, bf16);
     size_t bytes = round_up(p.counter_bytes, 256) + round_up(p.partial_bytes, 256) + round_up(p.eta_bytes, 256);
-    // a separate selection kernel: bf16 unless fused (<= 2 tokens, N:M); float32 for top-k / keep-all
-    const bool sel_kernel = (bf16 && !decode_fused(p.tpad, cfg->sel, K)) || cfg->sel == AS_SEL_TOPK ||
-                            cfg->sel == AS_SEL_ALL;
+    // a separate selection kernel (top-k; the non-cluster bf16 path beyond 2 tokens; keep-all)
+    const bool sel_kernel = decode_needs_select(T, K, n_out, bf16, cfg->out_dtype == AS_BF16, cfg->sel);
     if (sel_kernel) bytes += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
     if (sel_kernel && cfg->score == AS_SCORE_CLACT) bytes += round_up(colnorm_workspace(T, K), 256);
     return bytes;
@@ -417,7 +416,7 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     ws += round_up(plan.eta_bytes, 256);
 
     const uint32_t *mask_in = nullptr;
-    if ((bf16 && !decode_fused(plan.tpad, cfg->sel, K)) || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL) {
+    if (decode_needs_select(T, K, n_out, bf16, cfg->out_dtype == AS_BF16, cfg->sel)) {
         // per-token selection kernel first (bf16: always; float32: top-k needs the whole row)
         uint32_t *bm = reinterpret_cast<uint32_t *>(ws);
         ws += round_up((size_t)T * ((K + 31) / 32) * sizeof(uint32_t), 256);
@@ -478,12 +477,12 @@ as_status as_linear_decode(const void *x, as_dtype dt, int T, int K, int n_out, 
     return cuda_status(launch_decode(a, plan, stream));
 }
 
-as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int K, int n_out, const float *rowsum,
-                            const float *eta, const float *nu, const as_config *cfg, void *y, void *workspace,
-                            size_t ws_bytes, cudaStream_t stream)
+}  // extern "C"
+
+// Validation and GEMM arguments shared by the prefill entry points.
+static as_status prefill_args(const as_select_out *sel, const void *W, int T, int K, int n_out, const float *rowsum,
+                              const float *eta, const float *nu, const as_config *cfg, void *y, GemmArgs &a)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (!sel || !W || !y || T <= 0 || K <= 0 || n_out <= 0) return AS_ERR_INVALID_ARG;
     as_status st = check_cfg(cfg, K);
     if (st != AS_OK) return st;
@@ -497,7 +496,7 @@ as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int 
                           sel->x_compact_lo};
     for (const void *p : ptrs)
         if (!aligned16(p)) return AS_ERR_ALIGN;
-    GemmArgs a{};
+    a = GemmArgs{};
     a.A = sparse ? sel->x_compact : sel->x_masked;
     a.A_lo = sparse ? sel->x_compact_lo : sel->x_masked_lo;
     a.meta = sparse ? sel->meta24 : nullptr;
@@ -511,6 +510,49 @@ as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int 
     a.nu = cfg->var ? nu : nullptr;
     a.y = y;
     a.out_bf16 = cfg->out_dtype == AS_BF16;
+    return AS_OK;
+}
+
+extern "C" {
+
+as_status as_linear_prefill(const as_select_out *sel, const void *W, int T, int K, int n_out, const float *rowsum,
+                            const float *eta, const float *nu, const as_config *cfg, void *y, void *workspace,
+                            size_t ws_bytes, cudaStream_t stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    GemmArgs a;
+    const as_status st = prefill_args(sel, W, T, K, n_out, rowsum, eta, nu, cfg, y, a);
+    if (st != AS_OK) return st;
+    return cuda_status(launch_gemm(a, stream));
+}
+
+size_t as_rsparse_prefill_workspace(int T, int K, int r)
+{
+    if (T <= 0 || K <= 0 || (r != 64 && r != 128)) return (size_t)-1;
+    return rsp_layout(T, K, r).bytes;
+}
+
+as_status as_linear_prefill_rsparse(const as_select_out *sel, const void *x, const void *W, int T, int K, int n_out,
+                                    const float *rowsum, const float *eta, const as_config *cfg, int r,
+                                    const void *B, const void *A, void *y, void *workspace, size_t ws_bytes,
+                                    cudaStream_t stream)
+{
+    if (!x || !B || !A || !sel || !sel->bitmask) return AS_ERR_INVALID_ARG;
+    if (cfg && cfg->var) return AS_ERR_UNSUPPORTED;  // the pages define no VAR scale of the compensation
+    GemmArgs a;
+    as_status st = prefill_args(sel, W, T, K, n_out, rowsum, eta, nullptr, cfg, y, a);
+    if (st != AS_OK) return st;
+    if (r != 64 && r != 128) return AS_ERR_SHAPE;
+    for (const void *p : {x, B, A, (const void *)sel->bitmask, (const void *)workspace})
+        if (!aligned16(p)) return AS_ERR_ALIGN;
+    const RspLayout L = rsp_layout(T, K, r);
+    if (!workspace || ws_bytes < L.bytes) return AS_ERR_WORKSPACE;
+    cudaError_t e = launch_rsp_u(x, sel->bitmask, cfg->dpts ? eta : nullptr, B, T, K, r, workspace, stream);
+    if (e != cudaSuccess) return AS_ERR_CUDA;
+    a.U2 = static_cast<const char *>(workspace) + L.u;
+    a.Ar = A;
+    a.r = r;
     return cuda_status(launch_gemm(a, stream));
 }
 
@@ -528,8 +570,9 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
     a.eta_static = cfg->dpts == AS_PTS_STATIC ? cfg->eta_static : nullptr;
     a.bf16 = bf16;
     a.sel = cfg->sel;
+    a.out_bf16 = cfg->out_dtype == AS_BF16;
     int n = 0;
-    if ((bf16 && !decode_fused(plan.tpad, cfg->sel, K)) || cfg->sel == AS_SEL_TOPK || cfg->sel == AS_SEL_ALL)
+    if (decode_needs_select(T, K, n_out, bf16, a.out_bf16, cfg->sel))
         n += 1 + (cfg->score == AS_SCORE_CLACT ? 2 : 0);  // select kernel (+ column energy)
     return n + decode_launch_count(a, plan);
 }

@@ -6,6 +6,7 @@
 #include "gemm.cu"
 #include "fp8.cu"
 #include "rsparse.cu"
+#include "rsparse_prefill.cu"
 #include "hybrid.cu"
 #include "abi.cu"
 #include "noalloc.cu"

@@ -516,7 +516,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 // FUSED (at most 2 tokens): the kernel computes the means and the selection
 // itself (no select kernel before it).  Otherwise the select kernel precedes
 // it.  With several splits k_decode_reduce follows it in both cases.
@@ -1004,8 +1003,9 @@ bool decode_fused(int tpad, int sel, int K)
     return tpad <= 2 && (sel == AS_SEL_NM || sel == AS_SEL_THRESH) && K <= 8 * TC_THREADS * 8;
 }
 
-int decode_launch_count(const DecodeArgs &, const DecodePlan &p)
+int decode_launch_count(const DecodeArgs &a, const DecodePlan &p)
 {
+    (void)a;
     if (!p.tc) return 1;
     return 1 + (p.k_splits > 1 ? 1 : 0);  // decode (+ split-K reduction); the select kernel is counted by the caller
 }
@@ -1081,6 +1081,15 @@ static cudaError_t launch_tc(const DecodeArgs &a, const DecodePlan &p, cudaStrea
     set_pdl(rc, rattr);
     return cudaLaunchKernelEx(&rc, k_decode_reduce<TP>, (const float *)a.partial, p.k_splits, a.T, a.n_out,
                               a.dpts ? (const float *)a.eta_in : (const float *)nullptr, a.rowsum, a.y, a.out_bf16);
+}
+
+bool decode_needs_select(int T, int K, int n_out, int bf16, int out_bf16, int sel)
+{
+    (void)n_out;
+    (void)out_bf16;
+    if (sel == AS_SEL_TOPK) return true;  // top-k needs the whole row's scores
+    if (!bf16) return sel == AS_SEL_ALL;
+    return !decode_fused(tpad_of(T), sel, K) || sel == AS_SEL_ALL;
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)

@@ -69,8 +69,18 @@ struct GemmParams {
     void *y;
     int T, K, n_out, out_bf16;
     int m_tiles, n_tiles, k_blocks, meta_kt;
-    int kb_pass;  // K blocks of one pass over K; k_blocks = 2 kb_pass when a residual A operand follows
+    int kb_pass;  // K blocks of one pass over K
+    int kb_main;  // kb_pass, or 2 kb_pass when a residual A operand follows
+    int rblk;     // R-Sparse: 64-wide blocks of the rank (k_blocks = kb_main + 2 rblk)
 };
+
+// R-Sparse extra K block e (0 .. 2 rblk - 1): which part of U (0 hi, 1 lo)
+// and which 64-wide block of the rank it covers.
+__device__ __forceinline__ void extra_block(int e, int rblk, int &part, int &j)
+{
+    part = e / rblk;
+    j = e - part * rblk;
+}
 
 // Adds row `row`, columns col0 .. col0+31 of a float32 [T, n_out] term to 32
 // accumulator values (n_out % 8 == 0: a 4-column group past n_out is
@@ -100,7 +110,8 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
 template <bool SPARSE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmA2, GemmParams p)
+           const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmU,
+           const __grid_constant__ CUtensorMap tmR, GemmParams p)
 {
     using C = GemmCfg<SPARSE>;
     constexpr int BN = C::BN, S = C::STAGES;
@@ -154,6 +165,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 tile_coords(tile, p.m_tiles, p.n_tiles, mt, nt);
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                    if (kb >= p.kb_main) {  // R-Sparse: U (dense) against A_r, first B sub-tile only
+                        int part, j;
+                        extra_block(kb - p.kb_main, p.rblk, part, j);
+                        mbar_arrive_expect_tx(&full[stage], C::A_BYTES + (SPARSE ? C::B_BYTES / 2 : C::B_BYTES));
+                        tma_load_2d(sA + stage * C::A_BYTES, &tmU, &full[stage], j * 64, mt * GEMM_BM + part * p.T);
+                        tma_load_2d(sB + stage * C::B_BYTES, &tmR, &full[stage], j * 64, nt * BN);
+                        if (++stage == S) { stage = 0; phase ^= 1; }
+                        continue;
+                    }
                     mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + C::M_BYTES);
                     // second pass over K: the residual operand against the same W blocks
                     const bool lo = kb >= p.kb_pass;
@@ -194,7 +214,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
                     const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
                     const uint64_t a_desc = sdesc_kmajor_sw128(a_addr);
-                    if constexpr (SPARSE) {
+                    if (SPARSE && kb >= p.kb_main) {  // R-Sparse block: dense MMAs into the same accumulator
+                        const uint64_t b_desc = sdesc_kmajor_sw128(b_addr);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_bf16(d_tmem, a_desc + (uint64_t)((32 * j) >> 4), b_desc + (uint64_t)((32 * j) >> 4),
+                                     idesc_bf16(GEMM_BM, BN, false), 1u);
+                    } else if constexpr (SPARSE) {
                         const uint32_t e_tmem = meta_tmem + stage * 4;
                         tmem_cp_128x128b(e_tmem, sdesc_rows16(smem_u32(sM + stage * C::M_BYTES)));
 #pragma unroll
@@ -346,7 +372,8 @@ constexpr size_t pair_smem_bytes() { return 1024 + (size_t)PAIR_STAGES * PairCfg
 template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     k_gemm_sp_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmA2, GemmParams p)
+                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmA2,
+                   const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmR, GemmParams p)
 {
     using C = PairCfg<FP8>;
     constexpr int S = PAIR_STAGES;
@@ -406,6 +433,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                 const int echunk = (2 * mt + (int)rank) * p.meta_kt;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
+                    if (!FP8 && kb >= p.kb_main) {  // R-Sparse: U (dense) against A_r, first B sub-tile only
+                        int part, j;
+                        extra_block(kb - p.kb_main, p.rblk, part, j);
+                        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (PAIR_A_BYTES + 128 * 128));
+                        const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
+                        tma_load_2d_pair(sA + stage * PAIR_A_BYTES, &tmU, bar, j * 64, arow + part * p.T);
+                        tma_load_2d_pair(sB + stage * PAIR_B_BYTES, &tmR, bar, j * 64, brow);
+                        if (++stage == S) { stage = 0; phase ^= 1; }
+                        continue;
+                    }
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
                     const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
                     // second pass over K: the residual operand, same positions and W blocks
@@ -440,6 +477,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     tc_fence_after();
                     const uint32_t b_addr = smem_u32(sB + stage * PAIR_B_BYTES);
                     const uint64_t a_desc = sdesc_kmajor_sw128(smem_u32(sA + stage * PAIR_A_BYTES));
+                    if (!FP8 && kb >= p.kb_main) {  // R-Sparse block: dense MMAs into the same accumulator
+                        const uint64_t b_desc = sdesc_kmajor_sw128(b_addr);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_bf16_pair(tmem, a_desc + (uint64_t)((32 * j) >> 4), b_desc + (uint64_t)((32 * j) >> 4),
+                                          idesc_bf16(PAIR_BM, PAIR_BN, false), 1u);
+                        tc_commit_pair_mc(&empty[stage], 0x3);
+                        if (++stage == S) { stage = 0; phase ^= 1; }
+                        continue;
+                    }
                     const uint32_t e_tmem = meta_tmem + stage * C::META_COLS;
                     tmem_cp_128x128b_pair(e_tmem, sdesc_rows16(smem_u32(sM + stage * PAIR_M_BYTES)));
                     if constexpr (FP8)
@@ -568,7 +615,8 @@ constexpr size_t dense_pair_smem_bytes() { return 1024 + (size_t)DP_STAGES * DP_
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     k_gemm_dense_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmA2, GemmParams p)
+                      const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmU,
+                      const __grid_constant__ CUtensorMap tmR, GemmParams p)
 {
     constexpr int S = DP_STAGES;
     extern __shared__ unsigned char smem_raw[];
@@ -626,6 +674,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *(volatile int *)abort_flag = 1; break; }
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * DP_STAGE_BYTES);
                     const uint32_t bar = mapa_u32(smem_u32(&full[stage]), 0);
+                    if (kb >= p.kb_main) {  // R-Sparse: U against A_r
+                        int part, j;
+                        extra_block(kb - p.kb_main, p.rblk, part, j);
+                        tma_load_2d_pair(sA + stage * DP_A_BYTES, &tmU, bar, j * 64, arow + part * p.T);
+                        tma_load_2d_pair(sB + stage * DP_B_BYTES, &tmR, bar, j * 64, brow);
+                        if (++stage == S) { stage = 0; phase ^= 1; }
+                        continue;
+                    }
                     // second pass over K: the residual operand against the same W blocks
                     const bool lo = kb >= p.kb_pass;
                     const int kk = lo ? kb - p.kb_pass : kb;
@@ -826,6 +882,10 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     if (!make_map(&mA, a.A, (uint64_t)a.T, ka, GEMM_BM)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, C::BN)) return cudaErrorInvalidValue;
     if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, ka, GEMM_BM)) return cudaErrorInvalidValue;
+    CUtensorMap mU = mA, mR = mB;
+    if (a.r > 0 && (!make_map(&mU, a.U2, 2 * (uint64_t)a.T, (uint64_t)a.r, GEMM_BM) ||
+                    !make_map(&mR, a.Ar, (uint64_t)a.n_out, (uint64_t)a.r, C::BN)))
+        return cudaErrorInvalidValue;
     GemmParams p{};
     p.meta = a.meta;
     p.rowsum = a.rowsum;
@@ -840,14 +900,16 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     p.m_tiles = (a.T + GEMM_BM - 1) / GEMM_BM;
     p.n_tiles = (a.n_out + C::BN - 1) / C::BN;
     p.kb_pass = (a.K + C::KB - 1) / C::KB;
-    p.k_blocks = p.kb_pass * (a.A_lo ? 2 : 1);
+    p.kb_main = p.kb_pass * (a.A_lo ? 2 : 1);
+    p.rblk = a.r / 64;
+    p.k_blocks = p.kb_main + 2 * p.rblk;
     p.meta_kt = (a.K + 127) / 128;
     const size_t smem = gemm_smem_bytes<SPARSE>();
     cudaError_t e = cudaFuncSetAttribute(k_gemm<SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = std::min(tiles, sm_count());
-    k_gemm<SPARSE><<<grid, GEMM_THREADS, smem, st>>>(mA, mB, mA2, p);
+    k_gemm<SPARSE><<<grid, GEMM_THREADS, smem, st>>>(mA, mB, mA2, mU, mR, p);
     return cudaGetLastError();
 }
 
@@ -924,12 +986,18 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     p.m_tiles = mt128 / 2;
     p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
     p.kb_pass = (a.K + 127) / 128;
-    p.k_blocks = p.kb_pass * (a.A_lo ? 2 : 1);
+    p.kb_main = p.kb_pass * (a.A_lo ? 2 : 1);
+    p.rblk = a.r / 64;
+    p.k_blocks = p.kb_main + 2 * p.rblk;
     p.meta_kt = (a.K + 127) / 128;
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map_meta(&mE, a.meta, (uint64_t)mt128 * p.meta_kt)) return cudaErrorInvalidValue;
+    CUtensorMap mU = mA, mR = mB;
+    if (a.r > 0 && (!make_map(&mU, a.U2, 2 * (uint64_t)a.T, (uint64_t)a.r, 128) ||
+                    !make_map(&mR, a.Ar, (uint64_t)a.n_out, (uint64_t)a.r, 128)))
+        return cudaErrorInvalidValue;
     const size_t smem = pair_smem_bytes<false>();
     cudaError_t e = cudaFuncSetAttribute(k_gemm_sp_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -937,7 +1005,7 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_sp_pair<false><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, mA2, p);
+    k_gemm_sp_pair<false><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, mA2, mU, mR, p);
     return cudaGetLastError();
 }
 
@@ -957,16 +1025,22 @@ static cudaError_t launch_gemm_dense_pair(const GemmArgs &a, cudaStream_t st)
     p.m_tiles = mt128 / 2;
     p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
     p.kb_pass = (a.K + 63) / 64;
-    p.k_blocks = p.kb_pass * (a.A_lo ? 2 : 1);
+    p.kb_main = p.kb_pass * (a.A_lo ? 2 : 1);
+    p.rblk = a.r / 64;
+    p.k_blocks = p.kb_main + 2 * p.rblk;
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
+    CUtensorMap mU = mA, mR = mB;
+    if (a.r > 0 && (!make_map(&mU, a.U2, 2 * (uint64_t)a.T, (uint64_t)a.r, 128) ||
+                    !make_map(&mR, a.Ar, (uint64_t)a.n_out, (uint64_t)a.r, 128)))
+        return cudaErrorInvalidValue;
     const size_t smem = dense_pair_smem_bytes();
     const int clusters = dense_pair_clusters(smem);
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_dense_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mA2, p);
+    k_gemm_dense_pair<<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mA2, mU, mR, p);
     return cudaGetLastError();
 }
 
@@ -989,6 +1063,8 @@ cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st)
     p.n_tiles = (a.n_out + PAIR_BN - 1) / PAIR_BN;
     p.k_blocks = (a.K + 255) / 256;
     p.kb_pass = p.k_blocks;
+    p.kb_main = p.k_blocks;
+    p.rblk = 0;
     p.meta_kt = p.k_blocks;
     if (!make_map_u8(&mA, a.x8, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map_u8(&mB, a.Wq, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
@@ -1000,7 +1076,7 @@ cudaError_t launch_gemm_fp8(const Fp8GemmArgs &a, cudaStream_t st)
     if (clusters <= 0) return cudaErrorNotSupported;
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = 2 * std::min(tiles, clusters);
-    k_gemm_sp_pair<true><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, mA, p);
+    k_gemm_sp_pair<true><<<grid, PAIR_THREADS, smem, st>>>(mA, mB, mE, mA, mA, mB, p);
     return cudaGetLastError();
 }
 

@@ -68,6 +68,8 @@ struct DecodePlan {
     size_t partial_bytes, counter_bytes, eta_bytes, smem_bytes;
 };
 DecodePlan decode_plan(int T, int K, int n_out, int bf16);
+// Whether a decode call runs a separate selection kernel first.
+bool decode_needs_select(int T, int K, int n_out, int bf16, int out_bf16, int sel);
 int decode_launch_count(const DecodeArgs &a, const DecodePlan &p);
 // True when a bf16 decode of this token pad and selection is one fused launch.
 bool decode_fused(int tpad, int sel, int K);
@@ -85,7 +87,20 @@ struct GemmArgs {
     void *y;
     int out_bf16;
     const float *addend = nullptr;  // float32 [T, n_out] added to the accumulator (2:4 only)
+    // R-Sparse compensation: U2 bf16 [2T, r] (U hi rows, then U lo rows) and
+    // A_r bf16 [n_out, r], run as 2 r/64 extra K blocks after the main ones
+    const void *U2 = nullptr;
+    const void *Ar = nullptr;
+    int r = 0;
 };
+// R-Sparse prefill U = (xhat (.) (1 - m)) B_r (rsparse_prefill.cu)
+struct RspLayout {
+    int splits, blocks_per_split;
+    size_t part, u, bytes;
+};
+RspLayout rsp_layout(int T, int K, int r);
+cudaError_t launch_rsp_u(const void *x, const uint32_t *mask, const float *eta, const void *B, int T, int K, int r,
+                         void *ws, cudaStream_t st);
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 
 // FP8 2:4 prefill (fp8.cu, gemm.cu).

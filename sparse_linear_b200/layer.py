@@ -12,8 +12,9 @@ import torch
 from . import (AS_BF16, AS_F32, AS_MODE_24, AS_MODE_DENSE, AS_MODE_SPLIT, AS_OP_AMBER, AS_OP_DECODE,
                AS_OP_PREFILL, AS_OP_SELECT, AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SCORE_MAG, AS_SEL_ALL, AS_SEL_NM,
                as_block_sparsity, as_hybrid_dense_blocks, as_hybrid_workspace, as_linear_decode, as_linear_prefill,
-               as_linear_prefill_hybrid, as_meta24_words, as_prefill_mode, as_select, as_weight_prep,
-               as_weight_prep_amber, as_workspace_size, config, select_out)
+               as_linear_prefill_hybrid, as_linear_prefill_rsparse, as_meta24_words, as_prefill_mode,
+               as_rsparse_prefill_workspace, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size,
+               config, select_out)
 
 
 _MODE_NAMES = {AS_MODE_24: "2:4", AS_MODE_SPLIT: "split", AS_MODE_DENSE: "dense"}
@@ -178,6 +179,23 @@ class SparseLinear:
         if code == AS_MODE_24:
             return self.prefill_from(bufs, T, stream=stream), mode, s
         return self.prefill_hybrid_from(x, bufs, as_hybrid_dense_blocks(self.K, dense_frac), stream=stream), mode, s
+
+    def prefill_rsparse(self, x: torch.Tensor, B: torch.Tensor, A: torch.Tensor, stream=None):
+        """Selection + prefill with the R-Sparse compensation of the dropped
+        channels (overview page, section 3.3): B [K, r], A [n_out, r] bf16
+        factors of W, r in {64, 128}.  Returns (y, bufs)."""
+        T = x.shape[0]
+        bufs = self.select_buffers(T, x.device)
+        self.select(x, bufs, stream=stream)
+        key = ("rsparse", T, A.shape[1])
+        if key not in self._ws:
+            self._ws[key] = workspace(as_rsparse_prefill_workspace(T, self.K, A.shape[1]), x.device)
+        y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=x.device)
+        sel = select_out(**{k: v for k, v in bufs.items()
+                            if k in ("bitmask", "x_masked", "x_compact", "meta24", "x_masked_lo", "x_compact_lo")})
+        as_linear_prefill_rsparse(sel, x, self.W, self.cfg, y, B, A, rowsum=self.rowsum, eta=bufs.get("eta"),
+                                  workspace=self._ws[key], stream=stream)
+        return y, bufs
 
     def prefill(self, x: torch.Tensor, running_var=None, first_batch: bool = False, stream=None):
         bufs = self.select_buffers(x.shape[0], x.device)

@@ -311,3 +311,32 @@ def test_noalloc_refusals_enqueue_nothing(lib):
     assert call(x=fake + 4) == lib.AS_ERR_ALIGN
     assert call(mask=fake + 8) == lib.AS_ERR_ALIGN
     assert call(T=16, K=11008, n_out=16384, cfg=lib.config(sel=lib.AS_SEL_NM, n=8, m=16)) == lib.AS_ERR_WORKSPACE
+
+
+def test_rsparse_prefill_validation_launches_nothing(lib):
+    fake = 1 << 20
+    f = lib._lib.as_linear_prefill_rsparse
+    assert lib.as_rsparse_prefill_workspace(4096, 14336, 64) > 4096 * 64 * 2 * 2
+    for r in (0, 32, 96, 256):
+        with pytest.raises(lib.ASError):
+            lib.as_rsparse_prefill_workspace(16, 1024, r)
+    sel = lib.as_select_out()
+    sel.bitmask = fake
+    sel.x_compact = fake
+    sel.meta24 = fake
+    cfg = lib.config(sel=lib.AS_SEL_NM, n=2, m=4)
+    ws = lib.as_rsparse_prefill_workspace(16, 1024, 64)
+
+    def call(s=sel, x=fake, r=64, c=cfg, B=fake, wb=ws, T=16):
+        return f(ctypes.byref(s), x, fake, T, 1024, 64, None, None, ctypes.byref(c), r, B, fake, fake, fake, wb, None)
+
+    assert call(r=32) == lib.AS_ERR_SHAPE
+    assert call(x=None) == lib.AS_ERR_INVALID_ARG
+    assert call(B=None) == lib.AS_ERR_INVALID_ARG
+    assert call(c=lib.config(var=True, sel=lib.AS_SEL_NM, n=2, m=4)) == lib.AS_ERR_UNSUPPORTED
+    assert call(B=fake + 4) == lib.AS_ERR_ALIGN
+    assert call(wb=ws - 1) == lib.AS_ERR_WORKSPACE
+    nomask = lib.as_select_out()
+    nomask.x_compact = fake
+    nomask.meta24 = fake
+    assert call(s=nomask) == lib.AS_ERR_INVALID_ARG

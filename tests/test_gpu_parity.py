@@ -216,6 +216,29 @@ def test_decode_keep_all_is_dense(sl):
     assert mask.all()
 
 
+def test_decode_plan_stable_across_calls(sl):
+    """Workspace sizes and launch counts asked for up front stay valid after
+    calls of other token counts have run (the plan must not depend on which
+    calls ran before it)."""
+    x, W, _ = synth.decode_downproj(16)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
+    from sparse_linear_b200.layer import SparseLinear, workspace
+    L = SparseLinear(dev(W), cfg, alpha=0.5)
+    Ts = (1, 8, 16, 2, 4)
+    sizes = {T: sl.as_workspace_size(sl.AS_OP_DECODE, T, 11008, 4096, cfg) for T in Ts}
+    launches = {T: sl.as_decode_launches(T, 11008, 4096, sl.AS_BF16, cfg) for T in Ts}
+    wss = {T: workspace(sizes[T], "cuda") for T in Ts}
+    xd = dev(x)
+    for _ in range(2):
+        for T in Ts:
+            y = torch.empty(T, 4096, dtype=torch.bfloat16, device="cuda")
+            sl.as_linear_decode(xd[:T], L.Wt, cfg, y, g=L.g, rowsum=L.rowsum, workspace=wss[T])
+            assert sl.as_workspace_size(sl.AS_OP_DECODE, T, 11008, 4096, cfg) == sizes[T]
+            assert sl.as_decode_launches(T, 11008, 4096, sl.AS_BF16, cfg) == launches[T]
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+
+
 def test_decode_deterministic(sl):
     x, W, _ = synth.decode_downproj(8)
     cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
@@ -639,6 +662,68 @@ def test_rsparse_decode(sl, T, K, n_out, r, dpts, svd):
     sl.as_rsparse_decode(xd, mask_d, dev(B), dev(A), y2, eta=eta_d if dpts else None, workspace=ws)
     torch.cuda.synchronize()
     assert rel_l2(f32(y2) - f32(y0), comp) <= TOL_F32
+
+
+# (T, K, n_out, r, selection, shift, out, factors): even tile counts run the
+# CTA-pair kernels, T = 300 the one-SM kernels; 2:4 runs the sparse GEMM with
+# dense R-Sparse K blocks, the others the masked dense GEMM
+@pytest.mark.parametrize("T,K,n_out,r,sel,dpts,out,svd", [
+    (256, 1024, 264, 64, "2:4", True, "f32", True),
+    (300, 1024, 264, 128, "8:16", True, "f32", True),
+    (300, 2048, 520, 64, "2:4", False, "bf16", False),
+    (512, 1024, 1024, 64, "top-k", False, "f32", True),
+    (256, 1024, 264, 128, "2:4", False, "f32", True),
+])
+def test_rsparse_prefill(sl, T, K, n_out, r, sel, dpts, out, svd):
+    """Prefill with R-Sparse: the selection bit-exact, y against the oracle's
+    pruned product plus its float64 compensation with the same bf16 factors
+    (numpy SVD of W, or random)."""
+    x, W = synth.random_layer(T, K, n_out, seed=81 + T, dist="sqrelu" if sel == "2:4" else "laplace")
+    odt = sl.AS_F32 if out == "f32" else sl.AS_BF16
+    if sel == "2:4":
+        cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, dpts=dpts, out_dtype=odt)
+    elif sel == "8:16":
+        cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=dpts, out_dtype=odt)
+    else:
+        cfg = sl.config(sel=sl.AS_SEL_TOPK, k_keep=K // 3, dpts=dpts, out_dtype=odt)
+    L = layer(sl, W, cfg, 0.5)
+    if svd:
+        A64, B64 = oracle.rsparse_factors(W, r)
+        A, B = _bf16r(A64), _bf16r(B64)
+    else:
+        rng = np.random.default_rng(83)
+        A, B = _bf16r(rng.normal(0, 0.05, (n_out, r))), _bf16r(rng.normal(0, 0.02, (K, r)))
+    y, bufs = L.prefill_rsparse(dev(x), dev(B), dev(A))
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    xf, Wf = x.float().numpy(), W.float().numpy()
+    eta32 = f32(bufs["eta"]) if dpts else None
+    f = f32(L.g) if sel == "8:16" else None
+    mask = ref_selection(sl, oracle.score(xf, eta=eta32, f=f), cfg)
+    np.testing.assert_array_equal(unpack_bitmask(bufs["bitmask"], K), mask)
+    eta64 = oracle.token_mean(xf) if dpts else None
+    _, rs = oracle.weight_prep(Wf, 1.0)
+    ref = oracle.linear(xf, mask, Wf, eta=eta64, rowsum=rs if dpts else None)
+    comp = oracle.rsparse(xf, mask, B.float().numpy(), A.float().numpy(), eta=eta64)
+    err = rel_l2(f32(y), ref + comp)
+    assert err <= (TOL_F32 if out == "f32" else TOL_BF16), err
+    if out == "f32":  # the compensation is really in y: without it the error is far larger
+        assert rel_l2(ref, ref + comp) > 20 * err
+
+
+def test_rsparse_prefill_full_rank_restores_dense(sl):
+    """Full-rank factors (r = K = 128): W = A B^T up to the factors' bf16
+    rounding, so the compensated prefill of a 2:4 selection gives the dense
+    product of the unpruned input."""
+    T, K, n_out, r = 256, 128, 256, 128
+    x, W = synth.random_layer(T, K, n_out, seed=91, dist="laplace")
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=2, m=4, out_dtype=sl.AS_F32)
+    L = layer(sl, W, cfg)
+    A64, B64 = oracle.rsparse_factors(W, r)
+    y, _ = L.prefill_rsparse(dev(x), dev(_bf16r(B64)), dev(_bf16r(A64)))
+    torch.cuda.synchronize()
+    dense = x.double().numpy() @ W.double().numpy().T
+    assert rel_l2(f32(y), dense) <= 1e-2
 
 
 def test_rsparse_keep_all_adds_nothing(sl):
