@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
 // rows are in flight while one is scored), the channel factors once per
 // CTA.  Statistics, score, selection and outputs are those of k_select.
 constexpr int SR_THREADS = 256;
-constexpr int SR_BUFS = 3;
+constexpr int SR_BUFS = 4;
 constexpr uint32_t SR_PIECE = 16384;  // bytes per bulk copy instruction
 
 __device__ __forceinline__ void bulk_load_pieces(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
@@ -379,9 +379,14 @@ __device__ __forceinline__ void bulk_load_pieces(void *dst, const void *src, uin
 }
 
 // M: block size fixed at compile time (0: from the arguments); COMPACT: the
-// 2:4 outputs (compact operand + positions; no masked copy, no VAR).
-template <typename TX, int M, bool COMPACT>
-__global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
+// 2:4 outputs (compact operand + positions; no masked copy, no VAR).  FREG:
+// the channel factors stay in registers (a thread scores the same channels
+// of every row; at most SR_FREG_TILES tiles), freeing their shared memory for
+// more CTAs per SM.
+constexpr int SR_FREG_TILES = 4;
+
+template <typename TX, int M, bool COMPACT, bool FREG>
+__global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(SelectArgs a)
 {
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ double red[2][SR_THREADS / 32];
@@ -390,7 +395,17 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
     const int ngroups = K >> 3, ntiles = (ngroups + SR_THREADS - 1) / SR_THREADS, kt = (K + 127) >> 7;
     const int Tpad = a.meta24 ? (T + 127) / 128 * 128 : T;
     const bool has_f = a.f != nullptr;
-    const uint32_t fbytes = has_f ? (uint32_t)K * 4u : 0u, rowbytes = (uint32_t)K * (uint32_t)sizeof(TX);
+    const uint32_t fbytes = (has_f && !FREG) ? (uint32_t)K * 4u : 0u, rowbytes = (uint32_t)K * (uint32_t)sizeof(TX);
+    float fr[FREG ? SR_FREG_TILES : 1][8];
+    if constexpr (FREG) {
+#pragma unroll
+        for (int tile = 0; tile < SR_FREG_TILES; ++tile) {
+            const int g = tile * SR_THREADS + tid;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) fr[tile][e] = 1.0f;
+            if (g < ngroups) load8f(a.f + 8 * g, fr[tile]);
+        }
+    }
     float *sf = reinterpret_cast<float *>(sm);
     TX *rows = reinterpret_cast<TX *>(sm + fbytes);
     const TX *x = static_cast<const TX *>(a.x);
@@ -402,7 +417,7 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
     }
     __syncthreads();
     if (tid == 0) {
-        if (has_f) {
+        if (fbytes) {
             mbar_arrive_expect_tx(&bars[SR_BUFS], fbytes);
             bulk_load_pieces(sf, a.f, fbytes, &bars[SR_BUFS]);
         }
@@ -414,7 +429,7 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
             }
         }
     }
-    if (has_f && !mbar_wait(&bars[SR_BUFS], 0)) return;
+    if (fbytes && !mbar_wait(&bars[SR_BUFS], 0)) return;
 
     int it = 0;
     for (int t = blockIdx.x; t < Tpad; t += gridDim.x, ++it) {
@@ -510,16 +525,15 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
             }
         }
         double skm = 0.0, skmm = 0.0;
-        for (int tile = 0; tile < ntiles; ++tile) {
+        // one tile of 8 channels per thread; fv: the tile's channel factors
+        auto tile_step = [&](int tile, const float (&fvin)[8]) {
             const int g = tile * SR_THREADS + tid, c0 = 8 * g;
             const bool act = g < ngroups;
-            if constexpr (COMPACT) {
-                if (plain) break;  // done by the 16-channel loop above
-            }
             float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, fv[8] = {1, 1, 1, 1, 1, 1, 1, 1}, xh[8], sc[8];
             if (act) {
                 load8(xr + c0, v);
-                if (has_f) load8f(sf + c0, fv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) fv[e] = fvin[e];
             }
             score8v(v, a.dpts, eta, act && has_f, fv, xh, sc);
             uint32_t keep;
@@ -528,7 +542,8 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                 keep = a.sel == AS_SEL_NM       ? nm_keep_dispatch(sc, lane, a.n, a.m)
                        : a.sel == AS_SEL_THRESH ? keep_thresh(sc, a.tau)
                                                 : 0xFFu;
-            else if constexpr (M >= 8) keep = nm_keep_sorted<M>(sc, lane, a.n);
+            else if constexpr (M >= 16) keep = 2 * a.n == M ? nm_keep_half<M>(sc, lane, a.n) : nm_keep_sorted<M>(sc, lane, a.n);
+            else if constexpr (M == 8) keep = nm_keep_sorted<M>(sc, lane, a.n);
             else keep = nm_keep<M>(sc, lane, a.n);
             if (act) {
                 if (a.bitmask) {
@@ -573,6 +588,17 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
                     mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
                 }
             }
+        };
+        if constexpr (FREG) {
+#pragma unroll
+            for (int tile = 0; tile < SR_FREG_TILES; ++tile)
+                if (tile < ntiles) tile_step(tile, fr[tile]);  // compile-time index: fr stays in registers
+        } else if (!(COMPACT && plain)) {  // the plain 2:4 case was done by the 16-channel loop above
+            for (int tile = 0; tile < ntiles; ++tile) {
+                float fv[8] = {1, 1, 1, 1, 1, 1, 1, 1};
+                if (has_f && tile * SR_THREADS + tid < ngroups) load8f(sf + 8 * (tile * SR_THREADS + tid), fv);
+                tile_step(tile, fv);
+            }
         }
         if (a.meta24 && tid < 16 * kt - ngroups)  // channel padding of the last 128-channel tile
             *meta_byte(a.meta24, t, 8 * (ngroups + tid), kt) = 0x44;
@@ -605,57 +631,133 @@ __global__ void __launch_bounds__(SR_THREADS) k_select_rows(SelectArgs a)
 }
 
 // ---------------------------------------------------------------- CLACT
-// partial[s][i] = sum over rows [s*rows_per, ...) of x[t, i]^2; a thread
-// owns 8 consecutive channels (16-byte loads), rows unrolled by 8.
-template <typename TX>
-__global__ void __launch_bounds__(128) k_colsq_rows(const TX *__restrict__ x, int T, int K, int rows_per,
-                                                    double *__restrict__ part)
+// Column energy c_j = sqrt(sum_t x_tj^2) over the T rows.
+// k_colsq_ring: persistent, one CTA per SM; CTA b takes rows b, b + G, ...
+// of a window of up to CN_WIN channels.  Whole rows of the window arrive in
+// shared memory by 1-D bulk copies (a ring of CN_BUFS rows, 192 KB, the next
+// rows in flight while one is summed); thread i keeps the float64 sums of channels
+// 8i .. 8i+7, 8i+2048 .. and so on in registers and writes them as the CTA's
+// partial [b][K] at the end.  k_colnorm_final sums the G partials of a
+// channel in a fixed order (8 threads per channel, then a fixed shuffle
+// tree), so c is deterministic.
+constexpr int CN_THREADS = 256;
+constexpr int CN_WIN = 8 * 4 * CN_THREADS;  // 8192 channels: 4 groups of 8 per thread
+constexpr int CN_BUFS_BF16 = 12;  // 192 KB of 16 KB rows in flight per SM
+constexpr int CN_BUFS_F32 = 6;    // 192 KB of 32 KB rows
+
+template <typename TX, int CN_BUFS>
+__global__ void __launch_bounds__(CN_THREADS) k_colsq_ring(const TX *__restrict__ x, int T, int K,
+                                                           double *__restrict__ part)
 {
-    const int i8 = blockIdx.x * blockDim.x + threadIdx.x, s = blockIdx.y;
-    if (8 * i8 >= K) return;
-    const int t0 = s * rows_per, t1 = min(T, t0 + rows_per);
-    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int tb = t0; tb < t1; tb += 8) {
-        float v[8][8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-            if (tb + r < t1) load8(x + (size_t)(tb + r) * K + 8 * i8, v[r]);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-            if (tb + r < t1)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] += (double)v[r][e] * (double)v[r][e];
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ __align__(8) uint64_t bars[CN_BUFS];
+    const int tid = threadIdx.x;
+    const int c_lo = blockIdx.y * CN_WIN, nwin = min(CN_WIN, K - c_lo);  // nwin % 8 == 0
+    const uint32_t rowbytes = (uint32_t)nwin * (uint32_t)sizeof(TX);
+    TX *rows = reinterpret_cast<TX *>(sm);
+    if (tid == 0) {
+        for (int b = 0; b < CN_BUFS; ++b) mbar_init(&bars[b], 1);
+        fence_mbar_init();
     }
+    __syncthreads();
+    if (tid == 0)
+        for (int b = 0; b < CN_BUFS; ++b) {
+            const int t = blockIdx.x + b * gridDim.x;
+            if (t < T) {
+                mbar_arrive_expect_tx(&bars[b], rowbytes);
+                bulk_load_pieces(rows + (size_t)b * CN_WIN, x + (size_t)t * K + c_lo, rowbytes, &bars[b]);
+            }
+        }
+    double acc[4][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[(size_t)s * K + 8 * i8 + e] = acc[e];
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[q][e] = 0.0;
+    int it = 0;
+    for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
+        const int buf = it % CN_BUFS;
+        if (!mbar_wait(&bars[buf], (uint32_t)(it / CN_BUFS) & 1u)) break;
+        const TX *xr = rows + (size_t)buf * CN_WIN;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int c0 = 8 * (tid + q * CN_THREADS);
+            if (c0 < nwin) {
+                float v[8];
+                load8(xr + c0, v);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[q][e] += (double)v[e] * (double)v[e];
+            }
+        }
+        __syncthreads();  // every thread is done with the buffer: the row CN_BUFS ahead goes into it
+        if (tid == 0) {
+            const int tn = t + CN_BUFS * gridDim.x;
+            if (tn < T) {
+                mbar_arrive_expect_tx(&bars[buf], rowbytes);
+                bulk_load_pieces(rows + (size_t)buf * CN_WIN, x + (size_t)tn * K + c_lo, rowbytes, &bars[buf]);
+            }
+        }
+    }
+    double *pr = part + (size_t)blockIdx.x * K + c_lo;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int c0 = 8 * (tid + q * CN_THREADS);
+        if (c0 < nwin)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pr[c0 + e] = acc[q][e];
+    }
 }
 
-__global__ void k_colnorm_final(const double *__restrict__ part, int slabs, int K, float *__restrict__ c)
+// c[i] = sqrt(sum over the G partials), 8 threads per channel: thread k of
+// a channel sums partials k, k + 8, ... in order, then a fixed shuffle tree.
+__global__ void k_colnorm_final(const double *__restrict__ part, int G, int K, float *__restrict__ c)
 {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= K) return;
+    const int gi = blockIdx.x * blockDim.x + threadIdx.x;
+    const int i = gi >> 3, k = gi & 7;
     double s = 0.0;
-    for (int j = 0; j < slabs; ++j) s += part[(size_t)j * K + i];
-    c[i] = (float)sqrt(s);
+    if (i < K)
+        for (int j = k; j < G; j += 8) s += part[(size_t)j * K + i];
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    if (i < K && k == 0) c[i] = (float)sqrt(s);
 }
 
-static int colnorm_slabs(int T) { return (T + 127) / 128; }
+static int colnorm_ctas(int T)
+{
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    return T < sms ? (T > 0 ? T : 1) : sms;
+}
 
 size_t colnorm_workspace(int T, int K)
 {
-    return (size_t)colnorm_slabs(T) * (size_t)K * sizeof(double) + (size_t)K * sizeof(float);
+    return (size_t)colnorm_ctas(T) * (size_t)K * sizeof(double) + (size_t)K * sizeof(float);
 }
 
 cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void *ws, cudaStream_t st)
 {
-    const int slabs = colnorm_slabs(T);
+    const int G = colnorm_ctas(T);
     double *part = static_cast<double *>(ws);
-    dim3 grid((K / 8 + 127) / 128, slabs);  // K % 8 == 0
-    if (bf16)
-        k_colsq_rows<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), T, K, 128, part);
-    else
-        k_colsq_rows<float><<<grid, 128, 0, st>>>(static_cast<const float *>(x), T, K, 128, part);
-    k_colnorm_final<<<(K + 255) / 256, 256, 0, st>>>(part, slabs, K, c);
+    dim3 grid(G, (K + CN_WIN - 1) / CN_WIN);  // K % 8 == 0
+    cudaError_t e;
+    if (bf16) {
+        const size_t smem = (size_t)CN_BUFS_BF16 * CN_WIN * 2;
+        static int done[64];
+        e = smem_limit_once(k_colsq_ring<__nv_bfloat16, CN_BUFS_BF16>, smem, done);
+        if (e == cudaSuccess)
+            k_colsq_ring<__nv_bfloat16, CN_BUFS_BF16><<<grid, CN_THREADS, smem, st>>>(
+                static_cast<const __nv_bfloat16 *>(x), T, K, part);
+    } else {
+        const size_t smem = (size_t)CN_BUFS_F32 * CN_WIN * 4;
+        static int done[64];
+        e = smem_limit_once(k_colsq_ring<float, CN_BUFS_F32>, smem, done);
+        if (e == cudaSuccess)
+            k_colsq_ring<float, CN_BUFS_F32><<<grid, CN_THREADS, smem, st>>>(static_cast<const float *>(x), T, K, part);
+    }
+    if (e != cudaSuccess) return e;
+    const long long threads = (long long)K * 8;
+    k_colnorm_final<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(part, G, K, c);
     return cudaGetLastError();
 }
 
@@ -671,23 +773,33 @@ static cudaError_t launch_select_t(const SelectArgs &a, size_t smem, int grid, c
     return cudaGetLastError();
 }
 
-template <typename TX, int M, bool COMPACT>
-static cudaError_t launch_select_rows_t(const SelectArgs &a, cudaStream_t st)
+template <typename TX, int M, bool COMPACT, bool FREG>
+static cudaError_t launch_select_rows_f(const SelectArgs &a, cudaStream_t st)
 {
-    const size_t smem = (a.f ? (size_t)a.K * 4 : 0) + (size_t)SR_BUFS * a.K * sizeof(TX);
+    const size_t smem = ((a.f && !FREG) ? (size_t)a.K * 4 : 0) + (size_t)SR_BUFS * a.K * sizeof(TX);
     static int done[64];
-    cudaError_t e = smem_limit_once(k_select_rows<TX, M, COMPACT>, smem, done);
+    cudaError_t e = smem_limit_once(k_select_rows<TX, M, COMPACT, FREG>, smem, done);
     if (e != cudaSuccess) return e;
     int per_sm = 0, dev = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_select_rows<TX, M, COMPACT>, SR_THREADS, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_select_rows<TX, M, COMPACT, FREG>, SR_THREADS, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int rows = a.meta24 ? (a.T + 127) / 128 * 128 : a.T;
     const int grid = std::min(rows, per_sm * sms);
-    k_select_rows<TX, M, COMPACT><<<grid, SR_THREADS, smem, st>>>(a);
+    k_select_rows<TX, M, COMPACT, FREG><<<grid, SR_THREADS, smem, st>>>(a);
     return cudaGetLastError();
+}
+
+// Channel factors in registers when every thread scores at most
+// SR_FREG_TILES tiles of 8 channels (K <= 8192).
+template <typename TX, int M, bool COMPACT>
+static cudaError_t launch_select_rows_t(const SelectArgs &a, cudaStream_t st)
+{
+    const int ntiles = (a.K / 8 + SR_THREADS - 1) / SR_THREADS;
+    if (!COMPACT && a.f && ntiles <= SR_FREG_TILES) return launch_select_rows_f<TX, M, COMPACT, true>(a, st);
+    return launch_select_rows_f<TX, M, COMPACT, false>(a, st);
 }
 
 template <typename TX>

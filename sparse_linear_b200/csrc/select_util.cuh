@@ -188,6 +188,108 @@ __device__ __forceinline__ uint32_t nm_keep_sorted(const float (&s)[8], int lane
     return keep;
 }
 
+// The n = M/2 -th largest score of the M-block (M = 16 or 32; the block's
+// M/8 consecutive lanes hold 8 scores each), without a full sort:
+//   1. each lane sorts its 8 scores (descending bitonic network);
+//   2. M = 32: lanes q, q^1 merge into one sorted 16-list (half-cleaner on
+//      A ++ reverse(B), then a bitonic merge in each lane; the even lane
+//      holds ranks 0..7, the odd lane 8..15);
+//   3. the n largest of two sorted lists A, B (n = M/2 each) are
+//      {max(A[i], B[n-1-i])} (half-cleaner of a bitonic sequence), so their
+//      minimum is the n-th largest of the block.
+// Every lane of the block gets the same value.  All 32 lanes must call.
+__device__ __forceinline__ void sort8_desc(float (&v)[8])
+{
+#pragma unroll
+    for (int size = 2; size <= 8; size <<= 1)
+#pragma unroll
+        for (int d = size >> 1; d > 0; d >>= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if ((e & d) == 0) {
+                    const float hi = fmaxf(v[e], v[e | d]), lo = fminf(v[e], v[e | d]);
+                    const bool desc = (e & size) == 0;
+                    v[e] = desc ? hi : lo;
+                    v[e | d] = desc ? lo : hi;
+                }
+}
+
+template <int M>
+__device__ __forceinline__ float theta_half(const float (&s)[8], int lane)
+{
+    static_assert(M == 16 || M == 32, "theta_half: M = 16 or 32");
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = s[e];
+    sort8_desc(v);
+    if constexpr (M == 32) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p[e] = __shfl_xor_sync(0xffffffffu, v[7 - e], 1);
+        const bool upper = (lane & 1) == 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = upper ? fmaxf(v[e], p[e]) : fminf(v[e], p[e]);
+#pragma unroll
+        for (int d = 4; d > 0; d >>= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if ((e & d) == 0) {
+                    const float hi = fmaxf(v[e], v[e | d]), lo = fminf(v[e], v[e | d]);
+                    v[e] = hi;
+                    v[e | d] = lo;
+                }
+    }
+    constexpr int partner = M == 32 ? 3 : 1;  // the lane holding the reversed ranks of the other list
+    float mn = __int_as_float(0x7f800000);      // +inf
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mn = fminf(mn, fmaxf(v[e], __shfl_xor_sync(0xffffffffu, v[7 - e], partner)));
+    if constexpr (M == 32) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+    return mn;
+}
+
+// Exactly n of every M-block kept (rank < n for "higher score first, equal
+// scores by lower index") from the block's n-th largest score theta: every
+// score > theta, and of the scores == theta the lowest-indexed ones until n.
+template <int M>
+__device__ __forceinline__ uint32_t keep_from_theta(const float (&s)[8], int lane, int n, float th)
+{
+    constexpr int G = M / 8;  // lanes per block
+    const int q = lane & (G - 1);
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        gt |= (uint32_t)(s[e] > th) << e;
+        eq |= (uint32_t)(s[e] == th) << e;
+    }
+    const int neq = __popc(eq);
+    int ngt = __popc(gt), inc = neq;
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) {
+        const int up = __shfl_up_sync(0xffffffffu, inc, o);
+        if (q >= o) inc += up;
+    }
+    int before = inc - neq;  // equal scores in the lower lanes of the block
+    const int room = n - ngt;  // equal scores that still fit
+    uint32_t keep = gt;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        if ((eq >> e) & 1u) {
+            keep |= (uint32_t)(before < room) << e;
+            ++before;
+        }
+    }
+    return keep;
+}
+
+// n = M/2 selection through theta_half (M = 16, 32).
+template <int M>
+__device__ __forceinline__ uint32_t nm_keep_half(const float (&s)[8], int lane, int n)
+{
+    return keep_from_theta<M>(s, lane, n, theta_half<M>(s, lane));
+}
+
 // 2:4 blocks inside the lane: one comparison per pair of the block decides
 // for both (j ahead of i: s_j > s_i, or s_j == s_i and j < i).  S is float
 // (scores) or uint32_t (bf16 magnitude bits, which order like the values).
@@ -233,8 +335,8 @@ __device__ __forceinline__ uint32_t nm_keep_dispatch(const float (&s)[8], int la
     case 2: return nm_keep<2>(s, lane, n);
     case 4: return n == 2 ? keep_2of4(s) : nm_keep<4>(s, lane, n);
     case 8: return nm_keep_sorted<8>(s, lane, n);
-    case 16: return nm_keep_sorted<16>(s, lane, n);
-    default: return nm_keep_sorted<32>(s, lane, n);
+    case 16: return n == 8 ? nm_keep_half<16>(s, lane, n) : nm_keep_sorted<16>(s, lane, n);
+    default: return n == 16 ? nm_keep_half<32>(s, lane, n) : nm_keep_sorted<32>(s, lane, n);
     }
 }
 
