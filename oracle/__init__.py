@@ -26,8 +26,9 @@ Functions and the passages they follow (page title, section):
   (``token_mean``) or a calibrated table.
 * ``var_scale``     overview §3.2.
 * ``linear``        overview §3.1 / §3.2 and the layer definition y = prune(x) W^T.
-* ``block_nnz``, ``pick_dense``, ``hybrid_mode``, ``hybrid_mask``  2:4 +
-                    Squared-ReLU page §3.2-3.3 (sparse/dense split, mode switch).
+* ``block_nnz``, ``pick_dense``, ``hybrid_mode``, ``hybrid_mask``, ``nm_split``
+                    2:4 + Squared-ReLU page §3.2-3.3 (sparse/dense split of a
+                    2:4 activation and of an N:M selection, mode switch).
 * ``rsparse``, ``rsparse_factors``  overview §3.3 (R-Sparse low-rank compensation;
                     the factors from a truncated SVD, numpy's).
 * ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
@@ -375,6 +376,48 @@ def hybrid_mode(sparsity: float) -> str:
     if sparsity >= 0.90:
         return "split"
     return "dense"
+
+
+def nm_split(s, mask_nm, xm, n_dense: int):
+    """The hybrid 2:4 decomposition of an N:M selection (2:4 + Squared-ReLU
+    page §3.2, the sparse/dense feature split, applied to an N:M selection;
+    §3.3 for the mode).  Readings:
+    * the 2:4-compliant part takes, in every 4-channel block, the two
+      channels ranked first by (kept by the N:M selection, then higher
+      float32 score, then lower index); a block with fewer than two kept
+      channels fills its positions with the lowest-indexed dropped ones,
+      whose values are zero (``pos``, exactly 2 per block);
+    * ``part`` = the kept channels inside the 2:4 part;
+    * the dense blocks D are the n_dense blocks with the most nonzeros of
+      the masked activation xm = xhat * mask over the tokens (ties to the
+      lower block index), as in ``hybrid_mask``;
+    * the split keeps ``part`` plus every kept channel of D:
+      m_split = part | (mask_nm & D); with D covering every block whose
+      kept channels do not fit 2:4, m_split equals mask_nm.
+    s, mask_nm, xm: [T, k]; returns dict(pos, part, idx, m_split, sparsity)."""
+    s = np.asarray(s, np.float32)
+    kept = np.asarray(mask_nm, np.uint8).astype(bool)
+    T, k = s.shape
+    sb = s.reshape(T, k // 4, 4)
+    kb = kept.reshape(T, k // 4, 4)
+    rank = np.zeros((T, k // 4, 4), np.int64)
+    for i in range(4):
+        for j in range(4):
+            if i == j:
+                continue
+            beats = (kb[..., j] & ~kb[..., i]) | ((kb[..., j] == kb[..., i]) &
+                                                  ((sb[..., j] > sb[..., i]) | ((sb[..., j] == sb[..., i]) & (j < i))))
+            rank[..., i] += beats
+    pos = (rank < 2).reshape(T, k)
+    part = pos & kept
+    nnz, total = block_nnz(np.asarray(xm, np.float32))
+    idx = pick_dense(nnz, n_dense)
+    dense = np.zeros(k, bool)
+    for b in idx:
+        dense[4 * b:4 * b + 4] = True
+    m_split = part | (kept & dense[None, :])
+    return dict(pos=pos.astype(np.uint8), part=part.astype(np.uint8), idx=idx,
+                m_split=m_split.astype(np.uint8), sparsity=1.0 - total / float(T * k))
 
 
 def hybrid_mask(x, n_dense: int):

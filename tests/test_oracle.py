@@ -700,3 +700,68 @@ def test_hybrid_recovers_dropped_nonzeros_of_dense_blocks(oracle_lib):
             assert not lost[:, 4 * b:4 * b + 4].any()
     assert dropped[0] > 0 and all(a >= b for a, b in zip(dropped, dropped[1:])) and dropped[-1] == 0
     np.testing.assert_allclose(oracle_lib.linear(xf, mask, Wf), dense, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- hybrid split of an N:M selection
+def test_nm_split_worked_blocks(oracle_lib):
+    """Hand-worked 4-blocks (2:4 + Squared-ReLU page §3.2 reading): the two
+    kept channels with the highest scores form the 2:4 part, ties to the
+    lower index; a block with one kept channel pads with the lowest dropped
+    one."""
+    s = np.array([[5, 3, 4, 9, 2, 2, 2, 2, 0, 0, 7, 0, 1, 8, 6, 3]], np.float32)
+    m = np.array([[1, 1, 1, 0, 0, 1, 1, 1, 0, 0, 1, 0, 1, 1, 1, 1]], np.uint8)
+    r = oracle_lib.nm_split(s, m, s * m, 0)
+    assert r["part"].tolist() == [[1, 0, 1, 0, 0, 1, 1, 0, 0, 0, 1, 0, 0, 1, 1, 0]]
+    assert r["pos"].tolist() == [[1, 0, 1, 0, 0, 1, 1, 0, 1, 0, 1, 0, 0, 1, 1, 0]]
+    assert r["m_split"].tolist() == r["part"].tolist()  # no dense block
+
+
+def test_nm_split_invariants_and_extremes(oracle_lib):
+    """On random 8:16 and 16:32 selections: positions exactly 2 per block,
+    part within the selection, top-2 property per block; every block dense
+    gives back the N:M selection; a selection that already fits 2:4 is its
+    own 2:4 part for any number of dense blocks."""
+    rng = np.random.default_rng(7)
+    for n, m in ((8, 16), (16, 32)):
+        x = rng.laplace(0, 0.3, size=(6, 128)).astype(np.float32)
+        s = oracle_lib.score(x)
+        mask = oracle_lib.select_nm(s, n, m)
+        r = oracle_lib.nm_split(s, mask, x * mask, 0)
+        pos, part = r["pos"].reshape(6, 32, 4), r["part"].reshape(6, 32, 4)
+        assert (pos.sum(-1) == 2).all()
+        assert ((part == 1) <= (mask.reshape(6, 32, 4) == 1)).all()
+        kb = mask.reshape(6, 32, 4).astype(bool)
+        assert (part.sum(-1) == np.minimum(kb.sum(-1), 2)).all()
+        sb = s.reshape(6, 32, 4)
+        over = kb & ~part.astype(bool)
+        lo = np.where(part.astype(bool), sb, np.inf).min(-1)
+        hi = np.where(over, sb, -np.inf).max(-1)
+        assert (lo >= hi).all()
+        full = oracle_lib.nm_split(s, mask, x * mask, 32)
+        np.testing.assert_array_equal(full["m_split"], mask)
+    # a 2:4 selection viewed as 8:16: already 2:4-compliant
+    x = rng.laplace(0, 0.3, size=(5, 64)).astype(np.float32)
+    s = oracle_lib.score(x)
+    m24 = oracle_lib.select_nm(s, 2, 4)
+    for nd in (0, 4, 16):
+        np.testing.assert_array_equal(oracle_lib.nm_split(s, m24, x * m24, nd)["m_split"], m24)
+
+
+def test_nm_split_exact_when_dense_blocks_cover_the_overflow(oracle_lib):
+    """The split product equals the N:M product when the dense blocks cover
+    every block whose kept channels exceed 2 for some token; with fewer
+    dense blocks the overflow outside them is what is dropped."""
+    rng = np.random.default_rng(8)
+    x = rng.laplace(0, 0.3, size=(8, 256)).astype(np.float32)
+    W = rng.normal(0, 0.02, size=(40, 256)).astype(np.float32)
+    s = oracle_lib.score(x)
+    mask = oracle_lib.select_nm(s, 8, 16)
+    y_nm = oracle_lib.linear(x, mask, W)
+    over_blocks = np.unique(np.nonzero((mask.reshape(8, 64, 4).sum(-1) > 2))[1])
+    r = oracle_lib.nm_split(s, mask, x * mask, 64)
+    np.testing.assert_allclose(oracle_lib.linear(x, r["m_split"], W), y_nm, rtol=0, atol=1e-12)
+    r0 = oracle_lib.nm_split(s, mask, x * mask, 0)
+    dropped = mask.astype(bool) & ~r0["m_split"].astype(bool)
+    np.testing.assert_allclose(oracle_lib.linear(x, r0["m_split"], W) + (x * dropped) @ W.T.astype(np.float64),
+                               y_nm, rtol=0, atol=1e-12)
+    assert len(over_blocks) > 0
