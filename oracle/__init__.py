@@ -405,8 +405,13 @@ def nm_split(s, mask_nm, xm, n_dense: int):
         for j in range(4):
             if i == j:
                 continue
-            beats = (kb[..., j] & ~kb[..., i]) | ((kb[..., j] == kb[..., i]) &
-                                                  ((sb[..., j] > sb[..., i]) | ((sb[..., j] == sb[..., i]) & (j < i))))
+            # kept before dropped; kept ones by score, then index; dropped
+            # ones (zero-valued padding) by index alone
+            both_kept = kb[..., j] & kb[..., i]
+            both_dropped = ~kb[..., j] & ~kb[..., i]
+            beats = (kb[..., j] & ~kb[..., i]) | (both_kept & ((sb[..., j] > sb[..., i]) |
+                                                               ((sb[..., j] == sb[..., i]) & (j < i)))) | \
+                    (both_dropped & (j < i))
             rank[..., i] += beats
     pos = (rank < 2).reshape(T, k)
     part = pos & kept

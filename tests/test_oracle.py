@@ -708,11 +708,13 @@ def test_nm_split_worked_blocks(oracle_lib):
     kept channels with the highest scores form the 2:4 part, ties to the
     lower index; a block with one kept channel pads with the lowest dropped
     one."""
-    s = np.array([[5, 3, 4, 9, 2, 2, 2, 2, 0, 0, 7, 0, 1, 8, 6, 3]], np.float32)
-    m = np.array([[1, 1, 1, 0, 0, 1, 1, 1, 0, 0, 1, 0, 1, 1, 1, 1]], np.uint8)
+    s = np.array([[5, 3, 4, 9, 2, 2, 2, 2, 0, 0, 7, 0, 1, 8, 6, 3, 1, 0, 9, 5]], np.float32)
+    m = np.array([[1, 1, 1, 0, 0, 1, 1, 1, 0, 0, 1, 0, 1, 1, 1, 1, 0, 0, 1, 0]], np.uint8)
     r = oracle_lib.nm_split(s, m, s * m, 0)
-    assert r["part"].tolist() == [[1, 0, 1, 0, 0, 1, 1, 0, 0, 0, 1, 0, 0, 1, 1, 0]]
-    assert r["pos"].tolist() == [[1, 0, 1, 0, 0, 1, 1, 0, 1, 0, 1, 0, 0, 1, 1, 0]]
+    assert r["part"].tolist() == [[1, 0, 1, 0, 0, 1, 1, 0, 0, 0, 1, 0, 0, 1, 1, 0, 0, 0, 1, 0]]
+    # the last block pads with channel 0, the lowest-indexed dropped one,
+    # although dropped channel 3 has the higher score
+    assert r["pos"].tolist() == [[1, 0, 1, 0, 0, 1, 1, 0, 1, 0, 1, 0, 0, 1, 1, 0, 1, 0, 1, 0]]
     assert r["m_split"].tolist() == r["part"].tolist()  # no dense block
 
 
