@@ -642,10 +642,66 @@ def bench_prefill(sl, dev, pk):
         eight_batches_vs_cublas_dense=statistics.median(per_batch) / t_dense)
     del xs, x
     torch.cuda.empty_cache()
+    out["nm_split"] = bench_nm_split(sl, dev, ev_time)
     assert sl.as_stream_status() == sl.AS_OK
     out["timing"] = (f"median of {PREFILL_REPS} launches, CUDA events, each after writing a "
                      f"{L2_FLUSH_BYTES >> 20} MB buffer (L2 flushed)")
     return out
+
+
+def bench_nm_split(sl, dev, ev_time):
+    """The hybrid 2:4 decomposition of an N:M selection (2:4 part on the
+    sparse tensor cores, the kept channels of the busiest blocks dense) next
+    to the masked dense GEMM of the same selection and cuBLAS, on two inputs:
+    the CLACT + VAR 16:32 layer (x about 50 % zeros after the selection: the
+    page's mode rule picks dense) and an 8:16 selection of hot-channel
+    squared-ReLU activations (about 94 % zeros: the split regime)."""
+    from sparse_linear_b200.layer import SparseLinear, workspace
+    res = {}
+    cases = {
+        "clact_var_16of32": (lambda: (synth.prefill_clact_batch(0), synth.prefill_clact_weight()),
+                             sl.config(score=sl.AS_SCORE_CLACT, sel=sl.AS_SEL_NM, n=16, m=32, var=True)),
+        "sqrelu_hot_8of16": (lambda: synth.prefill_sqrelu_hot()[1:3],
+                             sl.config(sel=sl.AS_SEL_NM, n=8, m=16)),
+    }
+    for name, (make, cfg) in cases.items():
+        x, W = make()
+        x, W = x.to(dev), W.to(dev)
+        T, K = x.shape
+        n_out = W.shape[0]
+        L = SparseLinear(W, cfg, keep_wt=False)
+        run = torch.zeros(T, dtype=torch.float32, device=dev) if cfg.var else None
+        bufs = L.select_buffers(T)
+        bufs["x_compact"] = torch.empty(T, K // 2, dtype=torch.bfloat16, device=dev)
+        bufs["meta24"] = torch.empty(sl.as_meta24_words(T, K), dtype=torch.int32, device=dev)
+        bufs["bitmask24"] = torch.empty(T, (K + 31) // 32, dtype=torch.int32, device=dev)
+        L.select(x, bufs, running_var=run, first_batch=True)
+        sp = torch.empty(1, dtype=torch.float32, device=dev)
+        ws_sp = workspace(sl.as_hybrid_workspace(T, K, 0, 0), dev)
+        sl.as_block_sparsity(bufs["x_masked"], sp, workspace=ws_sp)
+        sparsity = float(sp.item())
+        sel = sl.select_out(**{k: bufs[k] for k in ("x_masked", "x_compact", "meta24", "bitmask24")})
+        y_nm = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
+        t_dense_masked = ev_time(lambda: L.prefill_from(bufs, T, y_nm))
+        t_cublas = ev_time(lambda: torch.matmul(x, W.t()))
+        ref = y_nm.float()
+        entry = dict(shape=[T, K, n_out], masked_sparsity=sparsity,
+                     mode_rule=["2:4", "split", "dense"][sl.as_prefill_mode(sparsity)],
+                     masked_dense_gemm_us=t_dense_masked * 1e6, cublas_dense_us=t_cublas * 1e6)
+        for label, nd in (("dense_5pct", sl.as_hybrid_dense_blocks(K, 0.05)), ("all_blocks_dense", K // 4)):
+            wsh = workspace(sl.as_hybrid_workspace(T, K, n_out, nd), dev)
+            y = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
+            fn = lambda nd=nd, wsh=wsh, y=y: sl.as_linear_prefill_nm_split(  # noqa: E731
+                sel, T, W, cfg, y, nd, rowsum=L.rowsum, eta=bufs.get("eta"), nu=bufs.get("nu"), workspace=wsh)
+            t = ev_time(fn)
+            err = float(torch.linalg.norm(y.float() - ref) / torch.linalg.norm(ref))
+            entry[label] = dict(n_dense=nd, us=t * 1e6, rel_err_vs_nm_product=err,
+                                speedup_vs_masked_dense=t_dense_masked / t, speedup_vs_cublas=t_cublas / t)
+            del wsh, y
+        res[name] = entry
+        del x, W, L, bufs, sel, y_nm, ref
+        torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------- CPU oracle

@@ -146,6 +146,17 @@ typedef struct as_select_out {
                             2^-17 relative).  Needs x_masked. */
     void *x_compact_lo;  /* 2:4 only, bf16 [T, K/2]: the same residual of
                             x_compact (zeros when no shift).  Needs x_compact. */
+    uint32_t *bitmask24; /* N:M with m a multiple of 4 and m >= 8 (optional,
+                            with x_masked, x_compact and meta24): the 2:4-
+                            compliant part of the selection ([SQR] 3.2 applied
+                            to an N:M selection).  In every 4-block the two
+                            channels ranked first by (kept, higher score,
+                            lower index) form the part; x_compact/meta24 hold
+                            their values xhat*m (zero for a dropped channel
+                            that pads a block with fewer than two kept) and
+                            positions, and bitmask24 [T, ceil(K/32)] the kept
+                            channels inside the part.  See
+                            as_linear_prefill_nm_split. */
 } as_select_out;
 
 /* --------------------------------------------------------------------------
@@ -332,6 +343,33 @@ as_status as_linear_prefill_hybrid(const as_select_out *sel, const void *x, int 
                                    void *workspace, size_t ws_bytes, cudaStream_t stream);
 as_status as_block_sparsity(const void *x, int T, int K, int n_dense, int32_t *dense_idx, float *sparsity,
                             void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Hybrid 2:4 decomposition of an N:M selection ([SQR] 3.2: the densest
+ * features dense, the rest 2:4 on the sparse tensor cores; here applied to
+ * an N:M selection that is not 2:4-compliant, 8:16 or 16:32):
+ *   y = epilogue((xm (.) p) W^T + (xm (.) (1 - p))[:, D] W[:, D]^T),
+ * xm = xhat (.) m the masked activation (sel->x_masked), p the 2:4 part
+ * (sel->bitmask24, x_compact, meta24 from as_select), D the n_dense
+ * 4-channel blocks with the most nonzeros of xm over the T tokens (ties to
+ * the lower block index).  Kept channels outside p and outside D are
+ * dropped, so the result is the N:M product exactly when D covers every
+ * block with more than two kept channels for some token (n_dense = K/4
+ * always does); fewer dense blocks trade that remainder for speed.  The
+ * epilogue is as_linear_prefill's (x nu_t with VAR, + eta_t rowsum_o with a
+ * token shift, rounding to cfg->out_dtype).
+ *   cfg      the as_select configuration: AS_SEL_NM, m a multiple of 4 and
+ *            m >= 8.
+ *   n_dense  0 <= n_dense <= K/4, a multiple of 16.  K % 64 == 0,
+ *            K <= 32768, n_out % 8 == 0, T < 2^22.
+ *   dense_idx, sparsity: as as_linear_prefill_hybrid (sparsity: of xm).
+ * Workspace: as_hybrid_workspace(T, K, n_out, n_dense), no zero-fill.
+ * as_block_sparsity on xm gives the sparsity for as_prefill_mode.
+ * ------------------------------------------------------------------------ */
+as_status as_linear_prefill_nm_split(const as_select_out *sel, int T, int K, const void *W, int n_out, int n_dense,
+                                     const as_config *cfg, const float *rowsum, const float *eta, const float *nu,
+                                     void *y, int32_t *dense_idx, float *sparsity, void *workspace, size_t ws_bytes,
+                                     cudaStream_t stream);
 
 /* The inference mode switch ([SQR] 3.3), host-only.  The page keys the mode
  * on the layer's measured activation sparsity (as_block_sparsity's output):

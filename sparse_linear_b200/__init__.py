@@ -43,7 +43,7 @@ EXPORTS = [
     "as_weight_prep_amber", "as_meta8_words", "as_weight_quant_fp8", "as_select_sqrelu24_fp8",
     "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode", "as_hybrid_workspace",
     "as_linear_prefill_hybrid", "as_block_sparsity", "as_prefill_mode", "as_hybrid_dense_blocks",
-    "as_rsparse_prefill_workspace", "as_linear_prefill_rsparse",
+    "as_rsparse_prefill_workspace", "as_linear_prefill_rsparse", "as_linear_prefill_nm_split",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -59,7 +59,7 @@ class as_config(ctypes.Structure):
 class as_select_out(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in (
         "bitmask", "eta", "colnorm", "var_dense", "var_kept", "nu", "x_masked",
-        "x_compact", "meta24", "x_masked_lo", "x_compact_lo")]
+        "x_compact", "meta24", "x_masked_lo", "x_compact_lo", "bitmask24")]
 
 
 _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -93,6 +93,8 @@ _sig = {
     "as_abi_version": ([], _I),
     "as_prefill_mode": ([ctypes.c_double], _I),
     "as_rsparse_prefill_workspace": ([_I, _I, _I], _S),
+    "as_linear_prefill_nm_split": ([ctypes.POINTER(as_select_out), _I, _I, _P, _I, _I, ctypes.POINTER(as_config),
+                                    _P, _P, _P, _P, _P, _P, _P, _S, _P], _I),
     "as_linear_prefill_rsparse": ([ctypes.POINTER(as_select_out), _P, _P, _I, _I, _I, _P, _P,
                                    ctypes.POINTER(as_config), _I, _P, _P, _P, _P, _S, _P], _I),
     "as_hybrid_dense_blocks": ([_I, ctypes.c_double], _I),
@@ -359,6 +361,17 @@ def as_linear_prefill_rsparse(sel: as_select_out, x, W, cfg: as_config, y, B, A,
     _check(_lib.as_linear_prefill_rsparse(ctypes.byref(sel), _ptr(x), _ptr(W), T, K, n_out, _ptr(rowsum), _ptr(eta),
                                           ctypes.byref(cfg), r, _ptr(B), _ptr(A), _ptr(y), _ptr(workspace), ws_bytes,
                                           _stream(stream)), "as_linear_prefill_rsparse")
+
+
+def as_linear_prefill_nm_split(sel: as_select_out, T: int, W, cfg: as_config, y, n_dense: int, rowsum=None,
+                               eta=None, nu=None, dense_idx=None, sparsity=None, workspace=None, stream=None) -> None:
+    """Hybrid 2:4 decomposition of an N:M selection (see include/actsparse.h)."""
+    n_out, K = W.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.as_linear_prefill_nm_split(ctypes.byref(sel), T, K, _ptr(W), n_out, int(n_dense), ctypes.byref(cfg),
+                                           _ptr(rowsum), _ptr(eta), _ptr(nu), _ptr(y), _ptr(dense_idx),
+                                           _ptr(sparsity), _ptr(workspace), ws_bytes, _stream(stream)),
+           "as_linear_prefill_nm_split")
 
 
 def as_stream_status(stream=None) -> int:

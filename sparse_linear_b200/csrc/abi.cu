@@ -216,6 +216,47 @@ int as_hybrid_dense_blocks(int K, double dense_frac)
     return n < 16 ? 16 : (n > hi ? hi : n);
 }
 
+as_status as_linear_prefill_nm_split(const as_select_out *sel, int T, int K, const void *W, int n_out, int n_dense,
+                                     const as_config *cfg, const float *rowsum, const float *eta, const float *nu,
+                                     void *y, int32_t *dense_idx, float *sparsity, void *workspace, size_t ws_bytes,
+                                     cudaStream_t stream)
+{
+    if (!sel || !W || !y || !sel->x_masked || !sel->x_compact || !sel->meta24 || !sel->bitmask24)
+        return AS_ERR_INVALID_ARG;
+    if (n_out <= 0) return AS_ERR_INVALID_ARG;
+    as_status st = check_cfg(cfg, K);
+    if (st != AS_OK) return st;
+    if (cfg->sel != AS_SEL_NM || cfg->m < 8 || cfg->m % 4 != 0) return AS_ERR_UNSUPPORTED;
+    st = hybrid_shape(T, K, n_out, n_dense);
+    if (st != AS_OK) return st;
+    if (cfg->dpts && (!rowsum || !eta)) return AS_ERR_INVALID_ARG;
+    if (cfg->var && !nu) return AS_ERR_INVALID_ARG;
+    const void *ptrs[] = {W, y, sel->x_masked, sel->x_compact, sel->meta24, sel->bitmask24, workspace, rowsum,
+                          eta, nu};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return AS_ERR_ALIGN;
+    if (!workspace || ws_bytes < hybrid_layout(T, K, n_out, n_dense).bytes) return AS_ERR_WORKSPACE;
+    HybridArgs a{};
+    a.x = sel->x_masked;  // the masked activation: its nonzeros pick D, its overflow is the dense remainder
+    a.bitmask = sel->bitmask24;
+    a.x_compact = sel->x_compact;
+    a.meta24 = sel->meta24;
+    a.W = W;
+    a.T = T;
+    a.K = K;
+    a.n_out = n_out;
+    a.n_dense = n_dense;
+    a.y = y;
+    a.out_bf16 = cfg->out_dtype == AS_BF16;
+    a.idx_out = dense_idx;
+    a.sparsity_out = sparsity;
+    a.workspace = workspace;
+    a.rowsum = cfg->dpts ? rowsum : nullptr;
+    a.eta = cfg->dpts ? eta : nullptr;
+    a.nu = cfg->var ? nu : nullptr;
+    return cuda_status(launch_hybrid(a, stream));
+}
+
 static bool rsparse_rank_ok(int r) { return r == 32 || r == 64 || r == 128; }
 
 size_t as_rsparse_workspace(int T, int K, int r)
@@ -312,13 +353,20 @@ as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *c
     if (K % 8 != 0) return AS_ERR_SHAPE;
     if (cfg->score == AS_SCORE_WEIGHT && !chan_factor) return AS_ERR_INVALID_ARG;
     if (cfg->var && !running_var) return AS_ERR_INVALID_ARG;
-    if ((out->x_compact || out->meta24) && (!is24(cfg) || dt != AS_BF16 || K % 16 != 0)) return AS_ERR_UNSUPPORTED;
+    // the 2:4 part of an N:M selection (bitmask24 with x_compact, meta24 and x_masked)
+    const bool part24 = out->bitmask24 != nullptr;
+    if (part24) {
+        if (cfg->sel != AS_SEL_NM || cfg->m < 8 || cfg->m % 4 != 0) return AS_ERR_UNSUPPORTED;
+        if (!out->x_compact || !out->meta24 || !out->x_masked) return AS_ERR_INVALID_ARG;
+    }
+    if ((out->x_compact || out->meta24) && ((!is24(cfg) && !part24) || dt != AS_BF16 || K % 16 != 0))
+        return AS_ERR_UNSUPPORTED;
     if ((out->x_compact == nullptr) != (out->meta24 == nullptr)) return AS_ERR_INVALID_ARG;
     if ((out->x_masked_lo && (!out->x_masked || dt != AS_BF16)) || (out->x_compact_lo && !out->x_compact))
         return AS_ERR_INVALID_ARG;
     const void *ptrs[] = {x, chan_factor, running_var, out->bitmask, out->eta, out->colnorm, out->var_dense,
                           out->var_kept, out->nu, out->x_masked, out->x_compact, out->meta24, workspace,
-                          out->x_masked_lo, out->x_compact_lo};
+                          out->x_masked_lo, out->x_compact_lo, out->bitmask24};
     for (const void *p : ptrs)
         if (!aligned16(p)) return AS_ERR_ALIGN;
     if (cfg->sel == AS_SEL_TOPK && cfg->k_keep > 0 && cfg->k_keep < K && (size_t)K * 4 > 200 * 1024)
@@ -364,6 +412,8 @@ as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *c
     a.meta24 = out->meta24;
     a.x_masked_lo = out->x_masked_lo;
     a.x_compact_lo = out->x_compact_lo;
+    a.bitmask24 = out->bitmask24;
+    if (part24 && !select_rows_kernel(a)) return AS_ERR_UNSUPPORTED;  // written by the row kernel only
     return cuda_status(launch_select(a, stream));
 }
 

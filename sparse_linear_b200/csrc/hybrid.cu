@@ -275,6 +275,9 @@ cudaError_t launch_hybrid(const HybridArgs &a, cudaStream_t st)
     s.y = a.y;
     s.out_bf16 = a.out_bf16;
     s.addend = addend;
+    s.rowsum = a.rowsum;
+    s.eta = a.eta;
+    s.nu = a.nu;
     return launch_gemm(s, st);
 }
 

@@ -34,11 +34,14 @@ struct SelectArgs {
     uint32_t *meta24;
     void *x_masked_lo;   // bf16 residuals of x_masked (float32-output GEMM operand), or nullptr
     void *x_compact_lo;  // bf16 residuals of x_compact, or nullptr
+    uint32_t *bitmask24; // N:M selection: kept channels of its 2:4 part (x_compact/meta24 hold the part)
 };
 // CLACT column energy c_j = sqrt(sum_t x_tj^2), float64 partials in ws.
 size_t colnorm_workspace(int T, int K);
 cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void *ws, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st, int wide = 0);
+// Whether launch_select (not wide) runs the row kernel for these arguments.
+bool select_rows_kernel(const SelectArgs &a);
 // N:M selection of a decode call: keep words and eta only (grid token x chunk).
 cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st);
 
@@ -140,6 +143,7 @@ struct HybridArgs {
     int *idx_out;             // [n_dense] or NULL
     float *sparsity_out;      // [1] or NULL
     void *workspace;
+    const float *rowsum = nullptr, *eta = nullptr, *nu = nullptr;  // epilogue terms of the 2:4 GEMM
 };
 struct HybridLayout {
     size_t nnz, total, idx, xr, wd, yd, bytes;

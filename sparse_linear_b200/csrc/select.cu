@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
         // (its channel offset within a 32-channel block is the same in
         // every tile).
         uint8_t *mrow = nullptr;
-        if constexpr (COMPACT) mrow = meta_byte(a.meta24, t, 8 * tid, kt);
+        if (a.meta24) mrow = meta_byte(a.meta24, t, 8 * tid, kt);
         constexpr size_t mstride = (size_t)(8 * SR_THREADS / 128) * 2048;  // bytes per tile
         const bool plain = !a.dpts && !has_f;  // score = |x|
         if constexpr (COMPACT) {
@@ -566,6 +566,38 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
                     if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
                     if (a.x_masked_lo)
                         store8_lo(static_cast<__nv_bfloat16 *>(a.x_masked_lo) + (size_t)t * K + c0, km);
+                    if (a.bitmask24) {
+                        // the 2:4 part of the N:M selection: per 4-block the two channels
+                        // ranked first by (kept, higher score, lower index); dropped
+                        // channels rank below every kept one (score -1)
+                        float s2[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s2[e] = ((keep >> e) & 1u) ? sc[e] : -1.0f;
+                        const uint32_t pos = keep_2of4(s2);
+                        float cv[4];
+                        uint32_t nib[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            int i0, i1;
+                            pos_2of4((pos >> (4 * h)) & 0xFu, i0, i1);
+                            cv[2 * h] = pick4(km, 4 * h, i0);
+                            cv[2 * h + 1] = pick4(km, 4 * h, i1);
+                            nib[h] = (uint32_t)i0 | ((uint32_t)i1 << 2);
+                        }
+                        const __nv_bfloat162 p0 = __floats2bfloat162_rn(cv[0], cv[1]);
+                        const __nv_bfloat162 p1 = __floats2bfloat162_rn(cv[2], cv[3]);
+                        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact) + (size_t)t * (K / 2) +
+                                                   c0 / 2) =
+                            make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
+                        if (a.x_compact_lo)
+                            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
+                                                       c0 / 2) = lo4(cv);
+                        mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
+                        uint8_t *b24 = reinterpret_cast<uint8_t *>(a.bitmask24 + (size_t)t * words);
+                        b24[g] = (uint8_t)(pos & keep);
+                        if (g == ngroups - 1)
+                            for (int b = ngroups; b < words * 4; ++b) b24[b] = 0;
+                    }
                 }
                 if constexpr (COMPACT) {
                     float cv[4];
@@ -806,7 +838,7 @@ template <typename TX>
 static cudaError_t launch_select_rows(const SelectArgs &a, cudaStream_t st)
 {
     if (a.sel == AS_SEL_NM) {
-        if (a.x_compact) {
+        if (a.x_compact && !a.bitmask24) {  // a 2:4 selection (bitmask24: the 2:4 part of an N:M one)
             if constexpr (std::is_same<TX, __nv_bfloat16>::value) return launch_select_rows_t<TX, 4, true>(a, st);
         }
         switch (a.m) {
@@ -827,9 +859,11 @@ static bool select_rows_fits(const SelectArgs &a)
     return (a.f ? (size_t)a.K * 4 : 0) + (size_t)SR_BUFS * a.K * elem <= 200 * 1024;
 }
 
+bool select_rows_kernel(const SelectArgs &a) { return a.sel != AS_SEL_TOPK && select_rows_fits(a); }
+
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st, int wide)
 {
-    if (!wide && a.sel != AS_SEL_TOPK && select_rows_fits(a))
+    if (!wide && select_rows_kernel(a))
         return a.bf16 ? launch_select_rows<__nv_bfloat16>(a, st) : launch_select_rows<float>(a, st);
     const bool topk = a.sel == AS_SEL_TOPK && a.k_keep > 0 && a.k_keep < a.K;
     const size_t smem = topk ? (size_t)a.K * sizeof(uint32_t) : 0;

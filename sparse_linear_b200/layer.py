@@ -12,7 +12,8 @@ import torch
 from . import (AS_BF16, AS_F32, AS_MODE_24, AS_MODE_DENSE, AS_MODE_SPLIT, AS_OP_AMBER, AS_OP_DECODE,
                AS_OP_PREFILL, AS_OP_SELECT, AS_OP_WEIGHT_PREP, AS_SCORE_CLACT, AS_SCORE_MAG, AS_SEL_ALL, AS_SEL_NM,
                as_block_sparsity, as_hybrid_dense_blocks, as_hybrid_workspace, as_linear_decode, as_linear_prefill,
-               as_linear_prefill_hybrid, as_linear_prefill_rsparse, as_meta24_words, as_prefill_mode,
+               as_linear_prefill_hybrid, as_linear_prefill_nm_split, as_linear_prefill_rsparse, as_meta24_words,
+               as_prefill_mode,
                as_rsparse_prefill_workspace, as_select, as_weight_prep, as_weight_prep_amber, as_workspace_size,
                config, select_out)
 
@@ -195,6 +196,29 @@ class SparseLinear:
                             if k in ("bitmask", "x_masked", "x_compact", "meta24", "x_masked_lo", "x_compact_lo")})
         as_linear_prefill_rsparse(sel, x, self.W, self.cfg, y, B, A, rowsum=self.rowsum, eta=bufs.get("eta"),
                                   workspace=self._ws[key], stream=stream)
+        return y, bufs
+
+    def prefill_nm_split(self, x: torch.Tensor, n_dense: int, running_var=None, first_batch: bool = False,
+                         dense_idx=None, sparsity=None, stream=None):
+        """Selection with the 2:4 part of this layer's N:M configuration, then
+        the hybrid split: the 2:4 part on the sparse tensor cores, the kept
+        channels of the n_dense busiest blocks dense (2:4 + Squared-ReLU page,
+        section 3.2).  Returns (y, bufs)."""
+        T, K = x.shape
+        dev = x.device
+        bufs = self.select_buffers(T, dev)
+        bufs["x_compact"] = torch.empty(T, K // 2, dtype=torch.bfloat16, device=dev)
+        bufs["meta24"] = torch.empty(as_meta24_words(T, K), dtype=torch.int32, device=dev)
+        bufs["bitmask24"] = torch.empty(T, (K + 31) // 32, dtype=torch.int32, device=dev)
+        self.select(x, bufs, running_var=running_var, first_batch=first_batch, stream=stream)
+        key = ("hybrid", T, n_dense)
+        if key not in self._ws:
+            self._ws[key] = workspace(as_hybrid_workspace(T, K, self.n_out, n_dense), dev)
+        y = torch.empty(T, self.n_out, dtype=self.out_dtype(), device=dev)
+        sel = select_out(**{k: v for k, v in bufs.items() if k in ("x_masked", "x_compact", "meta24", "bitmask24")})
+        as_linear_prefill_nm_split(sel, T, self.W, self.cfg, y, n_dense, rowsum=self.rowsum, eta=bufs.get("eta"),
+                                   nu=bufs.get("nu"), dense_idx=dense_idx, sparsity=sparsity,
+                                   workspace=self._ws[key], stream=stream)
         return y, bufs
 
     def prefill(self, x: torch.Tensor, running_var=None, first_batch: bool = False, stream=None):

@@ -340,3 +340,32 @@ def test_rsparse_prefill_validation_launches_nothing(lib):
     nomask.x_compact = fake
     nomask.meta24 = fake
     assert call(s=nomask) == lib.AS_ERR_INVALID_ARG
+
+
+def test_nm_split_validation_launches_nothing(lib):
+    fake = 1 << 20
+    cfg = lib.config(sel=lib.AS_SEL_NM, n=16, m=32)
+    sel = lib.select_out(x_masked=fake, x_compact=fake, meta24=fake, bitmask24=fake)
+    f = lib._lib.as_linear_prefill_nm_split
+    ws = lib.as_hybrid_workspace(256, 1024, 256, 16)
+
+    def call(s=sel, c=cfg, nd=16, wb=ws, K=1024):
+        return f(ctypes.byref(s), 256, K, fake, 256, nd, ctypes.byref(c), None, None, None, fake, None, None, fake,
+                 wb, None)
+
+    assert call(c=lib.config(sel=lib.AS_SEL_NM, n=2, m=4)) == lib.AS_ERR_UNSUPPORTED   # already 2:4
+    assert call(c=lib.config(sel=lib.AS_SEL_TOPK, k_keep=10)) == lib.AS_ERR_UNSUPPORTED
+    assert call(nd=17) == lib.AS_ERR_SHAPE
+    assert call(K=1000) == lib.AS_ERR_SHAPE
+    assert call(s=lib.select_out(x_masked=fake, x_compact=fake, meta24=fake)) == lib.AS_ERR_INVALID_ARG
+    assert call(c=lib.config(sel=lib.AS_SEL_NM, n=16, m=32, dpts=True)) == lib.AS_ERR_INVALID_ARG  # no eta/rowsum
+    assert call(wb=ws - 1) == lib.AS_ERR_WORKSPACE
+    # as_select: the 2:4 part needs an N:M selection with m a multiple of 4, m >= 8
+    sel_f = lib._lib.as_select
+    out = lib.select_out(x_masked=fake, x_compact=fake, meta24=fake, bitmask24=fake)
+    for c in (lib.config(sel=lib.AS_SEL_NM, n=2, m=4), lib.config(sel=lib.AS_SEL_TOPK, k_keep=3)):
+        assert sel_f(fake, lib.AS_BF16, 4, 64, ctypes.byref(c), None, None, 0, ctypes.byref(out), None, 0,
+                     None) == lib.AS_ERR_UNSUPPORTED
+    nomask = lib.select_out(x_compact=fake, meta24=fake, bitmask24=fake)
+    assert sel_f(fake, lib.AS_BF16, 4, 64, ctypes.byref(cfg), None, None, 0, ctypes.byref(nomask), None, 0,
+                 None) == lib.AS_ERR_INVALID_ARG

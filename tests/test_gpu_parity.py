@@ -783,6 +783,74 @@ def test_hybrid_without_dense_blocks_is_the_24_prefill(sl):
     assert torch.equal(y, y0)
 
 
+def check_nm_split(sl, T, K, n_out, n, m, score, dpts, var, n_dense, out, seed=61):
+    """The hybrid decomposition of an N:M selection through the C ABI: the
+    selection, its 2:4 part (kept bits, positions, compact values) and the
+    dense blocks bit-exact against the oracle; y against the oracle's split
+    product with the same epilogue."""
+    x, W = synth.random_layer(T, K, n_out, seed=seed, dist="t3" if score == sl.AS_SCORE_CLACT else "laplace")
+    cfg = sl.config(score=score, sel=sl.AS_SEL_NM, n=n, m=m, dpts=dpts, var=var, out_dtype=out)
+    L = layer(sl, W, cfg, 0.5)
+    running = torch.zeros(T, dtype=torch.float32, device="cuda") if var else None
+    idx = torch.full((max(n_dense, 1),), -1, dtype=torch.int32, device="cuda")
+    sp = torch.empty(1, dtype=torch.float32, device="cuda")
+    y, bufs = L.prefill_nm_split(dev(x), n_dense, running_var=running, first_batch=True, dense_idx=idx, sparsity=sp)
+    torch.cuda.synchronize()
+    assert sl.as_stream_status() == sl.AS_OK
+    xf, Wf = x.float().numpy(), W.float().numpy()
+    f = f32(bufs["colnorm"]) if score == sl.AS_SCORE_CLACT else (f32(L.g) if score == sl.AS_SCORE_WEIGHT else None)
+    eta32 = f32(bufs["eta"]) if dpts else None
+    sc = oracle.score(xf, eta=eta32, f=f)
+    mask = oracle.select_nm(sc, n, m)
+    np.testing.assert_array_equal(unpack_bitmask(bufs["bitmask"], K), mask)
+    xm = f32(bufs["x_masked"])
+    r = oracle.nm_split(sc, mask, xm, n_dense)
+    np.testing.assert_array_equal(unpack_bitmask(bufs["bitmask24"], K), r["part"])
+    pos = decode_meta24(bufs["meta24"], T, K)
+    ref_pos = np.nonzero(r["pos"].reshape(T, K // 4, 4))[2].reshape(T, K // 4, 2)
+    np.testing.assert_array_equal(pos, ref_pos)
+    vals = np.take_along_axis(xm.reshape(T, K // 4, 4), ref_pos, axis=2).reshape(T, K // 2)
+    np.testing.assert_array_equal(f32(bufs["x_compact"]), vals)
+    if n_dense:
+        np.testing.assert_array_equal(idx.cpu().numpy(), r["idx"])
+    assert sp.item() == np.float32(r["sparsity"])
+    nu = None
+    if var:
+        nu = oracle.var_scale(xf, mask, None, cfg.var_momentum, cfg.var_eps)["nu"]
+    eta64 = oracle.token_mean(xf) if dpts else None
+    _, rs = oracle.weight_prep(Wf, 1.0)
+    ref = oracle.linear(xf, r["m_split"], Wf, eta=eta64, rowsum=rs if dpts else None, nu=nu)
+    err = rel_l2(f32(y), ref)
+    assert err <= (TOL_BF16 if out == sl.AS_BF16 else TOL_F32), err
+    return y, mask, r
+
+
+# (T, K, n_out, n, m, score, dpts, var, n_dense, out): T = 300 runs the
+# one-SM kernels, the others the CTA pairs
+@pytest.mark.parametrize("T,K,n_out,n,m,score,dpts,var,n_dense,out", [
+    (256, 1024, 264, 8, 16, 1, True, False, 16, 1),     # weight-aware 8:16 with D-PTS
+    (300, 2048, 264, 16, 32, 2, False, True, 64, 0),    # CLACT + VAR 16:32, float32 out
+    (256, 1024, 256, 16, 32, 0, False, False, 0, 0),    # no dense block: the 2:4 part alone
+    (512, 2048, 520, 8, 16, 0, False, False, 32, 1),
+])
+def test_nm_split(sl, T, K, n_out, n, m, score, dpts, var, n_dense, out):
+    check_nm_split(sl, T, K, n_out, n, m, score, dpts, var, n_dense, out)
+
+
+def test_nm_split_all_blocks_dense_is_the_nm_product(sl):
+    """With every block dense the split is exactly the 16:32 selection's
+    product: against the oracle and the masked dense prefill of the same
+    selection."""
+    T, K, n_out = 256, 1024, 256
+    y, mask, r = check_nm_split(sl, T, K, n_out, 16, 32, 0, False, False, K // 4, 0)
+    np.testing.assert_array_equal(r["m_split"], mask)
+    x, W = synth.random_layer(T, K, n_out, seed=61, dist="laplace")
+    cfg = sl.config(sel=sl.AS_SEL_NM, n=16, m=32, out_dtype=sl.AS_F32)
+    y_nm, _ = layer(sl, W, cfg).prefill(dev(x))
+    torch.cuda.synchronize()
+    assert rel_l2(f32(y), f32(y_nm)) <= TOL_F32
+
+
 def test_hybrid_full_size(sl):
     """The down-projection shape with hot channels (T 4096, K 14336, n_out
     4096, 192 dense blocks = 768 channels), sampled rows of every tile."""
