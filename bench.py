@@ -643,6 +643,14 @@ def bench_prefill(sl, dev, pk):
     del xs, x
     torch.cuda.empty_cache()
     out["nm_split"] = bench_nm_split(sl, dev, ev_time)
+    # read-only stream of this box (a library reduction over 256 MB of bf16):
+    # what a kernel that only reads HBM can reach, next to the copy peak
+    big = torch.ones(128 << 20, dtype=torch.bfloat16, device=dev)
+    t_read = ev_time(lambda: big.sum(dtype=torch.float32))
+    out["read_stream_calibration"] = dict(what="torch.sum over 256 MB bf16 (reads only)",
+                                          gbs=big.numel() * 2 / t_read / 1e9,
+                                          frac_of_copy_peak=big.numel() * 2 / t_read / 1e9 / pk["hbm_gbs"])
+    del big
     assert sl.as_stream_status() == sl.AS_OK
     out["timing"] = (f"median of {PREFILL_REPS} launches, CUDA events, each after writing a "
                      f"{L2_FLUSH_BYTES >> 20} MB buffer (L2 flushed)")
