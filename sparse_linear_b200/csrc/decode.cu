@@ -987,7 +987,7 @@ template <typename TW, int TP, int VEC>
 static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &p, cudaStream_t st)
 {
     const size_t smem = DecCfg<TP, VEC, TW>::smem;
-    if (smem > 48 * 1024) {
+    if (smem > 40 * 1024) {  // the 48 KB default also counts the kernel's static shared memory (< 8 KB)
         cudaError_t e = cudaFuncSetAttribute(k_decode<TW, TP, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;

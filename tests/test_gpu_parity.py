@@ -239,6 +239,31 @@ def test_decode_plan_stable_across_calls(sl):
     assert sl.as_stream_status() == sl.AS_OK
 
 
+def test_decode_repeated_and_graph(sl):
+    """Many calls in a row, eagerly and replayed from a CUDA graph, give the
+    same result as the first (the workspace's counters return to zero after
+    every call), with no timeout recorded."""
+    x, W, _ = synth.decode_downproj(16)
+    cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
+    L = layer(sl, W, cfg, 0.5)
+    xd = dev(x)
+    y0 = L.decode(xd).clone()
+    for _ in range(20):
+        assert torch.equal(L.decode(xd), y0)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        L.decode(xd)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            yg = L.decode(xd)
+    for _ in range(10):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg, y0)
+    assert sl.as_stream_status() == sl.AS_OK
+
+
 def test_decode_deterministic(sl):
     x, W, _ = synth.decode_downproj(8)
     cfg = sl.config(score=sl.AS_SCORE_WEIGHT, sel=sl.AS_SEL_NM, n=8, m=16, dpts=True)
