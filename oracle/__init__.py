@@ -32,6 +32,8 @@ Functions and the passages they follow (page title, section):
 * ``rsparse``, ``rsparse_factors``  overview §3.3 (R-Sparse low-rank compensation;
                     the factors from a truncated SVD, numpy's).
 * ``compress_nm``   2:4 + Squared-ReLU page §3.3 (kept values stored contiguously).
+* ``select_stats``  2:4 + Squared-ReLU page §2.3 (natural nonzeros a 2:4
+                    selection must drop) and the kept count per token.
 * ``e4m3_encode``/``e4m3_decode``, ``quant_rows_fp8``, ``sqrelu24_fp8``,
   ``linear_fp8``    2:4 + Squared-ReLU page §3.1 (fused Squared-ReLU + 2:4 +
                     FP8 producer, FP8 row-scaled GEMM) and §5.3 (sparsify
@@ -349,6 +351,18 @@ def rsparse(x, mask, B, A, eta=None):
     comp = np.empty((T, n_out), np.float64)
     _load().or_rsparse(_ptr(x), _ptr(mask), T, k, _ptr(e), _ptr(B), _ptr(A), n_out, r, _ptr(comp))
     return comp
+
+
+def select_stats(x, mask):
+    """Per token: the number of kept channels and the number of channels with
+    x != 0 that the selection dropped (the 2:4 + Squared-ReLU page §2.3: a
+    4-block with three natural nonzeros has to lose one of them).  Plain
+    counting over the definition; int64 [T] each."""
+    x = np.asarray(x, np.float64)
+    mask = np.asarray(mask).astype(bool)
+    kept = mask.sum(axis=1, dtype=np.int64)
+    dropped = ((x != 0.0) & ~mask).sum(axis=1, dtype=np.int64)
+    return kept, dropped
 
 
 def block_nnz(x):

@@ -767,3 +767,36 @@ def test_nm_split_exact_when_dense_blocks_cover_the_overflow(oracle_lib):
     np.testing.assert_allclose(oracle_lib.linear(x, r0["m_split"], W) + (x * dropped) @ W.T.astype(np.float64),
                                y_nm, rtol=0, atol=1e-12)
     assert len(over_blocks) > 0
+
+
+def test_select_stats_worked_row(oracle_lib):
+    """Two 4-blocks by magnitude (2:4): [0, 3, -1, 2] keeps 3 and 2 and drops
+    the natural nonzero -1; [0, 0, 5, 0] keeps 5 and the lowest-indexed zero,
+    dropping no nonzero."""
+    x = np.array([[0.0, 3.0, -1.0, 2.0, 0.0, 0.0, 5.0, 0.0]])
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    np.testing.assert_array_equal(mask, [[0, 1, 0, 1, 1, 0, 1, 0]])
+    kept, dropped = oracle_lib.select_stats(x, mask)
+    assert kept.tolist() == [4] and dropped.tolist() == [1]
+
+
+def test_select_stats_force_dropped_closed_form(oracle_lib):
+    """2:4 + Squared-ReLU page §2.3: a 4-block with k > 2 natural nonzeros
+    loses k - 2 of them.  For z ~ N(-1.2, 1), max(0, z)^2 is nonzero with
+    p = 1 - Phi(1.2), k ~ Binomial(4, p), so the expected number dropped per
+    block is 4 p^3 (1 - p) + 2 p^4 (0.0057 here: 1.25 % of the nonzeros,
+    the page's 'about 1 %' at this sparsity).  Checked within 5 sigma over
+    2^20 blocks; every token keeps exactly K / 2."""
+    rng = np.random.default_rng(2024)
+    T, K = 1024, 4096
+    x = np.maximum(rng.normal(-1.2, 1.0, size=(T, K)), 0.0) ** 2
+    mask = oracle_lib.select_nm(oracle_lib.score(x), 2, 4)
+    kept, dropped = oracle_lib.select_stats(x, mask)
+    assert (kept == K // 2).all()
+    p = 0.5 * math.erfc(1.2 / math.sqrt(2.0))
+    mu = 4 * p**3 * (1 - p) + 2 * p**4
+    var = 4 * p**3 * (1 - p) + 4 * p**4 - mu * mu
+    n_blocks = T * K // 4
+    assert abs(dropped.sum() / n_blocks - mu) <= 5.0 * math.sqrt(var / n_blocks)
+    share = dropped.sum() / (x != 0).sum()
+    assert 0.010 < share < 0.015
