@@ -21,6 +21,7 @@ reports the max over ranks.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import math
@@ -46,6 +47,16 @@ METRIC = "decode tokens/s & achieved HBM GB/s; prefill sparse TFLOP/s vs dense, 
 
 
 # ---------------------------------------------------------------- helpers
+@contextlib.contextmanager
+def nvtx(name: str):
+    """NVTX range around a bench section (visible to ncu --nvtx filters)."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -258,7 +269,8 @@ def bench_decode(sl, dev, steps, warmup, world):
     with torch.cuda.stream(stream):
         run_steps(max(3, warmup))
     torch.cuda.synchronize()
-    t_local = timed(lambda j: run_steps(steps) if j == 0 else None, 1)
+    with nvtx("decode timed region"):
+        t_local = timed(lambda j: run_steps(steps) if j == 0 else None, 1)
     # per-T kernel durations: graphs of 8 back-to-back calls of one T
     per_t = {}
     reps = max(8, steps // N_ROT)
@@ -949,13 +961,18 @@ def main():
     import sparse_linear_b200 as sl
     dev = torch.device("cuda", torch.cuda.current_device())
     pk, pk_src = peaks()
-    d = bench_decode(sl, dev, args.steps, args.warmup, world)
+    with nvtx("decode down-projection"):
+        d = bench_decode(sl, dev, args.steps, args.warmup, world)
     prefill = None
     if not args.no_prefill and rank == 0:
-        prefill = bench_prefill(sl, dev, pk)
+        with nvtx("prefill"):
+            prefill = bench_prefill(sl, dev, pk)
     extra = None
     if not args.no_prefill and rank == 0:
-        extra = {"decode_block_T1": bench_block(sl, dev), "tiny_fp32_decode": bench_tiny(sl, dev)}
+        with nvtx("decode block"):
+            blk = bench_block(sl, dev)
+        with nvtx("tiny fp32 layer"):
+            extra = {"decode_block_T1": blk, "tiny_fp32_decode": bench_tiny(sl, dev)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         tps, threads, sample = oracle_decode_sample(budget_s=15.0)

@@ -216,6 +216,22 @@ as_status as_select(const void *x, as_dtype dt, int T, int K, const as_config *c
                     cudaStream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Per-token statistics of a selection ([SQR] 2.3: where a 4-block holds
+ * three natural nonzeros, the 2:4 selection has to drop one of them; the
+ * page puts that near 1 % of the values at 95 % sparsity).
+ *   x        [T, K] in `dt` (AS_BF16 or AS_F32): the activations selected from.
+ *   bitmask  [T, ceil(K/32)] keep words (bit c%32 of word c/32), as written
+ *            by as_select or by the decode's mask_out.
+ *   kept     [T] int32 (may be NULL): kept channels of each token.
+ *   nz_dropped [T] int32 (may be NULL): channels with x != 0 that were not
+ *            kept.
+ * K % 8 == 0; pointers 16-byte aligned.  No workspace.  One kernel on
+ * `stream`; exact integer counts.
+ * ------------------------------------------------------------------------ */
+as_status as_select_stats(const void *x, as_dtype dt, const uint32_t *bitmask, int T, int K, int32_t *kept,
+                          int32_t *nz_dropped, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
  * Decode: 1 <= T <= 16 tokens against the channel-major weight Wt [K, n_out].
  * For N:M selection the score, block top-N, D-PTS mean and the contraction
  * run in one kernel that streams only the union over the T tokens of the

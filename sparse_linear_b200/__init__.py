@@ -44,6 +44,7 @@ EXPORTS = [
     "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode", "as_hybrid_workspace",
     "as_linear_prefill_hybrid", "as_block_sparsity", "as_prefill_mode", "as_hybrid_dense_blocks",
     "as_rsparse_prefill_workspace", "as_linear_prefill_rsparse", "as_linear_prefill_nm_split",
+    "as_select_stats",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -72,6 +73,7 @@ _sig = {
     "as_linear_prefill_hybrid": ([ctypes.POINTER(as_select_out), _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, _S,
                                   _P], _I),
     "as_block_sparsity": ([_P, _I, _I, _I, _P, _P, _P, _S, _P], _I),
+    "as_select_stats": ([_P, _I, _P, _I, _I, _P, _P, _P], _I),
     "as_rsparse_decode": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P], _I),
     "as_weight_quant_fp8": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "as_select_sqrelu24_fp8": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
@@ -221,6 +223,14 @@ def as_block_sparsity(x, sparsity, n_dense: int = 0, dense_idx=None, workspace=N
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_lib.as_block_sparsity(_ptr(x), T, K, int(n_dense), _ptr(dense_idx), _ptr(sparsity), _ptr(workspace),
                                   ws_bytes, _stream(stream)), "as_block_sparsity")
+
+
+def as_select_stats(x, bitmask, kept=None, nz_dropped=None, stream=None) -> None:
+    """Per-token kept count and natural nonzeros dropped (int32 [T] each)."""
+    T, K = x.shape
+    dt = AS_BF16 if x.dtype == torch.bfloat16 else AS_F32
+    _check(_lib.as_select_stats(_ptr(x), dt, _ptr(bitmask), T, K, _ptr(kept), _ptr(nz_dropped), _stream(stream)),
+           "as_select_stats")
 
 
 def as_prefill_mode(sparsity: float) -> int:

@@ -169,6 +169,18 @@ as_status as_block_sparsity(const void *x, int T, int K, int n_dense, int32_t *d
     return cuda_status(launch_block_sparsity(x, T, K, n_dense, dense_idx, sparsity, workspace, stream));
 }
 
+as_status as_select_stats(const void *x, as_dtype dt, const uint32_t *bitmask, int T, int K, int32_t *kept,
+                          int32_t *nz_dropped, cudaStream_t stream)
+{
+    if (!x || !bitmask) return AS_ERR_INVALID_ARG;
+    if (dt != AS_F32 && dt != AS_BF16) return AS_ERR_DTYPE;
+    if (T <= 0 || K <= 0 || K % 8 != 0) return AS_ERR_SHAPE;
+    for (const void *q : {x, (const void *)bitmask, (const void *)kept, (const void *)nz_dropped})
+        if (!aligned16(q)) return AS_ERR_ALIGN;
+    if (!kept && !nz_dropped) return AS_OK;
+    return cuda_status(launch_select_stats(x, dt == AS_BF16, bitmask, T, K, kept, nz_dropped, stream));
+}
+
 as_status as_linear_prefill_hybrid(const as_select_out *sel, const void *x, int T, int K, const void *W, int n_out,
                                    int n_dense, as_dtype out_dtype, void *y, int32_t *dense_idx, float *sparsity,
                                    void *workspace, size_t ws_bytes, cudaStream_t stream)

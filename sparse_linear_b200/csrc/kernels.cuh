@@ -44,6 +44,9 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st, int wide = 0);
 bool select_rows_kernel(const SelectArgs &a);
 // N:M selection of a decode call: keep words and eta only (grid token x chunk).
 cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st);
+// Kept count and natural nonzeros dropped per token (as_select_stats).
+cudaError_t launch_select_stats(const void *x, int bf16, const uint32_t *bitmask, int T, int K, int32_t *kept,
+                                int32_t *nz_dropped, cudaStream_t st);
 
 // ------------------------------------------------------------ decode
 struct DecodeArgs {

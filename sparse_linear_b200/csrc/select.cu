@@ -967,4 +967,64 @@ cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st)
     return cudaLaunchKernelEx(&cfg, k_select_nm_decode, a);
 }
 
+// ---------------------------------------------------------------- statistics
+// Per-token kept count and natural nonzeros dropped by a selection: one CTA
+// per token (grid-strided), 8 channels per thread per step, exact integer
+// counts reduced over the block.
+template <typename TX>
+__global__ void __launch_bounds__(256) k_select_stats(const TX *__restrict__ x, const uint32_t *__restrict__ bitmask,
+                                                      int T, int K, int32_t *kept, int32_t *nz_dropped)
+{
+    __shared__ int red[2][8];
+    const int words = (K + 31) >> 5, ng = K >> 3;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        const TX *xr = x + (size_t)t * K;
+        const uint8_t *bm = reinterpret_cast<const uint8_t *>(bitmask + (size_t)t * words);
+        int nk = 0, nd = 0;
+        for (int g = threadIdx.x; g < ng; g += blockDim.x) {
+            float v[8];
+            load8(xr + 8 * g, v);
+            uint32_t nz = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) nz |= (uint32_t)(v[e] != 0.0f) << e;
+            const uint32_t keep = bm[g];
+            nk += __popc(keep);
+            nd += __popc(nz & ~keep);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            nk += __shfl_xor_sync(0xffffffffu, nk, o);
+            nd += __shfl_xor_sync(0xffffffffu, nd, o);
+        }
+        if (lane == 0) {
+            red[0][warp] = nk;
+            red[1][warp] = nd;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int a = 0, b = 0;
+            for (int w = 0; w < 8; ++w) {
+                a += red[0][w];
+                b += red[1][w];
+            }
+            if (kept) kept[t] = a;
+            if (nz_dropped) nz_dropped[t] = b;
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_select_stats(const void *x, int bf16, const uint32_t *bitmask, int T, int K, int32_t *kept,
+                                int32_t *nz_dropped, cudaStream_t st)
+{
+    const int grid = T < 4096 ? T : 4096;
+    if (bf16)
+        k_select_stats<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), bitmask, T, K,
+                                                             kept, nz_dropped);
+    else
+        k_select_stats<float><<<grid, 256, 0, st>>>(static_cast<const float *>(x), bitmask, T, K, kept, nz_dropped);
+    return cudaGetLastError();
+}
+
 }  // namespace as

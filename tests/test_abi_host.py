@@ -369,3 +369,15 @@ def test_nm_split_validation_launches_nothing(lib):
     nomask = lib.select_out(x_compact=fake, meta24=fake, bitmask24=fake)
     assert sel_f(fake, lib.AS_BF16, 4, 64, ctypes.byref(cfg), None, None, 0, ctypes.byref(nomask), None, 0,
                  None) == lib.AS_ERR_INVALID_ARG
+
+
+def test_select_stats_validation(lib):
+    fake = 1 << 20
+    f = lib._lib.as_select_stats
+    assert f(None, lib.AS_BF16, fake, 4, 64, fake, fake, None) == lib.AS_ERR_INVALID_ARG
+    assert f(fake, lib.AS_BF16, None, 4, 64, fake, fake, None) == lib.AS_ERR_INVALID_ARG
+    assert f(fake, 7, fake, 4, 64, fake, fake, None) == lib.AS_ERR_DTYPE
+    assert f(fake, lib.AS_BF16, fake, 0, 64, fake, fake, None) == lib.AS_ERR_SHAPE
+    assert f(fake, lib.AS_BF16, fake, 4, 60, fake, fake, None) == lib.AS_ERR_SHAPE
+    assert f(fake + 4, lib.AS_BF16, fake, 4, 64, fake, fake, None) == lib.AS_ERR_ALIGN
+    assert f(fake, lib.AS_BF16, fake, 4, 64, None, None, None) == lib.AS_OK  # nothing asked, nothing launched

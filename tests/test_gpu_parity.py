@@ -347,6 +347,37 @@ def test_prefill_24_full_size(sl):
     dropped = (nz & (nzm == 0)).sum() / nz.sum()
     p = 0.5 * math.erfc(1.2 / math.sqrt(2))
     assert abs(dropped - (4 * p ** 3 * (1 - p) + 2 * p ** 4) / (4 * p)) < 2e-4
+    # the same counts per token from as_select_stats, exact against the oracle
+    kept = torch.empty(x.shape[0], dtype=torch.int32, device="cuda")
+    nzd = torch.empty_like(kept)
+    sl.as_select_stats(dev(x), bufs["bitmask"], kept, nzd)
+    torch.cuda.synchronize()
+    ref_k, ref_d = oracle.select_stats(x.float().numpy(), nzm)
+    np.testing.assert_array_equal(kept.cpu().numpy(), ref_k)
+    np.testing.assert_array_equal(nzd.cpu().numpy(), ref_d)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_select_stats_ragged(sl, dtype):
+    """Kept and natural-nonzero-dropped counts for an arbitrary keep mask
+    (K = 1000: a partial last keep word), float32 and bf16 activations with
+    exact zeros, against the oracle's counts."""
+    T, K = 7, 1000
+    rng = np.random.default_rng(11)
+    x64 = rng.normal(size=(T, K)) * (rng.random((T, K)) < 0.3)
+    mask = (rng.random((T, K)) < 0.4).astype(np.uint8)
+    words = np.zeros((T, (K + 31) // 32), np.uint32)
+    for t in range(T):
+        for c in np.flatnonzero(mask[t]):
+            words[t, c // 32] |= np.uint32(1) << np.uint32(c % 32)
+    x = torch.from_numpy(x64).to(dtype)
+    kept = torch.empty(T, dtype=torch.int32, device="cuda")
+    nzd = torch.empty_like(kept)
+    sl.as_select_stats(dev(x), torch.from_numpy(words.view(np.int32)).cuda(), kept, nzd)
+    torch.cuda.synchronize()
+    ref_k, ref_d = oracle.select_stats(x.float().numpy(), mask)
+    np.testing.assert_array_equal(kept.cpu().numpy(), ref_k)
+    np.testing.assert_array_equal(nzd.cpu().numpy(), ref_d)
 
 
 def check_prefill_masked(sl, xs, W, cfg, alpha=0.0, rows=None, eta_static=None):
