@@ -29,6 +29,10 @@
  *     and an invalid call launches nothing.  A kernel that gives up a bounded
  *     wait records AS_ERR_TIMEOUT in a device status word that
  *     as_stream_status() reports.  No entry point aborts, exits or traps.
+ *   - A library built with -DAS_BOUNDS_CHECK (libactsparse_checked.so)
+ *     checks the kernels' global and shared-memory indices against the
+ *     buffers they address; a failed check skips that access and records
+ *     AS_ERR_BOUNDS in the same status word.  Default builds have no checks.
  *   - Device pointers must be 16-byte aligned (AS_ERR_ALIGN otherwise).
  *   - Channel selection is deterministic: exactly N per M-block (or exactly
  *     k_keep per token), equal float32 scores broken towards the lower channel
@@ -57,7 +61,8 @@ typedef enum as_status {
     AS_ERR_UNSUPPORTED = 5,  /* valid but unsupported combination */
     AS_ERR_WORKSPACE = 6,    /* workspace NULL or smaller than required */
     AS_ERR_CUDA = 7,         /* a CUDA runtime/driver call failed */
-    AS_ERR_TIMEOUT = 8       /* a device-side bounded wait gave up */
+    AS_ERR_TIMEOUT = 8,      /* a device-side bounded wait gave up */
+    AS_ERR_BOUNDS = 9        /* a checked build found an index outside its buffer */
 } as_status;
 
 typedef enum as_dtype { AS_F32 = 0, AS_BF16 = 1 } as_dtype;
@@ -509,6 +514,11 @@ as_status as_linear_prefill_fp8(const uint8_t *x8, const uint32_t *meta8, const 
  * as AS_ERR_TIMEOUT recorded by a kernel of this library, or AS_ERR_CUDA if
  * the stream itself failed. */
 as_status as_stream_status(cudaStream_t stream);
+
+/* Checked builds (-DAS_BOUNDS_CHECK): the source line of the first index
+ * check that failed since the last call (0 if none; always 0 in default
+ * builds), then cleared.  -1 if the device could not be read. */
+int as_checked_line(void);
 
 /* Self-test of the failure path: launches on `stream` one small kernel
  * whose bounded wait (`polls` polls, 1 .. 1<<20) is on an mbarrier that

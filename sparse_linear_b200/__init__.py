@@ -28,6 +28,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 # ---------------------------------------------------------------- constants
 AS_OK, AS_ERR_INVALID_ARG, AS_ERR_SHAPE, AS_ERR_DTYPE, AS_ERR_ALIGN = 0, 1, 2, 3, 4
 AS_ERR_UNSUPPORTED, AS_ERR_WORKSPACE, AS_ERR_CUDA, AS_ERR_TIMEOUT = 5, 6, 7, 8
+AS_ERR_BOUNDS = 9
 AS_F32, AS_BF16 = 0, 1
 AS_SCORE_MAG, AS_SCORE_WEIGHT, AS_SCORE_CLACT = 0, 1, 2
 AS_SEL_NM, AS_SEL_TOPK, AS_SEL_ALL, AS_SEL_THRESH = 0, 1, 2, 3
@@ -44,7 +45,7 @@ EXPORTS = [
     "as_linear_prefill_fp8", "as_rsparse_workspace", "as_rsparse_decode", "as_hybrid_workspace",
     "as_linear_prefill_hybrid", "as_block_sparsity", "as_prefill_mode", "as_hybrid_dense_blocks",
     "as_rsparse_prefill_workspace", "as_linear_prefill_rsparse", "as_linear_prefill_nm_split",
-    "as_select_stats",
+    "as_select_stats", "as_checked_line",
 ]
 AS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -74,6 +75,7 @@ _sig = {
                                   _P], _I),
     "as_block_sparsity": ([_P, _I, _I, _I, _P, _P, _P, _S, _P], _I),
     "as_select_stats": ([_P, _I, _P, _I, _I, _P, _P, _P], _I),
+    "as_checked_line": ([], _I),
     "as_rsparse_decode": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P], _I),
     "as_weight_quant_fp8": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "as_select_sqrelu24_fp8": ([_P, _I, _I, _P, _P, _P, _P, _P], _I),
@@ -223,6 +225,11 @@ def as_block_sparsity(x, sparsity, n_dense: int = 0, dense_idx=None, workspace=N
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_lib.as_block_sparsity(_ptr(x), T, K, int(n_dense), _ptr(dense_idx), _ptr(sparsity), _ptr(workspace),
                                   ws_bytes, _stream(stream)), "as_block_sparsity")
+
+
+def as_checked_line() -> int:
+    """Checked builds: source line of the first failed index check (0: none)."""
+    return _lib.as_checked_line()
 
 
 def as_select_stats(x, bitmask, kept=None, nz_dropped=None, stream=None) -> None:

@@ -78,6 +78,7 @@ const char *as_status_string(as_status s)
     case AS_ERR_WORKSPACE: return "AS_ERR_WORKSPACE: workspace missing or too small";
     case AS_ERR_CUDA: return "AS_ERR_CUDA: a CUDA call failed";
     case AS_ERR_TIMEOUT: return "AS_ERR_TIMEOUT: a device-side bounded wait gave up";
+    case AS_ERR_BOUNDS: return "AS_ERR_BOUNDS: a checked build found an index outside its buffer";
     }
     return "unknown as_status";
 }
@@ -658,6 +659,14 @@ as_status as_probe_timeout(unsigned polls, cudaStream_t stream)
     if (polls < 1 || polls > (1u << 20)) return AS_ERR_INVALID_ARG;
     k_probe_timeout<<<1, 32, 0, stream>>>(polls);
     return cuda_status(cudaGetLastError());
+}
+
+int as_checked_line(void)
+{
+    int line = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&line, as::g_bounds_line, sizeof(int)) != cudaSuccess) return -1;
+    if (line != 0 && cudaMemcpyToSymbol(as::g_bounds_line, &zero, sizeof(int)) != cudaSuccess) return -1;
+    return line;
 }
 
 as_status as_stream_status(cudaStream_t stream)

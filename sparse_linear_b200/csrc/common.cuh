@@ -29,6 +29,26 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Index checks of the checked build (-DAS_BOUNDS_CHECK): as_in(i, n) is
+// true when 0 <= i < n; otherwise it records AS_ERR_BOUNDS and the caller
+// skips the access.  In default builds it is the constant true and the
+// checks compile away.
+// The source line of the first failed check is kept for as_checked_line().
+__device__ int g_bounds_line = 0;
+#ifdef AS_BOUNDS_CHECK
+__device__ __forceinline__ bool as_in_at(long long i, long long n, int line)
+{
+    if (i >= 0 && i < n) return true;
+    record_status(AS_ERR_BOUNDS);
+    atomicCAS(&g_bounds_line, 0, line);
+    return false;
+}
+#define as_in(i, n) as_in_at((i), (n), __LINE__)
+#else
+__device__ __forceinline__ constexpr bool as_in_at(long long, long long, int) { return true; }
+#define as_in(i, n) as_in_at((i), (n), 0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

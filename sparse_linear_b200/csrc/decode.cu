@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
                     }
                     if (act && t == 0 && slice == 0 && a.colnorm_out) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) a.colnorm_out[c0 + e] = f[e];
+                        for (int e = 0; e < 8; ++e)
+                            if (as_in(c0 + e, K)) a.colnorm_out[c0 + e] = f[e];
                     }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
@@ -221,7 +222,8 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
             const int wl = 8 * wt + (lane >> 2);
             if ((lane & 3) == 0 && wl < nw) {
                 s_keep[t][wl] = word;
-                if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
+                if (a.mask_out && slice == 0 && as_in((long long)t * nwords + w0 + wl, (long long)T * nwords))
+                    a.mask_out[(size_t)t * nwords + w0 + wl] = word;
             }
         }
     }
@@ -319,7 +321,7 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
 
     auto emit = [&](int t, int c, float v) {
         const int o = slice * DEC_NS + c;
-        if (t < T && o < n_out) {
+        if (t < T && o < n_out && as_in((long long)t * n_out + o, (long long)T * n_out)) {
             if (a.dpts) v = fmaf(s_eta[t], a.rowsum[o], v);
             if (a.out_bf16)
                 static_cast<__nv_bfloat16 *>(a.y)[(size_t)t * n_out + o] = __float2bfloat16_rn(v);
@@ -334,7 +336,8 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(DecodeArgs a, int words_
     }
     for (int i = tid; i < TP * DEC_NS; i += DEC_THREADS) {
         const int t = i / DEC_NS, c = i % DEC_NS, o = slice * DEC_NS + c;
-        if (t < T && o < n_out) a.partial[((size_t)split * T + t) * n_out + o] = red[i];
+        if (t < T && o < n_out && as_in(((long long)split * T + t) * n_out + o, (long long)k_splits * T * n_out))
+            a.partial[((size_t)split * T + t) * n_out + o] = red[i];
     }
     __threadfence();
     __syncthreads();
@@ -476,12 +479,13 @@ __global__ void __launch_bounds__(256) k_decode_reduce(const float *__restrict__
     if (i >= n_out * G) return;
     const int o = i / G, j = i % G;
     if (R::VW * j >= T) return;
+    if (!as_in((long long)(k_splits - 1) * n_out * G + i, (long long)k_splits * n_out * G)) return;
     const V s = sum_splits<V, 24>(reinterpret_cast<const V *>(partial) + i, (size_t)n_out * G, k_splits);
     const float rs = eta ? rowsum[o] : 0.0f;
 #pragma unroll
     for (int k = 0; k < R::VW; ++k) {
         const int t = R::VW * j + k;
-        if (t < T) {
+        if (t < T && as_in((long long)t * n_out + o, (long long)T * n_out)) {
             float v = vget(s, k);
             if (eta) v = fmaf(eta[t], rs, v);
             if (out_bf16)
@@ -589,7 +593,8 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             const int pos = st * TC_KS + row;
             const int cl = DENSE ? (pos < nch ? pos : TC_PAD) : list_cl[pos];
             const int col = col0 + 8 * c16;
-            const bool ok = cl != TC_PAD && col < n_out;
+            bool ok = cl != TC_PAD && col < n_out;
+            if (ok) ok = as_in((long long)(c_begin + cl) * n_out + col + 7, (long long)K * n_out);
             const void *src = ok ? (const void *)(wt + (size_t)cl * n_out + col) : (const void *)wt;
             cp_async16(base + row * TC_WROWP + c16 * 16, src, ok ? 16u : 0u);  // 0 bytes: zero fill
         }
@@ -671,7 +676,7 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
                     q += v * v;
                 }
                 s_f[i] = (float)sqrt(q);
-                if (slice == 0 && a.colnorm_out) a.colnorm_out[c_begin + i] = s_f[i];
+                if (slice == 0 && a.colnorm_out && as_in(c_begin + i, K)) a.colnorm_out[c_begin + i] = s_f[i];
             }
             __syncthreads();
         }
@@ -705,7 +710,8 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             }
             if (lane == 0) {
                 s_keep[t][wl] = word;
-                if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
+                if (a.mask_out && slice == 0 && as_in((long long)t * nwords + w0 + wl, (long long)T * nwords))
+                    a.mask_out[(size_t)t * nwords + w0 + wl] = word;
             }
             __syncwarp();
         }
@@ -728,8 +734,9 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             const int i = tid + r * TC_THREADS;
             if (i < TP * ngc) {
                 const int t = i / ngc, g = i % ngc;
-                chv[r] = t < T ? *reinterpret_cast<const uint4 *>(x + (size_t)t * K + c_begin + 8 * g)
-                               : make_uint4(0, 0, 0, 0);
+                chv[r] = (t < T && as_in((long long)t * K + c_begin + 8 * g + 7, (long long)T * K))
+                             ? *reinterpret_cast<const uint4 *>(x + (size_t)t * K + c_begin + 8 * g)
+                             : make_uint4(0, 0, 0, 0);
             }
         }
         // DENSE: the first stages of the weight stream, also before the wait
@@ -742,7 +749,7 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         for (int i = tid; i < TP * nw; i += TC_THREADS) {
             const int t = i / nw, wl = i % nw;
             uint32_t word = 0u;
-            if (t < T) {
+            if (t < T && as_in((long long)t * nwords + w0 + wl, (long long)T * nwords)) {
                 word = a.mask_in[(size_t)t * nwords + w0 + wl];
                 if (a.mask_out && slice == 0) a.mask_out[(size_t)t * nwords + w0 + wl] = word;
             }
@@ -792,7 +799,8 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
         for (int wl = warp; wl < nw; wl += TC_WARPS) {
             const uint32_t uw = __shfl_sync(0xffffffffu, u, wl);
             const int base = __shfl_sync(0xffffffffu, inc - cnt, wl);
-            if ((uw >> lane) & 1u) list_cl[base + __popc(uw & ((1u << lane) - 1u))] = 32 * wl + lane;
+            const int li = base + __popc(uw & ((1u << lane) - 1u));
+            if (((uw >> lane) & 1u) && as_in(li, TC_MAXL) && as_in(32 * wl + lane, nch)) list_cl[li] = 32 * wl + lane;
         }
     }
     const int Lp = (L + TC_KS - 1) / TC_KS * TC_KS;
@@ -879,6 +887,11 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
             for (int nt = 0; nt < C::NT; ++nt) {
                 const int o = col0 + mt * 16 + g8;
                 const int t = nt * 8 + 2 * q4;
+                // (checked build) the last float this lane stores
+                const long long pbase = (long long)split * n_out * TP, pn = (long long)k_splits * n_out * TP;
+                const bool t_ok = o < n_out && (TP == 1 ? q4 == 0 : t < TP);
+                if (t_ok && !as_in(pbase + (long long)(o + 8 < n_out ? o + 8 : o) * TP + (TP == 1 ? 0 : t + 1), pn))
+                    continue;
                 if constexpr (TP == 1) {
                     if (q4 == 0) {
                         if (o < n_out) pp[o] = acc[mt][nt][0];
@@ -914,7 +927,7 @@ __global__ void __launch_bounds__(TC_THREADS, TcCfg<TP>::MINB)
     const int ocol0 = slice * C::NS;
     for (int i = tid; i < T * C::NS; i += TC_THREADS) {
         const int t = i / C::NS, c = i % C::NS, o = ocol0 + c;
-        if (o >= n_out) continue;
+        if (o >= n_out || !as_in((long long)t * n_out + o, (long long)T * n_out)) continue;
         float v = red[t * C::NS + c];
         if (a.dpts) v = fmaf(s_eta[t], a.rowsum[o], v);
         if (a.out_bf16)

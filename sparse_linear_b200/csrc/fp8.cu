@@ -122,9 +122,12 @@ __global__ void __launch_bounds__(F8_THREADS) k_sqrelu24_fp8(const __nv_bfloat16
     const int nch = K / 8;          // real 8-channel chunks
     const int nch_pad = kt * 32;    // chunks the metadata tiles cover
     const int tid = threadIdx.x;
-    for (int c = nch + tid; c < nch_pad; c += F8_THREADS) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
+    const long long meta_bytes = (long long)((T + 255) / 256) * 2 * kt * 1024 * 4;
+    for (int c = nch + tid; c < nch_pad; c += F8_THREADS)
+        if (as_in((long long)meta8_byte(t, c, kt), meta_bytes)) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
     if (t >= T) {                   // padding rows of the last 256-row pair tile
-        for (int c = tid; c < nch; c += F8_THREADS) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
+        for (int c = tid; c < nch; c += F8_THREADS)
+            if (as_in((long long)meta8_byte(t, c, kt), meta_bytes)) meta8[meta8_byte(t, c, kt)] = F8_PAD_META;
         return;
     }
     const __nv_bfloat16 *zr = z + (size_t)t * K;
@@ -166,6 +169,9 @@ __global__ void __launch_bounds__(F8_THREADS) k_sqrelu24_fp8(const __nv_bfloat16
             sqrelu8(held[r], x);
             uint32_t codes, meta, keep;
             chunk_codes(x, inv, codes, meta, keep);
+            if (!as_in((long long)t * (K / 2) + 4 * c + 3, (long long)T * (K / 2)) ||
+                !as_in((long long)(mb0 + (size_t)r * (F8_THREADS / 32) * 4096), meta_bytes))
+                continue;
             *reinterpret_cast<uint32_t *>(xr + 4 * c) = codes;
             meta8[mb0 + (size_t)r * (F8_THREADS / 32) * 4096] = (uint8_t)meta;
             if (bitmask) bitmask[bm_row + c] = (uint8_t)keep;

@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 tmem_ld_wait();
                 const int col0 = nt * BN + ch * 32;
                 if (!row_ok || col0 >= p.n_out) continue;
+                if (!as_in((long long)row * p.n_out + min(col0 + 31, p.n_out - 1), (long long)p.T * p.n_out)) continue;
                 if (SPARSE && p.addend) add_addend(r, p.addend, row, col0, p.n_out);
                 float v[32];
 #pragma unroll
@@ -540,6 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
             for (int ch = 0; ch < 4; ++ch) {
                 const int col0 = nt * PAIR_BN + 128 * h + 32 * ch;
                 if (col0 >= p.n_out) continue;
+                if (!as_in((long long)row * p.n_out + min(col0 + 31, p.n_out - 1), (long long)p.T * p.n_out)) continue;
                 if (!FP8 && p.addend) add_addend(r[ch], p.addend, row, col0, p.n_out);
                 if constexpr (FP8) {
                     // n_out % 8 == 0: every 4-column group past col0 starts in range
@@ -754,6 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
             for (int ch = 0; ch < 4; ++ch) {
                 const int col0 = nt * PAIR_BN + 128 * h + 32 * ch;
                 if (col0 >= p.n_out) continue;
+                if (!as_in((long long)row * p.n_out + min(col0 + 31, p.n_out - 1), (long long)p.T * p.n_out)) continue;
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {

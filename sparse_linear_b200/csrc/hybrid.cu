@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *
     for (int b = b0; b < b1; ++b) {
         const unsigned v = nnz[b];
         const bool t = v > theta || (v == theta && r++ < need);
-        if (t) idx[pos++] = b;
+        if (t && as_in(pos, n_dense)) idx[pos++] = b;
     }
 }
 
@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(HY_THREADS) k_gather_dense(const __nv_bfloat16
     const int q = blockIdx.x * HY_THREADS + threadIdx.x;
     if (q >= n_dense) return;
     const int b = idx[q];
+    if (!as_in(b, K / 4)) return;  // a dense block index outside the row
     const long long rows = (long long)T + n_out;
     for (long long r = blockIdx.y; r < rows; r += gridDim.y) {
         if (r < T) {

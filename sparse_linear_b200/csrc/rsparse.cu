@@ -98,7 +98,8 @@ __global__ void __launch_bounds__(RS_THREADS) k_rs_u(const TW *__restrict__ x, c
         float s = 0.0f;
 #pragma unroll
         for (int w = 0; w < RS_WARPS; ++w) s += s_red[((size_t)w * TP + t) * R + j];
-        part[((size_t)blockIdx.x * T + t) * R + j] = s;
+        if (as_in(((long long)blockIdx.x * T + t) * R + j, (long long)gridDim.x * T * R))
+            part[((size_t)blockIdx.x * T + t) * R + j] = s;
     }
 }
 
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(RS_THREADS) k_rs_apply(const float *__restrict
             acc = fmaf(s_u[8 * q + 2 * e + 1], __uint_as_float(ws[e] & 0xffff0000u), acc);
         }
     }
-    y[(size_t)t * n_out + o] += acc;
+    if (as_in((long long)t * n_out + o, (long long)T * n_out)) y[(size_t)t * n_out + o] += acc;
 }
 
 size_t rsparse_workspace(int T, int K, int r) { return (size_t)((K + RS_CHUNK - 1) / RS_CHUNK) * T * r * 4; }

@@ -75,6 +75,14 @@ __device__ __forceinline__ uint8_t *meta_byte(uint32_t *meta, int t, int c0, int
     return reinterpret_cast<uint8_t *>(meta) + (size_t)tile * 2048 + lane * 16 + j * 4 + byte;
 }
 
+// Writes one 2:4 metadata byte (the checked build verifies that the address
+// lies in the ceil(T / 128) x kt tiles of 2048 bytes).
+__device__ __forceinline__ void meta_put(uint32_t *meta, int t, int c0, int kt, int T, uint8_t v)
+{
+    uint8_t *b = meta_byte(meta, t, c0, kt);
+    if (as_in(b - reinterpret_cast<uint8_t *>(meta), (long long)((T + 127) / 128) * kt * 2048)) *b = v;
+}
+
 // v[base + i] for i in 0..3 without a dynamic register index.
 __device__ __forceinline__ float pick4(const float (&v)[8], int base, int i)
 {
@@ -152,7 +160,7 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
 
     if (t >= a.T) {  // padding rows of the 2:4 metadata tiles
         if (a.meta24)
-            for (int g = tid; g < kt * 16; g += NT) *meta_byte(a.meta24, t, 8 * g, kt) = 0x44;
+            for (int g = tid; g < kt * 16; g += NT) meta_put(a.meta24, t, 8 * g, kt, a.T, 0x44);
         return;
     }
     const TX *xr = static_cast<const TX *>(a.x) + (size_t)t * K;
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
             } else {
                 keep = 0xFF;
             }
-            if (act) {
+            if (act && as_in((long long)t * K + c0 + 7, (long long)a.T * K)) {
                 if (a.bitmask) {
                     uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
                     bm[g] = (uint8_t)keep;
@@ -337,13 +345,13 @@ __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
                     if (a.x_compact_lo)
                         *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
                                                    c0 / 2) = lo4(cv);
-                    if (a.meta24) *meta_byte(a.meta24, t, c0, kt) = (uint8_t)(nib[0] | (nib[1] << 4));
+                    if (a.meta24) meta_put(a.meta24, t, c0, kt, a.T, (uint8_t)(nib[0] | (nib[1] << 4)));
                 }
             }  // act
         }  // u
     }
     if (a.meta24 && tid < 16 * kt - ngroups)  // channel padding of the last 128-channel tile
-        *meta_byte(a.meta24, t, 8 * (ngroups + tid), kt) = 0x44;
+        meta_put(a.meta24, t, 8 * (ngroups + tid), kt, a.T, 0x44);
 
     // ---- VAR: variances, running average, scale
     if (a.var) {
@@ -434,7 +442,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
     int it = 0;
     for (int t = blockIdx.x; t < Tpad; t += gridDim.x, ++it) {
         if (t >= T) {  // padding rows of the 2:4 metadata tiles
-            for (int g = tid; g < kt * 16; g += SR_THREADS) *meta_byte(a.meta24, t, 8 * g, kt) = 0x44;
+            for (int g = tid; g < kt * 16; g += SR_THREADS) meta_put(a.meta24, t, 8 * g, kt, a.T, 0x44);
             continue;
         }
         const int buf = it % SR_BUFS;
@@ -481,6 +489,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
                     const int g16 = tile * SR_THREADS + tid;
                     if (g16 >= ng16) continue;
                     const int c0 = 16 * g16;
+                    if (!as_in((long long)t * K + c0 + 15, (long long)T * K)) continue;
                     const uint4 r0 = *reinterpret_cast<const uint4 *>(xr + c0);
                     const uint4 r1 = *reinterpret_cast<const uint4 *>(xr + c0 + 8);
                     const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
@@ -520,7 +529,9 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
                     if (a.x_compact_lo)  // unshifted bf16 values: nothing is lost in rounding
                         *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
                                                    c0 / 2) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint16_t *>(m16 + tile * mst16) = (uint16_t)metab;
+                    if (as_in(m16 + tile * mst16 + 1 - reinterpret_cast<uint8_t *>(a.meta24),
+                              (long long)((T + 127) / 128) * kt * 2048))
+                        *reinterpret_cast<uint16_t *>(m16 + tile * mst16) = (uint16_t)metab;
                 }
             }
         }
@@ -536,6 +547,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
                 for (int e = 0; e < 8; ++e) fv[e] = fvin[e];
             }
             score8v(v, a.dpts, eta, act && has_f, fv, xh, sc);
+            const bool in_rows = act && as_in((long long)t * K + c0 + 7, (long long)T * K);
             uint32_t keep;
             if constexpr (COMPACT) keep = keep_2of4(sc);
             else if constexpr (M == 0)
@@ -545,7 +557,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
             else if constexpr (M >= 16) keep = 2 * a.n == M ? nm_keep_half<M>(sc, lane, a.n) : nm_keep_sorted<M>(sc, lane, a.n);
             else if constexpr (M == 8) keep = nm_keep_sorted<M>(sc, lane, a.n);
             else keep = nm_keep<M>(sc, lane, a.n);
-            if (act) {
+            if (act && in_rows) {
                 if (a.bitmask) {
                     uint8_t *bm = reinterpret_cast<uint8_t *>(a.bitmask + (size_t)t * words);
                     bm[g] = (uint8_t)keep;
@@ -592,6 +604,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
                         if (a.x_compact_lo)
                             *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
                                                        c0 / 2) = lo4(cv);
+                        if (as_in(mrow + tile * mstride - reinterpret_cast<uint8_t *>(a.meta24), (long long)((T + 127) / 128) * kt * 2048))
                         mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
                         uint8_t *b24 = reinterpret_cast<uint8_t *>(a.bitmask24 + (size_t)t * words);
                         b24[g] = (uint8_t)(pos & keep);
@@ -617,7 +630,8 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
                     if (a.x_compact_lo)
                         *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.x_compact_lo) + (size_t)t * (K / 2) +
                                                    c0 / 2) = lo4(cv);
-                    mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
+                    if (as_in(mrow + tile * mstride - reinterpret_cast<uint8_t *>(a.meta24), (long long)((T + 127) / 128) * kt * 2048))
+                        mrow[tile * mstride] = (uint8_t)(nib[0] | (nib[1] << 4));
                 }
             }
         };
@@ -633,7 +647,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
             }
         }
         if (a.meta24 && tid < 16 * kt - ngroups)  // channel padding of the last 128-channel tile
-            *meta_byte(a.meta24, t, 8 * (ngroups + tid), kt) = 0x44;
+            meta_put(a.meta24, t, 8 * (ngroups + tid), kt, a.T, 0x44);
 
         // ---- VAR: variances, running average, scale
         if (!COMPACT && a.var) {
@@ -948,7 +962,8 @@ __global__ void __launch_bounds__(SELD_THREADS) k_select_nm_decode(SelectArgs a)
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
     word |= __shfl_xor_sync(0xffffffffu, word, 2);
     const int wi = c0 >> 5;
-    if ((lane & 3) == 0 && act) a.bitmask[(size_t)t * words + wi] = word;
+    if ((lane & 3) == 0 && act && as_in((long long)t * words + wi, (long long)a.T * words))
+        a.bitmask[(size_t)t * words + wi] = word;
 }
 
 cudaError_t launch_select_nm_decode(const SelectArgs &a, cudaStream_t st)
@@ -988,7 +1003,7 @@ __global__ void __launch_bounds__(256) k_select_stats(const TX *__restrict__ x, 
             uint32_t nz = 0;
 #pragma unroll
             for (int e = 0; e < 8; ++e) nz |= (uint32_t)(v[e] != 0.0f) << e;
-            const uint32_t keep = bm[g];
+            const uint32_t keep = as_in((long long)t * words * 4 + g, (long long)T * words * 4) ? bm[g] : 0u;
             nk += __popc(keep);
             nd += __popc(nz & ~keep);
         }
