@@ -341,9 +341,9 @@ int as_decode_launches(int T, int K, int n_out, as_dtype dt, const as_config *cf
  * nonzeros of x over the T tokens, ties to the lower block index; the result
  * is the masked product with D's blocks kept whole and 2:4 elsewhere:
  *   y = (x (.) m) W^T + (x (.) (1 - m))[:, D] W[:, D]^T,
- * m the 2:4 magnitude selection of x.  The second term is a dense tcgen05
- * GEMM over the 4*n_dense gathered channels (float32) that the 2:4 GEMM adds
- * in its epilogue.
+ * m the 2:4 magnitude selection of x.  The second term runs inside the 2:4
+ * GEMM: the gathered remainder of D's blocks and their W columns are extra
+ * dense tcgen05 K blocks after the sparse ones, into the same accumulator.
  *   sel      the as_select outputs of x with sel = AS_SEL_NM, n = 2, m = 4,
  *            score AS_SCORE_MAG, no token shift or VAR: bitmask, x_compact
  *            and meta24 are required.

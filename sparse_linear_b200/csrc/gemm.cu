@@ -71,11 +71,11 @@ struct GemmParams {
     int m_tiles, n_tiles, k_blocks, meta_kt;
     int kb_pass;  // K blocks of one pass over K
     int kb_main;  // kb_pass, or 2 kb_pass when a residual A operand follows
-    int rblk;     // R-Sparse: 64-wide blocks of the rank (k_blocks = kb_main + 2 rblk)
+    int rblk;     // extra dense blocks: 64-wide blocks of r (k_blocks = kb_main + u_parts rblk)
 };
 
-// R-Sparse extra K block e (0 .. 2 rblk - 1): which part of U (0 hi, 1 lo)
-// and which 64-wide block of the rank it covers.
+// Extra K block e (0 .. u_parts rblk - 1): which part of U (R-Sparse: 0 hi,
+// 1 lo) and which 64-wide block of r it covers.
 __device__ __forceinline__ void extra_block(int e, int rblk, int &part, int &j)
 {
     part = e / rblk;
@@ -886,7 +886,7 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, C::BN)) return cudaErrorInvalidValue;
     if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, ka, GEMM_BM)) return cudaErrorInvalidValue;
     CUtensorMap mU = mA, mR = mB;
-    if (a.r > 0 && (!make_map(&mU, a.U2, 2 * (uint64_t)a.T, (uint64_t)a.r, GEMM_BM) ||
+    if (a.r > 0 && (!make_map(&mU, a.U2, (uint64_t)a.u_parts * a.T, (uint64_t)a.r, GEMM_BM) ||
                     !make_map(&mR, a.Ar, (uint64_t)a.n_out, (uint64_t)a.r, C::BN)))
         return cudaErrorInvalidValue;
     GemmParams p{};
@@ -905,7 +905,7 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     p.kb_pass = (a.K + C::KB - 1) / C::KB;
     p.kb_main = p.kb_pass * (a.A_lo ? 2 : 1);
     p.rblk = a.r / 64;
-    p.k_blocks = p.kb_main + 2 * p.rblk;
+    p.k_blocks = p.kb_main + a.u_parts * p.rblk;
     p.meta_kt = (a.K + 127) / 128;
     const size_t smem = gemm_smem_bytes<SPARSE>();
     cudaError_t e = cudaFuncSetAttribute(k_gemm<SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -991,14 +991,14 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     p.kb_pass = (a.K + 127) / 128;
     p.kb_main = p.kb_pass * (a.A_lo ? 2 : 1);
     p.rblk = a.r / 64;
-    p.k_blocks = p.kb_main + 2 * p.rblk;
+    p.k_blocks = p.kb_main + a.u_parts * p.rblk;
     p.meta_kt = (a.K + 127) / 128;
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, (uint64_t)a.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map_meta(&mE, a.meta, (uint64_t)mt128 * p.meta_kt)) return cudaErrorInvalidValue;
     CUtensorMap mU = mA, mR = mB;
-    if (a.r > 0 && (!make_map(&mU, a.U2, 2 * (uint64_t)a.T, (uint64_t)a.r, 128) ||
+    if (a.r > 0 && (!make_map(&mU, a.U2, (uint64_t)a.u_parts * a.T, (uint64_t)a.r, 128) ||
                     !make_map(&mR, a.Ar, (uint64_t)a.n_out, (uint64_t)a.r, 128)))
         return cudaErrorInvalidValue;
     const size_t smem = pair_smem_bytes<false>();
@@ -1030,12 +1030,12 @@ static cudaError_t launch_gemm_dense_pair(const GemmArgs &a, cudaStream_t st)
     p.kb_pass = (a.K + 63) / 64;
     p.kb_main = p.kb_pass * (a.A_lo ? 2 : 1);
     p.rblk = a.r / 64;
-    p.k_blocks = p.kb_main + 2 * p.rblk;
+    p.k_blocks = p.kb_main + a.u_parts * p.rblk;
     if (!make_map(&mA, a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mB, a.W, (uint64_t)a.n_out, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     if (!make_map(&mA2, a.A_lo ? a.A_lo : a.A, (uint64_t)a.T, (uint64_t)a.K, 128)) return cudaErrorInvalidValue;
     CUtensorMap mU = mA, mR = mB;
-    if (a.r > 0 && (!make_map(&mU, a.U2, 2 * (uint64_t)a.T, (uint64_t)a.r, 128) ||
+    if (a.r > 0 && (!make_map(&mU, a.U2, (uint64_t)a.u_parts * a.T, (uint64_t)a.r, 128) ||
                     !make_map(&mR, a.Ar, (uint64_t)a.n_out, (uint64_t)a.r, 128)))
         return cudaErrorInvalidValue;
     const size_t smem = dense_pair_smem_bytes();

@@ -214,7 +214,6 @@ HybridLayout hybrid_layout(int T, int K, int n_out, int n_dense)
     L.idx = off;    off += up((size_t)(n_dense > 0 ? n_dense : 1) * 4);
     L.xr = off;     off += up((size_t)T * 4 * n_dense * 2);
     L.wd = off;     off += up((size_t)n_out * 4 * n_dense * 2);
-    L.yd = off;     off += up((size_t)T * n_out * 4);
     L.bytes = off;
     return L;
 }
@@ -242,30 +241,22 @@ cudaError_t launch_hybrid(const HybridArgs &a, cudaStream_t st)
     float *sp = a.sparsity_out ? a.sparsity_out : reinterpret_cast<float *>(base + L.total + 16);
     cudaError_t e = launch_block_sparsity(a.x, a.T, a.K, a.n_dense, idx, sp, a.workspace, st);
     if (e != cudaSuccess) return e;
-    const float *addend = nullptr;
+    GemmArgs s{};
     if (a.n_dense > 0) {
         __nv_bfloat16 *xr = reinterpret_cast<__nv_bfloat16 *>(base + L.xr);
         __nv_bfloat16 *wd = reinterpret_cast<__nv_bfloat16 *>(base + L.wd);
-        float *yd = reinterpret_cast<float *>(base + L.yd);
         const long long rows = (long long)a.T + a.n_out;
         dim3 g((a.n_dense + HY_THREADS - 1) / HY_THREADS, (unsigned)(rows < HY_GATHER_ROWS ? rows : HY_GATHER_ROWS));
         k_gather_dense<<<g, HY_THREADS, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.x), a.bitmask,
                                                  static_cast<const __nv_bfloat16 *>(a.W), a.T, a.K, a.n_out, idx,
                                                  a.n_dense, xr, wd);
-        GemmArgs d{};
-        d.A = xr;
-        d.W = wd;
-        d.T = a.T;
-        d.K = 4 * a.n_dense;
-        d.n_out = a.n_out;
-        d.sparse = 0;
-        d.y = yd;
-        d.out_bf16 = 0;
-        e = launch_gemm(d, st);
-        if (e != cudaSuccess) return e;
-        addend = yd;
+        // the gathered remainder against the dense blocks' W columns: extra
+        // dense K blocks of the 2:4 GEMM, into the same accumulator
+        s.U2 = xr;
+        s.Ar = wd;
+        s.r = 4 * a.n_dense;
+        s.u_parts = 1;
     }
-    GemmArgs s{};
     s.A = a.x_compact;
     s.meta = a.meta24;
     s.W = a.W;
@@ -275,7 +266,6 @@ cudaError_t launch_hybrid(const HybridArgs &a, cudaStream_t st)
     s.sparse = 1;
     s.y = a.y;
     s.out_bf16 = a.out_bf16;
-    s.addend = addend;
     s.rowsum = a.rowsum;
     s.eta = a.eta;
     s.nu = a.nu;

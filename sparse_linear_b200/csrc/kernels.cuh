@@ -93,11 +93,15 @@ struct GemmArgs {
     void *y;
     int out_bf16;
     const float *addend = nullptr;  // float32 [T, n_out] added to the accumulator (2:4 only)
-    // R-Sparse compensation: U2 bf16 [2T, r] (U hi rows, then U lo rows) and
-    // A_r bf16 [n_out, r], run as 2 r/64 extra K blocks after the main ones
+    // Extra dense K blocks after the main ones: U2 bf16 [u_parts T, r] against
+    // Ar bf16 [n_out, r], u_parts r/64 blocks of 64 into the same accumulator.
+    // R-Sparse: u_parts 2 (U hi rows, then U lo rows), Ar = A_r.  Hybrid
+    // split: u_parts 1, the gathered remainder of the dense blocks against
+    // their W columns.
     const void *U2 = nullptr;
     const void *Ar = nullptr;
     int r = 0;
+    int u_parts = 2;
 };
 // R-Sparse prefill U = (xhat (.) (1 - m)) B_r (rsparse_prefill.cu)
 struct RspLayout {
@@ -149,7 +153,7 @@ struct HybridArgs {
     const float *rowsum = nullptr, *eta = nullptr, *nu = nullptr;  // epilogue terms of the 2:4 GEMM
 };
 struct HybridLayout {
-    size_t nnz, total, idx, xr, wd, yd, bytes;
+    size_t nnz, total, idx, xr, wd, bytes;
 };
 HybridLayout hybrid_layout(int T, int K, int n_out, int n_dense);
 cudaError_t launch_block_sparsity(const void *x, int T, int K, int n_dense, int *idx, float *sparsity, void *ws,

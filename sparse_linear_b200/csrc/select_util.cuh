@@ -299,7 +299,7 @@ __device__ __forceinline__ uint32_t keep_2of4(const S (&s)[8])
     uint32_t keep = 0;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const float a = s[4 * h], b = s[4 * h + 1], c = s[4 * h + 2], d = s[4 * h + 3];
+        const S a = s[4 * h], b = s[4 * h + 1], c = s[4 * h + 2], d = s[4 * h + 3];  // no conversion
         const int ab = b > a, ac = c > a, ad = d > a, bc = c > b, bd = d > b, cd = d > c;
         const int ra = ab + ac + ad;
         const int rb = (1 - ab) + bc + bd;
