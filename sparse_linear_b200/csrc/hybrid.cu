@@ -169,10 +169,9 @@ __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *
 }
 
 // Rows 0..T-1: the dropped values of the dense blocks; rows T..T+n_out-1:
-// the weight columns of the dense blocks.  One thread per (row, block); the
-// rows are strided over gridDim.y (at most HY_GATHER_ROWS CTAs), so any
-// T + n_out fits the launch.
-constexpr int HY_GATHER_ROWS = 16384;
+// the weight columns of the dense blocks.  A CTA takes HY_GROWS rows and its
+// threads run over their (row, block) items, several loads in flight each.
+constexpr int HY_GROWS = 16;
 
 __global__ void __launch_bounds__(HY_THREADS) k_gather_dense(const __nv_bfloat16 *__restrict__ x,
                                                              const uint32_t *__restrict__ bitmask,
@@ -181,12 +180,16 @@ __global__ void __launch_bounds__(HY_THREADS) k_gather_dense(const __nv_bfloat16
                                                              __nv_bfloat16 *__restrict__ xr,
                                                              __nv_bfloat16 *__restrict__ wd)
 {
-    const int q = blockIdx.x * HY_THREADS + threadIdx.x;
-    if (q >= n_dense) return;
-    const int b = idx[q];
-    if (!as_in(b, K / 4)) return;  // a dense block index outside the row
     const long long rows = (long long)T + n_out;
-    for (long long r = blockIdx.y; r < rows; r += gridDim.y) {
+    const long long r0 = (long long)blockIdx.x * HY_GROWS;
+    const int items = HY_GROWS * n_dense;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < items; i += HY_THREADS) {
+        const long long r = r0 + i / n_dense;
+        const int q = i % n_dense;
+        if (r >= rows) continue;
+        const int b = idx[q];
+        if (!as_in(b, K / 4)) continue;  // a dense block index outside the row
         if (r < T) {
             uint2 v = *reinterpret_cast<const uint2 *>(x + (size_t)r * K + 4 * b);
             const uint32_t m = (bitmask[(size_t)r * ((K + 31) / 32) + (b >> 3)] >> (4 * (b & 7))) & 15u;
@@ -246,8 +249,7 @@ cudaError_t launch_hybrid(const HybridArgs &a, cudaStream_t st)
         __nv_bfloat16 *xr = reinterpret_cast<__nv_bfloat16 *>(base + L.xr);
         __nv_bfloat16 *wd = reinterpret_cast<__nv_bfloat16 *>(base + L.wd);
         const long long rows = (long long)a.T + a.n_out;
-        dim3 g((a.n_dense + HY_THREADS - 1) / HY_THREADS, (unsigned)(rows < HY_GATHER_ROWS ? rows : HY_GATHER_ROWS));
-        k_gather_dense<<<g, HY_THREADS, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.x), a.bitmask,
+        k_gather_dense<<<(unsigned)((rows + HY_GROWS - 1) / HY_GROWS), HY_THREADS, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.x), a.bitmask,
                                                  static_cast<const __nv_bfloat16 *>(a.W), a.T, a.K, a.n_out, idx,
                                                  a.n_dense, xr, wd);
         // the gathered remainder against the dense blocks' W columns: extra
