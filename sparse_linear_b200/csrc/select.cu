@@ -166,7 +166,10 @@ __device__ __forceinline__ uint2 lo4(const float (&cv)[4])
 template <typename TX, int NT>
 __global__ void __launch_bounds__(NT) k_select(SelectArgs a)
 {
-    // a decode kernel chained after this one may start its own loads now
+    // launched programmatically: wait for the previous kernel in the stream
+    // (it may have written x), then let a decode kernel chained after this
+    // one start its own loads (it relies on this wait having returned)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(16) uint32_t keys[];  // [K] score bits (top-k only)
     __shared__ double red[2][NT / 32];
@@ -848,13 +851,24 @@ cudaError_t launch_colnorm(const void *x, int bf16, int T, int K, float *c, void
 template <typename TX, int NT>
 static cudaError_t launch_select_t(const SelectArgs &a, size_t smem, int grid, cudaStream_t st)
 {
-    if (smem > 48 * 1024) {
+    if (smem > 40 * 1024) {  // the 48 KB default also counts the kernel's static shared memory
         static int done[64];
         cudaError_t e = smem_limit_once(k_select<TX, NT>, smem, done);
         if (e != cudaSuccess) return e;
     }
-    k_select<TX, NT><<<grid, NT, smem, st>>>(a);
-    return cudaGetLastError();
+    // programmatic launch: the CTAs become resident while the previous
+    // kernel finishes and wait for it before their first load
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_select<TX, NT>, a);
 }
 
 template <typename TX, int M, bool COMPACT, bool FREG>
