@@ -65,7 +65,6 @@ struct GemmParams {
     const uint32_t *meta;
     const float *rowsum, *eta, *nu;
     const float *xscale, *wscale;  // FP8 row scales (tokens, output rows)
-    const float *addend;           // float32 [T, n_out] added to the accumulator (2:4 kernels)
     void *y;
     int T, K, n_out, out_bf16;
     int m_tiles, n_tiles, k_blocks, meta_kt;
@@ -80,22 +79,6 @@ __device__ __forceinline__ void extra_block(int e, int rblk, int &part, int &j)
 {
     part = e / rblk;
     j = e - part * rblk;
-}
-
-// Adds row `row`, columns col0 .. col0+31 of a float32 [T, n_out] term to 32
-// accumulator values (n_out % 8 == 0: a 4-column group past n_out is
-// clamped to the last one, whose values are not stored).
-__device__ __forceinline__ void add_addend(uint32_t (&r)[32], const float *addend, int row, int col0, int n_out)
-{
-    const float *ar = addend + (size_t)row * n_out;
-#pragma unroll
-    for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 a4 = *reinterpret_cast<const float4 *>(ar + min(col0 + 4 * c4, n_out - 4));
-        r[4 * c4] = __float_as_uint(__uint_as_float(r[4 * c4]) + a4.x);
-        r[4 * c4 + 1] = __float_as_uint(__uint_as_float(r[4 * c4 + 1]) + a4.y);
-        r[4 * c4 + 2] = __float_as_uint(__uint_as_float(r[4 * c4 + 2]) + a4.z);
-        r[4 * c4 + 3] = __float_as_uint(__uint_as_float(r[4 * c4 + 3]) + a4.w);
-    }
 }
 
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int &mt, int &nt)
@@ -278,7 +261,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const int col0 = nt * BN + ch * 32;
                 if (!row_ok || col0 >= p.n_out) continue;
                 if (!as_in((long long)row * p.n_out + min(col0 + 31, p.n_out - 1), (long long)p.T * p.n_out)) continue;
-                if (SPARSE && p.addend) add_addend(r, p.addend, row, col0, p.n_out);
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -542,7 +524,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                 const int col0 = nt * PAIR_BN + 128 * h + 32 * ch;
                 if (col0 >= p.n_out) continue;
                 if (!as_in((long long)row * p.n_out + min(col0 + 31, p.n_out - 1), (long long)p.T * p.n_out)) continue;
-                if (!FP8 && p.addend) add_addend(r[ch], p.addend, row, col0, p.n_out);
                 if constexpr (FP8) {
                     // n_out % 8 == 0: every 4-column group past col0 starts in range
                     // or is clamped to the last one (its values are not stored)
@@ -894,7 +875,6 @@ static cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t st)
     p.rowsum = a.rowsum;
     p.eta = a.eta;
     p.nu = a.nu;
-    p.addend = a.addend;
     p.y = a.y;
     p.T = a.T;
     p.K = a.K;
@@ -980,7 +960,6 @@ static cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t st)
     p.rowsum = a.rowsum;
     p.eta = a.eta;
     p.nu = a.nu;
-    p.addend = a.addend;
     p.y = a.y;
     p.T = a.T;
     p.K = a.K;

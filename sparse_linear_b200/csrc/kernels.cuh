@@ -92,7 +92,6 @@ struct GemmArgs {
     const float *rowsum, *eta, *nu;  // epilogue terms (optional)
     void *y;
     int out_bf16;
-    const float *addend = nullptr;  // float32 [T, n_out] added to the accumulator (2:4 only)
     // Extra dense K blocks after the main ones: U2 bf16 [u_parts T, r] against
     // Ar bf16 [n_out, r], u_parts r/64 blocks of 64 into the same accumulator.
     // R-Sparse: u_parts 2 (U hi rows, then U lo rows), Ar = A_r.  Hybrid

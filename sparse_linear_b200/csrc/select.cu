@@ -40,26 +40,6 @@ __device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[N
     __syncthreads();
 }
 
-template <int NT>
-__device__ __forceinline__ void block_sum4(double (&v)[4], double (*red)[NT / 32])
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        v[k] = warp_sum_f64(v[k]);
-        if (lane == 0) red[k][warp] = v[k];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        double t = 0.0;
-#pragma unroll
-        for (int w = 0; w < NT / 32; ++w) t += red[k][w];
-        v[k] = t;
-    }
-    __syncthreads();
-}
-
 // Exclusive prefix sum over the block in thread order; returns the prefix,
 // `total` receives the block total.
 template <int NT>
@@ -420,7 +400,7 @@ template <typename TX, int M, bool COMPACT, bool FREG>
 __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(SelectArgs a)
 {
     extern __shared__ __align__(128) unsigned char sm[];
-    __shared__ double red[4][SR_THREADS / 32];
+    __shared__ double red[2][SR_THREADS / 32];
     __shared__ __align__(8) uint64_t bars[SR_BUFS + 1];
     const int K = a.K, T = a.T, tid = threadIdx.x, lane = tid & 31;
     const int ngroups = K >> 3, ntiles = (ngroups + SR_THREADS - 1) / SR_THREADS, kt = (K + 127) >> 7;
@@ -472,11 +452,9 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
         if (!mbar_wait(&bars[buf], (uint32_t)(it / SR_BUFS) & 1u)) return;
         const TX *xr = rows + (size_t)buf * K;
 
-        // ---- row statistics: sum x, sum x^2 (float64).  D-PTS needs the mean
-        // before selecting, so it takes a pass of its own; VAR alone (no
-        // token shift) gathers them in the selection pass below.
+        // ---- row statistics: sum x, sum x^2 (float64)
         double sx = 0.0, sxx = 0.0;
-        if (a.dpts == AS_PTS_DYNAMIC) {
+        if (a.dpts == AS_PTS_DYNAMIC || a.var) {
             for (int g = tid; g < ngroups; g += SR_THREADS) {
                 float v[8];
                 load8(xr + 8 * g, v);
@@ -488,7 +466,6 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
             }
             block_sum2<SR_THREADS>(sx, sxx, red);
         }
-        const bool var_stats = a.var && a.dpts != AS_PTS_DYNAMIC;  // the row sums come from the selection pass
         const float eta =
             a.dpts == AS_PTS_STATIC ? a.eta_static[t] : (a.dpts ? (float)(sx / (double)K) : 0.0f);
         if (a.dpts && a.eta && tid == 0) a.eta[t] = eta;
@@ -595,21 +572,11 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
 #pragma unroll
                     for (int e = 0; e < 8; ++e) km[e] = ((keep >> e) & 1u) ? xh[e] : 0.0f;
                     if (a.var) {
-                        // float32 sums of the tile's 8 values, accumulated in float64
-                        float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            s0 += v[e];
-                            s1 = fmaf(v[e], v[e], s1);
-                            s2 += km[e];
-                            s3 = fmaf(km[e], km[e], s3);
+                            skm += (double)km[e];
+                            skmm += (double)km[e] * (double)km[e];
                         }
-                        if (var_stats) {
-                            sx += (double)s0;
-                            sxx += (double)s1;
-                        }
-                        skm += (double)s2;
-                        skmm += (double)s3;
                     }
                     if (a.x_masked) store8<TX>(static_cast<TX *>(a.x_masked) + (size_t)t * K + c0, km);
                     if (a.x_masked_lo)
@@ -687,12 +654,7 @@ __global__ void __launch_bounds__(SR_THREADS, FREG ? 3 : 1) k_select_rows(Select
 
         // ---- VAR: variances, running average, scale
         if (!COMPACT && a.var) {
-            double v4[4] = {sx, sxx, skm, skmm};
-            block_sum4<SR_THREADS>(v4, red);
-            sx = v4[0];
-            sxx = v4[1];
-            skm = v4[2];
-            skmm = v4[3];
+            block_sum2<SR_THREADS>(skm, skmm, red);
             if (tid == 0) {
                 const double Kd = (double)K;
                 const double vd = (sxx - sx * sx / Kd) / (Kd - 1.0);
