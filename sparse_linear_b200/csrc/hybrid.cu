@@ -96,7 +96,11 @@ __device__ __forceinline__ int run_scan(int cnt, int *s_warp, int *sum)
 // One CTA.  theta = the n_dense-th largest count, by an MSB-first radix
 // select over three 8-bit digits (counts < 2^24); taken = count > theta, or
 // count == theta among the lowest-indexed (by a prefix count of the equal
-// ones) until n_dense; then the taken blocks in ascending order.
+// ones) until n_dense; then the taken blocks in ascending order.  A thread
+// holds its (at most HY_PICK_PER) consecutive counts in registers; warp 0
+// finds each digit with a shuffle scan over the 256 bins.
+constexpr int HY_PICK_PER = 8;  // K <= 32768: at most 8192 blocks over 1024 threads
+
 __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *__restrict__ nnz, int nb, int n_dense,
                                                                 const unsigned long long *__restrict__ total,
                                                                 double elems, int *__restrict__ idx,
@@ -105,11 +109,14 @@ __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *
     __shared__ unsigned s_hist[256];
     __shared__ unsigned s_prefix, s_rem;
     __shared__ int s_warp[HY_PICK_THREADS / 32];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     if (tid == 0) *sparsity = (float)(1.0 - (double)*total / elems);
     if (n_dense <= 0) return;
     const int per = (nb + HY_PICK_THREADS - 1) / HY_PICK_THREADS;
     const int b0 = min(nb, tid * per), b1 = min(nb, b0 + per);
+    unsigned v[HY_PICK_PER];
+#pragma unroll
+    for (int k = 0; k < HY_PICK_PER; ++k) v[k] = (k < per && b0 + k < b1) ? nnz[b0 + k] : 0u;
     if (tid == 0) {
         s_prefix = 0;
         s_rem = (unsigned)n_dense;  // rank (1-based, from the top) still to find
@@ -119,20 +126,35 @@ __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *
         __syncthreads();
         const unsigned hi_mask = shift == 16 ? 0u : (0xffffffu << (shift + 8)) & 0xffffffu;
         const unsigned prefix = s_prefix;
-        for (int b = b0; b < b1; ++b) {
-            const unsigned v = nnz[b];
-            if ((v & hi_mask) == prefix) atomicAdd(&s_hist[(v >> shift) & 255u], 1u);
-        }
+#pragma unroll
+        for (int k = 0; k < HY_PICK_PER; ++k)
+            if (b0 + k < b1 && (v[k] & hi_mask) == prefix) atomicAdd(&s_hist[(v[k] >> shift) & 255u], 1u);
         __syncthreads();
-        if (tid == 0) {
-            unsigned cum = 0, rem = s_rem;
-            for (int d = 255; d >= 0; --d) {
-                if (cum + s_hist[d] >= rem) {
-                    s_prefix = prefix | ((unsigned)d << shift);
-                    s_rem = rem - cum;
-                    break;
+        if (tid < 32) {
+            // lane l owns digits 255-8l .. 248-8l (highest first)
+            unsigned c = 0;
+#pragma unroll
+            for (int d = 0; d < 8; ++d) c += s_hist[255 - 8 * lane - d];
+            unsigned inc = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned u = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += u;
+            }
+            const unsigned rem = s_rem;
+            const unsigned hit = __ballot_sync(0xffffffffu, inc >= rem);
+            const int L = __ffs(hit) - 1;
+            if (lane == L) {
+                unsigned cum = inc - c;
+                for (int d = 0; d < 8; ++d) {
+                    const unsigned h = s_hist[255 - 8 * lane - d];
+                    if (cum + h >= rem) {
+                        s_prefix = prefix | ((unsigned)(255 - 8 * lane - d) << shift);
+                        s_rem = rem - cum;
+                        break;
+                    }
+                    cum += h;
                 }
-                cum += s_hist[d];
             }
         }
         __syncthreads();
@@ -140,32 +162,36 @@ __global__ void __launch_bounds__(HY_PICK_THREADS) k_pick_dense(const unsigned *
     const unsigned theta = s_prefix;
     // blocks above theta, and the equal ones in index order
     int gt = 0, eq = 0;
-    for (int b = b0; b < b1; ++b) {
-        gt += nnz[b] > theta;
-        eq += nnz[b] == theta;
-    }
+#pragma unroll
+    for (int k = 0; k < HY_PICK_PER; ++k)
+        if (b0 + k < b1) {
+            gt += v[k] > theta;
+            eq += v[k] == theta;
+        }
     int n_gt;
     run_scan(gt, s_warp, &n_gt);
     int n_eq;
-    int eq_rank = run_scan(eq, s_warp, &n_eq);
+    const int eq_rank = run_scan(eq, s_warp, &n_eq);
     const int need = n_dense - n_gt;  // equal blocks to take, lowest indices first
     int take = 0;
     {
         int r = eq_rank;
-        for (int b = b0; b < b1; ++b) {
-            const unsigned v = nnz[b];
-            if (v > theta) ++take;
-            else if (v == theta) take += r++ < need;
-        }
+#pragma unroll
+        for (int k = 0; k < HY_PICK_PER; ++k)
+            if (b0 + k < b1) {
+                if (v[k] > theta) ++take;
+                else if (v[k] == theta) take += r++ < need;
+            }
     }
     int n_take;
     int pos = run_scan(take, s_warp, &n_take);
     int r = eq_rank;
-    for (int b = b0; b < b1; ++b) {
-        const unsigned v = nnz[b];
-        const bool t = v > theta || (v == theta && r++ < need);
-        if (t && as_in(pos, n_dense)) idx[pos++] = b;
-    }
+#pragma unroll
+    for (int k = 0; k < HY_PICK_PER; ++k)
+        if (b0 + k < b1) {
+            const bool t = v[k] > theta || (v[k] == theta && r++ < need);
+            if (t && as_in(pos, n_dense)) idx[pos++] = b0 + k;
+        }
 }
 
 // Rows 0..T-1: the dropped values of the dense blocks; rows T..T+n_out-1:
