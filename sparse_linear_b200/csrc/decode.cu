@@ -480,7 +480,10 @@ __global__ void __launch_bounds__(256) k_decode_reduce(const float *__restrict__
     const int o = i / G, j = i % G;
     if (R::VW * j >= T) return;
     if (!as_in((long long)(k_splits - 1) * n_out * G + i, (long long)k_splits * n_out * G)) return;
-    const V s = sum_splits<V, 24>(reinterpret_cast<const V *>(partial) + i, (size_t)n_out * G, k_splits);
+    // one token: scalar partials, so every split's load is in flight at once
+    // (T = 1 runs ~37 splits); wider vectors in batches of 24 (registers)
+    constexpr int B = R::VW == 1 ? TC_SPLIT_BATCH : 24;
+    const V s = sum_splits<V, B>(reinterpret_cast<const V *>(partial) + i, (size_t)n_out * G, k_splits);
     const float rs = eta ? rowsum[o] : 0.0f;
 #pragma unroll
     for (int k = 0; k < R::VW; ++k) {
