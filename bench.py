@@ -420,12 +420,13 @@ def bench_decode(sl, dev, steps, warmup, world):
 
     # the same steps captured once per rotation index, copies included.  The
     # graph of step i decodes step i's inputs (copied in by the previous
-    # step) and forks the input copies of step i + 1 onto the H2D stream up
-    # front and each output copy onto the D2H stream after its decode, then
-    # joins them: one step's input copies overlap the previous step's
-    # decodes, every step still copies its own inputs in and its outputs out
-    # inside the timed region (step 0's inputs by a copy before the first
-    # replay; the last replay also copies the inputs of a step not run).
+    # step) while it forks the input copies of step i + 1 onto the H2D
+    # stream and the output copies of step i - 1 onto the D2H stream, then
+    # joins them: every step's inputs are copied in and its outputs copied
+    # out inside the timed region, one step ahead and one step behind its
+    # decodes (step 0's inputs by a copy before the first replay, the last
+    # step's outputs by a copy after the last; the first replay also copies
+    # out stale outputs and the last copies in inputs of a step not run).
     xg = [{T: torch.empty(T, K_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS} for _ in range(2)]
     yg = [{T: torch.empty(T, N_DOWN, dtype=torch.bfloat16, device=dev) for T in DECODE_TS} for _ in range(N_ROT)]
     yhg = [{T: torch.empty(T, N_DOWN, dtype=torch.bfloat16).pin_memory() for T in DECODE_TS} for _ in range(N_ROT)]
@@ -434,6 +435,10 @@ def bench_decode(sl, dev, steps, warmup, world):
         for T in DECODE_TS:
             xg[i % 2][T].copy_(xh[T][i % N_ROT], non_blocking=True)
 
+    def copy_out(i):
+        for T in DECODE_TS:
+            yhg[i % N_ROT][T].copy_(yg[i % N_ROT][T], non_blocking=True)
+
     def step_forked(i):
         fork = torch.cuda.Event()
         fork.record(stream)
@@ -441,13 +446,10 @@ def bench_decode(sl, dev, steps, warmup, world):
         d2h_s.wait_event(fork)
         with torch.cuda.stream(h2d_s):
             copy_in(i + 1)
+        with torch.cuda.stream(d2h_s):
+            copy_out(i - 1)
         for T in DECODE_TS:
             calls[(i, T)](xg[i % 2][T], yg[i][T])
-            e_out = torch.cuda.Event()
-            e_out.record(stream)
-            with torch.cuda.stream(d2h_s):
-                d2h_s.wait_event(e_out)
-                yhg[i][T].copy_(yg[i][T], non_blocking=True)
         j_h, j_d = torch.cuda.Event(), torch.cuda.Event()
         j_h.record(h2d_s)
         j_d.record(d2h_s)
@@ -469,9 +471,10 @@ def bench_decode(sl, dev, steps, warmup, world):
 
     def e2e_replay(j):
         if j == 0:
-            with torch.cuda.stream(stream):
-                copy_in(0)
+            copy_in(0)
         e2e_graphs[j % N_ROT].replay()
+        if j == steps - 1:
+            copy_out(j)
 
     t_e2e = max_over_ranks(timed(e2e_replay, steps), world)
     clk.__exit__(None, None, None)
@@ -1027,8 +1030,8 @@ def main():
                 "d2h_bytes_per_step": d["d2h"],
                 "mode": "per step: the pinned x of each call copied in and its y copied out (separate "
                         "copy streams); the step captured once per rotation index in a CUDA graph through "
-                        "sl.DecodeCall and replayed, each step's graph also copying in the next step's x "
-                        "(double-buffered) while it decodes",
+                        "sl.DecodeCall and replayed, each step's graph copying in the next step's x "
+                        "(double-buffered) and copying out the previous step's y while it decodes",
                 "eager_value": d["e2e_eager"],
                 "eager_mode": "the same pipelined step issued eagerly from Python every step"},
         "gpu_launches": d["launches"],
