@@ -44,6 +44,8 @@ K_DOWN, N_DOWN = 11008, 4096
 N_ROT = 8  # rotating weight/activation copies: 8 x 90 MB defeats the 126 MB L2
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "decode tokens/s & achieved HBM GB/s; prefill sparse TFLOP/s vs dense, 1 B200"
+WORKLOAD = ("decode down-projection, Llama-7B shape: x bf16 [T, 11008] for T = 1, 8, 16 per step, "
+            "W bf16 [4096, 11008], 8:16 weight-aware alpha=0.5, D-PTS")
 
 
 # ---------------------------------------------------------------- helpers
@@ -934,8 +936,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decode down-projection Llama-7B shape, x bf16 [T in {1,8,16}, 11008], "
-                                   "W bf16 [4096, 11008], 8:16 weight-aware alpha=0.5, D-PTS"},
+            "config": {"workload": WORKLOAD},
             "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -1009,8 +1010,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; Laplace(0,0.3) activations with 1% x20 outlier channels, N(0,0.02^2) "
                 "weights; no model weights)",
-        "config": {"workload": "decode down-projection, Llama-7B shape: x bf16 [T, 11008] for T = 1, 8, 16 "
-                               "per step, W bf16 [4096, 11008], 8:16 weight-aware alpha=0.5, D-PTS",
+        "config": {"workload": WORKLOAD,
                    "tokens_per_step": d["tokens_per_step"], "parallelism": f"replicas x{world}",
                    "l2": f"{N_ROT} rotating weight copies ({N_ROT * 90} MB) and activation sets per step cycle",
                    "timing": "CUDA graphs of one step replayed; CUDA events on the launching stream"},
